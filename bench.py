@@ -1,0 +1,391 @@
+"""Throughput of the VideoMLA latent-KV attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1]
+
+One step = one chunk of an autoregressive rollout through the whole path, on one batch of
+synthetic Wan2.1-1.3B-shaped input (the 6-frame window full, a 3-frame chunk of 4680 queries):
+query projection with fused 3D-RoPE, chunk latents (joint KV down-projection), attention over
+the ring plus the chunk with the W_UV up-projection fused, and the ring append.  Steps advance
+the rollout (chunk 2, 3, 4, ... of a 6-frame window), so every step has the same work.
+
+Timing: W untimed warm-up steps, then K steps between a barrier + device synchronisation on
+both sides.  L2 is flushed before every step (a 256 MiB device memset, outside the per-step
+CUDA-event intervals).  Device time per step = sum of per-step event intervals on the launch
+stream; the job time is the max over ranks.  With N > 1 every rank runs its own independent
+sample (weak scaling: no data-path collective exists on this path).
+
+value      attention algorithmic TFLOP/s of the whole step: 2*(D + d_c) = 832 flop per
+           (query row, attended key, head), divided by the whole-step device time
+e2e        the same metric through the public API with host buffers: pinned host -> device copy
+           of the step's tokens and device -> host copy of its output inside the timed interval
+roofline   the attention call (rotated-key pre-pass + tensor-core kernel), timed on its own
+           stream with CUDA events inside the timed region, against the measured bf16 peak
+cpu_baseline  the float64 CPU oracle on a bounded sample of the same chunk (rank 0, N = 1)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA attention TFLOP/s & query tokens/s (Wan-1.3B shape), % of B200 BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                s, m = float(parts[0]), float(parts[1])
+                bits = int(parts[3], 16) if parts[3].startswith("0x") else int(parts[3])
+            except ValueError:
+                continue
+            sm.append(s)
+            mx.append(m)
+            for bit, name in REASON_BITS.items():
+                if bits & bit and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+class OracleSample:
+    """The float64 oracle on sampled query rows of the measured chunk (window full).  Inputs and
+    the window are prepared once; each call times one evaluation."""
+
+    def __init__(self, cfg):
+        import oracle
+        from mla_latent_kv_attn_b200 import inputs
+        self.cfg, self.oracle, self.inputs = cfg, oracle, inputs
+        self.d = oracle.dims_from(cfg)
+        self.lw = inputs.layer_weights(cfg)
+        self.win = oracle.SlidingWindow(self.d)
+        for ch in range(cfg.measured_chunk):
+            x = inputs.chunk_x(cfg, ch)[0]
+            c, k = oracle.down_project(x, self.lw.w_dkv, self.lw.w_kr)
+            self.win.append_chunk(cfg.first_frame(ch), c, k)
+        self.x = inputs.chunk_x(cfg, cfg.measured_chunk)[0]
+
+    def __call__(self, rows: int, seed_tag: int = 7):
+        cfg = self.cfg
+        sel = self.inputs.sample_rows(cfg.n_q, rows, tag=seed_tag)
+        t0 = time.perf_counter()
+        self.oracle.chunk_step(self.d, self.lw, self.x, self.win,
+                               cfg.first_frame(cfg.measured_chunk), rows=sel, append=False)
+        dt = time.perf_counter() - t0
+        flops = 2.0 * (cfg.d_latent + cfg.d_c) * len(sel) * \
+            cfg.keys_per_query(cfg.measured_chunk) * cfg.n_heads
+        return flops, dt, len(sel)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, cfg):
+    """--impl reference: the CPU oracle as it stands, each step a bounded row sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = args.ref_rows
+    times, flops = [], 0.0
+    sample = OracleSample(cfg)
+    for i in range(args.warmup + args.steps):
+        f, dt, n = sample(rows, seed_tag=100 + i)
+        if i >= args.warmup:
+            times.append(dt)
+            flops += f
+    total = sum(times)
+    value = flops / total / 1e12
+    tok = rows * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "n_q": cfg.n_q,
+                   "keys_per_query": cfg.keys_per_query(cfg.measured_chunk),
+                   "sample": f"{rows} query rows x all heads per step"},
+        "query_tokens_per_s": tok,
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"{rows} sampled query rows of one chunk per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU path
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+    from mla_latent_kv_attn_b200 import api, inputs, rollout
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    c = api.make_config(cfg)
+    lw = inputs.layer_weights(cfg)
+    w = rollout.upload_weights(c, lw, device=dev)
+    ring = rollout.Ring(c, device=dev)
+    buf = rollout.ChunkBuffers(c, device=dev)
+    # independent sample per rank: inputs drawn with the rank as the sample index
+    n_pool = 4
+    pool = [torch.from_numpy(inputs.chunk_x(cfg, cfg.measured_chunk + i,
+                                            samples=range(rank, rank + cfg.batch)))
+            .to(device=dev, dtype=torch.bfloat16) for i in range(n_pool)]
+    for ch in range(cfg.measured_chunk):
+        buf.x.copy_(torch.from_numpy(inputs.chunk_x(cfg, ch, samples=range(rank, rank + cfg.batch)))
+                    .to(torch.bfloat16))
+        rollout.prefill_chunk(c, w, ring, buf, ch)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 6   # c_Q GEMM, Q' GEMM+RoPE, KV GEMM, rope-key pre-pass, attention, append
+
+    first_chunk = cfg.measured_chunk
+    flops_step = cfg.attention_flops(first_chunk)   # same for every later chunk (window full)
+
+    def step(i, ev=None, x=None):
+        ch = first_chunk + i
+        x = pool[i % n_pool] if x is None else x
+        first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, ch)
+        api.mla_query_proj(c, x, w.w_dq, w.w_qcat, buf.c_q, buf.q, first)
+        api.mla_cache_append(c, x, w.w_dkv_kr, buf.chunk_lat, ring.cache, ring.slot_frame,
+                             first, api.MLA_PROJECT)
+        if ev is not None:
+            ev[0].record(stream)
+        api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid,
+                              first, w.w_uv, buf.o, buf.lse, buf.workspace, buf.dev_status)
+        if ev is not None:
+            ev[1].record(stream)
+        api.mla_cache_append(c, None, None, buf.chunk_lat, ring.cache, ring.slot_frame, first,
+                             api.MLA_APPEND)
+
+    # warm-up
+    for i in range(args.warmup):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    # ---- device-timed region
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.25)
+        for i in range(args.steps):
+            flush.zero_()
+            ev_s[i].record(stream)
+            step(args.warmup + i, ev_a[i])
+            ev_e[i].record(stream)
+        torch.cuda.synchronize()
+        time.sleep(0.25)
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(ev_s, ev_e)]
+    attn_ms = [a.elapsed_time(b) for a, b in ev_a]
+    total_ms = sum(step_ms)
+    total_t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(total_t, op=dist.ReduceOp.MAX)
+    total_ms = float(total_t.item())
+    status = int(buf.dev_status.item())
+    if status != 0:
+        raise RuntimeError(f"a kernel reported status {status}")
+
+    # ---- end to end through the public API with host buffers
+    x_host = [p.cpu().pin_memory() for p in pool]
+    o_host = torch.empty(buf.o.shape, dtype=buf.o.dtype).pin_memory()
+    h2d = x_host[0].numel() * x_host[0].element_size()
+    d2h = o_host.numel() * o_host.element_size()
+    e2e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e2e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    base = args.warmup + args.steps
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_s[i].record(stream)
+        buf.x.copy_(x_host[(base + i) % n_pool], non_blocking=True)
+        step(base + i, x=buf.x)
+        o_host.copy_(buf.o, non_blocking=True)
+        e2e_e[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))], device=dev,
+                          dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(e2e_ms.item())
+
+    peaks, peak_kind = load_peaks()
+    n_units_all = world * cfg.batch
+    ms_per_step = total_ms / args.steps
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    tok_s = world * cfg.batch * cfg.n_q * args.steps / (total_ms * 1e-3)
+    attn_avg_ms = statistics.mean(attn_ms)
+    achieved = flops_step / (attn_avg_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tr_path):
+        tr = json.load(open(tr_path))
+        if tr.get("kernel_sha") == kernel_sha():
+            traffic = tr.get("bytes_per_launch")
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "n_q": cfg.n_q,
+                   "window_frames": cfg.window_frames, "chunk_frames": cfg.chunk_frames,
+                   "keys_per_query": cfg.keys_per_query(first_chunk), "heads": cfg.n_heads,
+                   "parallelism": f"replicas x{world} (independent samples)",
+                   "l2": "flushed before every step (256 MiB memset outside the event intervals)"},
+        "query_tokens_per_s": tok_s,
+        "pct_of_bf16_peak": 100.0 * value / peak,
+        "attention_call_ms": attn_avg_ms,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "mla_attention_fwd (rotated-key pre-pass + attention_tc_kernel)",
+                     "peak_kind": f"{peak_kind} burst bf16",
+                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
+        "e2e": {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12,
+                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, dt, n = OracleSample(cfg)(args.cpu_rows)
+        result["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s",
+                                  "cores": blas_threads(), "kind": "oracle",
+                                  "sample": f"{n} sampled query rows x 12 heads of one chunk "
+                                            f"({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def kernel_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("attention_sm100.cu", "sm100.cuh", "common.cuh", "kernels.h"):
+        h.update(open(os.path.join(ROOT, "mla_latent_kv_attn_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--cpu-rows", type=int, default=192)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from mla_latent_kv_attn_b200 import inputs
+    cfg = inputs.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,262 @@
+/*
+ * mla.h - C ABI of the VideoMLA latent-KV attention library for NVIDIA B200 (sm_100a).
+ *
+ * The library implements the attention hot path of VideoMLA ("VideoMLA: Low-Rank Latent KV
+ * Cache for Minute-Scale Autoregressive Video Diffusion"): multi-head latent attention over a
+ * rolling, frame-granular sliding-window cache that stores, per token, only a content latent
+ * c_KV (d_c scalars) and one head-shared, unrotated positional key k_R (d_rope scalars).
+ * Sources, cited by page and section:
+ *   [M]  hyper.ai summary of VideoMLA (English edition), "Method"; identical to the Chinese
+ *        edition's "方法" section.
+ *   [A]  chatpaper abstract of the paper, English abstract.
+ *   [F1] ai-papers.net article "VideoMLAとは？", the paragraph after Figure 1 (Wan2.1-1.3B base,
+ *        192-wide content latent, 3,072 -> 224 cached scalars per token).
+ *   [I]  hyper.ai summary, "Introduction" (rolling key-value cache; chunk-wise students).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer named as device memory must be a device (or managed) pointer on the current
+ *   device, 16-byte aligned, to a dense row-major array of the stated shape.  "T" is the
+ *   configuration's element type: bfloat16 (MLA_BF16) or float32 (MLA_FP32).
+ * - The caller owns every buffer.  The library never allocates device memory, never
+ *   synchronises the device or a stream, and keeps no pointer after a call returns.
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All work is
+ *   enqueued on it, asynchronously.
+ * - Arguments are checked on the host before anything is launched.  A rejected call returns a
+ *   non-zero mla_status, launches nothing and leaves every buffer untouched;
+ *   mla_last_error() then describes the problem.  A launch that fails returns MLA_ERR_CUDA.
+ * - Errors that only the device can see (a bounded wait inside a kernel that ran out) are
+ *   written to the optional `dev_status` word (see mla_attention_fwd); kernels never trap.
+ * - Entry points are thread-safe; mla_last_error() is per host thread.
+ *
+ * Token order.  A chunk holds chunk_frames latent frames of frame_h x frame_w tokens; tokens
+ * are ordered by frame, then row h, then column w.  Positions used by 3D-RoPE are
+ * (t, h, w) = (absolute latent-frame index since the rollout began, row, column).
+ */
+#ifndef MLA_LATENT_KV_ATTN_H_
+#define MLA_LATENT_KV_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_ABI_VERSION 1
+
+typedef enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,    /* a null pointer, a bad size or an inconsistent configuration */
+  MLA_ERR_UNSUPPORTED = 2,    /* a valid request this build does not implement */
+  MLA_ERR_ALIGNMENT = 3,      /* a pointer that is not 16-byte aligned */
+  MLA_ERR_CUDA = 4,           /* a CUDA runtime or driver call failed */
+  MLA_ERR_DEVICE_TIMEOUT = 5, /* value a kernel writes to dev_status when a bounded wait ran out */
+  MLA_ERR_WORKSPACE = 6       /* workspace missing or smaller than required */
+} mla_status;
+
+typedef enum mla_dtype { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype;
+
+/* Which kernels serve a call.  MLA_PATH_AUTO picks the tensor-core (tcgen05/TMA) kernels when
+ * the shape allows (bf16; for attention d_c = 192, d_rope = 32 and, with the W_UV epilogue,
+ * d_head = 128) and the CUDA-core kernels otherwise.  MLA_PATH_SIMT forces the CUDA-core
+ * kernels (every dtype and shape; slow but simple, used as a cross-check). */
+typedef enum mla_kernel_path { MLA_PATH_AUTO = 0, MLA_PATH_SIMT = 1 } mla_kernel_path;
+
+/* Layer shape, frame geometry and rollout geometry ([M], [F1]).
+ * D = d_c + d_rope is the cached width per token; tpf = frame_h * frame_w;
+ * n_q = chunk_frames * tpf query tokens per sample; the ring holds window_frames * tpf tokens
+ * per sample.  3D-RoPE: axis a in (t, h, w) owns rope_pairs_a adjacent channel pairs of the
+ * d_rope channels (t band first); pair i of axis a turns by pos_a * rope_base^(-i/rope_pairs_a);
+ * (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos).  The pages only say "3D-RoPE"; this is the
+ * reading adopted.  softmax_scale multiplies q.k before the softmax (1/sqrt(d_head + d_rope)
+ * in every preset). */
+typedef struct mla_config {
+  int32_t d_model;        /* token width of x                                  (Wan: 1536) */
+  int32_t n_heads;        /* H                                                 (Wan: 12)   */
+  int32_t d_head;         /* per-head width of k_nope, v and the output        (Wan: 128)  */
+  int32_t d_c;            /* content latent width                              (Wan: 192)  */
+  int32_t d_rope;         /* positional key width, = 2*(sum of rope pairs)     (Wan: 32)   */
+  int32_t d_cq;           /* query latent width                                (Wan: 512)  */
+  int32_t rope_pairs_t;   /* rotary pairs on the temporal axis                 (Wan: 4)    */
+  int32_t rope_pairs_h;   /* rotary pairs on the row axis                      (Wan: 6)    */
+  int32_t rope_pairs_w;   /* rotary pairs on the column axis                   (Wan: 6)    */
+  float rope_base;        /* rotary base                                       (10000)     */
+  float softmax_scale;    /* score scale                                       (1/sqrt(160)) */
+  int32_t frame_h;        /* latent frame height in tokens                     (Wan: 30)   */
+  int32_t frame_w;        /* latent frame width in tokens                      (Wan: 52)   */
+  int32_t chunk_frames;   /* C: frames generated per chunk                                 */
+  int32_t window_frames;  /* W: frames the ring keeps; chunk_frames <= window_frames       */
+  int32_t batch;          /* B: independent samples, each with its own ring                */
+  int32_t dtype;          /* mla_dtype of every T array                                    */
+  int32_t kernel_path;    /* mla_kernel_path                                               */
+} mla_config;
+
+/* Returns a static, human-readable name of a status code. */
+const char* mla_status_string(int32_t status);
+
+/* Returns a description of the last error raised on the calling host thread ("" if none). */
+const char* mla_last_error(void);
+
+/* Returns MLA_ABI_VERSION of the loaded library. */
+int32_t mla_abi_version(void);
+
+/* Checks a configuration without touching the device.  Errors: MLA_ERR_INVALID_ARG for
+ * non-positive sizes, d_rope != 2*(pairs), odd d_rope, chunk_frames > window_frames or an unknown
+ * dtype/path. */
+mla_status mla_config_check(const mla_config* cfg);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_cache_append: joint down-projection and ring-buffer append ([M]: "each video latent token
+ * is compressed into a shared content latent via a joint down-projection, written to the
+ * compressed KV cache"; "a single head-shared positional key k_R is computed from x via W_R^K
+ * and stored in the cache", unrotated; [A]: fixed-size sliding-window KV cache; [I]: rolling
+ * cache).
+ *
+ *   mode & MLA_PROJECT : chunk_lat[b, n, :] = [W_down^KV x[b, n] || W_R^K x[b, n]]   (T, fp32 acc.)
+ *   mode & MLA_APPEND  : for each frame f = first_frame + j, j < chunk_frames:
+ *                          slot = f mod window_frames,
+ *                          cache[b, slot*tpf + i, :] = chunk_lat[b, j*tpf + i, :]   (exact copy)
+ *                          slot_frame[b, slot] = f
+ *   MLA_PROJECT_AND_APPEND does both (the ring gets the same rounded values as chunk_lat).
+ *
+ *   x          device T [B, n_q, d_model]      (read if mode & MLA_PROJECT)
+ *   w_dkv_kr   device T [d_c + d_rope, d_model] rows 0..d_c-1 = W_down^KV, rows d_c.. = W_R^K
+ *   chunk_lat  device T [B, n_q, D]            written by PROJECT, read by APPEND
+ *   cache      device T [B, window_frames*tpf, D]  the ring (read/written only by APPEND)
+ *   slot_frame device int32 [B, window_frames] absolute frame held by each slot; -1 = empty.
+ *              The caller initialises it to -1 before the first chunk.
+ *   first_frame >= 0: absolute index of the chunk's first frame.
+ * Append a chunk only after its own attention (the ring slots it overwrites may still be in the
+ * window of that chunk).  Errors: MLA_ERR_INVALID_ARG (null pointer needed by mode, bad mode,
+ * first_frame < 0), MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+#define MLA_PROJECT 1
+#define MLA_APPEND 2
+#define MLA_PROJECT_AND_APPEND 3
+mla_status mla_cache_append(const mla_config* cfg, const void* x, const void* w_dkv_kr,
+                            void* chunk_lat, void* cache, int32_t* slot_frame,
+                            int32_t first_frame, int32_t mode, void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_rope3d: in-place 3D-RoPE ([M]: the unrotated positional key is rotated by 3D-RoPE at
+ * attention time; the positional query is rotated; [F1]: 3-D rotary position encoding).
+ *
+ *   data        device T [n_samples, rows_per_sample, row_width]; for every row, n_vec vectors
+ *               of d_rope channels start at columns col_offset + v*vec_stride (v < n_vec) and are
+ *               rotated in place (fp32 math, one rounding to T).
+ *   Row r of a sample is token i = r mod tpf of frame slot fi = r / tpf, so (h, w) =
+ *   (i / frame_w, i mod frame_w) and t = frame_table[sample*frame_table_stride + fi] when
+ *   frame_table (device int32) is non-null, else first_frame + fi.  Rows whose t is negative
+ *   (an empty ring slot) are left unchanged.  rows_per_sample must be a multiple of tpf.
+ * Errors: MLA_ERR_INVALID_ARG (sizes, vectors beyond row_width), MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_rope3d(const mla_config* cfg, void* data, int32_t n_samples,
+                      int32_t rows_per_sample, int32_t row_width, int32_t col_offset,
+                      int32_t n_vec, int32_t vec_stride, const int32_t* frame_table,
+                      int32_t frame_table_stride, int32_t first_frame, void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_key_positions: the integer (t, h, w) of every key a chunk attends to, in the order
+ * mla_attention_fwd walks them: ring slots 0 .. n_valid_frames*tpf - 1 (t from slot_frame), then
+ * the chunk's own n_q tokens (t = first_frame + j).  Which keys are attended is the window rule
+ * of [A]/[I]: the valid ring frames plus the whole chunk, bidirectionally.
+ *   slot_frame device int32 [B, window_frames]; pos_out device int32 [B, n_keys, 3] with
+ *   n_keys = (n_valid_frames + chunk_frames)*tpf.  0 <= n_valid_frames <= window_frames.
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_key_positions(const mla_config* cfg, const int32_t* slot_frame,
+                             int32_t n_valid_frames, int32_t first_frame, int32_t* pos_out,
+                             void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_compose_query_weights: weight absorption of the key up-projection into the query path.
+ * The content score q_nope_h . (W_UK_h c_KV) equals (W_UK_h^T W_UQ_h c_Q) . c_KV, so attention
+ * can run on the latent directly.  (The pages define the two-part score [M]; absorption is exact
+ * algebra, not a statement of the pages.)
+ *   w_uq  device T [H, d_head, d_cq]   per-head content-query up-projection (q_nope = W_UQ_h c_Q)
+ *   w_uk  device T [H, d_head, d_c]    per-head key up-projection
+ *   w_qr  device T [H, d_rope, d_cq]   per-head positional-query projection
+ *   w_qcat device T [H, D, d_cq]       out: rows 0..d_c-1 = W_UK_h^T W_UQ_h (fp32 accumulation,
+ *                                      one rounding to T), rows d_c.. = W_QR_h (copied)
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_compose_query_weights(const mla_config* cfg, const void* w_uq, const void* w_uk,
+                                     const void* w_qr, void* w_qcat, void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_query_proj: the query path ([M]: query latent c_Q derived from x; head-specific positional
+ * query computed from c_Q and rotated), in absorbed form.
+ *   c_q[b, n]      = W_down^Q x[b, n]                                  (T, fp32 accumulation)
+ *   q[b, n, h, :]  = [ w_qcat[h, 0:d_c] c_q  ||  RoPE3D(w_qcat[h, d_c:D] c_q, pos(b, n)) ]
+ * pos(b, n) = (first_frame + n / tpf, row, column) of chunk token n.  q is not scaled.
+ *   x      device T [B, n_q, d_model]     w_dq  device T [d_cq, d_model]
+ *   w_qcat device T [H, D, d_cq] (from mla_compose_query_weights)
+ *   c_q    device T [B, n_q, d_cq] (out)  q     device T [B, n_q, H, D] (out)
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_query_proj(const mla_config* cfg, const void* x, const void* w_dq,
+                          const void* w_qcat, void* c_q, void* q, int32_t first_frame,
+                          void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_attention_workspace_bytes: device scratch mla_attention_fwd needs for a call with the
+ * given number of valid ring frames (rotated positional keys of every attended key, tile-padded).
+ * Returns 0 for an invalid configuration.
+ * ------------------------------------------------------------------------------------------ */
+size_t mla_attention_workspace_bytes(const mla_config* cfg, int32_t n_valid_frames);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_attention_fwd: latent-space multi-head attention of one chunk against the ring plus
+ * itself ([M]: the score of head h combines q_nope.k_nope and q_rope.k_rope; per-head keys and
+ * values are reconstructed from c_KV only when needed; [A]: sliding window).
+ * Keys: ring slots 0 .. n_valid_frames*tpf - 1 (their frames from slot_frame), then the chunk's
+ * own tokens; every query of the chunk sees every one of these keys (block-causal across chunks,
+ * bidirectional inside the chunk).  For key m with latent L_m = [c_m || k_R,m]:
+ *   K'_m   = [c_m || RoPE3D(k_R,m, pos_m)]
+ *   s      = softmax_scale * q[b, n, h, :] . K'_m
+ *   p      = softmax over m (fp32)
+ *   O_lat  = sum_m p c_m                                   (the value of head h is W_UV_h c_m)
+ *   out    = W_UV_h O_lat  (if w_uv != NULL)  else  O_lat
+ *
+ *   q          device T [B, n_q, H, D]         from mla_query_proj
+ *   chunk_lat  device T [B, n_q, D]            the chunk's own latents (MLA_PROJECT)
+ *   cache      device T [B, window_frames*tpf, D] the ring; slots >= n_valid_frames*tpf unused
+ *   slot_frame device int32 [B, window_frames]
+ *   n_valid_frames  0..window_frames, first_frame >= 0
+ *   w_uv       device T [H, d_head, d_c] or NULL
+ *   out        device T [B, n_q, H*d_head] (w_uv given; heads concatenated in head order)
+ *              or device T [B, n_q, H, d_c] (w_uv NULL)
+ *   lse        device float [B, H, n_q] natural-log softmax denominators of the scaled scores,
+ *              or NULL
+ *   workspace  device scratch of >= mla_attention_workspace_bytes(cfg, n_valid_frames) bytes,
+ *              256-byte aligned; its contents on entry do not matter
+ *   dev_status device int32 word or NULL.  The caller sets it to 0; a kernel writes
+ *              MLA_ERR_DEVICE_TIMEOUT there if one of its bounded waits ran out (results are then
+ *              undefined).  The host reads it after synchronising.
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_WORKSPACE, MLA_ERR_UNSUPPORTED,
+ * MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_attention_fwd(const mla_config* cfg, const void* q, const void* chunk_lat,
+                             const void* cache, const int32_t* slot_frame,
+                             int32_t n_valid_frames, int32_t first_frame, const void* w_uv,
+                             void* out, float* lse, void* workspace, size_t workspace_bytes,
+                             int32_t* dev_status, void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_out_proj: value up-projection of latent outputs and the optional output projection
+ * ([M]: v_{t,h} is reconstructed from c_KV by W_UV_h; the output projection is the usual
+ * attention-layer output map, which the pages do not describe).
+ *   o[b, n, h*d_head:(h+1)*d_head] = W_UV_h o_lat[b, n, h]        (T, fp32 accumulation)
+ *   y[b, n] = W_O o[b, n]                                          (only if w_o and y non-null)
+ *   o_lat device T [B, n_q, H, d_c]   w_uv device T [H, d_head, d_c]   o device T [B, n_q, H*d_head]
+ *   w_o   device T [d_model, H*d_head] or NULL                        y device T [B, n_q, d_model]
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_out_proj(const mla_config* cfg, const void* o_lat, const void* w_uv,
+                        const void* w_o, void* o, void* y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_LATENT_KV_ATTN_H_ */

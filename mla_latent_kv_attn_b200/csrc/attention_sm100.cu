@@ -1,0 +1,452 @@
+// attention_sm100.cu - latent-space multi-head attention of one chunk against the ring plus
+// itself, on the sm_100a tensor cores (VideoMLA: hyper.ai summary, "Method": the score of head h
+// adds q_nope.k_nope and q_rope.k_rope; keys/values are rebuilt from c_KV only when needed).
+//
+// In absorbed form every head is a query against the same keys K'_m = [c_m || RoPE(k_R,m)]
+// (224 wide) and the same values c_m (192 wide, the first 192 columns of K'): 12-head MQA.
+//
+// One CTA = one 128-row query tile of one head of one sample.  Roles (192 threads):
+//   warps 0-3  softmax: one TMEM lane (= query row) per thread; online softmax in the log2
+//              domain with lazy rescaling of O (only when the running max grows by > 8);
+//              write P (bf16) back into TMEM over the S buffer it came from; final 1/l,
+//              optional W_UV epilogue, stores and lse.
+//   warp 4     TMA producer: Q tile once, then 128-key K' tiles into a 2-stage ring: three
+//              128x64 (128B-swizzled) content blocks from the ring/chunk latents and one 128x32
+//              (64B-swizzled) block of pre-rotated positional keys; then the W_UV_h tile.
+//   warp 5     TMEM allocation; one thread issues every tcgen05.mma:
+//                S_j   = Q K'_j^T          M=128, N=128, K=224 (12 SW128 + 2 SW64 k-steps)
+//                O    += P_j V_j           M=128, N=192, K=128; P from TMEM, V = content
+//                                          blocks of the same stage read MN-major
+//                o     = O_lat W_UV_h^T    M=128, N=128, K=192 (epilogue, O_lat bf16 in smem)
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,448); the epilogue result reuses S0.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace mla {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;           // query rows per CTA
+constexpr int kBN = kKeyTile;      // keys per tile
+constexpr int kDc = 192;           // content latent width
+constexpr int kDr = 32;            // positional key width
+constexpr int kD = kDc + kDr;      // 224
+constexpr int kDh = 128;           // head width of the W_UV epilogue
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+
+constexpr int kBlk = kBM * 128;                  // one 128-row x 128-byte block: 16 KB
+constexpr int kRopeBlk = kBN * kDr * 2;          // 8 KB
+constexpr int kTile = 3 * kBlk + kRopeBlk;       // 56 KB: Q tile or one K' stage
+constexpr int kSmem = (1 + kStages) * kTile + 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;
+
+struct AttnParams {
+  int n_q, H, nc, nc_pad, nt_ring, nt;
+  float scale_log2;
+  int has_w_uv;
+  void* out;
+  float* lse;
+  int32_t* dev_status;
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Bounded wait that also gives up once another role has given up.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int32_t* dev_status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long start = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - start > kWaitLimitCycles) {
+      *abort_flag = 1;
+      if (dev_status != nullptr) atomicExch(dev_status, static_cast<int32_t>(MLA_ERR_DEVICE_TIMEOUT));
+      return false;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
+                        const __grid_constant__ CUtensorMap tm_cache,
+                        const __grid_constant__ CUtensorMap tm_chunk,
+                        const __grid_constant__ CUtensorMap tm_ws,
+                        const __grid_constant__ CUtensorMap tm_wuv, AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_full;
+  __shared__ __align__(8) uint64_t kv_full[kStages];
+  __shared__ __align__(8) uint64_t kv_empty[kStages];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t p_full[2];
+  __shared__ __align__(8) uint64_t pv_done;
+  __shared__ __align__(8) uint64_t w_full;
+  __shared__ __align__(8) uint64_t olat_full;
+  __shared__ __align__(8) uint64_t epi_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sQ = sbase;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int q0 = qt * kBM;
+  volatile int* abort_flag = &abort_sh;
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(smem_u32(&q_full), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&kv_full[s]), 1);
+      mbar_init(smem_u32(&kv_empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&p_full[i]), 128);
+    }
+    mbar_init(smem_u32(&pv_done), 1);
+    mbar_init(smem_u32(&w_full), 1);
+    mbar_init(smem_u32(&olat_full), 128);
+    mbar_init(smem_u32(&epi_done), 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_chunk);
+      tma_prefetch_desc(&tm_ws);
+      const uint32_t qb = smem_u32(&q_full);
+      mbar_arrive_expect_tx(qb, kTile);
+      for (int i = 0; i < 3; ++i) tma_load_4d(sQ + i * kBlk, &tm_q, qb, 64 * i, h, q0, b);
+      tma_load_4d(sQ + 3 * kBlk, &tm_qr, qb, kDc, h, q0, b);
+      for (int j = 0; j <= p.nt; ++j) {
+        const int s = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        if (j == p.nt && !p.has_w_uv) break;
+        if (!wait_bar(smem_u32(&kv_empty[s]), ph ^ 1, abort_flag, p.dev_status)) break;
+        const uint32_t dst = sbase + (1 + s) * kTile;
+        if (j == p.nt) {   // W_UV_h tile [128 x 192] into the content blocks of this stage
+          const uint32_t wb = smem_u32(&w_full);
+          mbar_arrive_expect_tx(wb, 3 * kBlk);
+          for (int i = 0; i < 3; ++i) tma_load_2d(dst + i * kBlk, &tm_wuv, wb, 64 * i, h * kDh);
+          break;
+        }
+        const uint32_t fb = smem_u32(&kv_full[s]);
+        mbar_arrive_expect_tx(fb, kTile);
+        if (j < p.nt_ring) {
+          const int r0 = j * kBN;
+          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlk, &tm_cache, fb, 64 * i, r0, b);
+          tma_load_3d(dst + 3 * kBlk, &tm_ws, fb, 0, r0, b);
+        } else {
+          const int r0 = (j - p.nt_ring) * kBN;
+          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlk, &tm_chunk, fb, 64 * i, r0, b);
+          tma_load_3d(dst + 3 * kBlk, &tm_ws, fb, 0, p.nc_pad + r0, b);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDc, 0, 1);
+      constexpr uint32_t idesc_uv = idesc_bf16_f32(kBM, kDh, 0, 0);
+      bool ok = wait_bar(smem_u32(&q_full), 0, abort_flag, p.dev_status);
+      auto issue_qk = [&](int j) {
+        const int s = j % kStages;
+        const uint32_t kt = sbase + (1 + s) * kTile;
+        const uint32_t d = tmem + (j & 1) * kBN;
+#pragma unroll
+        for (int blk = 0; blk < 3; ++blk)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc(sQ + blk * kBlk + 32 * kk, 16, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(kt + blk * kBlk + 32 * kk, 16, 1024, kSwizzle128B);
+            mma_ss(d, ad, bd, idesc_qk, (blk | kk) != 0 ? 1u : 0u);
+          }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint64_t ad = smem_desc(sQ + 3 * kBlk + 32 * kk, 16, 512, kSwizzle64B);
+          const uint64_t bd = smem_desc(kt + 3 * kBlk + 32 * kk, 16, 512, kSwizzle64B);
+          mma_ss(d, ad, bd, idesc_qk, 1u);
+        }
+        mma_commit(smem_u32(&s_full[j & 1]));
+      };
+      if (ok) ok = wait_bar(smem_u32(&kv_full[0]), 0, abort_flag, p.dev_status);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0);
+      }
+      for (int j = 0; j < p.nt && ok; ++j) {
+        if (j + 1 < p.nt) {
+          const int s1 = (j + 1) % kStages;
+          ok = wait_bar(smem_u32(&kv_full[s1]), ((j + 1) / kStages) & 1, abort_flag, p.dev_status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(j + 1);
+        }
+        ok = wait_bar(smem_u32(&p_full[j & 1]), (j >> 1) & 1, abort_flag, p.dev_status);
+        if (!ok) break;
+        tc_fence_after();
+        const int s = j % kStages;
+        const uint32_t vt = sbase + (1 + s) * kTile;
+        const uint32_t pa = tmem + (j & 1) * kBN;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // V rows kk*16 .. +15: 16 rows x 128 B further per step; N blocks 16 KB apart
+          const uint64_t bd = smem_desc(vt + kk * 2048, kBlk, 1024, kSwizzle128B);
+          mma_ts(tmem + kColO, pa + kk * 8, bd, idesc_pv, (j | kk) != 0 ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&kv_empty[s]));
+        mma_commit(smem_u32(&pv_done));
+      }
+      if (ok && p.has_w_uv) {
+        ok = wait_bar(smem_u32(&w_full), 0, abort_flag, p.dev_status) &&
+             wait_bar(smem_u32(&olat_full), 0, abort_flag, p.dev_status);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t wt = sbase + (1 + p.nt % kStages) * kTile;
+#pragma unroll
+          for (int blk = 0; blk < 3; ++blk)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc(sQ + blk * kBlk + 32 * kk, 16, 1024, kSwizzle128B);
+              const uint64_t bd = smem_desc(wt + blk * kBlk + 32 * kk, 16, 1024, kSwizzle128B);
+              mma_ss(tmem, ad, bd, idesc_uv, (blk | kk) != 0 ? 1u : 0u);
+            }
+          mma_commit(smem_u32(&epi_done));
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warps 0..3
+    const int row = warp * 32 + lane;                 // TMEM lane and query row in the tile
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int n = q0 + row;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < p.nt; ++j) {
+      ok = __all_sync(0xffffffffu,
+                      wait_bar(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_flag, p.dev_status));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t sc = tmem + lane_off + (j & 1) * kBN;
+      float s[kBN];
+      {
+        uint32_t r[kBN];
+        tmem_ld128_wait(sc, r);
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
+      }
+      const int valid = j < p.nt_ring ? min(kBN, p.nc - j * kBN)
+                                      : min(kBN, p.n_q - (j - p.nt_ring) * kBN);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        s[c] = c < valid ? s[c] * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, s[c]);
+      }
+      if (j == 0) {
+        m_run = mx;
+      } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
+        // O must be rescaled: wait until PV(j-1) has landed, then scale this warp's rows.
+        ok = __all_sync(0xffffffffu,
+                        wait_bar(smem_u32(&pv_done), (j - 1) & 1, abort_flag, p.dev_status));
+        if (!ok) break;
+        tc_fence_after();
+        const float m_new = fmaxf(m_run, mx);
+        const float alpha = fast_exp2(m_run - m_new);
+        l_run *= alpha;
+        m_run = m_new;
+#pragma unroll 1
+        for (int c = 0; c < kDc; c += 16) {
+          uint32_t r[16];
+          tmem_ld16_wait(tmem + lane_off + kColO + c, r);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st16(tmem + lane_off + kColO + c, r);
+        }
+        tmem_wait_st();
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBN; c += 32) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(s[c + 2 * i] - m_run);
+          const float p1 = fast_exp2(s[c + 2 * i + 1] - m_run);
+          sum += p0 + p1;
+          w[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(sc + c / 2, w);
+      }
+      l_run += sum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&p_full[j & 1]));
+    }
+    if (ok)
+      ok = __all_sync(0xffffffffu,
+                      wait_bar(smem_u32(&pv_done), (p.nt - 1) & 1, abort_flag, p.dev_status));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      if (p.lse != nullptr && n < p.n_q)
+        p.lse[(static_cast<int64_t>(b) * p.H + h) * p.n_q + n] =
+            (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      if (!p.has_w_uv) {
+        bf16* orow = static_cast<bf16*>(p.out) +
+                     ((static_cast<int64_t>(b) * p.n_q + n) * p.H + h) * kDc;
+#pragma unroll 1
+        for (int c = 0; c < kDc; c += 32) {
+          uint32_t r[32];
+          tmem_ld32_wait(tmem + lane_off + kColO + c, r);
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+          if (n < p.n_q) {
+            uint4* d4 = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+      } else {
+        // O_lat (bf16) -> shared memory, 128B-swizzled K-major, over the dead Q tile.
+        uint8_t* qsm = smem_raw + (sQ - smem_u32(smem_raw));
+#pragma unroll 1
+        for (int c = 0; c < kDc; c += 32) {
+          uint32_t r[32];
+          tmem_ld32_wait(tmem + lane_off + kColO + c, r);
+          const int blk = c / 64;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {         // four 16-byte chunks of 8 values
+            const int chunk = (c % 64) / 8 + ch;   // chunk index within the 128-byte row
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(r[8 * ch + 0]) * inv_l, __uint_as_float(r[8 * ch + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(r[8 * ch + 2]) * inv_l, __uint_as_float(r[8 * ch + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(r[8 * ch + 4]) * inv_l, __uint_as_float(r[8 * ch + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(r[8 * ch + 6]) * inv_l, __uint_as_float(r[8 * ch + 7]) * inv_l);
+            const int off = blk * kBlk + row * 128 + ((chunk ^ (row & 7)) * 16);
+            *reinterpret_cast<uint4*>(qsm + off) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&olat_full));
+        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&epi_done), 0, abort_flag, p.dev_status));
+        if (ok) {
+          tc_fence_after();
+          bf16* orow = static_cast<bf16*>(p.out) +
+                       (static_cast<int64_t>(b) * p.n_q + n) * (static_cast<int64_t>(p.H) * kDh) +
+                       static_cast<int64_t>(h) * kDh;
+#pragma unroll 1
+          for (int c = 0; c < kDh; c += 32) {
+            uint32_t r[32];
+            tmem_ld32_wait(tmem + lane_off + c, r);
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            if (n < p.n_q) {
+              uint4* d4 = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool tc_attention_supported(const Dims& d, bool has_w_uv) {
+  return d.dtype == MLA_BF16 && d.d_c == kDc && d.d_rope == kDr && (!has_w_uv || d.d_head == kDh);
+}
+
+mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
+  const KeyWorkspace kw = key_workspace_layout(d, n_valid);
+  CUtensorMap tq, tqr, tcache, tchunk, tws, twuv;
+  mla_status st;
+  {
+    const uint64_t dims[4] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.H),
+                              static_cast<uint64_t>(d.n_q), static_cast<uint64_t>(d.B)};
+    const uint64_t strides[3] = {kD * 2ull, static_cast<uint64_t>(d.H) * kD * 2,
+                                 static_cast<uint64_t>(d.n_q) * d.H * kD * 2};
+    const uint32_t box[4] = {64, 1, kBM, 1};
+    if ((st = make_tmap_bf16(&tq, a.q, 4, dims, strides, box, 128)) != MLA_OK) return st;
+    const uint32_t box_r[4] = {kDr, 1, kBM, 1};
+    if ((st = make_tmap_bf16(&tqr, a.q, 4, dims, strides, box_r, 64)) != MLA_OK) return st;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.n_q),
+                              static_cast<uint64_t>(d.B)};
+    const uint64_t strides[2] = {kD * 2ull, static_cast<uint64_t>(d.n_q) * kD * 2};
+    const uint32_t box[3] = {64, kBN, 1};
+    if ((st = make_tmap_bf16(&tchunk, a.chunk_lat, 3, dims, strides, box, 128)) != MLA_OK) return st;
+  }
+  if (kw.nc > 0) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(kw.nc),
+                              static_cast<uint64_t>(d.B)};
+    const uint64_t strides[2] = {kD * 2ull, static_cast<uint64_t>(d.W) * d.tpf * kD * 2};
+    const uint32_t box[3] = {64, kBN, 1};
+    if ((st = make_tmap_bf16(&tcache, a.cache, 3, dims, strides, box, 128)) != MLA_OK) return st;
+  } else {
+    tcache = tchunk;  // never read: no ring tiles
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(kDr), static_cast<uint64_t>(kw.rows),
+                              static_cast<uint64_t>(d.B)};
+    const uint64_t strides[2] = {kDr * 2ull, static_cast<uint64_t>(kw.rows) * kDr * 2};
+    const uint32_t box[3] = {kDr, kBN, 1};
+    if ((st = make_tmap_bf16(&tws, a.ws, 3, dims, strides, box, 64)) != MLA_OK) return st;
+  }
+  if (a.w_uv != nullptr) {
+    const uint64_t dims[2] = {static_cast<uint64_t>(kDc), static_cast<uint64_t>(d.H) * kDh};
+    const uint64_t strides[1] = {kDc * 2ull};
+    const uint32_t box[2] = {64, kDh};
+    if ((st = make_tmap_bf16(&twuv, a.w_uv, 2, dims, strides, box, 128)) != MLA_OK) return st;
+  } else {
+    twuv = tchunk;    // never read
+  }
+  AttnParams p;
+  p.n_q = d.n_q; p.H = d.H; p.nc = kw.nc; p.nc_pad = kw.nc_pad;
+  p.nt_ring = ceil_div(kw.nc, kBN);
+  p.nt = p.nt_ring + ceil_div(d.n_q, kBN);
+  p.scale_log2 = d.scale * 1.4426950408889634f;
+  p.has_w_uv = a.w_uv != nullptr;
+  p.out = a.out; p.lse = a.lse; p.dev_status = a.dev_status;
+  MLA_CUDA_TRY(cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kSmem));
+  dim3 grid(ceil_div(d.n_q, kBM), d.H, d.B);
+  attention_tc_kernel<<<grid, kThreads, kSmem, s>>>(tq, tqr, tcache, tchunk, tws, twuv, p);
+  MLA_LAUNCH_CHECK("attention_tc");
+  return MLA_OK;
+}
+
+}  // namespace mla

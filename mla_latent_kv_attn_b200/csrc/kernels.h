@@ -1,0 +1,107 @@
+// kernels.h - internal launchers shared by the C ABI (mla_abi.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace mla {
+
+// Keys are walked in tiles of this many rows by every attention kernel; the rotated-key
+// workspace pads the ring part and the chunk part to a multiple of it.
+constexpr int kKeyTile = 128;
+
+// Strided batched GEMM  C[z](m, n) = sum_k A[z](m, k) B[z](n, k)  (element strides).
+struct GemmArgs {
+  const void* A;
+  const void* B;
+  void* C;
+  int M, N, K, batch;
+  int64_t a_sm, a_sk, a_batch;
+  int64_t b_sn, b_sk, b_batch;
+  int64_t c_sm, c_batch;
+};
+
+struct AttnArgs {
+  const void* q;          // [B, n_q, H, D]
+  const void* chunk_lat;  // [B, n_q, D]
+  const void* cache;      // [B, W*tpf, D]
+  const void* ws;         // rotated keys [B, rows, d_rope]
+  const void* w_uv;       // [H, d_head, d_c] or null
+  void* out;              // [B, n_q, H*d_head] or [B, n_q, H, d_c]
+  float* lse;             // [B, H, n_q] or null
+  int32_t* dev_status;    // or null
+};
+
+struct KeyWorkspace {
+  int nc;       // ring keys attended (n_valid * tpf)
+  int nc_pad;   // nc rounded up to kKeyTile: row of the first chunk key
+  int rows;     // rows per sample
+  size_t bytes; // whole workspace
+};
+
+KeyWorkspace key_workspace_layout(const Dims& d, int n_valid);
+
+// CUDA-core kernels (simt.cu)
+mla_status gemm_simt(const GemmArgs& g, int dtype, cudaStream_t s);
+mla_status rope3d_inplace(const Dims& d, void* data, int n_samples, int rows, int row_width,
+                          int col_offset, int n_vec, int vec_stride, const int32_t* frame_table,
+                          int frame_table_stride, int first_frame, cudaStream_t s);
+mla_status ring_append(const Dims& d, const void* chunk_lat, void* cache, int32_t* slot_frame,
+                       int first_frame, cudaStream_t s);
+mla_status key_positions(const Dims& d, const int32_t* slot_frame, int n_valid, int first_frame,
+                         int32_t* out, cudaStream_t s);
+mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_lat,
+                           const int32_t* slot_frame, int n_valid, int first_frame, void* ws,
+                           cudaStream_t s);
+mla_status attention_simt(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
+mla_status copy_rows(int dtype, const void* src, int64_t src_stride, void* dst,
+                     int64_t dst_stride, int rows, int cols, int64_t src_batch,
+                     int64_t dst_batch, int batch, cudaStream_t s);
+
+// Tensor-core kernels (gemm_sm100.cu, attention_sm100.cu)
+
+// Epilogues of the tcgen05 GEMM.
+enum GemmEpilogue : int {
+  kEpiStore = 0,     // C[m, n] = acc (bf16)
+  kEpiRopeQ = 1,     // as kEpiStore, and 3D-RoPE on the last d_rope columns of every
+                     // D-wide head block of the output row (query path)
+};
+
+struct TcGemmArgs {
+  // A: [batch][M, K] rows with element stride a_sm, batch stride a_batch; K contiguous.
+  const void* A;
+  int64_t a_sm, a_batch;
+  // B: [batch][N, K], K contiguous.
+  const void* B;
+  int64_t b_sn, b_batch;
+  // C: [batch][M, N] bf16, row stride c_sm, batch stride c_batch; N contiguous.
+  void* C;
+  int64_t c_sm, c_batch;
+  int M, N, K, batch;
+  int epilogue;
+  // kEpiRopeQ: rows are chunk tokens of samples of n_q rows; head blocks of width D.
+  int rope_D, rope_n_q, rope_first_frame;
+  RopeGeom rope;
+};
+
+bool tc_gemm_supported(int M, int N, int K, int64_t a_sm, int64_t b_sn);
+mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s);
+
+bool tc_attention_supported(const Dims& d, bool has_w_uv);
+mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
+
+}  // namespace mla
+
+#include <cuda.h>
+
+namespace mla {
+
+// Encodes a tiled TMA descriptor over a bf16 tensor.  dims[0] is the contiguous dimension;
+// strides_bytes[i] is the byte stride of dims[i + 1]; box[i] the tile extent per dimension;
+// swizzle_bytes 0, 32, 64 or 128.  Out-of-range elements of a tile read as zero.
+mla_status make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                          const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
+
+}  // namespace mla

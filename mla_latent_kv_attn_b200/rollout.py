@@ -1,0 +1,136 @@
+"""Host-side driver of a chunked rollout: the schedule, the ring state and the per-chunk calls.
+
+A rollout generates chunk after chunk of ``chunk_frames`` latent frames.  Chunk c covers frames
+c*C .. c*C + C - 1; it attends to the frames still in the window (at most W earlier frames) and
+to itself, then its latents enter the ring (hyper.ai summary of VideoMLA, "Introduction":
+streaming students generate frames with a rolling key-value cache; chatpaper abstract: the
+window has a fixed size).
+
+The ring stores frame f in slot f mod W.  Frames are appended in order from frame 0, so the
+first min(frames so far, W) slots are exactly the filled ones and attention walks slots
+0 .. n_valid*tpf - 1 (the softmax does not depend on key order).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Tuple
+
+import torch
+
+from . import api
+from .api import MLA_APPEND, MLA_PROJECT, MLA_PROJECT_AND_APPEND
+
+
+def chunk_schedule(chunk_frames: int, window_frames: int, chunk: int) -> Tuple[int, int]:
+    """(first_frame, n_valid_frames) of a chunk."""
+    first = chunk * chunk_frames
+    return first, min(first, window_frames)
+
+
+@dataclasses.dataclass
+class DeviceWeights:
+    """One layer's weights on the device, in the layouts the C ABI takes."""
+
+    w_dkv_kr: torch.Tensor   # [d_c + d_rope, d_model]
+    w_dq: torch.Tensor       # [d_cq, d_model]
+    w_qcat: torch.Tensor     # [H, d_c + d_rope, d_cq]  (composed on the device)
+    w_uv: torch.Tensor       # [H, d_head, d_c]
+    w_o: torch.Tensor        # [d_model, H*d_head]
+
+
+def upload_weights(c, lw, device="cuda", stream=None) -> DeviceWeights:
+    """Copies a layer's weights (numpy, already dtype-rounded) and composes the absorbed query
+    weights on the device."""
+    dt = api.torch_dtype(c)
+    t = lambda a: torch.from_numpy(a).to(device=device, dtype=dt).contiguous()
+    import numpy as np
+    w_uq, w_uk, w_qr = t(lw.w_uq), t(lw.w_uk), t(lw.w_qr)
+    w_qcat = torch.empty((c.n_heads, c.d_c + c.d_rope, c.d_cq), device=device, dtype=dt)
+    api.mla_compose_query_weights(c, w_uq, w_uk, w_qr, w_qcat, stream=stream)
+    return DeviceWeights(w_dkv_kr=t(np.concatenate([lw.w_dkv, lw.w_kr], 0)), w_dq=t(lw.w_dq),
+                         w_qcat=w_qcat, w_uv=t(lw.w_uv), w_o=t(lw.w_o))
+
+
+class Ring:
+    """The latent cache of one layer for B samples: cache [B, W*tpf, D] and slot_frame [B, W]."""
+
+    def __init__(self, c, device="cuda"):
+        tpf = c.frame_h * c.frame_w
+        self.c = c
+        self.cache = torch.zeros((c.batch, c.window_frames * tpf, c.d_c + c.d_rope),
+                                 device=device, dtype=api.torch_dtype(c))
+        self.slot_frame = torch.full((c.batch, c.window_frames), -1, device=device,
+                                     dtype=torch.int32)
+
+    def state_dict(self):
+        return {"cache": self.cache.clone(), "slot_frame": self.slot_frame.clone()}
+
+    def load_state_dict(self, sd):
+        self.cache.copy_(sd["cache"])
+        self.slot_frame.copy_(sd["slot_frame"])
+
+
+class ChunkBuffers:
+    """Per-chunk activations and scratch, allocated once per workload."""
+
+    def __init__(self, c, device="cuda", fuse_uv: bool = True):
+        tpf = c.frame_h * c.frame_w
+        n_q = c.chunk_frames * tpf
+        D = c.d_c + c.d_rope
+        dt = api.torch_dtype(c)
+        B, H = c.batch, c.n_heads
+        self.x = torch.empty((B, n_q, c.d_model), device=device, dtype=dt)
+        self.c_q = torch.empty((B, n_q, c.d_cq), device=device, dtype=dt)
+        self.q = torch.empty((B, n_q, H, D), device=device, dtype=dt)
+        self.chunk_lat = torch.empty((B, n_q, D), device=device, dtype=dt)
+        self.o = torch.empty((B, n_q, H * c.d_head), device=device, dtype=dt)
+        self.o_lat = torch.empty((B, n_q, H, c.d_c), device=device, dtype=dt)
+        self.lse = torch.empty((B, H, n_q), device=device, dtype=torch.float32)
+        ws = api.mla_attention_workspace_bytes(c, c.window_frames)
+        self.workspace = torch.empty((max(ws, 256),), device=device, dtype=torch.uint8)
+        self.dev_status = torch.zeros((1,), device=device, dtype=torch.int32)
+
+
+def attend_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
+                 fuse_uv: bool = True, stream=None) -> torch.Tensor:
+    """Query path, chunk latents and attention of one chunk (buf.x holds its tokens).
+    Returns buf.o (fused W_UV) or buf.o_lat (latent output)."""
+    first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
+    api.mla_query_proj(c, buf.x, w.w_dq, w.w_qcat, buf.c_q, buf.q, first, stream=stream)
+    api.mla_cache_append(c, buf.x, w.w_dkv_kr, buf.chunk_lat, ring.cache, ring.slot_frame, first,
+                         MLA_PROJECT, stream=stream)
+    out = buf.o if fuse_uv else buf.o_lat
+    api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid, first,
+                          w.w_uv if fuse_uv else None, out, buf.lse, buf.workspace,
+                          buf.dev_status, stream=stream)
+    return out
+
+
+def append_chunk(c, ring: Ring, buf: ChunkBuffers, chunk: int, stream=None) -> None:
+    """Moves the chunk's latents (buf.chunk_lat) into the ring, after its attention."""
+    first, _ = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
+    api.mla_cache_append(c, None, None, buf.chunk_lat, ring.cache, ring.slot_frame, first,
+                         MLA_APPEND, stream=stream)
+
+
+def prefill_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
+                  stream=None) -> None:
+    """Projects buf.x and appends it to the ring without attending (cache warm-up)."""
+    first, _ = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
+    api.mla_cache_append(c, buf.x, w.w_dkv_kr, buf.chunk_lat, ring.cache, ring.slot_frame, first,
+                         MLA_PROJECT_AND_APPEND, stream=stream)
+
+
+def run_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
+              fuse_uv: bool = True, stream=None) -> torch.Tensor:
+    """One whole chunk: attend, then append."""
+    out = attend_chunk(c, w, ring, buf, chunk, fuse_uv=fuse_uv, stream=stream)
+    append_chunk(c, ring, buf, chunk, stream=stream)
+    return out
+
+
+def check_device_status(buf: ChunkBuffers) -> None:
+    """Raises if a kernel reported a bounded wait that ran out (reads one int; synchronises)."""
+    v = int(buf.dev_status.item())
+    if v != 0:
+        raise api.MLAError("device", v, "a kernel's bounded wait ran out")

@@ -1,0 +1,197 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 CPU oracle, element by
+element, on identical seeded inputs.
+
+Floating point: bf16 workloads within max-abs 2e-2 and rel-L2 5e-3, fp32 within max-abs 1e-4,
+for every intermediate the ABI exposes (chunk latents, query latent, absorbed query, latent
+output, output, lse).  Integer work (key positions, ring slots) is bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_latent_kv_attn_b200 import api, inputs, rollout
+from parity_util import (GpuRun, OracleRun, check_chunk, check_ring, compare,
+                         expected_key_positions, to_np)
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"tc": api.MLA_PATH_AUTO, "simt": api.MLA_PATH_SIMT}
+
+
+def full_rollout(cfg, path, rows=None, check_positions=True):
+    g = GpuRun(cfg, path)
+    o = OracleRun(cfg, g.lw)
+    rows = np.arange(cfg.n_q) if rows is None else rows
+    report = {}
+    for ch in range(cfg.n_chunks):
+        x = inputs.chunk_x(cfg, ch)
+        first = cfg.first_frame(ch)
+        if check_positions:
+            pos = g.key_positions(ch)
+            for b in range(cfg.batch):
+                np.testing.assert_array_equal(pos[b], expected_key_positions(cfg, o.windows[b], first))
+        gres = g.attend(ch, x)
+        ores = o.step(ch, x, rows)
+        check_chunk(f"chunk{ch}", cfg, gres, ores, rows, report)
+        g.append(ch)
+        check_ring(cfg, g, o, report)
+    return report
+
+
+def test_toy_fp32_rollout_wraps_and_matches():
+    """Config 0: 4 chunks of 1 frame, window of 2 frames (the ring wraps at chunk 2)."""
+    full_rollout(inputs.CONFIGS[0], api.MLA_PATH_AUTO)
+
+
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_small_frames_bf16_rollout(path):
+    """Wan layer widths on 6x10 frames: 180 queries (2 tiles, ragged), 0..240 ring keys."""
+    full_rollout(inputs.small_bf16_config(), PATHS[path])
+
+
+def prefilled(cfg, path, upto):
+    g = GpuRun(cfg, path)
+    o = OracleRun(cfg, g.lw)
+    for ch in range(upto):
+        x = inputs.chunk_x(cfg, ch)
+        g.prefill(ch, x)
+        o.prefill(ch, x)
+    return g, o
+
+
+def test_wan_config1_sampled_rows():
+    """Config 1 at full size (B1, window 6 frames full, chunk of 3 frames), 384 sampled rows."""
+    cfg = inputs.CONFIGS[1]
+    g, o = prefilled(cfg, api.MLA_PATH_AUTO, cfg.measured_chunk)
+    check_ring(cfg, g, o)
+    ch = cfg.measured_chunk
+    x = inputs.chunk_x(cfg, ch)
+    rows = inputs.sample_rows(cfg.n_q, 384, tag=1)
+    pos = g.key_positions(ch)
+    np.testing.assert_array_equal(pos[0], expected_key_positions(cfg, o.windows[0], cfg.first_frame(ch)))
+    check_chunk("cfg1", cfg, g.attend(ch, x), o.step(ch, x, rows), rows)
+    g.append(ch)
+    check_ring(cfg, g, o)
+
+
+def test_wan_config3_batch8_sampled_rows():
+    """Config 3: 8 independent samples, window 9 frames, chunk 3 frames."""
+    cfg = inputs.CONFIGS[3]
+    g, o = prefilled(cfg, api.MLA_PATH_AUTO, cfg.measured_chunk)
+    ch = cfg.measured_chunk
+    x = inputs.chunk_x(cfg, ch)
+    rows = inputs.sample_rows(cfg.n_q, 48, tag=3)
+    check_chunk("cfg3", cfg, g.attend(ch, x), o.step(ch, x, rows), rows)
+
+
+def test_wan_config2_long_rollout_sampled():
+    """Config 2: 80 chunks, window 21 frames; temporal positions reach t = 239 and the ring
+    wraps every 7 chunks.  Every chunk runs the whole path on the GPU; the oracle evaluates
+    sampled rows at chunks while the window fills, across wraps and at the end."""
+    cfg = inputs.CONFIGS[2]
+    g = GpuRun(cfg, api.MLA_PATH_AUTO)
+    o = OracleRun(cfg, g.lw)
+    checked = {0, 1, 6, 7, 8, 40, 78, 79}
+    rows = inputs.sample_rows(cfg.n_q, 32, tag=2)
+    for ch in range(cfg.n_chunks):
+        x = inputs.chunk_x(cfg, ch)
+        if ch in checked:
+            pos = g.key_positions(ch)
+            np.testing.assert_array_equal(pos[0], expected_key_positions(cfg, o.windows[0], cfg.first_frame(ch)))
+            check_chunk(f"cfg2.chunk{ch}", cfg, g.attend(ch, x, want_latent=False),
+                        o.step(ch, x, rows), rows)
+        else:
+            g.attend(ch, x, want_latent=False)
+            o.prefill(ch, x)
+        g.append(ch)
+    check_ring(cfg, g, o)
+    assert int(g.ring.slot_frame.max()) == 239
+
+
+def test_tensor_core_and_cuda_core_paths_agree_on_config1():
+    """Diagnostic cross-check on every row of config 1 (GPU against GPU)."""
+    cfg = inputs.CONFIGS[1]
+    outs = []
+    for path in (api.MLA_PATH_AUTO, api.MLA_PATH_SIMT):
+        g, _ = prefilled(cfg, path, cfg.measured_chunk)
+        outs.append(g.attend(cfg.measured_chunk, inputs.chunk_x(cfg, cfg.measured_chunk)))
+    for k in ("o", "o_lat", "q", "chunk_lat"):
+        compare("tc_vs_simt." + k, outs[0][k], outs[1][k], "bf16")
+
+
+def test_standalone_rope3d_and_out_proj():
+    cfg = inputs.small_bf16_config()
+    g = GpuRun(cfg, api.MLA_PATH_AUTO)
+    o = OracleRun(cfg, g.lw)
+    d = oracle.dims_from(cfg)
+    x = inputs.chunk_x(cfg, 0)
+    g.prefill(0, x)
+    o.prefill(0, x)
+    # rotate the ring's positional keys in place (frames from slot_frame) and compare
+    rot = g.ring.cache.clone()
+    api.mla_rope3d(g.c, rot, n_vec=1, col_offset=cfg.d_c, vec_stride=0,
+                   frame_table=g.ring.slot_frame)
+    tpf = cfg.tokens_per_frame
+    sf = g.ring.slot_frame.cpu().numpy()
+    got = to_np(rot)
+    for b in range(cfg.batch):
+        for s, t in enumerate(sf[b]):
+            if t < 0:
+                np.testing.assert_array_equal(got[b, s * tpf:(s + 1) * tpf],
+                                              to_np(g.ring.cache)[b, s * tpf:(s + 1) * tpf])
+                continue
+            rec = [r for r in o.windows[b].frames if r.t == t][0]
+            ref = oracle.rope3d(rec.k_r, oracle.token_positions([t], d), d)
+            compare("rope3d", got[b, s * tpf:(s + 1) * tpf, cfg.d_c:], ref, "bf16")
+    # out_proj of a latent output and the optional W_O
+    x1 = inputs.chunk_x(cfg, 1)
+    res = g.attend(1, x1)
+    ores = o.step(1, x1, np.arange(cfg.n_q))
+    y = torch.empty((cfg.batch, cfg.n_q, cfg.d_model), device="cuda", dtype=torch.bfloat16)
+    api.mla_out_proj(g.c, g.buf.o_lat, g.w.w_uv, g.buf.o, w_o=g.w.w_o, y=y)
+    torch.cuda.synchronize()
+    for b in range(cfg.batch):
+        compare("out_proj.o", to_np(g.buf.o)[b], ores[b]["o"], "bf16")
+        compare("out_proj.y", to_np(y)[b], oracle.output_projection(ores[b]["o"], g.lw.w_o), "bf16")
+
+
+def test_ring_checkpoint_resume_is_bit_identical():
+    cfg = inputs.small_bf16_config()
+    a = GpuRun(cfg)
+    outs_a = []
+    for ch in range(cfg.n_chunks):
+        outs_a.append(a.attend(ch, inputs.chunk_x(cfg, ch), want_latent=False)["o"])
+        a.append(ch)
+        if ch == 1:
+            saved = a.ring.state_dict()
+    b = GpuRun(cfg)
+    b.ring.load_state_dict(saved)
+    for ch in range(2, cfg.n_chunks):
+        ob = b.attend(ch, inputs.chunk_x(cfg, ch), want_latent=False)["o"]
+        np.testing.assert_array_equal(ob, outs_a[ch])
+        b.append(ch)
+
+
+def test_bad_arguments_on_device():
+    cfg = inputs.small_bf16_config()
+    g = GpuRun(cfg)
+    x = inputs.chunk_x(cfg, 0)
+    g.load_x(x)
+    host = torch.empty_like(g.buf.chunk_lat, device="cpu")
+    with pytest.raises(api.MLAError) as e:
+        api.mla_cache_append(g.c, g.buf.x, g.w.w_dkv_kr, host, g.ring.cache, g.ring.slot_frame, 0,
+                             api.MLA_PROJECT)
+    assert e.value.status == 1
+    small_ws = torch.empty((64,), device="cuda", dtype=torch.uint8)
+    with pytest.raises(api.MLAError) as e:
+        api.mla_attention_fwd(g.c, g.buf.q, g.buf.chunk_lat, g.ring.cache, g.ring.slot_frame, 0, 0,
+                              None, g.buf.o_lat, workspace=small_ws)
+    assert e.value.status == 6
+    from mla_latent_kv_attn_b200 import _lib
+    import ctypes
+    st = _lib.lib().mla_rope3d(ctypes.byref(g.c), g.buf.chunk_lat.data_ptr() + 2, 1, cfg.n_q,
+                               224, 192, 1, 0, None, 0, 0, None)
+    assert st == 3
+    torch.cuda.synchronize()
+    assert int(g.buf.dev_status.item()) == 0
