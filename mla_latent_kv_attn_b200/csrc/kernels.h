@@ -21,6 +21,12 @@ struct GemmArgs {
   int64_t a_sm, a_sk, a_batch;
   int64_t b_sn, b_sk, b_batch;
   int64_t c_sm, c_batch;
+  // Optional fused 3D-RoPE of the query path: in every D-wide block of output columns, the
+  // pairs of columns d_c.. D-1 are rotated (fp32, before the one rounding) at the position of
+  // row m (chunk token m mod rope_n_q).  Needs even d_c.
+  int rope_epi;
+  int rope_D, rope_dc, rope_n_q, rope_first_frame;
+  RopeGeom rope;
 };
 
 struct AttnArgs {

@@ -246,6 +246,16 @@ mla_status mla_query_proj(const mla_config* cfg, const void* x, const void* w_dq
     g.rope = rope_geom(d);
     return gemm_tc(g, s);
   }
+  if (d.d_c % 2 == 0) {
+    GemmArgs g{};
+    g.A = c_q; g.a_sm = d.d_cq; g.a_sk = 1; g.a_batch = 0;
+    g.B = w_qcat; g.b_sn = d.d_cq; g.b_sk = 1; g.b_batch = 0;
+    g.C = q; g.c_sm = N; g.c_batch = 0;
+    g.M = M; g.N = N; g.K = d.d_cq; g.batch = 1;
+    g.rope_epi = 1; g.rope_D = d.D; g.rope_dc = d.d_c; g.rope_n_q = d.n_q;
+    g.rope_first_frame = first_frame; g.rope = rope_geom(d);
+    return gemm_simt(g, d.dtype, s);
+  }
   MLA_TRY(gemm(d, c_q, d.d_cq, 0, w_qcat, d.d_cq, 0, q, N, 0, M, N, d.d_cq, 1, s));
   return rope3d_inplace(d, q, d.B, d.n_q, N, d.d_c, d.H, d.D, nullptr, 0, first_frame, s);
 }

@@ -56,6 +56,23 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g) {
     }
     __syncthreads();
   }
+  if (g.rope_epi) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = m0 + ty * 4 + i;
+      const int nl = m % g.rope_n_q;
+      const int tok = nl % g.rope.tpf;
+      const int t = g.rope_first_frame + nl / g.rope.tpf;
+#pragma unroll
+      for (int j = 0; j < 4; j += 2) {
+        const int col = (n0 + tx * 4 + j) % g.rope_D;
+        if (col >= g.rope_dc)
+          rope_rotate(acc[i][j], acc[i][j + 1],
+                      rope_angle(g.rope, (col - g.rope_dc) / 2, t, tok / g.rope.frame_w,
+                                 tok % g.rope.frame_w));
+      }
+    }
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int m = m0 + ty * 4 + i;

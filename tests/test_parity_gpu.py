@@ -116,8 +116,12 @@ def test_tensor_core_and_cuda_core_paths_agree_on_config1():
     for path in (api.MLA_PATH_AUTO, api.MLA_PATH_SIMT):
         g, _ = prefilled(cfg, path, cfg.measured_chunk)
         outs.append(g.attend(cfg.measured_chunk, inputs.chunk_x(cfg, cfg.measured_chunk)))
+    # two correct bf16 results may differ by one or two units in the last place of a value
     for k in ("o", "o_lat", "q", "chunk_lat"):
-        compare("tc_vs_simt." + k, outs[0][k], outs[1][k], "bf16")
+        a, b = outs[0][k], outs[1][k]
+        err = a - b
+        assert np.abs(err).max() <= 2 * 2.0 ** -8 * max(1.0, np.abs(b).max()), k
+        assert np.linalg.norm(err) / np.linalg.norm(b) <= 5e-3, k
 
 
 def test_standalone_rope3d_and_out_proj():
