@@ -107,11 +107,10 @@ int32_t mla_abi_version(void);
 mla_status mla_config_check(const mla_config* cfg);
 
 /* --------------------------------------------------------------------------------------------
- * mla_cache_append: joint down-projection and ring-buffer append ([M]: "each video latent token
- * is compressed into a shared content latent via a joint down-projection, written to the
- * compressed KV cache"; "a single head-shared positional key k_R is computed from x via W_R^K
- * and stored in the cache", unrotated; [A]: fixed-size sliding-window KV cache; [I]: rolling
- * cache).
+ * mla_cache_append: joint down-projection and ring-buffer append.  [M]: a joint down-projection
+ * turns every token into the content latent that the cache keeps, and W_R^K turns it into the
+ * one positional key all heads share, cached before any rotation; [A]: the window of cached
+ * frames has a fixed size; [I]: the cache rolls forward chunk by chunk.
  *
  *   mode & MLA_PROJECT : chunk_lat[b, n, :] = [W_down^KV x[b, n] || W_R^K x[b, n]]   (T, fp32 acc.)
  *   mode & MLA_APPEND  : for each frame f = first_frame + j, j < chunk_frames:
@@ -242,6 +241,32 @@ mla_status mla_attention_fwd(const mla_config* cfg, const void* q, const void* c
                              int32_t n_valid_frames, int32_t first_frame, const void* w_uv,
                              void* out, float* lse, void* workspace, size_t workspace_bytes,
                              int32_t* dev_status, void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_attention_fwd_static_scratch: mla_attention_fwd without the workspace arguments, for
+ * callers that cannot allocate device memory.  The paper has no counterpart to this call; it
+ * exists for deployment.  Some callers have no way to hand the library a scratch buffer: code
+ * that issues its work while a stream is being captured into a CUDA graph (cudaMalloc is not
+ * allowed there), plugins whose host framework gives them only their input and output buffers,
+ * and services that forbid device allocation after start-up.  This call keeps its scratch (the
+ * rotated positional keys of the attended keys) in a fixed 16 MiB array compiled into the
+ * library, and calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Arguments, results and errors are those of mla_attention_fwd.  A call whose scratch,
+ *     mla_attention_workspace_bytes(cfg, n_valid_frames), exceeds 16 MiB (16777216 bytes) is
+ *     rejected with MLA_ERR_WORKSPACE before anything is launched.
+ *   - Every device that loads the library keeps those 16 MiB reserved until the process exits.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current); make that first call before any stream capture begins.
+ *   - All calls share the one array per device.  Calls whose kernels overlap on the GPU (on
+ *     different streams, or from different host threads) race on it and give wrong results;
+ *     order them on one stream.  Each call rewrites every part of the array it reads, so what an
+ *     earlier call left there does not matter.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q,
+                                            const void* chunk_lat, const void* cache,
+                                            const int32_t* slot_frame, int32_t n_valid_frames,
+                                            int32_t first_frame, const void* w_uv, void* out,
+                                            float* lse, int32_t* dev_status, void* stream);
 
 /* --------------------------------------------------------------------------------------------
  * mla_out_proj: value up-projection of latent outputs and the optional output projection

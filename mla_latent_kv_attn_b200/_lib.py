@@ -64,6 +64,8 @@ SIGNATURES = {
     "mla_attention_fwd": (c_int32, [_CFG, _P, _P, _P, _P, c_int32, c_int32, _P, _P, _P, _P,
                                     c_size_t, _P, _P]),
     "mla_out_proj": (c_int32, [_CFG, _P, _P, _P, _P, _P, _P]),
+    "mla_attention_fwd_static_scratch": (c_int32, [_CFG, _P, _P, _P, _P, c_int32, c_int32, _P,
+                                                   _P, _P, _P, _P]),
 }
 
 _lib = None

@@ -18,7 +18,8 @@ from ._lib import (MLA_APPEND, MLA_BF16, MLA_FP32, MLA_PATH_AUTO, MLA_PATH_SIMT,
 __all__ = [
     "make_config", "torch_dtype", "mla_config_check", "mla_cache_append", "mla_rope3d",
     "mla_key_positions", "mla_compose_query_weights", "mla_query_proj",
-    "mla_attention_workspace_bytes", "mla_attention_fwd", "mla_out_proj", "MLAError",
+    "mla_attention_workspace_bytes", "mla_attention_fwd", "mla_attention_fwd_static_scratch",
+    "mla_out_proj", "MLAError",
     "MLA_PROJECT", "MLA_APPEND", "MLA_PROJECT_AND_APPEND", "MLA_PATH_AUTO", "MLA_PATH_SIMT",
 ]
 
@@ -161,3 +162,23 @@ def mla_out_proj(c: MLAConfigC, o_lat, w_uv, o, w_o=None, y=None, stream=None) -
         _ptr(o, "o", dt, (B, n_q, H * c.d_head)), _ptr(y, "y", dt, (B, n_q, c.d_model)),
         _stream(stream))
     _lib.check("mla_out_proj", st)
+
+
+def mla_attention_fwd_static_scratch(c: MLAConfigC, q, chunk_lat, cache, slot_frame,
+                                     n_valid_frames: int, first_frame: int, w_uv, out, lse=None,
+                                     dev_status=None, stream=None) -> None:
+    """mla_attention_fwd for callers that cannot allocate: the scratch lives in the library's
+    built-in 16 MiB device array (one per device, shared by all calls; order calls on one
+    stream).  The first call on a device should come before any stream capture."""
+    tpf, n_q, D = _geom(c)
+    dt = torch_dtype(c)
+    B, H = c.batch, c.n_heads
+    out_shape = (B, n_q, H * c.d_head) if w_uv is not None else (B, n_q, H, c.d_c)
+    st = _lib.lib().mla_attention_fwd_static_scratch(
+        ctypes.byref(c), _ptr(q, "q", dt, (B, n_q, H, D)), _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)),
+        _ptr(cache, "cache", dt, (B, c.window_frames * tpf, D)),
+        _ptr(slot_frame, "slot_frame", torch.int32, (B, c.window_frames)), n_valid_frames,
+        first_frame, _ptr(w_uv, "w_uv", dt, (H, c.d_head, c.d_c)), _ptr(out, "out", dt, out_shape),
+        _ptr(lse, "lse", torch.float32, (B, H, n_q)), _ptr(dev_status, "dev_status", torch.int32),
+        _stream(stream))
+    _lib.check("mla_attention_fwd_static_scratch", st)

@@ -98,6 +98,13 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s);
 bool tc_attention_supported(const Dims& d, bool has_w_uv);
 mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
 
+// Attention with the scratch held in the library's built-in device array
+// (attention_static_ws.cu); args.ws is ignored.
+size_t static_scratch_bytes();
+mla_status attention_fwd_static_scratch(const Dims& d, const AttnArgs& args,
+                                        const int32_t* slot_frame, int n_valid, int first_frame,
+                                        cudaStream_t s);
+
 }  // namespace mla
 
 #include <cuda.h>

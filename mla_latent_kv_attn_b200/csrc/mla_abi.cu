@@ -303,6 +303,32 @@ mla_status mla_attention_fwd(const mla_config* cfg, const void* q, const void* c
   return attention_simt(d, a, n_valid_frames, s);
 }
 
+mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q,
+                                            const void* chunk_lat, const void* cache,
+                                            const int32_t* slot_frame, int32_t n_valid_frames,
+                                            int32_t first_frame, const void* w_uv, void* out,
+                                            float* lse, int32_t* dev_status, void* stream) {
+  set_last_error("");
+  MLA_TRY(check_cfg(cfg));
+  const Dims d = dims_of(*cfg);
+  MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
+                d.W);
+  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_ptr(q, "q"));
+  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
+  MLA_TRY(check_ptr(slot_frame, "slot_frame"));
+  MLA_TRY(check_ptr(out, "out"));
+  MLA_TRY(check_ptr(cache, "cache", n_valid_frames > 0));
+  MLA_TRY(check_ptr(w_uv, "w_uv", false));
+  MLA_TRY(check_ptr(lse, "lse", false));
+  MLA_TRY(check_ptr(dev_status, "dev_status", false));
+  AttnArgs a{};
+  a.q = q; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = nullptr; a.w_uv = w_uv;
+  a.out = out; a.lse = lse; a.dev_status = dev_status;
+  return attention_fwd_static_scratch(d, a, slot_frame, n_valid_frames, first_frame,
+                                      static_cast<cudaStream_t>(stream));
+}
+
 mla_status mla_out_proj(const mla_config* cfg, const void* o_lat, const void* w_uv,
                         const void* w_o, void* o, void* y, void* stream) {
   set_last_error("");
