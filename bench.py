@@ -192,6 +192,24 @@ def run_reference(args, cfg):
     return 0
 
 
+# --------------------------------------------------------------------------- ranks
+
+def rank_samples(rank: int, batch: int) -> range:
+    """Sample indices a rank draws: every rank runs its own, disjoint samples."""
+    return range(rank * batch, (rank + 1) * batch)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest value over all ranks (the local value without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # --------------------------------------------------------------------------- GPU path
 
 def run_ours(args, cfg):
@@ -215,12 +233,11 @@ def run_ours(args, cfg):
     buf = rollout.ChunkBuffers(c, device=dev)
     # independent sample per rank: inputs drawn with the rank as the sample index
     n_pool = 4
-    pool = [torch.from_numpy(inputs.chunk_x(cfg, cfg.measured_chunk + i,
-                                            samples=range(rank, rank + cfg.batch)))
+    samples = rank_samples(rank, cfg.batch)
+    pool = [torch.from_numpy(inputs.chunk_x(cfg, cfg.measured_chunk + i, samples=samples))
             .to(device=dev, dtype=torch.bfloat16) for i in range(n_pool)]
     for ch in range(cfg.measured_chunk):
-        buf.x.copy_(torch.from_numpy(inputs.chunk_x(cfg, ch, samples=range(rank, rank + cfg.batch)))
-                    .to(torch.bfloat16))
+        buf.x.copy_(torch.from_numpy(inputs.chunk_x(cfg, ch, samples=samples)).to(torch.bfloat16))
         rollout.prefill_chunk(c, w, ring, buf, ch)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -274,11 +291,7 @@ def run_ours(args, cfg):
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(ev_s, ev_e)]
     attn_ms = [a.elapsed_time(b) for a, b in ev_a]
-    total_ms = sum(step_ms)
-    total_t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(total_t, op=dist.ReduceOp.MAX)
-    total_ms = float(total_t.item())
+    total_ms = max_over_ranks(sum(step_ms), device=dev)
     status = int(buf.dev_status.item())
     if status != 0:
         raise RuntimeError(f"a kernel reported status {status}")
@@ -302,12 +315,9 @@ def run_ours(args, cfg):
         o_host.copy_(buf.o, non_blocking=True)
         e2e_e[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e))], device=dev,
-                          dtype=torch.float64)
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e)), device=dev)
     if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_ms = float(e2e_ms.item())
 
     peaks, peak_kind = load_peaks()
     n_units_all = world * cfg.batch

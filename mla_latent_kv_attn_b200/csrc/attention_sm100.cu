@@ -10,7 +10,7 @@
 //              domain with lazy rescaling of O (only when the running max grows by > 8);
 //              write P (bf16) back into TMEM over the S buffer it came from; final 1/l,
 //              optional W_UV epilogue, stores and lse.
-//   warp 4     TMA producer: Q tile once, then 128-key K' tiles into a 2-stage ring: three
+//   warp 4     TMA producer: Q tile once, then 128-key K' tiles into a 3-stage ring: three
 //              128x64 (128B-swizzled) content blocks from the ring/chunk latents and one 128x32
 //              (64B-swizzled) block of pre-rotated positional keys; then the W_UV_h tile.
 //   warp 5     TMEM allocation; one thread issues every tcgen05.mma:
@@ -34,7 +34,7 @@ constexpr int kDc = 192;           // content latent width
 constexpr int kDr = 32;            // positional key width
 constexpr int kD = kDc + kDr;      // 224
 constexpr int kDh = 128;           // head width of the W_UV epilogue
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kThreads = 192;
 
 constexpr int kBlk = kBM * 128;                  // one 128-row x 128-byte block: 16 KB

@@ -10,7 +10,7 @@ described on the VideoMLA pages:
 * hyper.ai summary of VideoMLA (English edition), section "Method"; the same
   paragraph appears in the Chinese edition, section "方法".  Every token x_t is
   compressed by a joint down-projection into a content latent c_KV (written to
-  the cache); a single head-shared positional key k_R = W_R^K x_t is stored
+  the cache); one positional key k_R = W_R^K x_t, common to all heads, is kept
   unrotated and rotated by 3D-RoPE only when attention runs; per-head keys and
   values are rebuilt from c_KV by per-head up-projections; the query side has a
   query latent c_Q from x_t and per-head positional queries computed from c_Q
@@ -20,9 +20,9 @@ described on the VideoMLA pages:
 * ai-papers.net article "VideoMLAとは？", paragraph after Figure 1: the base
   model is Wan2.1-1.3B, the content latent is 192 wide, and a token's cached
   state shrinks from 3,072 to 224 scalars.
-* chatpaper abstract (English): long rollouts use a fixed-size sliding-window
-  KV cache; the latent layout cuts per-token KV memory by 92.7% at every
-  cached layer.
+* chatpaper abstract (English): long rollouts keep a sliding window of fixed
+  size as their KV cache; with the latent layout each layer's cache needs
+  92.7% less memory per token.
 
 Where the pages are silent the oracle takes the plainest reading (each one is
 listed with its reason in the design notes):
@@ -123,8 +123,9 @@ def kv_reduction(d: Dims) -> float:
 
 
 # ---------------------------------------------------------------------------
-# positions and 3D-RoPE (hyper.ai summary, Method: the unrotated key is rotated
-# by 3D-RoPE at attention time; the positional query is rotated as well)
+# positions and 3D-RoPE (hyper.ai summary, Method: k_R stays unrotated in the
+# cache and gets its 3D-RoPE rotation when attention runs; so does the query's
+# positional part)
 
 def token_positions(frames: Sequence[int], d: Dims) -> np.ndarray:
     """(t, h, w) of every token of the given frames, frames in the order given,

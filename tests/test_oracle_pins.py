@@ -323,6 +323,16 @@ def test_positions_row_major():
                           [9, 0, 0], [9, 0, 1], [9, 0, 2], [9, 1, 0], [9, 1, 1], [9, 1, 2]]
 
 
+def test_output_projection_brute_force():
+    rng = np.random.default_rng(5)
+    o = rng.standard_normal((3, 4))
+    w_o = rng.standard_normal((5, 4))
+    y = oracle.output_projection(o, w_o)
+    for n in range(3):
+        for i in range(5):
+            assert abs(y[n, i] - sum(w_o[i, k] * o[n, k] for k in range(4))) < 1e-12
+
+
 # --------------------------------------------------------------------------
 # the pins above catch planted slips
 
@@ -332,7 +342,8 @@ PINS = [test_rope_identity_at_origin, test_rope_preserves_pair_norms,
         test_rope_worked_example, test_softmax_rows_sum_to_one, test_lse_is_log_of_denominator,
         test_absorbed_form_equals_non_absorbed, test_mha_special_case_matches_library_sdpa,
         test_brute_force_rollout_with_wraparound, test_window_holds_the_last_w_frames,
-        test_positions_row_major, test_cache_size_matches_pages]
+        test_positions_row_major, test_cache_size_matches_pages,
+        test_output_projection_brute_force]
 
 
 def _patch(monkeypatch, name, fn):
@@ -401,6 +412,9 @@ def _mutants():
     def dense_wrong(d):
         return d.n_heads * d.d_head
 
+    def out_proj_transposed(o, w_o):
+        return np.asarray(o, np.float64) @ np.asarray(w_o, np.float64)[:, :np.asarray(o).shape[1]]
+
     return {
         "rope rotates the wrong way": [("rope3d", rope_flipped)],
         "rope frequency exponent doubled": [("rope3d_angles", angles_wrong_exponent)],
@@ -414,6 +428,7 @@ def _mutants():
         "head outputs interleaved": [("attend", attend_heads_interleaved)],
         "window one frame short": [("SlidingWindow", ShortWindow)],
         "dense cache counted once": [("dense_scalars_per_token", dense_wrong)],
+        "output projection transposed": [("output_projection", out_proj_transposed)],
     }
 
 
@@ -428,3 +443,4 @@ def test_planted_mistakes_are_caught(name, monkeypatch):
         except Exception:
             failed.append(pin.__name__)
     assert failed, f"no pin caught the planted slip: {name}"
+
