@@ -257,11 +257,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int valid = j < p.nt_ring ? min(kBN, p.nc - j * kBN)
                                       : min(kBN, p.n_q - (j - p.nt_ring) * kBN);
-      float mx = -INFINITY;
+      if (valid < kBN) {                    // only the last tile of the ring or of the chunk
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        s[c] = c < valid ? s[c] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < kBN; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+      }
+      // Row max of the raw scores (the scale is positive), four independent chains.
+      float mx;
+      {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < kBN; c += 4)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) m4[u] = fmaxf(m4[u], s[c + u]);
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
       }
       if (j == 0) {
         m_run = mx;
@@ -285,19 +294,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
       }
-      float sum = 0.f;
+      // p = 2^(s * scale * log2(e) - m): one FFMA and one ex2 per score; P packed to bf16
+      // pairs and written over S in TMEM.  Four independent partial sums.
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      const float neg_m = -m_run;
 #pragma unroll
       for (int c = 0; c < kBN; c += 32) {
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(s[c + 2 * i] - m_run);
-          const float p1 = fast_exp2(s[c + 2 * i + 1] - m_run);
-          sum += p0 + p1;
+          const float p0 = fast_exp2(fmaf(s[c + 2 * i], p.scale_log2, neg_m));
+          const float p1 = fast_exp2(fmaf(s[c + 2 * i + 1], p.scale_log2, neg_m));
+          sum4[i & 3] += p0 + p1;
           w[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(sc + c / 2, w);
       }
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l_run += sum;
       tmem_wait_st();
       tc_fence_before();

@@ -199,3 +199,66 @@ def test_bad_arguments_on_device():
     assert st == 3
     torch.cuda.synchronize()
     assert int(g.buf.dev_status.item()) == 0
+
+
+def test_wan_config4_thirty_layer_stack():
+    """Config 4: 30 layers, each with its own weights and ring, batch 2, window 12 frames; every
+    chunk runs 4 denoising steps through all 30 layers against the frozen rings, then each layer
+    appends its last step's latents.  All 1200 attention calls run on the GPU.  The oracle checks
+    sampled rows of layer 29 at the last chunk (steps 0 and 3, ring wrapped, 23,400 keys) and of
+    layer 0 at chunks 0 and 1, plus both layers' ring slots."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    from parity_util import expected_slot_frame
+
+    cfg = inputs.CONFIGS[4]
+    c = api.make_config(cfg)
+    layers = [inputs.layer_weights(cfg, l) for l in range(cfg.n_layers)]
+    dev_w = [rollout.upload_weights(c, lw) for lw in layers]
+    rings = [rollout.Ring(c) for _ in range(cfg.n_layers)]
+    buf = rollout.ChunkBuffers(c)
+    last = cfg.n_steps - 1
+    checks = {(cfg.n_chunks - 1, 0, 29), (cfg.n_chunks - 1, last, 29), (0, 0, 0), (0, last, 0),
+              (1, last, 0)}
+    history = {29: range(cfg.n_chunks), 0: range(2)}
+    rows = inputs.sample_rows(cfg.n_q, 24, tag=4)
+    order = [(ch, s, l) for ch in range(cfg.n_chunks) for s in range(cfg.n_steps)
+             for l in range(cfg.n_layers)]
+    kept, gpu_out = {}, {}
+    workers = min(16, os.cpu_count() or 4)
+    pool = ThreadPoolExecutor(max_workers=workers)
+    futs = {}
+    for i, key in enumerate(order):
+        for k in order[i:i + workers + 4]:
+            if k not in futs:
+                futs[k] = pool.submit(inputs.chunk_x, cfg, k[0], k[1], k[2])
+        ch, s, l = key
+        x = futs.pop(key).result()
+        if key in checks or (l in history and s == last and ch in history[l]):
+            kept[key] = x
+        buf.x.copy_(torch.from_numpy(x).to(torch.bfloat16))
+        rollout.attend_chunk(c, dev_w[l], rings[l], buf, ch, fuse_uv=True)
+        if key in checks:
+            gpu_out[key] = (to_np(buf.o)[:, rows], to_np(buf.lse)[:, :, rows])
+        if s == last:
+            rollout.append_chunk(c, rings[l], buf, ch)
+    pool.shutdown()
+    torch.cuda.synchronize()
+    rollout.check_device_status(buf)
+
+    for l, chunks in history.items():
+        o = OracleRun(cfg, layers[l])
+        for ch in chunks:
+            for s in (0, last):
+                if (ch, s, l) in checks:
+                    res = o.step(ch, kept[(ch, s, l)], rows, append=False)
+                    g_o, g_lse = gpu_out[(ch, s, l)]
+                    for b in range(cfg.batch):
+                        compare(f"cfg4.l{l}.c{ch}.s{s}.b{b}.o", g_o[b], res[b]["o"], "bf16")
+                        compare(f"cfg4.l{l}.c{ch}.s{s}.b{b}.lse", g_lse[b], res[b]["lse"], "bf16")
+            o.prefill(ch, kept[(ch, last, l)])
+        if l == 29:
+            gpu_sf = rings[l].slot_frame.cpu().numpy()
+            for b in range(cfg.batch):
+                np.testing.assert_array_equal(gpu_sf[b], expected_slot_frame(cfg, o.windows[b]))
