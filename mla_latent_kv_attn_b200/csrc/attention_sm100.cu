@@ -5,20 +5,23 @@
 // In absorbed form every head is a query against the same keys K'_m = [c_m || RoPE(k_R,m)]
 // (224 wide) and the same values c_m (192 wide, the first 192 columns of K'): 12-head MQA.
 //
-// One CTA = one 128-row query tile of one head of one sample.  Roles (192 threads):
+// One CTA = one 128-row query tile of one head of one sample.  Roles (224 threads):
 //   warps 0-3  softmax: one TMEM lane (= query row) per thread; online softmax in the log2
 //              domain with lazy rescaling of O (only when the running max grows by > 8);
-//              write P (bf16) back into TMEM over the S buffer it came from; final 1/l,
+//              write P (bf16) into its TMEM buffer; final 1/l,
 //              optional W_UV epilogue, stores and lse.
 //   warp 4     TMA producer: Q tile once, then 128-key K' tiles into a 3-stage ring: three
 //              128x64 (128B-swizzled) content blocks from the ring/chunk latents and one 128x32
 //              (64B-swizzled) block of pre-rotated positional keys; then the W_UV_h tile.
-//   warp 5     TMEM allocation; one thread issues every tcgen05.mma:
+//   warps 5, 6 TMEM allocation (warp 5); one thread of warp 5 issues the QK products, one of
+//              warp 6 the PV products and the epilogue (two issuers keep the pipe fed):
 //                S_j   = Q K'_j^T          M=128, N=128, K=224 (12 SW128 + 2 SW64 k-steps)
 //                O    += P_j V_j           M=128, N=192, K=128; P from TMEM, V = content
 //                                          blocks of the same stage read MN-major
 //                o     = O_lat W_UV_h^T    M=128, N=128, K=192 (epilogue, O_lat bf16 in smem)
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,448); the epilogue result reuses S0.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,448), P [448,512); the epilogue result
+// reuses S0.  P has its own buffer so that a QK may overwrite an S buffer as soon as the
+// softmax has loaded it, instead of after the PV that reads its P.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -35,14 +38,22 @@ constexpr int kDr = 32;            // positional key width
 constexpr int kD = kDc + kDr;      // 224
 constexpr int kDh = 128;           // head width of the W_UV epilogue
 constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;   // warps 0-3: one TMEM lane (query row) per thread
+constexpr int kProducerWarp = 4;
+constexpr int kQkWarp = 5;              // also allocates and frees TMEM
+constexpr int kPvWarp = 6;
+constexpr int kThreads = 224;
 
-constexpr int kBlk = kBM * 128;                  // one 128-row x 128-byte block: 16 KB
-constexpr int kRopeBlk = kBN * kDr * 2;          // 8 KB
-constexpr int kTile = 3 * kBlk + kRopeBlk;       // 56 KB: Q tile or one K' stage
-constexpr int kSmem = (1 + kStages) * kTile + 1024;
+constexpr int kQBlk = kBM * 128;                 // 128 rows x 128 B: 16 KB (Q, O_lat, W_UV)
+constexpr int kKBlk = kBN * 128;                 // 128 rows x 128 B: 16 KB (K' content)
+constexpr int kQTile = 3 * kQBlk + kBM * kDr * 2;   // 56 KB
+constexpr int kKTile = 3 * kKBlk + kBN * kDr * 2;   // 56 KB: one K' stage
+constexpr int kSmem = kQTile + kStages * kKTile + 1024;
+static_assert(kKTile >= 3 * kQBlk, "the W_UV tile is loaded into one K' stage");
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 128;    // S buffers at columns 0 and 128
 constexpr uint32_t kColO = 256;
+constexpr uint32_t kColP = 448;    // kBN / 2 columns of packed bf16 P
 
 struct AttnParams {
   int n_q, H, nc, nc_pad, nt_ring, nt;
@@ -86,7 +97,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t kv_full[kStages];
   __shared__ __align__(8) uint64_t kv_empty[kStages];
   __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ __align__(8) uint64_t p_full[2];
+  __shared__ __align__(8) uint64_t s_free[2];
+  __shared__ __align__(8) uint64_t p_full;
   __shared__ __align__(8) uint64_t pv_done;
   __shared__ __align__(8) uint64_t w_full;
   __shared__ __align__(8) uint64_t olat_full;
@@ -110,15 +122,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&p_full[i]), 128);
+      mbar_init(smem_u32(&s_free[i]), kSoftmaxThreads);
     }
+    mbar_init(smem_u32(&p_full), kSoftmaxThreads);
     mbar_init(smem_u32(&pv_done), 1);
     mbar_init(smem_u32(&w_full), 1);
-    mbar_init(smem_u32(&olat_full), 128);
+    mbar_init(smem_u32(&olat_full), kSoftmaxThreads);
     mbar_init(smem_u32(&epi_done), 1);
+
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kQkWarp) {
     tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
     tmem_relinquish();
   }
@@ -127,111 +141,118 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_chunk);
       tma_prefetch_desc(&tm_ws);
       const uint32_t qb = smem_u32(&q_full);
-      mbar_arrive_expect_tx(qb, kTile);
-      for (int i = 0; i < 3; ++i) tma_load_4d(sQ + i * kBlk, &tm_q, qb, 64 * i, h, q0, b);
-      tma_load_4d(sQ + 3 * kBlk, &tm_qr, qb, kDc, h, q0, b);
-      for (int j = 0; j <= p.nt; ++j) {
+      mbar_arrive_expect_tx(qb, kQTile);
+      for (int i = 0; i < 3; ++i) tma_load_4d(sQ + i * kQBlk, &tm_q, qb, 64 * i, h, q0, b);
+      tma_load_4d(sQ + 3 * kQBlk, &tm_qr, qb, kDc, h, q0, b);
+      bool ok = true;
+      for (int j = 0; j < p.nt && ok; ++j) {
         const int s = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (j == p.nt && !p.has_w_uv) break;
-        if (!wait_bar(smem_u32(&kv_empty[s]), ph ^ 1, abort_flag, p.dev_status)) break;
-        const uint32_t dst = sbase + (1 + s) * kTile;
-        if (j == p.nt) {   // W_UV_h tile [128 x 192] into the content blocks of this stage
-          const uint32_t wb = smem_u32(&w_full);
-          mbar_arrive_expect_tx(wb, 3 * kBlk);
-          for (int i = 0; i < 3; ++i) tma_load_2d(dst + i * kBlk, &tm_wuv, wb, 64 * i, h * kDh);
-          break;
-        }
+        ok = wait_bar(smem_u32(&kv_empty[s]), ((j / kStages) & 1) ^ 1, abort_flag, p.dev_status);
+        if (!ok) break;
+        const uint32_t dst = sbase + kQTile + s * kKTile;
         const uint32_t fb = smem_u32(&kv_full[s]);
-        mbar_arrive_expect_tx(fb, kTile);
+        mbar_arrive_expect_tx(fb, kKTile);
         if (j < p.nt_ring) {
           const int r0 = j * kBN;
-          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlk, &tm_cache, fb, 64 * i, r0, b);
-          tma_load_3d(dst + 3 * kBlk, &tm_ws, fb, 0, r0, b);
+          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kKBlk, &tm_cache, fb, 64 * i, r0, b);
+          tma_load_3d(dst + 3 * kKBlk, &tm_ws, fb, 0, r0, b);
         } else {
           const int r0 = (j - p.nt_ring) * kBN;
-          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlk, &tm_chunk, fb, 64 * i, r0, b);
-          tma_load_3d(dst + 3 * kBlk, &tm_ws, fb, 0, p.nc_pad + r0, b);
+          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kKBlk, &tm_chunk, fb, 64 * i, r0, b);
+          tma_load_3d(dst + 3 * kKBlk, &tm_ws, fb, 0, p.nc_pad + r0, b);
+        }
+      }
+      if (ok && p.has_w_uv) {
+        // W_UV_h [128 x 192] (48 KB) goes into the stage a tile nt would use, once it is free.
+        const int s = p.nt % kStages;
+        if (wait_bar(smem_u32(&kv_empty[s]), ((p.nt / kStages) & 1) ^ 1, abort_flag, p.dev_status)) {
+          const uint32_t wb = smem_u32(&w_full);
+          mbar_arrive_expect_tx(wb, 3 * kQBlk);
+          for (int i = 0; i < 3; ++i)
+            tma_load_2d(sbase + kQTile + s * kKTile + i * kQBlk, &tm_wuv, wb, 64 * i, h * kDh);
         }
       }
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kQkWarp || warp == kPvWarp) {
+    // ------------------------------------------------------------------ MMA issuers
+    // Two threads issue MMAs: one the QK products, the other the PV products and the W_UV
+    // epilogue.  A tcgen05.mma issue takes about as long as the tensor pipe needs to start
+    // it, so the pipe only stays busy if some thread is always issuing; with two issuers one
+    // waits on a barrier while the other feeds the pipe.  Order between the two streams is
+    // explicit: QK(j) overwrites the S/P buffer that PV(j-2) reads, so it waits for PV(j-2).
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDc, 0, 1);
       constexpr uint32_t idesc_uv = idesc_bf16_f32(kBM, kDh, 0, 0);
-      bool ok = wait_bar(smem_u32(&q_full), 0, abort_flag, p.dev_status);
-      auto issue_qk = [&](int j) {
-        const int s = j % kStages;
-        const uint32_t kt = sbase + (1 + s) * kTile;
-        const uint32_t d = tmem + (j & 1) * kBN;
-#pragma unroll
-        for (int blk = 0; blk < 3; ++blk)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc(sQ + blk * kBlk + 32 * kk, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(kt + blk * kBlk + 32 * kk, 16, 1024, kSwizzle128B);
-            mma_ss(d, ad, bd, idesc_qk, (blk | kk) != 0 ? 1u : 0u);
-          }
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const uint64_t ad = smem_desc(sQ + 3 * kBlk + 32 * kk, 16, 512, kSwizzle64B);
-          const uint64_t bd = smem_desc(kt + 3 * kBlk + 32 * kk, 16, 512, kSwizzle64B);
-          mma_ss(d, ad, bd, idesc_qk, 1u);
-        }
-        mma_commit(smem_u32(&s_full[j & 1]));
-      };
-      if (ok) ok = wait_bar(smem_u32(&kv_full[0]), 0, abort_flag, p.dev_status);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0);
-      }
-      for (int j = 0; j < p.nt && ok; ++j) {
-        if (j + 1 < p.nt) {
-          const int s1 = (j + 1) % kStages;
-          ok = wait_bar(smem_u32(&kv_full[s1]), ((j + 1) / kStages) & 1, abort_flag, p.dev_status);
+      // Descriptors are built once; an operand at byte offset `off` from a descriptor's start
+      // is that descriptor plus off/16 (the start-address field is the low 14 bits and every
+      // address stays below 256 KB, so the add never carries out of the field).
+      constexpr uint32_t kQBlkD = kQBlk >> 4, kKBlkD = kKBlk >> 4, kKTileD = kKTile >> 4;
+      const uint64_t q_c = smem_desc(sQ, 16, 1024, kSwizzle128B);
+      const uint64_t q_r = smem_desc(sQ + 3 * kQBlk, 16, 512, kSwizzle64B);
+      const uint64_t k_c0 = smem_desc(sbase + kQTile, 16, 1024, kSwizzle128B);
+      const uint64_t k_r0 = smem_desc(sbase + kQTile + 3 * kKBlk, 16, 512, kSwizzle64B);
+      const uint64_t v_0 = smem_desc(sbase + kQTile, kKBlk, 1024, kSwizzle128B);
+      bool ok = true;
+      if (warp == kQkWarp) {
+        ok = wait_bar(smem_u32(&q_full), 0, abort_flag, p.dev_status);
+        for (int j = 0; j < p.nt && ok; ++j) {
+          const int s = j % kStages;
+          ok = wait_bar(smem_u32(&kv_full[s]), (j / kStages) & 1, abort_flag, p.dev_status);
+          if (ok && j >= 2)   // the softmax has loaded S(j-2) out of the buffer this QK overwrites
+            ok = wait_bar(smem_u32(&s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.dev_status);
           if (!ok) break;
           tc_fence_after();
-          issue_qk(j + 1);
-        }
-        ok = wait_bar(smem_u32(&p_full[j & 1]), (j >> 1) & 1, abort_flag, p.dev_status);
-        if (!ok) break;
-        tc_fence_after();
-        const int s = j % kStages;
-        const uint32_t vt = sbase + (1 + s) * kTile;
-        const uint32_t pa = tmem + (j & 1) * kBN;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // V rows kk*16 .. +15: 16 rows x 128 B further per step; N blocks 16 KB apart
-          const uint64_t bd = smem_desc(vt + kk * 2048, kBlk, 1024, kSwizzle128B);
-          mma_ts(tmem + kColO, pa + kk * 8, bd, idesc_pv, (j | kk) != 0 ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&kv_empty[s]));
-        mma_commit(smem_u32(&pv_done));
-      }
-      if (ok && p.has_w_uv) {
-        ok = wait_bar(smem_u32(&w_full), 0, abort_flag, p.dev_status) &&
-             wait_bar(smem_u32(&olat_full), 0, abort_flag, p.dev_status);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t wt = sbase + (1 + p.nt % kStages) * kTile;
+          const uint64_t kc = k_c0 + static_cast<uint32_t>(s) * kKTileD;
+          const uint64_t kr = k_r0 + static_cast<uint32_t>(s) * kKTileD;
+          const uint32_t d = tmem + (j & 1) * kColS;
 #pragma unroll
           for (int blk = 0; blk < 3; ++blk)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = smem_desc(sQ + blk * kBlk + 32 * kk, 16, 1024, kSwizzle128B);
-              const uint64_t bd = smem_desc(wt + blk * kBlk + 32 * kk, 16, 1024, kSwizzle128B);
-              mma_ss(tmem, ad, bd, idesc_uv, (blk | kk) != 0 ? 1u : 0u);
-            }
-          mma_commit(smem_u32(&epi_done));
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(d, q_c + (blk * kQBlkD + 2 * kk), kc + (blk * kKBlkD + 2 * kk), idesc_qk,
+                     (blk | kk) != 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) mma_ss(d, q_r + 2 * kk, kr + 2 * kk, idesc_qk, 1u);
+          mma_commit(smem_u32(&s_full[j & 1]));
+        }
+      } else {
+        for (int j = 0; j < p.nt && ok; ++j) {
+          ok = wait_bar(smem_u32(&p_full), j & 1, abort_flag, p.dev_status);
+          if (!ok) break;
+          tc_fence_after();
+          const int s = j % kStages;
+          const uint64_t vd = v_0 + static_cast<uint32_t>(s) * kKTileD;
+          const uint32_t pa = tmem + kColP;
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            // V rows kk*16 .. +15: 16 rows of 128 B further per step (2048 B = 128 units)
+            mma_ts(tmem + kColO, pa + kk * 8, vd + 128 * kk, idesc_pv, (j | kk) != 0 ? 1u : 0u);
+          mma_commit(smem_u32(&kv_empty[s]));
+          mma_commit(smem_u32(&pv_done));
+        }
+        if (ok && p.has_w_uv) {
+          ok = wait_bar(smem_u32(&w_full), 0, abort_flag, p.dev_status) &&
+               wait_bar(smem_u32(&olat_full), 0, abort_flag, p.dev_status);
+          if (ok) {
+            tc_fence_after();
+            const uint64_t w_c = smem_desc(sbase + kQTile + (p.nt % kStages) * kKTile, 16, 1024,
+                                           kSwizzle128B);
+#pragma unroll
+            for (int blk = 0; blk < 3; ++blk)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tmem, q_c + (blk * kQBlkD + 2 * kk), w_c + (blk * kQBlkD + 2 * kk), idesc_uv,
+                       (blk | kk) != 0 ? 1u : 0u);
+            mma_commit(smem_u32(&epi_done));
+          }
         }
       }
     }
@@ -247,14 +268,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                       wait_bar(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_flag, p.dev_status));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t sc = tmem + lane_off + (j & 1) * kBN;
       float s[kBN];
       {
         uint32_t r[kBN];
-        tmem_ld128_wait(sc, r);
+        tmem_ld128_wait(tmem + lane_off + (j & 1) * kColS, r);
 #pragma unroll
         for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
       }
+      // S(j) is in registers: its TMEM buffer may take QK(j+2) now.
+      tc_fence_before();
+      mbar_arrive(smem_u32(&s_free[j & 1]));
       const int valid = j < p.nt_ring ? min(kBN, p.nc - j * kBN)
                                       : min(kBN, p.n_q - (j - p.nt_ring) * kBN);
       if (valid < kBN) {                    // only the last tile of the ring or of the chunk
@@ -262,28 +285,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kBN; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
-      // Row max of the raw scores (the scale is positive), four independent chains.
+      // Row max of the raw scores (the scale is positive), eight independent chains.
       float mx;
       {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float m8[8];
 #pragma unroll
-        for (int c = 0; c < kBN; c += 4)
+        for (int u = 0; u < 8; ++u) m8[u] = s[u];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) m4[u] = fmaxf(m4[u], s[c + u]);
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
+        for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], s[c + u]);
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
       }
+      // Lazy rescaling: the running max moves only when a row's max grows by more than 8
+      // (a factor 256), so p stays below 256 and O is rescaled rarely.
+      bool rescale = false;
+      float alpha = 1.f;
       if (j == 0) {
         m_run = mx;
       } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
-        // O must be rescaled: wait until PV(j-1) has landed, then scale this warp's rows.
+        const float m_new = fmaxf(m_run, mx);
+        alpha = fast_exp2(m_run - m_new);
+        l_run *= alpha;
+        m_run = m_new;
+        rescale = true;
+      }
+      // p = 2^(s * scale * log2(e) - m): one FFMA and one ex2 per score, packed to bf16 pairs.
+      uint32_t w[kBN / 2];
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float neg_m = -m_run;
+#pragma unroll
+      for (int i = 0; i < kBN / 2; ++i) {
+        const float p0 = fast_exp2(fmaf(s[2 * i], p.scale_log2, neg_m));
+        const float p1 = fast_exp2(fmaf(s[2 * i + 1], p.scale_log2, neg_m));
+        sum8[i & 7] += p0 + p1;
+        w[i] = pack_bf16x2(p0, p1);
+      }
+      l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      // The P buffer and O are free once PV(j-1) has completed.
+      if (j > 0) {
         ok = __all_sync(0xffffffffu,
                         wait_bar(smem_u32(&pv_done), (j - 1) & 1, abort_flag, p.dev_status));
         if (!ok) break;
         tc_fence_after();
-        const float m_new = fmaxf(m_run, mx);
-        const float alpha = fast_exp2(m_run - m_new);
-        l_run *= alpha;
-        m_run = m_new;
+      }
+      if (rescale) {
 #pragma unroll 1
         for (int c = 0; c < kDc; c += 16) {
           uint32_t r[16];
@@ -292,29 +339,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
           tmem_st16(tmem + lane_off + kColO + c, r);
         }
-        tmem_wait_st();
       }
-      // p = 2^(s * scale * log2(e) - m): one FFMA and one ex2 per score; P packed to bf16
-      // pairs and written over S in TMEM.  Four independent partial sums.
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-      const float neg_m = -m_run;
 #pragma unroll
-      for (int c = 0; c < kBN; c += 32) {
-        uint32_t w[16];
+      for (int c = 0; c < kBN / 2; c += 16) {
+        uint32_t w16[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(s[c + 2 * i], p.scale_log2, neg_m));
-          const float p1 = fast_exp2(fmaf(s[c + 2 * i + 1], p.scale_log2, neg_m));
-          sum4[i & 3] += p0 + p1;
-          w[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(sc + c / 2, w);
+        for (int i = 0; i < 16; ++i) w16[i] = w[c + i];
+        tmem_st16(tmem + lane_off + kColP + c, w16);
       }
-      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      l_run += sum;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&p_full[j & 1]));
+      mbar_arrive(smem_u32(&p_full));
     }
     if (ok)
       ok = __all_sync(0xffffffffu,
@@ -358,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             v.y = pack_bf16x2(__uint_as_float(r[8 * ch + 2]) * inv_l, __uint_as_float(r[8 * ch + 3]) * inv_l);
             v.z = pack_bf16x2(__uint_as_float(r[8 * ch + 4]) * inv_l, __uint_as_float(r[8 * ch + 5]) * inv_l);
             v.w = pack_bf16x2(__uint_as_float(r[8 * ch + 6]) * inv_l, __uint_as_float(r[8 * ch + 7]) * inv_l);
-            const int off = blk * kBlk + row * 128 + ((chunk ^ (row & 7)) * 16);
+            const int off = blk * kQBlk + row * 128 + ((chunk ^ (row & 7)) * 16);
             *reinterpret_cast<uint4*>(qsm + off) = v;
           }
         }
@@ -390,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kQkWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

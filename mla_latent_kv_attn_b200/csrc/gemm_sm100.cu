@@ -226,9 +226,30 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s) {
       MLA_FAIL(MLA_ERR_UNSUPPORTED, "query RoPE epilogue needs 224-wide head blocks");
     return launch_gemm<224>(g, s);
   }
-  if (g.N <= 128) return launch_gemm<128>(g, s);
-  if (g.N <= 224) return launch_gemm<224>(g, s);
-  return launch_gemm<256>(g, s);
+  // Tile width: the one whose CTA count fills whole waves of 148 SMs best (ties to the wider
+  // tile, which re-reads A fewer times).  Projections here have few 128-row tiles, so a narrow
+  // N tile is what puts every SM to work.
+  constexpr int kSms = 148;
+  const int widths[4] = {256, 224, 128, 64};
+  int best = 256;
+  double best_eff = -1.0;
+  for (int w : widths) {
+    const long long ctas =
+        static_cast<long long>(ceil_div(g.M, kBM)) * ceil_div(g.N, w) * g.batch;
+    const long long waves = (ctas + kSms - 1) / kSms;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * kSms) *
+                       (static_cast<double>(g.N) / (ceil_div(g.N, w) * w));
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = w;
+    }
+  }
+  switch (best) {
+    case 64: return launch_gemm<64>(g, s);
+    case 128: return launch_gemm<128>(g, s);
+    case 224: return launch_gemm<224>(g, s);
+    default: return launch_gemm<256>(g, s);
+  }
 }
 
 }  // namespace mla
