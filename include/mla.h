@@ -281,6 +281,17 @@ mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q
 mla_status mla_out_proj(const mla_config* cfg, const void* o_lat, const void* w_uv,
                         const void* w_o, void* o, void* y, void* stream);
 
+/* --------------------------------------------------------------------------------------------
+ * mla_selftest_wait_timeout: checks, without faulting anything, that a kernel of this library
+ * whose bounded wait runs out reports it.  It launches one thread that waits, with the same
+ * bounded-wait routine the tensor-core kernels use, on a barrier that nothing ever completes;
+ * after about limit_us microseconds (1 .. 1e6) the wait gives up and the kernel writes
+ * MLA_ERR_DEVICE_TIMEOUT to *dev_status (device int32) and exits.  The caller zeroes
+ * *dev_status first and reads it after synchronising.  For failure-handling tests only.
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_selftest_wait_timeout(int32_t* dev_status, int32_t limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,7 @@ SIGNATURES = {
     "mla_out_proj": (c_int32, [_CFG, _P, _P, _P, _P, _P, _P]),
     "mla_attention_fwd_static_scratch": (c_int32, [_CFG, _P, _P, _P, _P, c_int32, c_int32, _P,
                                                    _P, _P, _P, _P]),
+    "mla_selftest_wait_timeout": (c_int32, [_P, c_int32, _P]),
 }
 
 _lib = None

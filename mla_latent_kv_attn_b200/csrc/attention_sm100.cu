@@ -70,20 +70,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Bounded wait that also gives up once another role has given up.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          int32_t* dev_status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long start = clock64();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - start > kWaitLimitCycles) {
-      *abort_flag = 1;
-      if (dev_status != nullptr) atomicExch(dev_status, static_cast<int32_t>(MLA_ERR_DEVICE_TIMEOUT));
-      return false;
-    }
-  }
+  return mbar_wait_or_abort(bar, parity, abort_flag, dev_status);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)

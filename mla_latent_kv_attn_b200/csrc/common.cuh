@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <string>
 
@@ -86,35 +88,48 @@ inline Dims dims_of(const mla_config& c) {
   return d;
 }
 
-// Geometry of the rotary bands, passed by value to kernels.
+// Geometry of the rotary bands, passed by value to kernels.  inv_freq[pair] =
+// rope_base^(-i / n_axis) for pair i of its axis band, computed on the host in double.
+constexpr int kMaxRopePairs = 64;
 struct RopeGeom {
   int pt, ph, pw;        // pairs per axis
   int frame_w, tpf;
-  float log2_base;       // log2(rope_base)
+  float inv_freq[kMaxRopePairs];
 };
 
 inline RopeGeom rope_geom(const Dims& d) {
-  RopeGeom g;
+  RopeGeom g{};
   g.pt = d.pt; g.ph = d.ph; g.pw = d.pw; g.frame_w = d.frame_w; g.tpf = d.tpf;
-  g.log2_base = static_cast<float>(std::log2(static_cast<double>(d.rope_base)));
+  const int n_axis[3] = {d.pt, d.ph, d.pw};
+  int pair = 0;
+  for (int a = 0; a < 3; ++a)
+    for (int i = 0; i < n_axis[a] && pair < kMaxRopePairs; ++i, ++pair)
+      g.inv_freq[pair] = static_cast<float>(
+          std::pow(static_cast<double>(d.rope_base), -static_cast<double>(i) / n_axis[a]));
   return g;
 }
 
 // Angle of rotary pair `pair` (0 .. pt+ph+pw-1) at position (t, h, w):
 // pos_axis * base^(-i / n_axis), i the pair's index inside its axis band.
 __device__ __forceinline__ float rope_angle(const RopeGeom& g, int pair, int t, int h, int w) {
-  int pos, i, n;
-  if (pair < g.pt) { pos = t; i = pair; n = g.pt; }
-  else if (pair < g.pt + g.ph) { pos = h; i = pair - g.pt; n = g.ph; }
-  else { pos = w; i = pair - g.pt - g.ph; n = g.pw; }
-  const float inv_freq = exp2f(-g.log2_base * static_cast<float>(i) / static_cast<float>(n));
-  return static_cast<float>(pos) * inv_freq;
+  const int pos = pair < g.pt ? t : (pair < g.pt + g.ph ? h : w);
+  return static_cast<float>(pos) * g.inv_freq[pair];
+}
+
+// sin and cos of an angle of moderate size (|a| < 2^15): Cody-Waite reduction by 2*pi
+// (2*pi split into its float value and the float remainder) to r in [-pi, pi], then the
+// hardware sin/cos approximations, which are accurate on that interval (error ~2^-21).
+__device__ __forceinline__ void rope_sincos(float a, float* s, float* c) {
+  const float k = rintf(a * 0.159154943091895336f);
+  float r = fmaf(-k, 6.28318548202514648f, a);
+  r = fmaf(-k, -1.74845553146951724e-7f, r);
+  __sincosf(r, s, c);
 }
 
 // Rotates one pair (x0, x1) by angle a.
 __device__ __forceinline__ void rope_rotate(float& x0, float& x1, float a) {
   float s, c;
-  sincosf(a, &s, &c);
+  rope_sincos(a, &s, &c);
   const float y0 = x0 * c - x1 * s;
   const float y1 = x0 * s + x1 * c;
   x0 = y0;

@@ -27,6 +27,8 @@ mla_status check_cfg(const mla_config* cfg) {
   MLA_CHECK_ARG(c.rope_pairs_t >= 0 && c.rope_pairs_h >= 0 && c.rope_pairs_w >= 0 &&
                     2 * (c.rope_pairs_t + c.rope_pairs_h + c.rope_pairs_w) == c.d_rope,
                 "d_rope (%d) must equal 2*(rope_pairs_t+rope_pairs_h+rope_pairs_w)", c.d_rope);
+  MLA_CHECK_ARG(c.rope_pairs_t + c.rope_pairs_h + c.rope_pairs_w <= kMaxRopePairs,
+                "at most %d rotary pairs are supported", kMaxRopePairs);
   MLA_CHECK_ARG(std::isfinite(c.rope_base) && c.rope_base > 1.f, "rope_base must be > 1");
   MLA_CHECK_ARG(std::isfinite(c.softmax_scale) && c.softmax_scale > 0.f,
                 "softmax_scale must be positive and finite");

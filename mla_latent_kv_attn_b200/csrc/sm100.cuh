@@ -7,6 +7,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include "mla.h"
+
 namespace mla {
 namespace sm100 {
 
@@ -57,6 +59,26 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (clock64() - start > kWaitLimitCycles) return false;
   }
   return true;
+}
+
+// Bounded wait used by kernels with several roles: gives up when the wait runs past
+// `limit_cycles`, or as soon as another role of the CTA has given up (abort flag).  On running
+// out it raises the abort flag and writes MLA_ERR_DEVICE_TIMEOUT to *dev_status (if given), so
+// the host learns of it after synchronising; the caller unwinds and frees what it holds.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity,
+                                                   volatile int* abort_flag, int32_t* dev_status,
+                                                   long long limit_cycles = kWaitLimitCycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long start = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - start > limit_cycles) {
+      *abort_flag = 1;
+      if (dev_status != nullptr) atomicExch(dev_status, static_cast<int32_t>(MLA_ERR_DEVICE_TIMEOUT));
+      return false;
+    }
+  }
 }
 
 // ---- TMA (tiled bulk tensor loads into this CTA's shared memory, no multicast) -------------

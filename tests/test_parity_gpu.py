@@ -262,3 +262,22 @@ def test_wan_config4_thirty_layer_stack():
             gpu_sf = rings[l].slot_frame.cpu().numpy()
             for b in range(cfg.batch):
                 np.testing.assert_array_equal(gpu_sf[b], expected_slot_frame(cfg, o.windows[b]))
+
+
+def test_device_wait_timeout_is_reported_and_context_survives():
+    """A bounded wait that runs out inside a kernel reports MLA_ERR_DEVICE_TIMEOUT through the
+    status word; nothing traps and the context keeps working afterwards."""
+    from mla_latent_kv_attn_b200 import _lib
+    status = torch.zeros(1, device="cuda", dtype=torch.int32)
+    st = _lib.lib().mla_selftest_wait_timeout(status.data_ptr(), 2000,
+                                              torch.cuda.current_stream().cuda_stream)
+    assert st == 0, _lib.last_error()
+    torch.cuda.synchronize()
+    assert int(status.item()) == _lib.MLA_ERR_DEVICE_TIMEOUT
+    # the device is still usable: a small rollout chunk runs and matches the oracle
+    cfg = inputs.CONFIGS[0]
+    g = GpuRun(cfg)
+    o = OracleRun(cfg, g.lw)
+    x = inputs.chunk_x(cfg, 0)
+    check_chunk("after_timeout", cfg, g.attend(0, x), o.step(0, x, np.arange(cfg.n_q)),
+                np.arange(cfg.n_q))
