@@ -4,22 +4,26 @@
 
 One step = one chunk of an autoregressive rollout through the whole path, on one batch of
 synthetic Wan2.1-1.3B-shaped input (the 6-frame window full, a 3-frame chunk of 4680 queries):
-query projection with fused 3D-RoPE, chunk latents (joint KV down-projection), attention over
-the ring plus the chunk with the W_UV up-projection fused, and the ring append.  Steps advance
+the projections of the chunk (query latent and chunk latents in one pass over x, then the
+absorbed query heads with fused 3D-RoPE), attention over the ring plus the chunk with the W_UV
+up-projection fused, and the ring append.  Steps advance
 the rollout (chunk 2, 3, 4, ... of a 6-frame window), so every step has the same work.
 
 Timing: W untimed warm-up steps, then K steps between a barrier + device synchronisation on
-both sides.  L2 is flushed before every step (a 256 MiB device memset, outside the per-step
-CUDA-event intervals).  Device time per step = sum of per-step event intervals on the launch
-stream; the job time is the max over ranks.  With N > 1 every rank runs its own independent
+both sides.  Each step's five kernels are captured beforehand as one CUDA graph per chunk
+(rollout.ChunkGraph) and replayed, so the device runs them back to back.  L2 is flushed before
+every step (a 256 MiB device memset, outside the per-step CUDA-event intervals).  Device time
+per step = sum of per-step event intervals on the launch stream; the job time is the max over
+ranks.  With N > 1 every rank runs its own independent
 sample (weak scaling: no data-path collective exists on this path).
 
 value      attention algorithmic TFLOP/s of the whole step: 2*(D + d_c) = 832 flop per
            (query row, attended key, head), divided by the whole-step device time
 e2e        the same metric through the public API with host buffers: pinned host -> device copy
            of the step's tokens and device -> host copy of its output inside the timed interval
-roofline   the attention call (rotated-key pre-pass + tensor-core kernel), timed on its own
-           stream with CUDA events inside the timed region, against the measured bf16 peak
+roofline   the attention call (rotated-key pre-pass + tensor-core kernel), timed with CUDA
+           events recorded inside each step's graph around that call, against the measured
+           bf16 peak
 cpu_baseline  the float64 CPU oracle on a bounded sample of the same chunk (rank 0, N = 1)
 """
 from __future__ import annotations
@@ -241,7 +245,8 @@ def run_ours(args, cfg):
         rollout.prefill_chunk(c, w, ring, buf, ch)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 6   # c_Q GEMM, Q' GEMM+RoPE, KV GEMM, rope-key pre-pass, attention, append
+    launches_per_step = 5   # x GEMM (c_Q || chunk latents), Q' GEMM+RoPE, rope-key pre-pass,
+                            # attention (+W_UV), ring append
 
     first_chunk = cfg.measured_chunk
     flops_step = cfg.attention_flops(first_chunk)   # same for every later chunk (window full)
@@ -250,9 +255,7 @@ def run_ours(args, cfg):
         ch = first_chunk + i
         x = pool[i % n_pool] if x is None else x
         first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, ch)
-        api.mla_query_proj(c, x, w.w_dq, w.w_qcat, buf.c_q, buf.q, first)
-        api.mla_cache_append(c, x, w.w_dkv_kr, buf.chunk_lat, ring.cache, ring.slot_frame,
-                             first, api.MLA_PROJECT)
+        api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
         if ev is not None:
             ev[0].record(stream)
         api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid,
@@ -262,10 +265,15 @@ def run_ours(args, cfg):
         api.mla_cache_append(c, None, None, buf.chunk_lat, ring.cache, ring.slot_frame, first,
                              api.MLA_APPEND)
 
+    # Each step is one CUDA graph (rollout.ChunkGraph): the chunk's five kernels replay back to
+    # back without per-launch host overhead.  Graphs are captured before the timed region (host
+    # set-up, like encoding a plan); capturing launches nothing.
+    graphs = [rollout.ChunkGraph(c, w, ring, buf, first_chunk + i, x=pool[i % n_pool], events=True)
+              for i in range(args.warmup + args.steps)]
     # warm-up
     for i in range(args.warmup):
         flush.zero_()
-        step(i)
+        graphs[i].replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -273,8 +281,6 @@ def run_ours(args, cfg):
     # ---- device-timed region
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -283,39 +289,67 @@ def run_ours(args, cfg):
         for i in range(args.steps):
             flush.zero_()
             ev_s[i].record(stream)
-            step(args.warmup + i, ev_a[i])
+            graphs[args.warmup + i].replay()
             ev_e[i].record(stream)
         torch.cuda.synchronize()
         time.sleep(0.25)
     if world > 1:
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(ev_s, ev_e)]
-    attn_ms = [a.elapsed_time(b) for a, b in ev_a]
+    attn_ms = [graphs[args.warmup + i].attention_ms() for i in range(args.steps)]
     total_ms = max_over_ranks(sum(step_ms), device=dev)
     status = int(buf.dev_status.item())
     if status != 0:
         raise RuntimeError(f"a kernel reported status {status}")
 
     # ---- end to end through the public API with host buffers
+    # Pinned host tokens in, pinned host output back, every copy inside the timed interval.
+    # Pipelined (rollout.HostStreamer): chunk n's copy-in overlaps chunk n-1's compute and its
+    # copy-out overlaps chunk n+1's compute; one interval from before the first copy-in to after
+    # the last copy-out, L2 flushes included.  The serial variant (copy-in, compute, copy-out
+    # one after the other on one stream) is reported beside it.
     x_host = [p.cpu().pin_memory() for p in pool]
-    o_host = torch.empty(buf.o.shape, dtype=buf.o.dtype).pin_memory()
+    o_host = [torch.empty(buf.o.shape, dtype=buf.o.dtype).pin_memory() for _ in range(2)]
     h2d = x_host[0].numel() * x_host[0].element_size()
-    d2h = o_host.numel() * o_host.element_size()
-    e2e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e2e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    d2h = o_host[0].numel() * o_host[0].element_size()
     base = args.warmup + args.steps
+    streamer = rollout.HostStreamer(c, w, ring, device=dev, compute_stream=stream)
+    for i in range(args.warmup):          # warm the streamer's own buffers and streams
+        flush.zero_()
+        streamer.submit(first_chunk + base + i, x_host[i % n_pool], o_host[i % 2])
+    streamer.finish()
+    torch.cuda.synchronize()
+    base += args.warmup
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e2e_a, e2e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_a.record(stream)
+    streamer.begin(e2e_a)
+    for i in range(args.steps):
+        flush.zero_()
+        streamer.submit(first_chunk + base + i, x_host[(base + i) % n_pool], o_host[i % 2])
+    streamer.finish()
+    e2e_b.record(stream)
+    torch.cuda.synchronize()
+    streamer.check_device_status()
+    e2e_ms = max_over_ranks(e2e_a.elapsed_time(e2e_b), device=dev)
+    base += args.steps
+    # serial variant
+    ser_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ser_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.zero_()
-        e2e_s[i].record(stream)
+        ser_s[i].record(stream)
         buf.x.copy_(x_host[(base + i) % n_pool], non_blocking=True)
         step(base + i, x=buf.x)
-        o_host.copy_(buf.o, non_blocking=True)
-        e2e_e[i].record(stream)
+        o_host[0].copy_(buf.o, non_blocking=True)
+        ser_e[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e)), device=dev)
+    ser_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(ser_s, ser_e)), device=dev)
     if world > 1:
         dist.barrier()
 
@@ -352,7 +386,12 @@ def run_ours(args, cfg):
                      "peak_kind": f"{peak_kind} burst bf16",
                      "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
         "e2e": {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12,
-                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps,
+                "mode": "pipelined: copy-in of chunk n+1 and copy-out of chunk n-1 overlap "
+                        "chunk n (rollout.HostStreamer); one interval incl. L2 flushes",
+                "serial_value": world * flops_step * args.steps / (ser_ms * 1e-3) / 1e12,
+                "serial_ms_per_step": ser_ms / args.steps},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }

@@ -199,6 +199,26 @@ mla_status mla_query_proj(const mla_config* cfg, const void* x, const void* w_dq
                           void* stream);
 
 /* --------------------------------------------------------------------------------------------
+ * mla_project_chunk: every projection of a chunk's tokens in one pass over x: the query path of
+ * mla_query_proj and the joint KV down-projection of mla_cache_append(MLA_PROJECT) ([M]: the
+ * query latent c_Q and the content latent c_KV are both down-projections of the token x, and
+ * k_R is W_R^K x).  The results equal those two calls:
+ *   c_q[b, n]        = W_down^Q x[b, n]
+ *   chunk_lat[b, n]  = [W_down^KV x[b, n] || W_R^K x[b, n]]
+ *   q[b, n, h, :]    = [ w_qcat[h, 0:d_c] c_q  ||  RoPE3D(w_qcat[h, d_c:D] c_q, pos(b, n)) ]
+ *   x      device T [B, n_q, d_model]
+ *   w_x    device T [d_cq + D, d_model]: rows 0..d_cq-1 = W_down^Q, rows d_cq..d_cq+d_c-1 =
+ *          W_down^KV, rows d_cq+d_c.. = W_R^K (the three down-projections stacked)
+ *   w_qcat device T [H, D, d_cq] (from mla_compose_query_weights)
+ *   c_q    device T [B, n_q, d_cq] (out)   q device T [B, n_q, H, D] (out)
+ *   chunk_lat device T [B, n_q, D] (out)
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w_x,
+                             const void* w_qcat, void* c_q, void* q, void* chunk_lat,
+                             int32_t first_frame, void* stream);
+
+/* --------------------------------------------------------------------------------------------
  * mla_attention_workspace_bytes: device scratch mla_attention_fwd needs for a call with the
  * given number of valid ring frames (rotated positional keys of every attended key, tile-padded).
  * Returns 0 for an invalid configuration.

@@ -17,7 +17,7 @@ from ._lib import (MLA_APPEND, MLA_BF16, MLA_FP32, MLA_PATH_AUTO, MLA_PATH_SIMT,
 
 __all__ = [
     "make_config", "torch_dtype", "mla_config_check", "mla_cache_append", "mla_rope3d",
-    "mla_key_positions", "mla_compose_query_weights", "mla_query_proj",
+    "mla_key_positions", "mla_compose_query_weights", "mla_query_proj", "mla_project_chunk",
     "mla_attention_workspace_bytes", "mla_attention_fwd", "mla_attention_fwd_static_scratch",
     "mla_out_proj", "MLAError",
     "MLA_PROJECT", "MLA_APPEND", "MLA_PROJECT_AND_APPEND", "MLA_PATH_AUTO", "MLA_PATH_SIMT",
@@ -128,6 +128,19 @@ def mla_query_proj(c: MLAConfigC, x, w_dq, w_qcat, c_q, q, first_frame: int, str
         _ptr(c_q, "c_q", dt, (B, n_q, c.d_cq)), _ptr(q, "q", dt, (B, n_q, H, D)), first_frame,
         _stream(stream))
     _lib.check("mla_query_proj", st)
+
+
+def mla_project_chunk(c: MLAConfigC, x, w_x, w_qcat, c_q, q, chunk_lat, first_frame: int,
+                      stream=None) -> None:
+    tpf, n_q, D = _geom(c)
+    dt = torch_dtype(c)
+    B, H = c.batch, c.n_heads
+    st = _lib.lib().mla_project_chunk(
+        ctypes.byref(c), _ptr(x, "x", dt, (B, n_q, c.d_model)),
+        _ptr(w_x, "w_x", dt, (c.d_cq + D, c.d_model)), _ptr(w_qcat, "w_qcat", dt, (H, D, c.d_cq)),
+        _ptr(c_q, "c_q", dt, (B, n_q, c.d_cq)), _ptr(q, "q", dt, (B, n_q, H, D)),
+        _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)), first_frame, _stream(stream))
+    _lib.check("mla_project_chunk", st)
 
 
 def mla_attention_workspace_bytes(c: MLAConfigC, n_valid_frames: int) -> int:

@@ -70,6 +70,33 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input FMNMX).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
+// Packed pairs of fp32 (sm_100 FFMA2 / FADD2: two lanes of fp32 arithmetic per instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          int32_t* dev_status) {
   return mbar_wait_or_abort(bar, parity, abort_flag, dev_status);
@@ -274,18 +301,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kBN; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
-      // Row max of the raw scores (the scale is positive), eight independent chains.
+      // Row max of the raw scores (the scale is positive): eight independent chains of
+      // three-input maxima, chain u covering columns u, u+8, ..., u+120.
       float mx;
       {
         float m8[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) m8[u] = s[u];
+        for (int u = 0; u < 8; ++u) {
+          float a = fmax3(s[u], s[u + 8], s[u + 16]);
 #pragma unroll
-        for (int c = 8; c < kBN; c += 8)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], s[c + u]);
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
+          for (int c = 24; c < kBN - 8; c += 16) a = fmax3(a, s[c + u], s[c + 8 + u]);
+          m8[u] = fmaxf(a, s[kBN - 8 + u]);
+        }
+        mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) *
+             p.scale_log2;
       }
       // Lazy rescaling: the running max moves only when a row's max grows by more than 8
       // (a factor 256), so p stays below 256 and O is rescaled rarely.
@@ -300,18 +329,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
         rescale = true;
       }
-      // p = 2^(s * scale * log2(e) - m): one FFMA and one ex2 per score, packed to bf16 pairs.
+      // p = 2^(s * scale * log2(e) - m): one packed FFMA2 per two scores, one ex2 per score,
+      // packed to bf16 pairs; the row sum runs in four packed FADD2 chains.
       uint32_t w[kBN / 2];
-      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const float neg_m = -m_run;
+      {
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(-m_run, -m_run);
+        uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int i = 0; i < kBN / 2; ++i) {
-        const float p0 = fast_exp2(fmaf(s[2 * i], p.scale_log2, neg_m));
-        const float p1 = fast_exp2(fmaf(s[2 * i + 1], p.scale_log2, neg_m));
-        sum8[i & 7] += p0 + p1;
-        w[i] = pack_bf16x2(p0, p1);
+        for (int i = 0; i < kBN / 2; ++i) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sc2, nm2), x0, x1);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
+          sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(p0, p1));
+          w[i] = pack_bf16x2(p0, p1);
+        }
+        const uint64_t t2 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
+        float l0, l1;
+        f2_unpack(t2, l0, l1);
+        l_run += l0 + l1;
       }
-      l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       // The P buffer and O are free once PV(j-1) has completed.
       if (j > 0) {
         ok = __all_sync(0xffffffffu,

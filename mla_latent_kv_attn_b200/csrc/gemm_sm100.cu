@@ -1,13 +1,28 @@
 // gemm_sm100.cu - bf16 GEMM on the 5th-generation tensor cores for the projections of the
-// path (KV down-projection, query latent, absorbed query heads, value up-projection, W_O).
+// path (joint query/KV down-projection, absorbed query heads, value up-projection, W_O).
 //
 //   C[z](m, n) = sum_k A[z](m, k) * B[z](n, k)     bf16 operands, fp32 accumulation in TMEM
 //
-// One CTA computes a 128 x BN tile.  Warp 0 streams 128x64 (A) and BNx64 (B) K-slices into a
-// 4-stage ring of 128B-swizzled shared-memory buffers with TMA; warp 1 allocates TMEM and one of
-// its threads issues tcgen05.mma (M=128, N=BN, K=16 per instruction) and commits each stage
-// back to the producer; warps 2..5 drain the fp32 accumulator from TMEM (one lane = one row),
-// optionally rotate the positional-query columns (3D-RoPE), and store bf16 rows.
+// Persistent: a grid of at most one CTA per SM walks the 128 x BN output tiles (tile index
+// n-fastest, so CTAs working at the same time share the A rows through L2), each CTA taking
+// every gridDim.x-th tile.  Roles (192 threads):
+//   warp 0     TMA producer: 128x64 (A) and BNx64 (B) K-slices into a ring of 128B-swizzled
+//              buffers as deep as shared memory allows (4 to 8 stages); the ring runs on across
+//              tile boundaries.
+//   warp 1     allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) into one of two
+//              TMEM accumulators (tiles alternate), committing each stage back to the producer
+//              and each finished accumulator to the epilogue.
+//   warps 2-5  epilogue: drain an accumulator (one TMEM lane = one output row per thread) 32
+//              columns at a time, optionally rotate the positional-query columns (3D-RoPE),
+//              write bf16 into a 64B-swizzled 128x32 staging buffer (two, alternating) that one
+//              thread stores with a TMA bulk-tensor store (whole lines, out-of-range rows and
+//              columns clipped), and hand the accumulator back; this overlaps the MMAs of the
+//              CTA's next tile.  Outputs whose strides TMA cannot take are stored row by row.
+// Before the first K-slice of a tile the producer asks L2 for its share of the tile's A panel
+// (when the panel is one contiguous range) with one bulk prefetch, so the panel streams from HBM
+// in long runs instead of one 128-byte piece per row and K-slice.
+// Optionally the columns n >= n_split go to a second output C2 (column n - n_split): one GEMM
+// over [W_1; W_2] then writes x W_1^T and x W_2^T to their own arrays.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -19,23 +34,43 @@ using namespace sm100;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;          // one 128-byte swizzle atom of bf16 per row
-constexpr int kStages = 4;
 constexpr int kThreads = 192;    // 6 warps
+constexpr int kEpiThreads = 128;
+
+constexpr int kMaxStages = 8;
+constexpr int kEpiCols = 32;                       // columns per staged store
+constexpr int kStageOut = kBM * kEpiCols * 2;      // 8 KB: one 128 x 32 bf16 staging buffer
+constexpr int kSmemBudget = 220 * 1024 - 2 * kStageOut;   // what the operand ring may use
 
 template <int BN>
 struct GemmCfg {
   static constexpr int kATile = kBM * kBK * 2;
   static constexpr int kBTile = BN * kBK * 2;
   static constexpr int kStage = kATile + kBTile;
-  static constexpr int kSmem = kStages * kStage + 1024;  // + slack to align to 1024 B
-  static constexpr int kTmemCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+  // As many stages as fit: the loads in flight per SM must cover the L2/HBM latency.
+  static constexpr int kStages = kSmemBudget / kStage < kMaxStages ? kSmemBudget / kStage : kMaxStages;
+  static constexpr int kOut = kStages * kStage;          // staging buffers after the ring
+  static constexpr int kSmem = kOut + 2 * kStageOut + 1024;  // + slack to align to 1024 B
+  // two accumulators, each starting on a power-of-two column
+  static constexpr int kAccStride = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+  static constexpr int kTmemCols = 2 * kAccStride;
+  static_assert(BN <= 256 && BN % 16 == 0, "tcgen05 M=128 needs N a multiple of 16 up to 256");
 };
 
 struct GemmParams {
-  int M, N, K;
+  int M, N, K, batch;
+  int n_tiles_m, n_tiles_n;
   int a_swapped, b_swapped;  // tensor map dims are (K, batch, rows) instead of (K, rows, batch)
   void* C;
   int64_t c_sm, c_batch;
+  void* C2;                  // columns >= n_split (0 = no split)
+  int64_t c2_sm, c2_batch;
+  int n_split;
+  int tma_store;             // 1: stores through tmC / tmC2 (see launch_gemm)
+  int c_swapped, c2_swapped; // output maps are (N, batch, rows) instead of (N, rows, batch)
+  int prefetch_a;            // 1: the A panel of a tile is one contiguous range
+  const void* A;
+  int64_t a_sm;
   int epilogue;
   int rope_D, rope_n_q, rope_first_frame;
   RopeGeom rope;
@@ -50,32 +85,57 @@ __device__ __forceinline__ void store_row32(bf16* dst, const float* v, int valid
 #pragma unroll
     for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
   } else {
-    for (int i = 0; i < valid && i < 32; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < valid) dst[i] = __float2bfloat16_rn(v[i]);
   }
+}
+
+struct TileCoord {
+  int z, m0, n0;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const GemmParams& p, int t) {
+  TileCoord c;
+  const int per_z = p.n_tiles_m * p.n_tiles_n;
+  c.z = t / per_z;
+  const int r = t - c.z * per_z;
+  c.m0 = (r / p.n_tiles_n) * kBM;
+  c.n0 = (r % p.n_tiles_n);
+  return c;
 }
 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                    GemmParams p) {
   using Cfg = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
+  constexpr int kStages = Cfg::kStages;
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
-  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ __align__(8) uint64_t acc_full[2];
+  __shared__ __align__(8) uint64_t acc_empty[2];
   __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM, z = blockIdx.z;
   const int nkb = ceil_div(p.K, kBK);
+  const int n_tiles = p.n_tiles_m * p.n_tiles_n * p.batch;
+  volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
+    abort_sh = 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
-    mbar_init(smem_u32(&acc_bar), 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&acc_full[a]), 1);
+      mbar_init(smem_u32(&acc_empty[a]), kEpiThreads);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -91,78 +151,155 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t ph = (kb / kStages) & 1;
-        if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1)) break;
-        const uint32_t a_dst = base + s * Cfg::kStage;
-        const uint32_t b_dst = a_dst + Cfg::kATile;
-        const uint32_t fb = smem_u32(&full_bar[s]);
-        mbar_arrive_expect_tx(fb, Cfg::kStage);
-        if (p.a_swapped) tma_load_3d(a_dst, &tmA, fb, kb * kBK, z, m0);
-        else tma_load_3d(a_dst, &tmA, fb, kb * kBK, m0, z);
-        if (p.b_swapped) tma_load_3d(b_dst, &tmB, fb, kb * kBK, z, n0);
-        else tma_load_3d(b_dst, &tmB, fb, kb * kBK, n0, z);
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_coord(p, t);
+        const int n0 = tc.n0 * BN;
+        if (p.prefetch_a) {
+          // share tc.n0 of n_tiles_n of the rows m0 .. m0+127 (all of K, contiguous)
+          const int rows = min(kBM, p.M - tc.m0);
+          const int r0 = rows * tc.n0 / p.n_tiles_n, r1 = rows * (tc.n0 + 1) / p.n_tiles_n;
+          const uint32_t row_bytes = static_cast<uint32_t>(p.a_sm) * 2u;
+          if (r1 > r0)
+            prefetch_l2_bulk(static_cast<const uint8_t*>(p.A) +
+                                 static_cast<int64_t>(tc.m0 + r0) * row_bytes,
+                             static_cast<uint32_t>(r1 - r0) * row_bytes);
+        }
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          ok = mbar_wait_or_abort(smem_u32(&empty_bar[s]), ph ^ 1, abort_flag, nullptr);
+          if (!ok) break;
+          const uint32_t a_dst = base + s * Cfg::kStage;
+          const uint32_t b_dst = a_dst + Cfg::kATile;
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          mbar_arrive_expect_tx(fb, Cfg::kStage);
+          if (p.a_swapped) tma_load_3d(a_dst, &tmA, fb, kb * kBK, tc.z, tc.m0);
+          else tma_load_3d(a_dst, &tmA, fb, kb * kBK, tc.m0, tc.z);
+          if (p.b_swapped) tma_load_3d(b_dst, &tmB, fb, kb * kBK, tc.z, n0);
+          else tma_load_3d(b_dst, &tmB, fb, kb * kBK, n0, tc.z);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, 0, 0);
+      int it = 0, lt = 0;
       bool ok = true;
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t ph = (kb / kStages) & 1;
-        ok = mbar_wait(smem_u32(&full_bar[s]), ph);
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++lt) {
+        const int acc = lt & 1;
+        // the epilogue has drained this accumulator (its previous tile); first use passes
+        ok = mbar_wait_or_abort(smem_u32(&acc_empty[acc]), ((lt >> 1) & 1) ^ 1, abort_flag, nullptr);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a_addr = base + s * Cfg::kStage;
-        const uint32_t b_addr = a_addr + Cfg::kATile;
+        const uint32_t d = tmem + acc * Cfg::kAccStride;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          ok = mbar_wait_or_abort(smem_u32(&full_bar[s]), ph, abort_flag, nullptr);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_addr = base + s * Cfg::kStage;
+          const uint32_t b_addr = a_addr + Cfg::kATile;
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          const uint64_t ad = smem_desc(a_addr + 32 * k, 16, 1024, kSwizzle128B);
-          const uint64_t bd = smem_desc(b_addr + 32 * k, 16, 1024, kSwizzle128B);
-          mma_ss(tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = smem_desc(a_addr + 32 * k, 16, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(b_addr + 32 * k, 16, 1024, kSwizzle128B);
+            mma_ss(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&empty_bar[s]));
         }
-        mma_commit(smem_u32(&empty_bar[s]));
+        if (ok) mma_commit(smem_u32(&acc_full[acc]));
       }
-      if (ok) mma_commit(smem_u32(&acc_bar));
     }
   } else {
     // epilogue warps 2..5 cover TMEM lane quadrants 2, 3, 0, 1
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int m = m0 + row;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_bar), 0));
-    tc_fence_after();
-    if (ok) {
-      bf16* crow = static_cast<bf16*>(p.C) + static_cast<int64_t>(z) * p.c_batch +
-                   static_cast<int64_t>(m) * p.c_sm;
-      const bool vec_ok = ((reinterpret_cast<uintptr_t>(p.C) & 15u) == 0) && (p.c_sm % 8 == 0) &&
-                          (p.c_batch % 8 == 0);
-      int t = 0, hh = 0, ww = 0;
+    const bool leader = threadIdx.x == 64;   // issues and waits for the TMA stores
+    const uint32_t out_base = base + Cfg::kOut;
+    const bool vec_ok = ((reinterpret_cast<uintptr_t>(p.C) & 15u) == 0) && (p.c_sm % 8 == 0) &&
+                        (p.c_batch % 8 == 0) &&
+                        (p.n_split == 0 || (((reinterpret_cast<uintptr_t>(p.C2) & 15u) == 0) &&
+                                            (p.c2_sm % 8 == 0) && (p.c2_batch % 8 == 0)));
+    int lt = 0, chunk = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&acc_full[acc]),
+                                                                  (lt >> 1) & 1, abort_flag, nullptr));
+      if (!ok) break;
+      tc_fence_after();
+      const TileCoord tc = tile_coord(p, t);
+      const int n0 = tc.n0 * BN;
+      const int m = tc.m0 + row;
+      int t_pos = 0, hh = 0, ww = 0;
       if (p.epilogue == kEpiRopeQ) {
         const int nl = m % p.rope_n_q;
         const int i = nl % p.rope.tpf;
-        t = p.rope_first_frame + nl / p.rope.tpf;
+        t_pos = p.rope_first_frame + nl / p.rope.tpf;
         hh = i / p.rope.frame_w;
         ww = i % p.rope.frame_w;
       }
+      const uint32_t tacc = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::kAccStride;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < BN; c0 += kEpiCols, ++chunk) {
+        const int n = n0 + c0;
+        if (n >= p.N) break;                   // uniform over the CTA
         uint32_t r[32];
-        tmem_ld32_wait(tmem + (static_cast<uint32_t>(quad * 32) << 16) + c0, r);
+        tmem_ld32_wait(tacc + c0, r);
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-        if (p.epilogue == kEpiRopeQ && ((n0 + c0) % p.rope_D) == p.rope_D - 32) {
+        if (p.epilogue == kEpiRopeQ && (n % p.rope_D) == p.rope_D - 32) {
 #pragma unroll
           for (int pr = 0; pr < 16; ++pr)
-            rope_rotate(v[2 * pr], v[2 * pr + 1], rope_angle(p.rope, pr, t, hh, ww));
+            rope_rotate(v[2 * pr], v[2 * pr + 1], rope_angle(p.rope, pr, t_pos, hh, ww));
         }
-        const int n = n0 + c0;
-        if (m < p.M && n < p.N) store_row32(crow + n, v, p.N - n, vec_ok);
+        const bool second = p.n_split > 0 && n >= p.n_split;
+        if (p.tma_store) {
+          const uint32_t buf = out_base + (chunk & 1) * kStageOut;
+          // the store that last read this buffer (two chunks ago) has finished reading it
+          if (leader) bulk_wait_group_read<1>();
+          named_bar_sync(1, kEpiThreads);
+          // row `row` is 64 B: four 16-byte pieces, piece j at j ^ ((row / 2) mod 4) (64B swizzle)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 w4 = make_uint4(pack_bf16x2(v[8 * j + 0], v[8 * j + 1]),
+                                        pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                        pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                                        pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+            const uint32_t dst = buf + row * 64 + ((j ^ ((row >> 1) & 3)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w4.x),
+                         "r"(w4.y), "r"(w4.z), "r"(w4.w)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, kEpiThreads);
+          if (leader) {
+            const CUtensorMap* map = second ? &tmC2 : &tmC;
+            const int col = second ? n - p.n_split : n;
+            if (second ? p.c2_swapped : p.c_swapped) tma_store_3d(map, buf, col, tc.z, tc.m0);
+            else tma_store_3d(map, buf, col, tc.m0, tc.z);
+            bulk_commit_group();
+          }
+        } else if (m < p.M) {
+          if (second) {
+            bf16* crow = static_cast<bf16*>(p.C2) + static_cast<int64_t>(tc.z) * p.c2_batch +
+                         static_cast<int64_t>(m) * p.c2_sm;
+            store_row32(crow + (n - p.n_split), v, p.N - n, vec_ok);
+          } else {
+            bf16* crow = static_cast<bf16*>(p.C) + static_cast<int64_t>(tc.z) * p.c_batch +
+                         static_cast<int64_t>(m) * p.c_sm;
+            store_row32(crow + n, v, (p.n_split > 0 ? p.n_split : p.N) - n, vec_ok);
+          }
+        }
       }
+      // accumulator drained: the MMA thread may start the CTA's next-but-one tile in it
+      tc_fence_before();
+      mbar_arrive(smem_u32(&acc_empty[acc]));
     }
+    if (leader) bulk_wait_group_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -172,24 +309,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Tensor map over one operand [batch][rows, K] (K contiguous).  TMA wants increasing strides,
-// so when the batch stride is below the row stride the map is built over (K, batch, rows).
-mla_status operand_map(CUtensorMap* map, const void* base, int K, int rows, int batch,
-                       int64_t row_stride, int64_t batch_stride, uint32_t box_rows, int* swapped) {
+// Tensor map over one bf16 matrix [batch][rows, cols] (cols contiguous), box (box_cols,
+// box_rows, 1).  TMA wants increasing strides, so when the batch stride is below the row stride
+// the map is built over (cols, batch, rows) and *swapped is set.
+mla_status matrix_map(CUtensorMap* map, const void* base, int cols, int rows, int batch,
+                      int64_t row_stride, int64_t batch_stride, uint32_t box_cols,
+                      uint32_t box_rows, int swizzle, int* swapped) {
   const int64_t bs = batch > 1 ? batch_stride : row_stride * rows;
   *swapped = (batch > 1 && bs < row_stride) ? 1 : 0;
   if (*swapped) {
-    const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(batch),
+    const uint64_t dims[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(batch),
                               static_cast<uint64_t>(rows)};
     const uint64_t strides[2] = {static_cast<uint64_t>(bs) * 2, static_cast<uint64_t>(row_stride) * 2};
-    const uint32_t box[3] = {static_cast<uint32_t>(kBK), 1, box_rows};
-    return make_tmap_bf16(map, base, 3, dims, strides, box, 128);
+    const uint32_t box[3] = {box_cols, 1, box_rows};
+    return make_tmap_bf16(map, base, 3, dims, strides, box, swizzle);
   }
-  const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows),
+  const uint64_t dims[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
                             static_cast<uint64_t>(batch)};
   const uint64_t strides[2] = {static_cast<uint64_t>(row_stride) * 2, static_cast<uint64_t>(bs) * 2};
-  const uint32_t box[3] = {static_cast<uint32_t>(kBK), box_rows, 1};
-  return make_tmap_bf16(map, base, 3, dims, strides, box, 128);
+  const uint32_t box[3] = {box_cols, box_rows, 1};
+  return make_tmap_bf16(map, base, 3, dims, strides, box, swizzle);
+}
+
+mla_status operand_map(CUtensorMap* map, const void* base, int K, int rows, int batch,
+                       int64_t row_stride, int64_t batch_stride, uint32_t box_rows, int* swapped) {
+  return matrix_map(map, base, K, rows, batch, row_stride, batch_stride, kBK, box_rows, 128, swapped);
+}
+
+// An output can take TMA stores when its base is 16-byte aligned and its strides are whole
+// multiples of 16 bytes.
+bool tma_storable(const void* c, int64_t c_sm, int64_t c_batch, int batch) {
+  return (reinterpret_cast<uintptr_t>(c) & 15u) == 0 && c_sm % 8 == 0 &&
+         (batch == 1 || c_batch % 8 == 0);
+}
+
+int num_sms() {
+  static int n = [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      return 148;
+    }
+    return v;
+  }();
+  return n;
 }
 
 template <int BN>
@@ -202,13 +366,40 @@ mla_status launch_gemm(const TcGemmArgs& g, cudaStream_t s) {
   st = operand_map(&tb, g.B, g.K, g.N, g.batch, g.b_sn, g.b_batch, BN, &b_sw);
   if (st != MLA_OK) return st;
   GemmParams p;
-  p.M = g.M; p.N = g.N; p.K = g.K; p.a_swapped = a_sw; p.b_swapped = b_sw; p.C = g.C; p.c_sm = g.c_sm; p.c_batch = g.c_batch;
+  p.M = g.M; p.N = g.N; p.K = g.K; p.batch = g.batch;
+  p.n_tiles_m = ceil_div(g.M, kBM); p.n_tiles_n = ceil_div(g.N, BN);
+  p.a_swapped = a_sw; p.b_swapped = b_sw;
+  p.C = g.C; p.c_sm = g.c_sm; p.c_batch = g.c_batch;
+  p.C2 = g.C2; p.c2_sm = g.c2_sm; p.c2_batch = g.c2_batch; p.n_split = g.n_split;
   p.epilogue = g.epilogue; p.rope_D = g.rope_D; p.rope_n_q = g.rope_n_q;
   p.rope_first_frame = g.rope_first_frame; p.rope = g.rope;
+  p.A = g.A; p.a_sm = g.a_sm;
+  p.prefetch_a = (g.batch == 1 && g.a_sm == g.K) ? 1 : 0;
+  // output maps: 32 x 128 boxes, 64B swizzle (the staging layout)
+  CUtensorMap tc, tc2;
+  p.tma_store = tma_storable(g.C, g.c_sm, g.c_batch, g.batch) &&
+                (g.n_split == 0 || tma_storable(g.C2, g.c2_sm, g.c2_batch, g.batch));
+  p.c_swapped = p.c2_swapped = 0;
+  if (p.tma_store) {
+    const int n1 = g.n_split > 0 ? g.n_split : g.N;
+    st = matrix_map(&tc, g.C, n1, g.M, g.batch, g.c_sm, g.c_batch, kEpiCols, kBM, 64, &p.c_swapped);
+    if (st != MLA_OK) return st;
+    if (g.n_split > 0) {
+      st = matrix_map(&tc2, g.C2, g.N - g.n_split, g.M, g.batch, g.c2_sm, g.c2_batch, kEpiCols,
+                      kBM, 64, &p.c2_swapped);
+      if (st != MLA_OK) return st;
+    } else {
+      tc2 = tc;   // never used
+    }
+  } else {
+    tc = ta;      // never used
+    tc2 = ta;
+  }
   MLA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     Cfg::kSmem));
-  dim3 grid(ceil_div(g.N, BN), ceil_div(g.M, kBM), g.batch);
-  gemm_tc_kernel<BN><<<grid, kThreads, Cfg::kSmem, s>>>(ta, tb, p);
+  const long long tiles = static_cast<long long>(p.n_tiles_m) * p.n_tiles_n * g.batch;
+  const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
+  gemm_tc_kernel<BN><<<grid, kThreads, Cfg::kSmem, s>>>(ta, tb, tc, tc2, p);
   MLA_LAUNCH_CHECK("gemm_tc");
   return MLA_OK;
 }
@@ -221,23 +412,26 @@ bool tc_gemm_supported(int M, int N, int K, int64_t a_sm, int64_t b_sn) {
 
 mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s) {
   if (g.M == 0 || g.N == 0) return MLA_OK;
+  if (g.n_split != 0 && (g.n_split % 32 != 0 || g.n_split >= g.N || g.C2 == nullptr))
+    MLA_FAIL(MLA_ERR_INVALID_ARG, "GEMM column split must be a multiple of 32 inside N");
   if (g.epilogue == kEpiRopeQ) {
     if (g.rope_D != 224 || g.N % 224 != 0)
       MLA_FAIL(MLA_ERR_UNSUPPORTED, "query RoPE epilogue needs 224-wide head blocks");
     return launch_gemm<224>(g, s);
   }
-  // Tile width: the one whose CTA count fills whole waves of 148 SMs best (ties to the wider
-  // tile, which re-reads A fewer times).  Projections here have few 128-row tiles, so a narrow
-  // N tile is what puts every SM to work.
-  constexpr int kSms = 148;
-  const int widths[4] = {256, 224, 128, 64};
+  // Tile width: the one whose tiles spread most evenly over the SMs (each persistent CTA takes
+  // ceil(tiles / SMs) tiles) with the least padding in N; ties go to the wider tile, which
+  // re-reads A fewer times.  Projections here have few 128-row tiles, so a narrower N tile is
+  // often what puts every SM to work.
+  const int sms = num_sms();
+  const int widths[5] = {256, 224, 192, 128, 64};
   int best = 256;
   double best_eff = -1.0;
   for (int w : widths) {
-    const long long ctas =
+    const long long tiles =
         static_cast<long long>(ceil_div(g.M, kBM)) * ceil_div(g.N, w) * g.batch;
-    const long long waves = (ctas + kSms - 1) / kSms;
-    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * kSms) *
+    const long long rounds = (tiles + sms - 1) / sms;
+    const double eff = static_cast<double>(tiles) / static_cast<double>(rounds * sms) *
                        (static_cast<double>(g.N) / (ceil_div(g.N, w) * w));
     if (eff > best_eff + 1e-9) {
       best_eff = eff;
@@ -247,6 +441,7 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s) {
   switch (best) {
     case 64: return launch_gemm<64>(g, s);
     case 128: return launch_gemm<128>(g, s);
+    case 192: return launch_gemm<192>(g, s);
     case 224: return launch_gemm<224>(g, s);
     default: return launch_gemm<256>(g, s);
   }

@@ -85,6 +85,11 @@ struct TcGemmArgs {
   // C: [batch][M, N] bf16, row stride c_sm, batch stride c_batch; N contiguous.
   void* C;
   int64_t c_sm, c_batch;
+  // Optional second output: when n_split > 0 (a multiple of 32, < N), columns n >= n_split go
+  // to C2 at column n - n_split (row stride c2_sm, batch stride c2_batch) instead of C.
+  void* C2;
+  int64_t c2_sm, c2_batch;
+  int n_split;
   int M, N, K, batch;
   int epilogue;
   // kEpiRopeQ: rows are chunk tokens of samples of n_q rows; head blocks of width D.

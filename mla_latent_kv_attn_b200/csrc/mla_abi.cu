@@ -105,6 +105,35 @@ mla_status gemm(const Dims& d, const void* A, int64_t a_sm, int64_t a_batch, con
   return gemm_simt(g, d.dtype, s);
 }
 
+// q[m, h, :] = [w_qcat[h, 0:d_c] c_q[m] || RoPE3D(w_qcat[h, d_c:D] c_q[m], pos(m))]
+mla_status query_heads(const Dims& d, const void* c_q, const void* w_qcat, void* q,
+                       int first_frame, cudaStream_t s) {
+  const int M = d.B * d.n_q;
+  const int N = d.H * d.D;
+  if (use_tc(d) && d.D == 224 && d.d_rope == 32 && tc_gemm_supported(M, N, d.d_cq, d.d_cq, d.d_cq)) {
+    TcGemmArgs g{};
+    g.A = c_q; g.a_sm = d.d_cq; g.a_batch = 0;
+    g.B = w_qcat; g.b_sn = d.d_cq; g.b_batch = 0;
+    g.C = q; g.c_sm = N; g.c_batch = 0;
+    g.M = M; g.N = N; g.K = d.d_cq; g.batch = 1;
+    g.epilogue = kEpiRopeQ; g.rope_D = d.D; g.rope_n_q = d.n_q; g.rope_first_frame = first_frame;
+    g.rope = rope_geom(d);
+    return gemm_tc(g, s);
+  }
+  if (d.d_c % 2 == 0) {
+    GemmArgs g{};
+    g.A = c_q; g.a_sm = d.d_cq; g.a_sk = 1; g.a_batch = 0;
+    g.B = w_qcat; g.b_sn = d.d_cq; g.b_sk = 1; g.b_batch = 0;
+    g.C = q; g.c_sm = N; g.c_batch = 0;
+    g.M = M; g.N = N; g.K = d.d_cq; g.batch = 1;
+    g.rope_epi = 1; g.rope_D = d.D; g.rope_dc = d.d_c; g.rope_n_q = d.n_q;
+    g.rope_first_frame = first_frame; g.rope = rope_geom(d);
+    return gemm_simt(g, d.dtype, s);
+  }
+  MLA_TRY(gemm(d, c_q, d.d_cq, 0, w_qcat, d.d_cq, 0, q, N, 0, M, N, d.d_cq, 1, s));
+  return rope3d_inplace(d, q, d.B, d.n_q, N, d.d_c, d.H, d.D, nullptr, 0, first_frame, s);
+}
+
 }  // namespace
 }  // namespace mla
 
@@ -237,29 +266,42 @@ mla_status mla_query_proj(const mla_config* cfg, const void* x, const void* w_dq
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int M = d.B * d.n_q;
   MLA_TRY(gemm(d, x, d.d_model, 0, w_dq, d.d_model, 0, c_q, d.d_cq, 0, M, d.d_cq, d.d_model, 1, s));
-  const int N = d.H * d.D;
-  if (use_tc(d) && d.D == 224 && d.d_rope == 32 && tc_gemm_supported(M, N, d.d_cq, d.d_cq, d.d_cq)) {
+  return query_heads(d, c_q, w_qcat, q, first_frame, s);
+}
+
+mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w_x,
+                             const void* w_qcat, void* c_q, void* q, void* chunk_lat,
+                             int32_t first_frame, void* stream) {
+  set_last_error("");
+  MLA_TRY(check_cfg(cfg));
+  const Dims d = dims_of(*cfg);
+  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_ptr(x, "x"));
+  MLA_TRY(check_ptr(w_x, "w_x"));
+  MLA_TRY(check_ptr(w_qcat, "w_qcat"));
+  MLA_TRY(check_ptr(c_q, "c_q"));
+  MLA_TRY(check_ptr(q, "q"));
+  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int M = d.B * d.n_q;
+  const int N = d.d_cq + d.D;
+  if (use_tc(d) && d.d_cq % 32 == 0 && tc_gemm_supported(M, N, d.d_model, d.d_model, d.d_model)) {
+    // one pass over x: columns 0..d_cq-1 are c_Q, the rest [c_KV || k_R]
     TcGemmArgs g{};
-    g.A = c_q; g.a_sm = d.d_cq; g.a_batch = 0;
-    g.B = w_qcat; g.b_sn = d.d_cq; g.b_batch = 0;
-    g.C = q; g.c_sm = N; g.c_batch = 0;
-    g.M = M; g.N = N; g.K = d.d_cq; g.batch = 1;
-    g.epilogue = kEpiRopeQ; g.rope_D = d.D; g.rope_n_q = d.n_q; g.rope_first_frame = first_frame;
-    g.rope = rope_geom(d);
-    return gemm_tc(g, s);
+    g.A = x; g.a_sm = d.d_model; g.a_batch = 0;
+    g.B = w_x; g.b_sn = d.d_model; g.b_batch = 0;
+    g.C = c_q; g.c_sm = d.d_cq; g.c_batch = 0;
+    g.C2 = chunk_lat; g.c2_sm = d.D; g.c2_batch = 0; g.n_split = d.d_cq;
+    g.M = M; g.N = N; g.K = d.d_model; g.batch = 1;
+    g.epilogue = kEpiStore;
+    MLA_TRY(gemm_tc(g, s));
+  } else {
+    const size_t es = dtype_size(d.dtype);
+    MLA_TRY(gemm(d, x, d.d_model, 0, w_x, d.d_model, 0, c_q, d.d_cq, 0, M, d.d_cq, d.d_model, 1, s));
+    MLA_TRY(gemm(d, x, d.d_model, 0, static_cast<const char*>(w_x) + es * d.d_cq * d.d_model,
+                 d.d_model, 0, chunk_lat, d.D, 0, M, d.D, d.d_model, 1, s));
   }
-  if (d.d_c % 2 == 0) {
-    GemmArgs g{};
-    g.A = c_q; g.a_sm = d.d_cq; g.a_sk = 1; g.a_batch = 0;
-    g.B = w_qcat; g.b_sn = d.d_cq; g.b_sk = 1; g.b_batch = 0;
-    g.C = q; g.c_sm = N; g.c_batch = 0;
-    g.M = M; g.N = N; g.K = d.d_cq; g.batch = 1;
-    g.rope_epi = 1; g.rope_D = d.D; g.rope_dc = d.d_c; g.rope_n_q = d.n_q;
-    g.rope_first_frame = first_frame; g.rope = rope_geom(d);
-    return gemm_simt(g, d.dtype, s);
-  }
-  MLA_TRY(gemm(d, c_q, d.d_cq, 0, w_qcat, d.d_cq, 0, q, N, 0, M, N, d.d_cq, 1, s));
-  return rope3d_inplace(d, q, d.B, d.n_q, N, d.d_c, d.H, d.D, nullptr, 0, first_frame, s);
+  return query_heads(d, c_q, w_qcat, q, first_frame, s);
 }
 
 size_t mla_attention_workspace_bytes(const mla_config* cfg, int32_t n_valid_frames) {

@@ -33,6 +33,7 @@ class DeviceWeights:
 
     w_dkv_kr: torch.Tensor   # [d_c + d_rope, d_model]
     w_dq: torch.Tensor       # [d_cq, d_model]
+    w_x: torch.Tensor        # [d_cq + d_c + d_rope, d_model]: W_down^Q, W_down^KV, W_R^K stacked
     w_qcat: torch.Tensor     # [H, d_c + d_rope, d_cq]  (composed on the device)
     w_uv: torch.Tensor       # [H, d_head, d_c]
     w_o: torch.Tensor        # [d_model, H*d_head]
@@ -47,8 +48,9 @@ def upload_weights(c, lw, device="cuda", stream=None) -> DeviceWeights:
     w_uq, w_uk, w_qr = t(lw.w_uq), t(lw.w_uk), t(lw.w_qr)
     w_qcat = torch.empty((c.n_heads, c.d_c + c.d_rope, c.d_cq), device=device, dtype=dt)
     api.mla_compose_query_weights(c, w_uq, w_uk, w_qr, w_qcat, stream=stream)
-    return DeviceWeights(w_dkv_kr=t(np.concatenate([lw.w_dkv, lw.w_kr], 0)), w_dq=t(lw.w_dq),
-                         w_qcat=w_qcat, w_uv=t(lw.w_uv), w_o=t(lw.w_o))
+    w_x = t(np.concatenate([lw.w_dq, lw.w_dkv, lw.w_kr], 0))
+    return DeviceWeights(w_dkv_kr=w_x[c.d_cq:], w_dq=w_x[:c.d_cq], w_x=w_x, w_qcat=w_qcat,
+                         w_uv=t(lw.w_uv), w_o=t(lw.w_o))
 
 
 class Ring:
@@ -96,9 +98,8 @@ def attend_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
     """Query path, chunk latents and attention of one chunk (buf.x holds its tokens).
     Returns buf.o (fused W_UV) or buf.o_lat (latent output)."""
     first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
-    api.mla_query_proj(c, buf.x, w.w_dq, w.w_qcat, buf.c_q, buf.q, first, stream=stream)
-    api.mla_cache_append(c, buf.x, w.w_dkv_kr, buf.chunk_lat, ring.cache, ring.slot_frame, first,
-                         MLA_PROJECT, stream=stream)
+    api.mla_project_chunk(c, buf.x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first,
+                          stream=stream)
     out = buf.o if fuse_uv else buf.o_lat
     api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid, first,
                           w.w_uv if fuse_uv else None, out, buf.lse, buf.workspace,
@@ -134,3 +135,115 @@ def check_device_status(buf: ChunkBuffers) -> None:
     v = int(buf.dev_status.item())
     if v != 0:
         raise api.MLAError("device", v, "a kernel's bounded wait ran out")
+
+
+class HostStreamer:
+    """Drives chunks whose tokens are in pinned host memory and whose outputs go back to pinned
+    host memory, with the copies overlapped with the device work of neighbouring chunks.
+
+    Two device buffer sets alternate.  Chunk n's tokens travel host -> device on one copy stream
+    while chunk n-1 computes; chunk n's output travels device -> host on a second copy stream
+    while chunk n+1 computes.  CUDA events order every reuse of a buffer:
+      - the copy into buffer set k waits until the chunk that last used set k has finished;
+      - the compute of a chunk waits for its tokens and for the copy-out of the output that
+        used the same buffer set two chunks earlier.
+    Chunks still compute strictly in order on the compute stream, so the ring sees exactly the
+    append order of run_chunk.  Nothing here synchronises the host.
+    """
+
+    def __init__(self, c, w: DeviceWeights, ring: Ring, device="cuda", compute_stream=None):
+        self.c, self.w, self.ring = c, w, ring
+        self.bufs = [ChunkBuffers(c, device=device), ChunkBuffers(c, device=device)]
+        self.compute = compute_stream or torch.cuda.current_stream(device)
+        self.h2d = torch.cuda.Stream(device=device)
+        self.d2h = torch.cuda.Stream(device=device)
+        self.x_free = [None, None]   # event: the compute that last read bufs[k] is done
+        self.o_free = [None, None]   # event: the copy-out of bufs[k].o is done
+        self.n = 0
+
+    def begin(self, event: torch.cuda.Event) -> None:
+        """Makes both copy streams wait for `event` (e.g. the start of a timed region)."""
+        self.h2d.wait_event(event)
+        self.d2h.wait_event(event)
+
+    def submit(self, chunk: int, x_host: torch.Tensor, o_host: torch.Tensor,
+               fuse_uv: bool = True) -> None:
+        """Enqueues chunk `chunk`: copy-in of x_host, attention, append, copy-out into o_host."""
+        k = self.n % 2
+        b = self.bufs[k]
+        with torch.cuda.stream(self.h2d):
+            if self.x_free[k] is not None:
+                self.h2d.wait_event(self.x_free[k])
+            b.x.copy_(x_host, non_blocking=True)
+            x_ready = torch.cuda.Event()
+            x_ready.record(self.h2d)
+        self.compute.wait_event(x_ready)
+        if self.o_free[k] is not None:
+            self.compute.wait_event(self.o_free[k])
+        out = run_chunk(self.c, self.w, self.ring, b, chunk, fuse_uv=fuse_uv, stream=self.compute)
+        done = torch.cuda.Event()
+        done.record(self.compute)
+        self.x_free[k] = done
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(done)
+            o_host.copy_(out, non_blocking=True)
+            o_done = torch.cuda.Event()
+            o_done.record(self.d2h)
+        self.o_free[k] = o_done
+        self.n += 1
+
+    def finish(self) -> None:
+        """Makes the compute stream wait for every copy issued so far."""
+        for e in self.o_free:
+            if e is not None:
+                self.compute.wait_event(e)
+
+    def check_device_status(self) -> None:
+        for b in self.bufs:
+            check_device_status(b)
+
+
+class ChunkGraph:
+    """One chunk's whole path (projections, attention, append) captured as a CUDA graph.
+
+    A chunk's kernels depend on its index only through launch parameters (first frame, valid
+    frames, ring slots), so each chunk index gets its own graph; capturing is host-side work
+    that can run ahead of the device, and a replay launches the chunk's kernels back to back
+    without per-kernel host overhead.  Buffers, ring and weights are bound at capture time and
+    must stay alive and in place while the graph is used.  `events=True` also records a pair of
+    timing events around the attention call inside the graph (attn_start / attn_end).
+    """
+
+    def __init__(self, c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
+                 x: Optional[torch.Tensor] = None, events: bool = False, fuse_uv: bool = True):
+        self.chunk = chunk
+        first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
+        x = buf.x if x is None else x
+        # external events: recorded by the graph at replay time (a plain event recorded during
+        # capture only orders the graph's nodes and cannot be timed)
+        self.attn_start = torch.cuda.Event(enable_timing=True, external=True) if events else None
+        self.attn_end = torch.cuda.Event(enable_timing=True, external=True) if events else None
+        self.graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(self.graph, stream=side, capture_error_mode="relaxed"):
+            api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
+            if events:
+                self.attn_start.record()
+            out = buf.o if fuse_uv else buf.o_lat
+            api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid,
+                                  first, w.w_uv if fuse_uv else None, out, buf.lse, buf.workspace,
+                                  buf.dev_status)
+            if events:
+                self.attn_end.record()
+            api.mla_cache_append(c, None, None, buf.chunk_lat, ring.cache, ring.slot_frame,
+                                 first, MLA_APPEND)
+        torch.cuda.current_stream().wait_stream(side)
+        self.out = out
+
+    def replay(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.out
+
+    def attention_ms(self) -> float:
+        return self.attn_start.elapsed_time(self.attn_end)

@@ -124,6 +124,91 @@ def test_tensor_core_and_cuda_core_paths_agree_on_config1():
         assert np.linalg.norm(err) / np.linalg.norm(b) <= 5e-3, k
 
 
+@pytest.mark.parametrize("cfg_id,path", [("small", "tc"), ("small", "simt"), ("1", "tc")])
+def test_project_chunk_matches_separate_projections(cfg_id, path):
+    """mla_project_chunk (one pass over x, two outputs) gives the results of mla_query_proj and
+    mla_cache_append(MLA_PROJECT), and both match the oracle."""
+    cfg = inputs.small_bf16_config() if cfg_id == "small" else inputs.CONFIGS[int(cfg_id)]
+    g = GpuRun(cfg, PATHS[path])
+    ch = cfg.measured_chunk
+    x = inputs.chunk_x(cfg, ch)
+    g.load_x(x)
+    first = cfg.first_frame(ch)
+    b = g.buf
+    api.mla_project_chunk(g.c, b.x, g.w.w_x, g.w.w_qcat, b.c_q, b.q, b.chunk_lat, first)
+    fused = {k: to_np(getattr(b, k)) for k in ("c_q", "q", "chunk_lat")}
+    for k in fused:
+        getattr(b, k).zero_()
+    api.mla_query_proj(g.c, b.x, g.w.w_dq, g.w.w_qcat, b.c_q, b.q, first)
+    api.mla_cache_append(g.c, b.x, g.w.w_dkv_kr, b.chunk_lat, g.ring.cache, g.ring.slot_frame,
+                         first, api.MLA_PROJECT)
+    sep = {k: to_np(getattr(b, k)) for k in ("c_q", "q", "chunk_lat")}
+    for k in fused:
+        err = np.abs(fused[k] - sep[k])
+        # same operands and fp32 accumulation; at most a last-place difference of a rounding
+        assert err.max() <= 2.0 ** -7 * max(1.0, np.abs(sep[k]).max()), k
+    rows = inputs.sample_rows(cfg.n_q, 96, tag=11)
+    d = oracle.dims_from(cfg)
+    for bi in range(cfg.batch):
+        xb = x[bi][rows]
+        c_kv, k_r = oracle.down_project(xb, g.lw.w_dkv, g.lw.w_kr)
+        c_q = oracle.query_latent(xb, g.lw.w_dq)
+        pos = oracle.token_positions(range(first, first + cfg.chunk_frames), d)[rows]
+        q_ref = oracle.absorbed_query(c_q, g.lw.w_uq, g.lw.w_uk, g.lw.w_qr, pos, d)
+        compare("fused.chunk_lat", fused["chunk_lat"][bi][rows],
+                np.concatenate([c_kv, k_r], axis=1), cfg.dtype)
+        compare("fused.c_q", fused["c_q"][bi][rows], c_q, cfg.dtype)
+        compare("fused.q", fused["q"][bi][rows], q_ref, cfg.dtype)
+
+
+def test_host_streamer_matches_serial_rollout():
+    """rollout.HostStreamer (pinned host tokens in, output out, copies overlapped with the
+    neighbouring chunks' compute) gives bit-identical outputs to run_chunk one chunk at a time."""
+    cfg = inputs.small_bf16_config()
+    xs = [torch.from_numpy(inputs.chunk_x(cfg, ch)).to(torch.bfloat16) for ch in range(cfg.n_chunks)]
+    a = GpuRun(cfg)
+    ref = []
+    for ch in range(cfg.n_chunks):
+        a.buf.x.copy_(xs[ch])
+        ref.append(rollout.run_chunk(a.c, a.w, a.ring, a.buf, ch).cpu().clone())
+    b = GpuRun(cfg)
+    st = rollout.HostStreamer(b.c, b.w, b.ring)
+    outs = [torch.empty_like(r).pin_memory() for r in ref]
+    for ch in range(cfg.n_chunks):
+        st.submit(ch, xs[ch].pin_memory(), outs[ch])
+    st.finish()
+    torch.cuda.synchronize()
+    st.check_device_status()
+    for ch in range(cfg.n_chunks):
+        assert torch.equal(outs[ch], ref[ch]), ch
+    assert torch.equal(a.ring.cache, b.ring.cache)
+    assert torch.equal(a.ring.slot_frame, b.ring.slot_frame)
+
+
+def test_chunk_graph_replay_matches_eager_rollout():
+    """rollout.ChunkGraph (a chunk's projections, attention and append captured as one CUDA
+    graph per chunk index) replays to bit-identical outputs and ring state as the eager calls."""
+    cfg = inputs.small_bf16_config()
+    xs = [torch.from_numpy(inputs.chunk_x(cfg, ch)).to(torch.bfloat16).cuda()
+          for ch in range(cfg.n_chunks)]
+    a = GpuRun(cfg)
+    ref = []
+    for ch in range(cfg.n_chunks):
+        a.buf.x.copy_(xs[ch])
+        ref.append(rollout.run_chunk(a.c, a.w, a.ring, a.buf, ch).clone())
+    b = GpuRun(cfg)
+    graphs = [rollout.ChunkGraph(b.c, b.w, b.ring, b.buf, ch, x=xs[ch], events=True)
+              for ch in range(cfg.n_chunks)]
+    for ch in range(cfg.n_chunks):
+        out = graphs[ch].replay().clone()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref[ch]), ch
+        assert graphs[ch].attention_ms() > 0.0
+    assert torch.equal(a.ring.cache, b.ring.cache)
+    assert torch.equal(a.ring.slot_frame, b.ring.slot_frame)
+    rollout.check_device_status(b.buf)
+
+
 def test_standalone_rope3d_and_out_proj():
     cfg = inputs.small_bf16_config()
     g = GpuRun(cfg, api.MLA_PATH_AUTO)
