@@ -43,6 +43,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MLA attention TFLOP/s & query tokens/s (Wan-1.3B shape), % of B200 BF16 peak"
+REF_BUDGET_S = 90.0     # target wall time of a whole --impl reference run
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -64,7 +65,9 @@ REASON_BITS = {
 
 
 class ClockSampler:
-    """nvidia-smi sampled every 100 ms while the timed region runs."""
+    """nvidia-smi sampled every 10 ms while the timed region runs.  The SM clock reported is the
+    median over the samples taken under load (GPU utilisation >= 50 %), since the B200 lowers its
+    clock under a sustained tensor load (power cap) and idle samples would hide that."""
 
     def __init__(self, index: int):
         self.index = index
@@ -75,8 +78,9 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index),
-                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "utilization.gpu",
+                 "--format=csv,noheader,nounits", "-lms", "10"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -98,25 +102,31 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
+        rows = []
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 4:
+            if len(parts) < 5:
                 continue
             try:
-                s, m = float(parts[0]), float(parts[1])
+                s, m, pw = float(parts[0]), float(parts[1]), float(parts[2])
                 bits = int(parts[3], 16) if parts[3].startswith("0x") else int(parts[3])
+                util = float(parts[4])
             except ValueError:
                 continue
-            sm.append(s)
-            mx.append(m)
-            for bit, name in REASON_BITS.items():
-                if bits & bit and name != "gpu_idle":
-                    reasons.add(name)
-        if not sm:
+            rows.append((s, m, pw, bits, util))
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        loaded = [r for r in rows if r[4] >= 50.0]
+        use = loaded if loaded else rows
+        reasons = set()
+        for r in use:
+            for bit, name in REASON_BITS.items():
+                if r[3] & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in use),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -162,13 +172,18 @@ def blas_threads() -> int:
 
 
 def run_reference(args, cfg):
-    """--impl reference: the CPU oracle as it stands, each step a bounded row sample."""
+    """--impl reference: the CPU oracle as it stands, each step a bounded row sample.  The rows
+    per step are sized from a calibration sample so that the whole --warmup + --steps run takes
+    about REF_BUDGET_S seconds (at most --ref-rows rows, at least 4)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    rows = args.ref_rows
-    times, flops = [], 0.0
     sample = OracleSample(cfg)
+    f, dt, n = sample(16, seed_tag=99)               # calibration (not counted)
+    per_row = dt / max(n, 1)
+    rows = int(REF_BUDGET_S / max(args.warmup + args.steps, 1) / max(per_row, 1e-6))
+    rows = max(4, min(args.ref_rows, rows))
+    times, flops = [], 0.0
     for i in range(args.warmup + args.steps):
         f, dt, n = sample(rows, seed_tag=100 + i)
         if i >= args.warmup:
@@ -408,6 +423,95 @@ def run_ours(args, cfg):
     return 0
 
 
+def run_stack(args, cfg):
+    """Workloads with a stack of layers and several denoising steps per chunk (the 30-layer
+    preset): one step = one whole rollout (every chunk, step and layer), each chunk replayed as
+    one CUDA graph (rollout.LayerStack.capture_chunk: ring keys rotated once per chunk and layer,
+    cached-ring attention, appends after the last step).  value = algorithmic attention flops of
+    the rollout / its device time.  Inputs: a pool of 8 seeded chunk inputs on the device,
+    cycled over (step, layer); the stack's rings and weights (over 700 MB) exceed L2, which is
+    also flushed before every rollout."""
+    import torch
+    import torch.distributed as dist
+    from mla_latent_kv_attn_b200 import api, inputs, rollout
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    steps = args.steps if args.steps_given else 3
+    c = api.make_config(cfg)
+    stack = rollout.LayerStack(c, [rollout.upload_weights(c, inputs.layer_weights(cfg, l), device=dev)
+                                   for l in range(cfg.n_layers)], device=dev)
+    samples = rank_samples(rank, cfg.batch)
+    pool = [torch.from_numpy(inputs.chunk_x(cfg, k, samples=samples)).to(device=dev,
+                                                                          dtype=torch.bfloat16)
+            for k in range(8)]
+    x_of = lambda s, l: pool[(s * cfg.n_layers + l) % len(pool)]
+    graphs = [stack.capture_chunk(ch, cfg.n_steps, x_of) for ch in range(cfg.n_chunks)]
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = sum(cfg.attention_flops(ch) for ch in range(cfg.n_chunks)) * cfg.n_steps * cfg.n_layers
+    calls = cfg.n_chunks * cfg.n_steps * cfg.n_layers
+    for _ in range(args.warmup):
+        flush.zero_()
+        for g in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    with ClockSampler(local) as clk:
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            for g in graphs:
+                g.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), device=dev)
+    rollout.check_device_status(stack.buf)
+    peaks, peak_kind = load_peaks()
+    value = world * flops * steps / (total_ms * 1e-3) / 1e12
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "n_q": cfg.n_q, "layers": cfg.n_layers,
+                   "denoising_steps": cfg.n_steps, "chunks": cfg.n_chunks,
+                   "window_frames": cfg.window_frames, "chunk_frames": cfg.chunk_frames,
+                   "attention_calls_per_step": calls,
+                   "parallelism": f"replicas x{world} (independent samples)",
+                   "l2": "inputs larger than L2 (30 layers' rings and weights), and flushed before "
+                         "every rollout"},
+        "query_tokens_per_s": world * cfg.batch * cfg.n_q * cfg.n_chunks * cfg.n_steps *
+                              cfg.n_layers * steps / (total_ms * 1e-3),
+        "pct_of_bf16_peak": 100.0 * value / peaks["bf16_tflops"],
+        "roofline": {"bound": "tensor", "achieved": value, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": value / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "whole rollout (attention flops / all kernels' time)",
+                     "peak_kind": f"{peak_kind} burst bf16"},
+        "e2e": None,
+        # per call: x-projection GEMM, Q' GEMM, chunk-key rotation, attention; per chunk and
+        # layer: the ring-key rotation (chunks with a non-empty window) and the append
+        "gpu_launches": steps * (calls * 4 + cfg.n_layers * (
+            cfg.n_chunks + sum(1 for ch in range(cfg.n_chunks) if cfg.valid_frames(ch) > 0))),
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def kernel_sha() -> str:
     import hashlib
     h = hashlib.sha256()
@@ -419,7 +523,7 @@ def kernel_sha() -> str:
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", type=int, default=1)
@@ -427,12 +531,17 @@ def main(argv=None):
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
+    args.steps_given = args.steps is not None
+    if args.steps is None:
+        args.steps = 200
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from mla_latent_kv_attn_b200 import inputs
     cfg = inputs.CONFIGS[args.config]
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if cfg.n_layers > 1:
+        return run_stack(args, cfg)
     return run_ours(args, cfg)
 
 

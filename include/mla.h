@@ -263,6 +263,34 @@ mla_status mla_attention_fwd(const mla_config* cfg, const void* q, const void* c
                              int32_t* dev_status, void* stream);
 
 /* --------------------------------------------------------------------------------------------
+ * Frozen-ring attention.  While a chunk is denoised in several steps, every step attends to the
+ * same ring ([I]: the rolling cache only moves on once a chunk is finished), so the rotation of
+ * the ring's positional keys ([M]: k_R is cached unrotated and rotated by 3D-RoPE when attention
+ * runs) gives the same values at every step.  These two calls split mla_attention_fwd so that
+ * rotation is done once per ring state:
+ *
+ * mla_rotate_ring_keys: writes RoPE3D(k_R) of ring slots 0 .. n_valid_frames*tpf - 1 (t from
+ *   slot_frame) into the ring part of an attention workspace (layout of
+ *   mla_attention_workspace_bytes(cfg, n_valid_frames)).  Arguments as in mla_attention_fwd.
+ *   Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.
+ *
+ * mla_attention_fwd_cached_ring: mla_attention_fwd for a workspace whose ring part already holds
+ *   the rotated ring keys written by mla_rotate_ring_keys with the same cache, slot_frame and
+ *   n_valid_frames, none of which may have changed since; only the chunk's own positional keys
+ *   are rotated.  Results are bit-identical to mla_attention_fwd.  Arguments, results and errors
+ *   are those of mla_attention_fwd.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_rotate_ring_keys(const mla_config* cfg, const void* cache,
+                                const int32_t* slot_frame, int32_t n_valid_frames,
+                                void* workspace, size_t workspace_bytes, void* stream);
+mla_status mla_attention_fwd_cached_ring(const mla_config* cfg, const void* q,
+                                         const void* chunk_lat, const void* cache,
+                                         const int32_t* slot_frame, int32_t n_valid_frames,
+                                         int32_t first_frame, const void* w_uv, void* out,
+                                         float* lse, void* workspace, size_t workspace_bytes,
+                                         int32_t* dev_status, void* stream);
+
+/* --------------------------------------------------------------------------------------------
  * mla_attention_fwd_static_scratch: mla_attention_fwd without the workspace arguments, for
  * callers that cannot allocate device memory.  The paper has no counterpart to this call; it
  * exists for deployment.  Some callers have no way to hand the library a scratch buffer: code

@@ -65,6 +65,9 @@ SIGNATURES = {
     "mla_attention_fwd": (c_int32, [_CFG, _P, _P, _P, _P, c_int32, c_int32, _P, _P, _P, _P,
                                     c_size_t, _P, _P]),
     "mla_out_proj": (c_int32, [_CFG, _P, _P, _P, _P, _P, _P]),
+    "mla_rotate_ring_keys": (c_int32, [_CFG, _P, _P, c_int32, _P, c_size_t, _P]),
+    "mla_attention_fwd_cached_ring": (c_int32, [_CFG, _P, _P, _P, _P, c_int32, c_int32, _P, _P,
+                                                _P, _P, c_size_t, _P, _P]),
     "mla_attention_fwd_static_scratch": (c_int32, [_CFG, _P, _P, _P, _P, c_int32, c_int32, _P,
                                                    _P, _P, _P, _P]),
     "mla_selftest_wait_timeout": (c_int32, [_P, c_int32, _P]),

@@ -19,6 +19,7 @@ __all__ = [
     "make_config", "torch_dtype", "mla_config_check", "mla_cache_append", "mla_rope3d",
     "mla_key_positions", "mla_compose_query_weights", "mla_query_proj", "mla_project_chunk",
     "mla_attention_workspace_bytes", "mla_attention_fwd", "mla_attention_fwd_static_scratch",
+    "mla_rotate_ring_keys", "mla_attention_fwd_cached_ring",
     "mla_out_proj", "MLAError",
     "MLA_PROJECT", "MLA_APPEND", "MLA_PROJECT_AND_APPEND", "MLA_PATH_AUTO", "MLA_PATH_SIMT",
 ]
@@ -147,22 +148,50 @@ def mla_attention_workspace_bytes(c: MLAConfigC, n_valid_frames: int) -> int:
     return int(_lib.lib().mla_attention_workspace_bytes(ctypes.byref(c), n_valid_frames))
 
 
-def mla_attention_fwd(c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_frames: int,
-                      first_frame: int, w_uv, out, lse=None, workspace=None, dev_status=None,
-                      stream=None) -> None:
+def _attention(fn_name: str, c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_frames: int,
+               first_frame: int, w_uv, out, lse, workspace, dev_status, stream) -> None:
     tpf, n_q, D = _geom(c)
     dt = torch_dtype(c)
     B, H = c.batch, c.n_heads
     out_shape = (B, n_q, H * c.d_head) if w_uv is not None else (B, n_q, H, c.d_c)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = _lib.lib().mla_attention_fwd(
+    st = getattr(_lib.lib(), fn_name)(
         ctypes.byref(c), _ptr(q, "q", dt, (B, n_q, H, D)), _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)),
         _ptr(cache, "cache", dt, (B, c.window_frames * tpf, D)),
         _ptr(slot_frame, "slot_frame", torch.int32, (B, c.window_frames)), n_valid_frames,
         first_frame, _ptr(w_uv, "w_uv", dt, (H, c.d_head, c.d_c)), _ptr(out, "out", dt, out_shape),
         _ptr(lse, "lse", torch.float32, (B, H, n_q)), _ptr(workspace, "workspace"), ws_bytes,
         _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
-    _lib.check("mla_attention_fwd", st)
+    _lib.check(fn_name, st)
+
+
+def mla_attention_fwd(c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_frames: int,
+                      first_frame: int, w_uv, out, lse=None, workspace=None, dev_status=None,
+                      stream=None) -> None:
+    _attention("mla_attention_fwd", c, q, chunk_lat, cache, slot_frame, n_valid_frames,
+               first_frame, w_uv, out, lse, workspace, dev_status, stream)
+
+
+def mla_attention_fwd_cached_ring(c: MLAConfigC, q, chunk_lat, cache, slot_frame,
+                                  n_valid_frames: int, first_frame: int, w_uv, out, lse=None,
+                                  workspace=None, dev_status=None, stream=None) -> None:
+    """mla_attention_fwd for a workspace whose ring part mla_rotate_ring_keys has filled for the
+    same (unchanged) ring; only the chunk's positional keys are rotated."""
+    _attention("mla_attention_fwd_cached_ring", c, q, chunk_lat, cache, slot_frame,
+               n_valid_frames, first_frame, w_uv, out, lse, workspace, dev_status, stream)
+
+
+def mla_rotate_ring_keys(c: MLAConfigC, cache, slot_frame, n_valid_frames: int, workspace,
+                         stream=None) -> None:
+    tpf, n_q, D = _geom(c)
+    dt = torch_dtype(c)
+    B = c.batch
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib.lib().mla_rotate_ring_keys(
+        ctypes.byref(c), _ptr(cache, "cache", dt, (B, c.window_frames * tpf, D)),
+        _ptr(slot_frame, "slot_frame", torch.int32, (B, c.window_frames)), n_valid_frames,
+        _ptr(workspace, "workspace"), ws_bytes, _stream(stream))
+    _lib.check("mla_rotate_ring_keys", st)
 
 
 def mla_out_proj(c: MLAConfigC, o_lat, w_uv, o, w_o=None, y=None, stream=None) -> None:

@@ -97,6 +97,67 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return r;
 }
 
+// 2^x on the FMA pipe, for a pair of arguments in packed form, so that part of the softmax's
+// exponentials bypass the MUFU unit (which otherwise sets the softmax's pace).  x = n + f with
+// n = rint(x) and f in [-1/2, 1/2]; 2^f by the degree-3 polynomial interpolating 2^f at the four
+// Chebyshev nodes of [-1/2, 1/2] (relative error below 1.0e-4, far under a bf16 half-ulp of P);
+// 2^n is added to the exponent field.  Arguments are clamped to >= -125 (2^-125 is zero for
+// the softmax's purposes and keeps the exponent field of the result positive); the softmax
+// never passes more than +8 (the lazy-rescale bound).
+constexpr float kExp2C0 = 0.9999245405197144f;
+constexpr float kExp2C1 = 0.6931367516517639f;
+constexpr float kExp2C2 = 0.2426394820213318f;
+constexpr float kExp2C3 = 0.05583828315138817f;
+constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23: x + this rounds x to an integer
+
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = f2_pack(kRoundMagic, kRoundMagic);
+  const uint64_t t = f2_add(x, magic);                              // magic + n, exactly
+  const uint64_t neg_n = f2_fma(t, f2_pack(-1.f, -1.f), magic);     // -n
+  const uint64_t f = f2_add(x, neg_n);                              // x - n
+  uint64_t q = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  // the low bits of t hold n (bits(t) = bits(magic) + n); shifted into the exponent field the
+  // bits of magic drop out, leaving n << 23
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Pairs (out of every 8) of a full key tile whose exponentials take the FMA-pipe polynomial.
+constexpr int kPolyPairsPer8 = 2;
+
+// p = 2^(s * scale_log2 - m) for one row of a key tile: packed to bf16 pairs in w, returning
+// the row sum.  kPoly: some pairs use exp2_poly_pair (full tiles; no masked -inf scores).
+template <bool kPoly>
+__device__ __forceinline__ float softmax_exp_row(const float (&s)[kKeyTile], float scale_log2,
+                                                 float m, uint32_t (&w)[kKeyTile / 2]) {
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int i = 0; i < kKeyTile / 2; ++i) {
+    float x0, x1, p0, p1;
+    f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sc2, nm2), x0, x1);
+    if (kPoly && (i & 7) < kPolyPairsPer8) {
+      exp2_poly_pair(x0, x1, p0, p1);
+    } else {
+      p0 = fast_exp2(x0);
+      p1 = fast_exp2(x1);
+    }
+    sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(p0, p1));
+    w[i] = pack_bf16x2(p0, p1);
+  }
+  const uint64_t t2 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
+  float l0, l1;
+  f2_unpack(t2, l0, l1);
+  return l0 + l1;
+}
+
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          int32_t* dev_status) {
   return mbar_wait_or_abort(bar, parity, abort_flag, dev_status);
@@ -329,27 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
         rescale = true;
       }
-      // p = 2^(s * scale * log2(e) - m): one packed FFMA2 per two scores, one ex2 per score,
-      // packed to bf16 pairs; the row sum runs in four packed FADD2 chains.
+      // p = 2^(s * scale * log2(e) - m): one packed FFMA2 per two scores, then ex2 on the MUFU
+      // unit or, for a fixed share of the pairs of full tiles, the FMA-pipe polynomial; packed
+      // to bf16 pairs; the row sum runs in four packed FADD2 chains.
       uint32_t w[kBN / 2];
-      {
-        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(-m_run, -m_run);
-        uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int i = 0; i < kBN / 2; ++i) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sc2, nm2), x0, x1);
-          const float p0 = fast_exp2(x0);
-          const float p1 = fast_exp2(x1);
-          sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(p0, p1));
-          w[i] = pack_bf16x2(p0, p1);
-        }
-        const uint64_t t2 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
-        float l0, l1;
-        f2_unpack(t2, l0, l1);
-        l_run += l0 + l1;
-      }
+      if (valid == kBN) l_run += softmax_exp_row<true>(s, p.scale_log2, m_run, w);
+      else l_run += softmax_exp_row<false>(s, p.scale_log2, m_run, w);
       // The P buffer and O are free once PV(j-1) has completed.
       if (j > 0) {
         ok = __all_sync(0xffffffffu,

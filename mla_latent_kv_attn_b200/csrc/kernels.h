@@ -58,9 +58,12 @@ mla_status ring_append(const Dims& d, const void* chunk_lat, void* cache, int32_
                        int first_frame, cudaStream_t s);
 mla_status key_positions(const Dims& d, const int32_t* slot_frame, int n_valid, int first_frame,
                          int32_t* out, cudaStream_t s);
+// Which rows of the rotated-key workspace build_rope_keys writes: all, the ring part (rows
+// [0, nc_pad)) or the chunk part (rows [nc_pad, rows)).
+enum RopeKeysPart : int { kRopeKeysAll = 0, kRopeKeysRing = 1, kRopeKeysChunk = 2 };
 mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_lat,
                            const int32_t* slot_frame, int n_valid, int first_frame, void* ws,
-                           cudaStream_t s);
+                           cudaStream_t s, int part = kRopeKeysAll);
 mla_status attention_simt(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
 mla_status copy_rows(int dtype, const void* src, int64_t src_stride, void* dst,
                      int64_t dst_stride, int rows, int cols, int64_t src_batch,

@@ -134,6 +134,50 @@ mla_status query_heads(const Dims& d, const void* c_q, const void* w_qcat, void*
   return rope3d_inplace(d, q, d.B, d.n_q, N, d.d_c, d.H, d.D, nullptr, 0, first_frame, s);
 }
 
+mla_status check_workspace(const Dims& d, int n_valid, const void* workspace,
+                           size_t workspace_bytes) {
+  const KeyWorkspace kw = key_workspace_layout(d, n_valid);
+  if (workspace == nullptr || workspace_bytes < kw.bytes)
+    MLA_FAIL(MLA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
+             kw.bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    MLA_FAIL(MLA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  return check_ptr(workspace, "workspace");
+}
+
+// Shared body of the attention entry points: checks, the rotated-key pre-pass (all of it, or
+// only the chunk's keys when the ring's rotated keys are already in the workspace), attention.
+mla_status attention_entry(const mla_config* cfg, const void* q, const void* chunk_lat,
+                           const void* cache, const int32_t* slot_frame, int32_t n_valid_frames,
+                           int32_t first_frame, const void* w_uv, void* out, float* lse,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                           void* stream, int rope_part) {
+  set_last_error("");
+  MLA_TRY(check_cfg(cfg));
+  const Dims d = dims_of(*cfg);
+  MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
+                d.W);
+  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_ptr(q, "q"));
+  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
+  MLA_TRY(check_ptr(slot_frame, "slot_frame"));
+  MLA_TRY(check_ptr(out, "out"));
+  MLA_TRY(check_ptr(cache, "cache", n_valid_frames > 0));
+  MLA_TRY(check_ptr(w_uv, "w_uv", false));
+  MLA_TRY(check_ptr(lse, "lse", false));
+  MLA_TRY(check_ptr(dev_status, "dev_status", false));
+  MLA_TRY(check_workspace(d, n_valid_frames, workspace, workspace_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MLA_TRY(build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid_frames, first_frame, workspace, s,
+                          rope_part));
+  AttnArgs a{};
+  a.q = q; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = workspace; a.w_uv = w_uv;
+  a.out = out; a.lse = lse; a.dev_status = dev_status;
+  if (use_tc(d) && tc_attention_supported(d, w_uv != nullptr))
+    return attention_tc(d, a, n_valid_frames, s);
+  return attention_simt(d, a, n_valid_frames, s);
+}
+
 }  // namespace
 }  // namespace mla
 
@@ -316,35 +360,34 @@ mla_status mla_attention_fwd(const mla_config* cfg, const void* q, const void* c
                              int32_t n_valid_frames, int32_t first_frame, const void* w_uv,
                              void* out, float* lse, void* workspace, size_t workspace_bytes,
                              int32_t* dev_status, void* stream) {
+  return attention_entry(cfg, q, chunk_lat, cache, slot_frame, n_valid_frames, first_frame, w_uv,
+                         out, lse, workspace, workspace_bytes, dev_status, stream, kRopeKeysAll);
+}
+
+mla_status mla_attention_fwd_cached_ring(const mla_config* cfg, const void* q,
+                                         const void* chunk_lat, const void* cache,
+                                         const int32_t* slot_frame, int32_t n_valid_frames,
+                                         int32_t first_frame, const void* w_uv, void* out,
+                                         float* lse, void* workspace, size_t workspace_bytes,
+                                         int32_t* dev_status, void* stream) {
+  return attention_entry(cfg, q, chunk_lat, cache, slot_frame, n_valid_frames, first_frame, w_uv,
+                         out, lse, workspace, workspace_bytes, dev_status, stream,
+                         kRopeKeysChunk);
+}
+
+mla_status mla_rotate_ring_keys(const mla_config* cfg, const void* cache,
+                                const int32_t* slot_frame, int32_t n_valid_frames,
+                                void* workspace, size_t workspace_bytes, void* stream) {
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
   MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
                 d.W);
-  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
-  MLA_TRY(check_ptr(q, "q"));
-  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
   MLA_TRY(check_ptr(slot_frame, "slot_frame"));
-  MLA_TRY(check_ptr(out, "out"));
   MLA_TRY(check_ptr(cache, "cache", n_valid_frames > 0));
-  MLA_TRY(check_ptr(w_uv, "w_uv", false));
-  MLA_TRY(check_ptr(lse, "lse", false));
-  MLA_TRY(check_ptr(dev_status, "dev_status", false));
-  const KeyWorkspace kw = key_workspace_layout(d, n_valid_frames);
-  if (workspace == nullptr || workspace_bytes < kw.bytes)
-    MLA_FAIL(MLA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
-             kw.bytes);
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    MLA_FAIL(MLA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
-  MLA_TRY(check_ptr(workspace, "workspace"));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  MLA_TRY(build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid_frames, first_frame, workspace, s));
-  AttnArgs a{};
-  a.q = q; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = workspace; a.w_uv = w_uv;
-  a.out = out; a.lse = lse; a.dev_status = dev_status;
-  if (use_tc(d) && tc_attention_supported(d, w_uv != nullptr))
-    return attention_tc(d, a, n_valid_frames, s);
-  return attention_simt(d, a, n_valid_frames, s);
+  MLA_TRY(check_workspace(d, n_valid_frames, workspace, workspace_bytes));
+  return build_rope_keys(d, cache, nullptr, slot_frame, n_valid_frames, 0, workspace,
+                         static_cast<cudaStream_t>(stream), kRopeKeysRing);
 }
 
 mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q,

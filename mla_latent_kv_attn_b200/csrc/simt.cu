@@ -259,14 +259,18 @@ template <typename T>
 __global__ void rope_keys_kernel(const T* __restrict__ cache, const T* __restrict__ chunk_lat,
                                  const int32_t* __restrict__ slot_frame, T* __restrict__ ws,
                                  int B, int W, int D, int d_c, int n_pairs, int n_q, int nc,
-                                 int nc_pad, int rows_ws, int first_frame, RopeGeom g) {
-  const int64_t total = static_cast<int64_t>(B) * rows_ws * n_pairs;
+                                 int nc_pad, int rows_ws, int row_begin, int row_end,
+                                 int first_frame, RopeGeom g) {
+  // rows [row_begin, row_end) of every sample's rows_ws workspace rows
+  const int span = row_end - row_begin;
+  const int64_t total = static_cast<int64_t>(B) * span * n_pairs;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int pair = static_cast<int>(e % n_pairs);
-    const int64_t rr = e / n_pairs;
-    const int r = static_cast<int>(rr % rows_ws);
-    const int b = static_cast<int>(rr / rows_ws);
+    const int64_t rs = e / n_pairs;
+    const int r = row_begin + static_cast<int>(rs % span);
+    const int b = static_cast<int>(rs / span);
+    const int64_t rr = static_cast<int64_t>(b) * rows_ws + r;
     T* dst = ws + rr * (2 * n_pairs) + 2 * pair;
     const T* src = nullptr;
     int m = -1;
@@ -304,22 +308,26 @@ KeyWorkspace key_workspace_layout(const Dims& d, int n_valid) {
 
 mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_lat,
                            const int32_t* slot_frame, int n_valid, int first_frame, void* ws,
-                           cudaStream_t s) {
+                           cudaStream_t s, int part) {
   const KeyWorkspace k = key_workspace_layout(d, n_valid);
   const int n_pairs = d.d_rope / 2;
-  const int64_t total = static_cast<int64_t>(d.B) * k.rows * n_pairs;
+  // the ring part is rows [0, nc_pad) (its padding rows included), the chunk part the rest
+  const int row_begin = part == kRopeKeysChunk ? k.nc_pad : 0;
+  const int row_end = part == kRopeKeysRing ? k.nc_pad : k.rows;
+  if (row_end <= row_begin) return MLA_OK;
+  const int64_t total = static_cast<int64_t>(d.B) * (row_end - row_begin) * n_pairs;
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));
   const RopeGeom g = rope_geom(d);
   if (d.dtype == MLA_FP32)
     rope_keys_kernel<float><<<blocks, 256, 0, s>>>(
         static_cast<const float*>(cache), static_cast<const float*>(chunk_lat), slot_frame,
         static_cast<float*>(ws), d.B, d.W, d.D, d.d_c, n_pairs, d.n_q, k.nc, k.nc_pad, k.rows,
-        first_frame, g);
+        row_begin, row_end, first_frame, g);
   else
     rope_keys_kernel<bf16><<<blocks, 256, 0, s>>>(
         static_cast<const bf16*>(cache), static_cast<const bf16*>(chunk_lat), slot_frame,
         static_cast<bf16*>(ws), d.B, d.W, d.D, d.d_c, n_pairs, d.n_q, k.nc, k.nc_pad, k.rows,
-        first_frame, g);
+        row_begin, row_end, first_frame, g);
   MLA_LAUNCH_CHECK("rope_keys");
   return MLA_OK;
 }

@@ -247,3 +247,75 @@ class ChunkGraph:
 
     def attention_ms(self) -> float:
         return self.attn_start.elapsed_time(self.attn_end)
+
+
+class LayerStack:
+    """A stack of attention layers, each with its own weights and ring, driven through a chunked
+    rollout with several denoising steps per chunk.
+
+    Every step of a chunk runs every layer's attention against that layer's ring, which stays
+    frozen until the chunk is finished (hyper.ai summary of VideoMLA, "Introduction": the cache
+    rolls forward chunk by chunk).  So the positional keys of each ring are rotated once per
+    chunk (mla_rotate_ring_keys into the layer's own workspace) and every step's attention only
+    rotates the chunk's keys (mla_attention_fwd_cached_ring).  At the last step each layer
+    appends the chunk's latents to its ring right after its attention.
+
+    One set of chunk activations (buf) is shared by all layers: a call's outputs are valid until
+    the next call.  capture_chunk() records a whole chunk (rotations, every step and layer,
+    appends) as one CUDA graph, with the step/layer inputs bound at capture time.
+    """
+
+    def __init__(self, c, weights, device="cuda", fuse_uv: bool = True):
+        self.c = c
+        self.w = list(weights)
+        self.rings = [Ring(c, device=device) for _ in self.w]
+        ws = max(api.mla_attention_workspace_bytes(c, c.window_frames), 256)
+        self.ws = [torch.empty((ws,), device=device, dtype=torch.uint8) for _ in self.w]
+        self.buf = ChunkBuffers(c, device=device)
+        self.fuse_uv = fuse_uv
+
+    @property
+    def n_layers(self) -> int:
+        return len(self.w)
+
+    def begin_chunk(self, chunk: int, stream=None) -> None:
+        """Rotates every layer's ring keys for this chunk's (frozen) ring state."""
+        _, n_valid = chunk_schedule(self.c.chunk_frames, self.c.window_frames, chunk)
+        for l in range(self.n_layers):
+            api.mla_rotate_ring_keys(self.c, self.rings[l].cache, self.rings[l].slot_frame,
+                                     n_valid, self.ws[l], stream=stream)
+
+    def attend(self, chunk: int, layer: int, x: torch.Tensor, append: bool = False,
+               stream=None) -> torch.Tensor:
+        """One layer's projections and attention for one step of the chunk (x: [B, n_q, d_model]
+        on the device); with append=True (the chunk's last step) the layer's ring takes the
+        chunk's latents afterwards.  Returns buf.o (or buf.o_lat without the W_UV epilogue)."""
+        c, b, w, ring = self.c, self.buf, self.w[layer], self.rings[layer]
+        first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
+        api.mla_project_chunk(c, x, w.w_x, w.w_qcat, b.c_q, b.q, b.chunk_lat, first, stream=stream)
+        out = b.o if self.fuse_uv else b.o_lat
+        api.mla_attention_fwd_cached_ring(c, b.q, b.chunk_lat, ring.cache, ring.slot_frame, n_valid,
+                                          first, w.w_uv if self.fuse_uv else None, out, b.lse,
+                                          self.ws[layer], b.dev_status, stream=stream)
+        if append:
+            api.mla_cache_append(c, None, None, b.chunk_lat, ring.cache, ring.slot_frame, first,
+                                 MLA_APPEND, stream=stream)
+        return out
+
+    def run_chunk(self, chunk: int, n_steps: int, x_of, stream=None) -> None:
+        """A whole chunk: n_steps steps through every layer; x_of(step, layer) gives the device
+        input of each call."""
+        self.begin_chunk(chunk, stream=stream)
+        for s in range(n_steps):
+            for l in range(self.n_layers):
+                self.attend(chunk, l, x_of(s, l), append=(s == n_steps - 1), stream=stream)
+
+    def capture_chunk(self, chunk: int, n_steps: int, x_of) -> torch.cuda.CUDAGraph:
+        """run_chunk recorded as one CUDA graph (inputs x_of(step, layer) bound at capture)."""
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+            self.run_chunk(chunk, n_steps, x_of)
+        torch.cuda.current_stream().wait_stream(side)
+        return g

@@ -209,6 +209,58 @@ def test_chunk_graph_replay_matches_eager_rollout():
     rollout.check_device_status(b.buf)
 
 
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_cached_ring_attention_is_bit_identical(path):
+    """mla_rotate_ring_keys once, then mla_attention_fwd_cached_ring, gives exactly the outputs
+    and lse of mla_attention_fwd, on a ring that has wrapped."""
+    cfg = inputs.small_bf16_config()
+    g = GpuRun(cfg, PATHS[path])
+    for ch in range(3):
+        g.prefill(ch, inputs.chunk_x(cfg, ch))
+    ch = 3
+    first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, ch)
+    g.load_x(inputs.chunk_x(cfg, ch))
+    b = g.buf
+    api.mla_project_chunk(g.c, b.x, g.w.w_x, g.w.w_qcat, b.c_q, b.q, b.chunk_lat, first)
+    api.mla_attention_fwd(g.c, b.q, b.chunk_lat, g.ring.cache, g.ring.slot_frame, n_valid, first,
+                          g.w.w_uv, b.o, b.lse, b.workspace, b.dev_status)
+    o_ref, lse_ref = b.o.clone(), b.lse.clone()
+    ws = torch.full_like(b.workspace, 0x5A)          # contents on entry must not matter
+    api.mla_rotate_ring_keys(g.c, g.ring.cache, g.ring.slot_frame, n_valid, ws)
+    for _ in range(2):                               # two steps against the same frozen ring
+        b.o.zero_()
+        api.mla_attention_fwd_cached_ring(g.c, b.q, b.chunk_lat, g.ring.cache, g.ring.slot_frame,
+                                          n_valid, first, g.w.w_uv, b.o, b.lse, ws, b.dev_status)
+        torch.cuda.synchronize()
+        assert torch.equal(b.o, o_ref)
+        assert torch.equal(b.lse, lse_ref)
+    rollout.check_device_status(b)
+
+
+def test_layer_stack_graph_matches_eager():
+    """A 3-layer, 2-step stack over 4 chunks (rings wrap): each chunk captured as one CUDA graph
+    replays to the eager run's rings and last outputs exactly."""
+    cfg = inputs.small_bf16_config()
+    c = api.make_config(cfg)
+    n_layers, n_steps = 3, 2
+    lws = [inputs.layer_weights(cfg, l) for l in range(n_layers)]
+    xs = {(ch, s, l): torch.from_numpy(inputs.chunk_x(cfg, ch, s, l)).to(torch.bfloat16).cuda()
+          for ch in range(cfg.n_chunks) for s in range(n_steps) for l in range(n_layers)}
+    eager = rollout.LayerStack(c, [rollout.upload_weights(c, lw) for lw in lws])
+    graphed = rollout.LayerStack(c, [rollout.upload_weights(c, lw) for lw in lws])
+    for ch in range(cfg.n_chunks):
+        x_of = lambda s, l, ch=ch: xs[(ch, s, l)]
+        eager.run_chunk(ch, n_steps, x_of)
+        o_eager = eager.buf.o.clone()
+        graphed.capture_chunk(ch, n_steps, x_of).replay()
+        torch.cuda.synchronize()
+        assert torch.equal(graphed.buf.o, o_eager), ch
+        for l in range(n_layers):
+            assert torch.equal(graphed.rings[l].cache, eager.rings[l].cache), (ch, l)
+            assert torch.equal(graphed.rings[l].slot_frame, eager.rings[l].slot_frame), (ch, l)
+    rollout.check_device_status(graphed.buf)
+
+
 def test_standalone_rope3d_and_out_proj():
     cfg = inputs.small_bf16_config()
     g = GpuRun(cfg, api.MLA_PATH_AUTO)
@@ -289,7 +341,8 @@ def test_bad_arguments_on_device():
 def test_wan_config4_thirty_layer_stack():
     """Config 4: 30 layers, each with its own weights and ring, batch 2, window 12 frames; every
     chunk runs 4 denoising steps through all 30 layers against the frozen rings, then each layer
-    appends its last step's latents.  All 1200 attention calls run on the GPU.  The oracle checks
+    appends its last step's latents.  All 1200 attention calls run on the GPU through
+    rollout.LayerStack (ring keys rotated once per chunk and layer, cached-ring attention).  The oracle checks
     sampled rows of layer 29 at the last chunk (steps 0 and 3, ring wrapped, 23,400 keys) and of
     layer 0 at chunks 0 and 1, plus both layers' ring slots."""
     import os
@@ -300,9 +353,9 @@ def test_wan_config4_thirty_layer_stack():
     cfg = inputs.CONFIGS[4]
     c = api.make_config(cfg)
     layers = [inputs.layer_weights(cfg, l) for l in range(cfg.n_layers)]
-    dev_w = [rollout.upload_weights(c, lw) for lw in layers]
-    rings = [rollout.Ring(c) for _ in range(cfg.n_layers)]
-    buf = rollout.ChunkBuffers(c)
+    stack = rollout.LayerStack(c, [rollout.upload_weights(c, lw) for lw in layers])
+    buf = stack.buf
+    rings = stack.rings
     last = cfg.n_steps - 1
     checks = {(cfg.n_chunks - 1, 0, 29), (cfg.n_chunks - 1, last, 29), (0, 0, 0), (0, last, 0),
               (1, last, 0)}
@@ -322,12 +375,12 @@ def test_wan_config4_thirty_layer_stack():
         x = futs.pop(key).result()
         if key in checks or (l in history and s == last and ch in history[l]):
             kept[key] = x
+        if s == 0 and l == 0:
+            stack.begin_chunk(ch)       # each layer's ring keys rotated once per chunk
         buf.x.copy_(torch.from_numpy(x).to(torch.bfloat16))
-        rollout.attend_chunk(c, dev_w[l], rings[l], buf, ch, fuse_uv=True)
+        stack.attend(ch, l, buf.x, append=(s == last))
         if key in checks:
             gpu_out[key] = (to_np(buf.o)[:, rows], to_np(buf.lse)[:, :, rows])
-        if s == last:
-            rollout.append_chunk(c, rings[l], buf, ch)
     pool.shutdown()
     torch.cuda.synchronize()
     rollout.check_device_status(buf)
