@@ -390,6 +390,7 @@ def run_ours(args, cfg):
         "config": {"workload": cfg.name, "batch": cfg.batch, "n_q": cfg.n_q,
                    "window_frames": cfg.window_frames, "chunk_frames": cfg.chunk_frames,
                    "keys_per_query": cfg.keys_per_query(first_chunk), "heads": cfg.n_heads,
+                   "d_c": cfg.d_c, "d_rope": cfg.d_rope,
                    "parallelism": f"replicas x{world} (independent samples)",
                    "l2": "flushed before every step (256 MiB memset outside the event intervals)"},
         "query_tokens_per_s": tok_s,
@@ -530,6 +531,10 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=192)
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--d-c", type=int, default=None,
+                    help="content-latent width (latent-size ablation shapes; default: the preset's)")
+    ap.add_argument("--d-rope", type=int, default=None,
+                    help="positional-key width (16, 32 or 64; default: the preset's)")
     args = ap.parse_args(argv)
     args.steps_given = args.steps is not None
     if args.steps is None:
@@ -538,6 +543,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     from mla_latent_kv_attn_b200 import inputs
     cfg = inputs.CONFIGS[args.config]
+    if args.d_c is not None or args.d_rope is not None:
+        cfg = inputs.with_latent_shape(cfg, args.d_c or cfg.d_c, args.d_rope or cfg.d_rope)
     if args.impl == "reference":
         return run_reference(args, cfg)
     if cfg.n_layers > 1:

@@ -218,6 +218,13 @@ mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w
                              const void* w_qcat, void* c_q, void* q, void* chunk_lat,
                              int32_t first_frame, void* stream);
 
+/* mla_attention_uses_tensor_cores: 1 if mla_attention_fwd with this configuration (and with the
+ * W_UV epilogue when with_w_uv != 0) runs the tcgen05 tensor-core kernel, 0 if it runs the
+ * CUDA-core kernel, -1 for an invalid configuration.  The tensor-core kernel covers bf16 with
+ * d_c in {128, 192, 256} and d_rope in {16, 32, 64} (and d_head = 128 with W_UV) unless
+ * kernel_path forces the CUDA-core path.  Host-only; launches nothing. */
+int32_t mla_attention_uses_tensor_cores(const mla_config* cfg, int32_t with_w_uv);
+
 /* --------------------------------------------------------------------------------------------
  * mla_attention_workspace_bytes: device scratch mla_attention_fwd needs for a call with the
  * given number of valid ring frames (rotated positional keys of every attended key, tile-padded).

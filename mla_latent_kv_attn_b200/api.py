@@ -19,7 +19,7 @@ __all__ = [
     "make_config", "torch_dtype", "mla_config_check", "mla_cache_append", "mla_rope3d",
     "mla_key_positions", "mla_compose_query_weights", "mla_query_proj", "mla_project_chunk",
     "mla_attention_workspace_bytes", "mla_attention_fwd", "mla_attention_fwd_static_scratch",
-    "mla_rotate_ring_keys", "mla_attention_fwd_cached_ring",
+    "mla_rotate_ring_keys", "mla_attention_fwd_cached_ring", "mla_attention_uses_tensor_cores",
     "mla_out_proj", "MLAError",
     "MLA_PROJECT", "MLA_APPEND", "MLA_PROJECT_AND_APPEND", "MLA_PATH_AUTO", "MLA_PATH_SIMT",
 ]
@@ -142,6 +142,13 @@ def mla_project_chunk(c: MLAConfigC, x, w_x, w_qcat, c_q, q, chunk_lat, first_fr
         _ptr(c_q, "c_q", dt, (B, n_q, c.d_cq)), _ptr(q, "q", dt, (B, n_q, H, D)),
         _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)), first_frame, _stream(stream))
     _lib.check("mla_project_chunk", st)
+
+
+def mla_attention_uses_tensor_cores(c: MLAConfigC, with_w_uv: bool = True) -> bool:
+    r = int(_lib.lib().mla_attention_uses_tensor_cores(ctypes.byref(c), 1 if with_w_uv else 0))
+    if r < 0:
+        raise MLAError("mla_attention_uses_tensor_cores", _lib.MLA_ERR_INVALID_ARG, _lib.last_error())
+    return bool(r)
 
 
 def mla_attention_workspace_bytes(c: MLAConfigC, n_valid_frames: int) -> int:

@@ -3,7 +3,9 @@
 // adds q_nope.k_nope and q_rope.k_rope; keys/values are rebuilt from c_KV only when needed).
 //
 // In absorbed form every head is a query against the same keys K'_m = [c_m || RoPE(k_R,m)]
-// (224 wide) and the same values c_m (192 wide, the first 192 columns of K'): 12-head MQA.
+// (D = DC + DR wide) and the same values c_m (DC wide, the first DC columns of K'): MQA.
+// The kernel is a template over the latent shape: DC in {128, 192, 256}, DR in {16, 32, 64}
+// (the Wan preset is DC 192, DR 32: D 224); the figures below are for that shape.
 //
 // One CTA = one 128-row query tile of one head of one sample.  Roles (224 threads):
 //   warps 0-3  softmax: one TMEM lane (= query row) per thread; online softmax in the log2
@@ -19,9 +21,11 @@
 //                O    += P_j V_j           M=128, N=192, K=128; P from TMEM, V = content
 //                                          blocks of the same stage read MN-major
 //                o     = O_lat W_UV_h^T    M=128, N=128, K=192 (epilogue, O_lat bf16 in smem)
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,448), P [448,512); the epilogue result
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+DC), P [256+DC,+64); the epilogue result
 // reuses S0.  P has its own buffer so that a QK may overwrite an S buffer as soon as the
-// softmax has loaded it, instead of after the PV that reads its P.
+// softmax has loaded it, instead of after the PV that reads its P.  With DC = 256 O fills the
+// rest of TMEM: P(j) is then written into S buffer j&1 and QK(j+2) waits for PV(j).
+// Stages of the K' ring: as many as shared memory holds, up to 4 (3 from D = 224 up).
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -33,11 +37,7 @@ using namespace sm100;
 
 constexpr int kBM = 128;           // query rows per CTA
 constexpr int kBN = kKeyTile;      // keys per tile
-constexpr int kDc = 192;           // content latent width
-constexpr int kDr = 32;            // positional key width
-constexpr int kD = kDc + kDr;      // 224
 constexpr int kDh = 128;           // head width of the W_UV epilogue
-constexpr int kStages = 3;
 constexpr int kSoftmaxThreads = 128;   // warps 0-3: one TMEM lane (query row) per thread
 constexpr int kProducerWarp = 4;
 constexpr int kQkWarp = 5;              // also allocates and frees TMEM
@@ -46,14 +46,37 @@ constexpr int kThreads = 224;
 
 constexpr int kQBlk = kBM * 128;                 // 128 rows x 128 B: 16 KB (Q, O_lat, W_UV)
 constexpr int kKBlk = kBN * 128;                 // 128 rows x 128 B: 16 KB (K' content)
-constexpr int kQTile = 3 * kQBlk + kBM * kDr * 2;   // 56 KB
-constexpr int kKTile = 3 * kKBlk + kBN * kDr * 2;   // 56 KB: one K' stage
-constexpr int kSmem = kQTile + kStages * kKTile + 1024;
-static_assert(kKTile >= 3 * kQBlk, "the W_UV tile is loaded into one K' stage");
+constexpr int kSmemMax = 227 * 1024;             // dynamic shared memory a CTA may use
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 128;    // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 256;
-constexpr uint32_t kColP = 448;    // kBN / 2 columns of packed bf16 P
+constexpr uint32_t kColO = 256;    // O: DC columns from here
+
+// Layout of one latent shape: content width DC (a multiple of 64: DC/64 blocks of 128 rows x
+// 128 B, 128-byte swizzle) and positional width DR (16, 32 or 64: one block of DR*2 bytes per
+// row with the swizzle of that width).  The Q tile and every K' stage have this layout.
+template <int DC_, int DR_>
+struct AttnShape {
+  static constexpr int DC = DC_, DR = DR_, D = DC + DR;
+  static_assert(DC % 64 == 0 && DC >= 64 && DC <= 256, "DC must be 64, 128, 192 or 256");
+  static_assert(DR == 16 || DR == 32 || DR == 64, "DR must be 16, 32 or 64");
+  static constexpr int kCBlk = DC / 64;
+  static constexpr int kRopeBytes = DR * 2;                // bytes per row of the rope block
+  static constexpr uint32_t kRopeSwz = DR == 16 ? kSwizzle32B : DR == 32 ? kSwizzle64B
+                                                                         : kSwizzle128B;
+  static constexpr int kRopeSbo = 8 * kRopeBytes;          // one swizzle atom: 8 rows
+  static constexpr int kRopeKSteps = DR / 16;
+  static constexpr int kQTile = kCBlk * kQBlk + kBM * kRopeBytes;
+  static constexpr int kKTile = kCBlk * kKBlk + kBN * kRopeBytes;
+  static constexpr int kFit = (kSmemMax - 1024 - kQTile) / kKTile;
+  static constexpr int kStages = kFit < 4 ? kFit : (D >= 224 ? 3 : 4);
+  static_assert(kStages >= 1, "the Q tile and one K' stage must fit in shared memory");
+  static constexpr int kSmem = kQTile + kStages * kKTile + 1024;
+  static_assert(kKTile >= kCBlk * kQBlk, "the W_UV tile is loaded into one K' stage");
+  // P (kBN/2 columns of packed bf16) gets its own TMEM columns after O when they fit; with a
+  // 256-wide O it is written into the S buffer it came from instead.
+  static constexpr bool kAliasP = kColO + DC + kBN / 2 > kTmemCols;
+  static constexpr uint32_t kColP = kAliasP ? 0u : kColO + DC;
+};
 
 struct AttnParams {
   int n_q, H, nc, nc_pad, nt_ring, nt;
@@ -163,12 +186,21 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   return mbar_wait_or_abort(bar, parity, abort_flag, dev_status);
 }
 
+template <int DC, int DR>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                         const __grid_constant__ CUtensorMap tm_cache,
                         const __grid_constant__ CUtensorMap tm_chunk,
                         const __grid_constant__ CUtensorMap tm_ws,
                         const __grid_constant__ CUtensorMap tm_wuv, AttnParams p) {
+  using Sh = AttnShape<DC, DR>;
+  constexpr int kDc = DC;
+  constexpr int kCBlk = Sh::kCBlk;
+  constexpr int kStages = Sh::kStages;
+  constexpr int kQTile = Sh::kQTile;
+  constexpr int kKTile = Sh::kKTile;
+  constexpr bool kAliasP = Sh::kAliasP;
+  constexpr uint32_t kColP = Sh::kColP;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full;
   __shared__ __align__(8) uint64_t kv_full[kStages];
@@ -177,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t s_free[2];
   __shared__ __align__(8) uint64_t p_full;
   __shared__ __align__(8) uint64_t pv_done;
+  __shared__ __align__(8) uint64_t pv_buf_done[2];   // PV(j) done, per S buffer (aliased P)
   __shared__ __align__(8) uint64_t w_full;
   __shared__ __align__(8) uint64_t olat_full;
   __shared__ __align__(8) uint64_t epi_done;
@@ -203,6 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&p_full), kSoftmaxThreads);
     mbar_init(smem_u32(&pv_done), 1);
+    mbar_init(smem_u32(&pv_buf_done[0]), 1);
+    mbar_init(smem_u32(&pv_buf_done[1]), 1);
     mbar_init(smem_u32(&w_full), 1);
     mbar_init(smem_u32(&olat_full), kSoftmaxThreads);
     mbar_init(smem_u32(&epi_done), 1);
@@ -226,8 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_ws);
       const uint32_t qb = smem_u32(&q_full);
       mbar_arrive_expect_tx(qb, kQTile);
-      for (int i = 0; i < 3; ++i) tma_load_4d(sQ + i * kQBlk, &tm_q, qb, 64 * i, h, q0, b);
-      tma_load_4d(sQ + 3 * kQBlk, &tm_qr, qb, kDc, h, q0, b);
+      for (int i = 0; i < kCBlk; ++i) tma_load_4d(sQ + i * kQBlk, &tm_q, qb, 64 * i, h, q0, b);
+      tma_load_4d(sQ + kCBlk * kQBlk, &tm_qr, qb, kDc, h, q0, b);
       bool ok = true;
       for (int j = 0; j < p.nt && ok; ++j) {
         const int s = j % kStages;
@@ -238,21 +273,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(fb, kKTile);
         if (j < p.nt_ring) {
           const int r0 = j * kBN;
-          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kKBlk, &tm_cache, fb, 64 * i, r0, b);
-          tma_load_3d(dst + 3 * kKBlk, &tm_ws, fb, 0, r0, b);
+          for (int i = 0; i < kCBlk; ++i) tma_load_3d(dst + i * kKBlk, &tm_cache, fb, 64 * i, r0, b);
+          tma_load_3d(dst + kCBlk * kKBlk, &tm_ws, fb, 0, r0, b);
         } else {
           const int r0 = (j - p.nt_ring) * kBN;
-          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kKBlk, &tm_chunk, fb, 64 * i, r0, b);
-          tma_load_3d(dst + 3 * kKBlk, &tm_ws, fb, 0, p.nc_pad + r0, b);
+          for (int i = 0; i < kCBlk; ++i) tma_load_3d(dst + i * kKBlk, &tm_chunk, fb, 64 * i, r0, b);
+          tma_load_3d(dst + kCBlk * kKBlk, &tm_ws, fb, 0, p.nc_pad + r0, b);
         }
       }
       if (ok && p.has_w_uv) {
-        // W_UV_h [128 x 192] (48 KB) goes into the stage a tile nt would use, once it is free.
+        // W_UV_h [128 x DC] goes into the stage a tile nt would use, once it is free.
         const int s = p.nt % kStages;
         if (wait_bar(smem_u32(&kv_empty[s]), ((p.nt / kStages) & 1) ^ 1, abort_flag, p.dev_status)) {
           const uint32_t wb = smem_u32(&w_full);
-          mbar_arrive_expect_tx(wb, 3 * kQBlk);
-          for (int i = 0; i < 3; ++i)
+          mbar_arrive_expect_tx(wb, kCBlk * kQBlk);
+          for (int i = 0; i < kCBlk; ++i)
             tma_load_2d(sbase + kQTile + s * kKTile + i * kQBlk, &tm_wuv, wb, 64 * i, h * kDh);
         }
       }
@@ -273,9 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // address stays below 256 KB, so the add never carries out of the field).
       constexpr uint32_t kQBlkD = kQBlk >> 4, kKBlkD = kKBlk >> 4, kKTileD = kKTile >> 4;
       const uint64_t q_c = smem_desc(sQ, 16, 1024, kSwizzle128B);
-      const uint64_t q_r = smem_desc(sQ + 3 * kQBlk, 16, 512, kSwizzle64B);
+      const uint64_t q_r = smem_desc(sQ + kCBlk * kQBlk, 16, Sh::kRopeSbo, Sh::kRopeSwz);
       const uint64_t k_c0 = smem_desc(sbase + kQTile, 16, 1024, kSwizzle128B);
-      const uint64_t k_r0 = smem_desc(sbase + kQTile + 3 * kKBlk, 16, 512, kSwizzle64B);
+      const uint64_t k_r0 = smem_desc(sbase + kQTile + kCBlk * kKBlk, 16, Sh::kRopeSbo, Sh::kRopeSwz);
       const uint64_t v_0 = smem_desc(sbase + kQTile, kKBlk, 1024, kSwizzle128B);
       bool ok = true;
       if (warp == kQkWarp) {
@@ -283,21 +318,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < p.nt && ok; ++j) {
           const int s = j % kStages;
           ok = wait_bar(smem_u32(&kv_full[s]), (j / kStages) & 1, abort_flag, p.dev_status);
-          if (ok && j >= 2)   // the softmax has loaded S(j-2) out of the buffer this QK overwrites
-            ok = wait_bar(smem_u32(&s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.dev_status);
+          if (ok && j >= 2) {
+            if constexpr (kAliasP)   // PV(j-2) has read P(j-2) out of the buffer this QK overwrites
+              ok = wait_bar(smem_u32(&pv_buf_done[j & 1]), ((j - 2) >> 1) & 1, abort_flag,
+                            p.dev_status);
+            else                     // the softmax has loaded S(j-2) out of that buffer
+              ok = wait_bar(smem_u32(&s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.dev_status);
+          }
           if (!ok) break;
           tc_fence_after();
           const uint64_t kc = k_c0 + static_cast<uint32_t>(s) * kKTileD;
           const uint64_t kr = k_r0 + static_cast<uint32_t>(s) * kKTileD;
           const uint32_t d = tmem + (j & 1) * kColS;
 #pragma unroll
-          for (int blk = 0; blk < 3; ++blk)
+          for (int blk = 0; blk < kCBlk; ++blk)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_ss(d, q_c + (blk * kQBlkD + 2 * kk), kc + (blk * kKBlkD + 2 * kk), idesc_qk,
                      (blk | kk) != 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk) mma_ss(d, q_r + 2 * kk, kr + 2 * kk, idesc_qk, 1u);
+          for (int kk = 0; kk < Sh::kRopeKSteps; ++kk)
+            mma_ss(d, q_r + 2 * kk, kr + 2 * kk, idesc_qk, 1u);
           mma_commit(smem_u32(&s_full[j & 1]));
         }
       } else {
@@ -307,13 +348,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const int s = j % kStages;
           const uint64_t vd = v_0 + static_cast<uint32_t>(s) * kKTileD;
-          const uint32_t pa = tmem + kColP;
+          const uint32_t pa = tmem + (kAliasP ? (j & 1) * kColS : kColP);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
             // V rows kk*16 .. +15: 16 rows of 128 B further per step (2048 B = 128 units)
             mma_ts(tmem + kColO, pa + kk * 8, vd + 128 * kk, idesc_pv, (j | kk) != 0 ? 1u : 0u);
           mma_commit(smem_u32(&kv_empty[s]));
           mma_commit(smem_u32(&pv_done));
+          if constexpr (kAliasP) mma_commit(smem_u32(&pv_buf_done[j & 1]));
         }
         if (ok && p.has_w_uv) {
           ok = wait_bar(smem_u32(&w_full), 0, abort_flag, p.dev_status) &&
@@ -323,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t w_c = smem_desc(sbase + kQTile + (p.nt % kStages) * kKTile, 16, 1024,
                                            kSwizzle128B);
 #pragma unroll
-            for (int blk = 0; blk < 3; ++blk)
+            for (int blk = 0; blk < kCBlk; ++blk)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_ss(tmem, q_c + (blk * kQBlkD + 2 * kk), w_c + (blk * kQBlkD + 2 * kk), idesc_uv,
@@ -352,9 +394,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
       }
-      // S(j) is in registers: its TMEM buffer may take QK(j+2) now.
-      tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[j & 1]));
+      // S(j) is in registers: its TMEM buffer may take QK(j+2) now (with P in its own buffer;
+      // an aliased P keeps the buffer until PV(j) has read it).
+      if constexpr (!kAliasP) {
+        tc_fence_before();
+        mbar_arrive(smem_u32(&s_free[j & 1]));
+      }
       const int valid = j < p.nt_ring ? min(kBN, p.nc - j * kBN)
                                       : min(kBN, p.n_q - (j - p.nt_ring) * kBN);
       if (valid < kBN) {                    // only the last tile of the ring or of the chunk
@@ -396,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t w[kBN / 2];
       if (valid == kBN) l_run += softmax_exp_row<true>(s, p.scale_log2, m_run, w);
       else l_run += softmax_exp_row<false>(s, p.scale_log2, m_run, w);
-      // The P buffer and O are free once PV(j-1) has completed.
-      if (j > 0) {
+      // The P buffer and O are free once PV(j-1) has completed (an aliased P needs only O).
+      if (j > 0 && (!kAliasP || rescale)) {
         ok = __all_sync(0xffffffffu,
                         wait_bar(smem_u32(&pv_done), (j - 1) & 1, abort_flag, p.dev_status));
         if (!ok) break;
@@ -418,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t w16[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) w16[i] = w[c + i];
-        tmem_st16(tmem + lane_off + kColP + c, w16);
+        tmem_st16(tmem + lane_off + (kAliasP ? (j & 1) * kColS : kColP) + c, w16);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -504,13 +549,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-}  // namespace
-
-bool tc_attention_supported(const Dims& d, bool has_w_uv) {
-  return d.dtype == MLA_BF16 && d.d_c == kDc && d.d_rope == kDr && (!has_w_uv || d.d_head == kDh);
-}
-
-mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
+template <int DC, int DR>
+mla_status attention_tc_impl(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
+  using Sh = AttnShape<DC, DR>;
+  constexpr int kD = Sh::D;
   const KeyWorkspace kw = key_workspace_layout(d, n_valid);
   CUtensorMap tq, tqr, tcache, tchunk, tws, twuv;
   mla_status st;
@@ -521,8 +563,9 @@ mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStrea
                                  static_cast<uint64_t>(d.n_q) * d.H * kD * 2};
     const uint32_t box[4] = {64, 1, kBM, 1};
     if ((st = make_tmap_bf16(&tq, a.q, 4, dims, strides, box, 128)) != MLA_OK) return st;
-    const uint32_t box_r[4] = {kDr, 1, kBM, 1};
-    if ((st = make_tmap_bf16(&tqr, a.q, 4, dims, strides, box_r, 64)) != MLA_OK) return st;
+    const uint32_t box_r[4] = {DR, 1, kBM, 1};
+    if ((st = make_tmap_bf16(&tqr, a.q, 4, dims, strides, box_r, Sh::kRopeBytes)) != MLA_OK)
+      return st;
   }
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.n_q),
@@ -541,15 +584,16 @@ mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStrea
     tcache = tchunk;  // never read: no ring tiles
   }
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(kDr), static_cast<uint64_t>(kw.rows),
+    const uint64_t dims[3] = {static_cast<uint64_t>(DR), static_cast<uint64_t>(kw.rows),
                               static_cast<uint64_t>(d.B)};
-    const uint64_t strides[2] = {kDr * 2ull, static_cast<uint64_t>(kw.rows) * kDr * 2};
-    const uint32_t box[3] = {kDr, kBN, 1};
-    if ((st = make_tmap_bf16(&tws, a.ws, 3, dims, strides, box, 64)) != MLA_OK) return st;
+    const uint64_t strides[2] = {DR * 2ull, static_cast<uint64_t>(kw.rows) * DR * 2};
+    const uint32_t box[3] = {DR, kBN, 1};
+    if ((st = make_tmap_bf16(&tws, a.ws, 3, dims, strides, box, Sh::kRopeBytes)) != MLA_OK)
+      return st;
   }
   if (a.w_uv != nullptr) {
-    const uint64_t dims[2] = {static_cast<uint64_t>(kDc), static_cast<uint64_t>(d.H) * kDh};
-    const uint64_t strides[1] = {kDc * 2ull};
+    const uint64_t dims[2] = {static_cast<uint64_t>(DC), static_cast<uint64_t>(d.H) * kDh};
+    const uint64_t strides[1] = {DC * 2ull};
     const uint32_t box[2] = {64, kDh};
     if ((st = make_tmap_bf16(&twuv, a.w_uv, 2, dims, strides, box, 128)) != MLA_OK) return st;
   } else {
@@ -562,12 +606,30 @@ mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStrea
   p.scale_log2 = d.scale * 1.4426950408889634f;
   p.has_w_uv = a.w_uv != nullptr;
   p.out = a.out; p.lse = a.lse; p.dev_status = a.dev_status;
-  MLA_CUDA_TRY(cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kSmem));
+  MLA_CUDA_TRY(cudaFuncSetAttribute(attention_tc_kernel<DC, DR>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmem));
   dim3 grid(ceil_div(d.n_q, kBM), d.H, d.B);
-  attention_tc_kernel<<<grid, kThreads, kSmem, s>>>(tq, tqr, tcache, tchunk, tws, twuv, p);
+  attention_tc_kernel<DC, DR><<<grid, kThreads, Sh::kSmem, s>>>(tq, tqr, tcache, tchunk, tws, twuv, p);
   MLA_LAUNCH_CHECK("attention_tc");
   return MLA_OK;
+}
+
+}  // namespace
+
+bool tc_attention_supported(const Dims& d, bool has_w_uv) {
+  return d.dtype == MLA_BF16 && (d.d_c == 128 || d.d_c == 192 || d.d_c == 256) &&
+         (d.d_rope == 16 || d.d_rope == 32 || d.d_rope == 64) && (!has_w_uv || d.d_head == kDh);
+}
+
+mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
+#define MLA_ATTN_CASE(DC, DR) \
+  if (d.d_c == DC && d.d_rope == DR) return attention_tc_impl<DC, DR>(d, a, n_valid, s);
+  MLA_ATTN_CASE(128, 16) MLA_ATTN_CASE(128, 32) MLA_ATTN_CASE(128, 64)
+  MLA_ATTN_CASE(192, 16) MLA_ATTN_CASE(192, 32) MLA_ATTN_CASE(192, 64)
+  MLA_ATTN_CASE(256, 16) MLA_ATTN_CASE(256, 32) MLA_ATTN_CASE(256, 64)
+#undef MLA_ATTN_CASE
+  MLA_FAIL(MLA_ERR_UNSUPPORTED, "no tensor-core attention kernel for d_c %d, d_rope %d", d.d_c,
+           d.d_rope);
 }
 
 }  // namespace mla

@@ -13,7 +13,8 @@
 //              TMEM accumulators (tiles alternate), committing each stage back to the producer
 //              and each finished accumulator to the epilogue.
 //   warps 2-5  epilogue: drain an accumulator (one TMEM lane = one output row per thread) 32
-//              columns at a time, optionally rotate the positional-query columns (3D-RoPE),
+//              columns at a time, optionally rotate the positional-query columns (the last
+//              d_rope columns of every head block: 3D-RoPE),
 //              write bf16 into a 64B-swizzled 128x32 staging buffer (two, alternating) that one
 //              thread stores with a TMA bulk-tensor store (whole lines, out-of-range rows and
 //              columns clipped), and hand the accumulator back; this overlaps the MMAs of the
@@ -72,7 +73,7 @@ struct GemmParams {
   const void* A;
   int64_t a_sm;
   int epilogue;
-  int rope_D, rope_n_q, rope_first_frame;
+  int rope_D, rope_dr, rope_n_q, rope_first_frame;
   RopeGeom rope;
 };
 
@@ -251,10 +252,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-        if (p.epilogue == kEpiRopeQ && (n % p.rope_D) == p.rope_D - 32) {
+        if (p.epilogue == kEpiRopeQ) {
+          // columns rope0 .. D-1 of every D-wide head block are the positional query; a 32-column
+          // chunk may start anywhere in a head block (D is a multiple of 16, not of 32)
+          const int cb0 = n % p.rope_D;
+          const int rope0 = p.rope_D - p.rope_dr;
+          if (cb0 + 32 > rope0) {
 #pragma unroll
-          for (int pr = 0; pr < 16; ++pr)
-            rope_rotate(v[2 * pr], v[2 * pr + 1], rope_angle(p.rope, pr, t_pos, hh, ww));
+            for (int pr = 0; pr < 16; ++pr) {
+              const int cb = cb0 + 2 * pr;
+              if (cb >= rope0 && cb < p.rope_D)
+                rope_rotate(v[2 * pr], v[2 * pr + 1],
+                            rope_angle(p.rope, (cb - rope0) >> 1, t_pos, hh, ww));
+            }
+          }
         }
         const bool second = p.n_split > 0 && n >= p.n_split;
         if (p.tma_store) {
@@ -371,7 +382,7 @@ mla_status launch_gemm(const TcGemmArgs& g, cudaStream_t s) {
   p.a_swapped = a_sw; p.b_swapped = b_sw;
   p.C = g.C; p.c_sm = g.c_sm; p.c_batch = g.c_batch;
   p.C2 = g.C2; p.c2_sm = g.c2_sm; p.c2_batch = g.c2_batch; p.n_split = g.n_split;
-  p.epilogue = g.epilogue; p.rope_D = g.rope_D; p.rope_n_q = g.rope_n_q;
+  p.epilogue = g.epilogue; p.rope_D = g.rope_D; p.rope_dr = g.rope_dr; p.rope_n_q = g.rope_n_q;
   p.rope_first_frame = g.rope_first_frame; p.rope = g.rope;
   p.A = g.A; p.a_sm = g.a_sm;
   p.prefetch_a = (g.batch == 1 && g.a_sm == g.K) ? 1 : 0;
@@ -414,11 +425,10 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s) {
   if (g.M == 0 || g.N == 0) return MLA_OK;
   if (g.n_split != 0 && (g.n_split % 32 != 0 || g.n_split >= g.N || g.C2 == nullptr))
     MLA_FAIL(MLA_ERR_INVALID_ARG, "GEMM column split must be a multiple of 32 inside N");
-  if (g.epilogue == kEpiRopeQ) {
-    if (g.rope_D != 224 || g.N % 224 != 0)
-      MLA_FAIL(MLA_ERR_UNSUPPORTED, "query RoPE epilogue needs 224-wide head blocks");
-    return launch_gemm<224>(g, s);
-  }
+  if (g.epilogue == kEpiRopeQ &&
+      (g.rope_D <= 0 || g.N % g.rope_D != 0 || g.rope_dr % 2 != 0 || g.rope_dr > g.rope_D ||
+       g.rope_dr / 2 > kMaxRopePairs))
+    MLA_FAIL(MLA_ERR_UNSUPPORTED, "query RoPE epilogue needs whole head blocks and even d_rope");
   // Tile width: the one whose tiles spread most evenly over the SMs (each persistent CTA takes
   // ceil(tiles / SMs) tiles) with the least padding in N; ties go to the wider tile, which
   // re-reads A fewer times.  Projections here have few 128-row tiles, so a narrower N tile is

@@ -74,8 +74,8 @@ mla_status copy_rows(int dtype, const void* src, int64_t src_stride, void* dst,
 // Epilogues of the tcgen05 GEMM.
 enum GemmEpilogue : int {
   kEpiStore = 0,     // C[m, n] = acc (bf16)
-  kEpiRopeQ = 1,     // as kEpiStore, and 3D-RoPE on the last d_rope columns of every
-                     // D-wide head block of the output row (query path)
+  kEpiRopeQ = 1,     // as kEpiStore, and 3D-RoPE on the last rope_dr columns of every
+                     // rope_D-wide head block of the output row (query path)
 };
 
 struct TcGemmArgs {
@@ -95,8 +95,9 @@ struct TcGemmArgs {
   int n_split;
   int M, N, K, batch;
   int epilogue;
-  // kEpiRopeQ: rows are chunk tokens of samples of n_q rows; head blocks of width D.
-  int rope_D, rope_n_q, rope_first_frame;
+  // kEpiRopeQ: rows are chunk tokens of samples of n_q rows; head blocks of width rope_D whose
+  // last rope_dr columns are rotated.
+  int rope_D, rope_dr, rope_n_q, rope_first_frame;
   RopeGeom rope;
 };
 

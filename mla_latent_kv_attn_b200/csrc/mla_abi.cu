@@ -110,13 +110,15 @@ mla_status query_heads(const Dims& d, const void* c_q, const void* w_qcat, void*
                        int first_frame, cudaStream_t s) {
   const int M = d.B * d.n_q;
   const int N = d.H * d.D;
-  if (use_tc(d) && d.D == 224 && d.d_rope == 32 && tc_gemm_supported(M, N, d.d_cq, d.d_cq, d.d_cq)) {
+  if (use_tc(d) && d.d_c % 2 == 0 && d.D % 8 == 0 &&
+      tc_gemm_supported(M, N, d.d_cq, d.d_cq, d.d_cq)) {
     TcGemmArgs g{};
     g.A = c_q; g.a_sm = d.d_cq; g.a_batch = 0;
     g.B = w_qcat; g.b_sn = d.d_cq; g.b_batch = 0;
     g.C = q; g.c_sm = N; g.c_batch = 0;
     g.M = M; g.N = N; g.K = d.d_cq; g.batch = 1;
-    g.epilogue = kEpiRopeQ; g.rope_D = d.D; g.rope_n_q = d.n_q; g.rope_first_frame = first_frame;
+    g.epilogue = kEpiRopeQ; g.rope_D = d.D; g.rope_dr = d.d_rope; g.rope_n_q = d.n_q;
+    g.rope_first_frame = first_frame;
     g.rope = rope_geom(d);
     return gemm_tc(g, s);
   }
@@ -346,6 +348,12 @@ mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w
                  d.d_model, 0, chunk_lat, d.D, 0, M, d.D, d.d_model, 1, s));
   }
   return query_heads(d, c_q, w_qcat, q, first_frame, s);
+}
+
+int32_t mla_attention_uses_tensor_cores(const mla_config* cfg, int32_t with_w_uv) {
+  if (check_cfg(cfg) != MLA_OK) return -1;
+  const Dims d = dims_of(*cfg);
+  return (use_tc(d) && tc_attention_supported(d, with_w_uv != 0)) ? 1 : 0;
 }
 
 size_t mla_attention_workspace_bytes(const mla_config* cfg, int32_t n_valid_frames) {

@@ -132,6 +132,24 @@ def small_bf16_config() -> MLAConfig:
                      **{**WAN, "frame_h": 6, "frame_w": 10})
 
 
+def rope_pairs_for(d_rope: int) -> Tuple[int, int, int]:
+    """Rotary pairs per (t, h, w) axis for a positional width: a quarter of the pairs on the
+    temporal axis, the rest split evenly between rows and columns (Wan: 32 -> (4, 6, 6))."""
+    n = d_rope // 2
+    pt = n // 4
+    ph = (n - pt) // 2
+    return pt, ph, n - pt - ph
+
+
+def with_latent_shape(cfg: MLAConfig, d_c: int, d_rope: int) -> MLAConfig:
+    """The same workload with another content-latent and positional-key width (the latent-size
+    ablation shapes); the name records the shape."""
+    if (d_c, d_rope) == (cfg.d_c, cfg.d_rope):
+        return cfg
+    return dataclasses.replace(cfg, d_c=d_c, d_rope=d_rope, rope_pairs=rope_pairs_for(d_rope),
+                               name=f"{cfg.name}_dc{d_c}_dr{d_rope}")
+
+
 # --------------------------------------------------------------------------
 # rounding helpers (dtype plumbing, not method arithmetic)
 

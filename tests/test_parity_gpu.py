@@ -50,6 +50,22 @@ def test_small_frames_bf16_rollout(path):
     full_rollout(inputs.small_bf16_config(), PATHS[path])
 
 
+LATENT_SHAPES = [(dc, dr) for dc in (128, 192, 256) for dr in (16, 32, 64)]
+
+
+@pytest.mark.parametrize("d_c,d_rope", LATENT_SHAPES)
+def test_latent_shape_sweep_tensor_cores_match_oracle(d_c, d_rope):
+    """The latent-size ablation shapes (d_c in {128, 192, 256} x d_rope in {16, 32, 64}) run on
+    the tensor-core kernels and match the oracle over a 4-chunk rollout whose ring wraps."""
+    cfg = inputs.with_latent_shape(inputs.small_bf16_config(), d_c, d_rope)
+    c = api.make_config(cfg)
+    assert api.mla_attention_uses_tensor_cores(c, True)
+    assert api.mla_attention_uses_tensor_cores(c, False)
+    report = full_rollout(cfg, api.MLA_PATH_AUTO)
+    worst = max(v[1] for k, v in report.items() if k.endswith(".o"))
+    assert worst <= 5e-3
+
+
 def prefilled(cfg, path, upto):
     g = GpuRun(cfg, path)
     o = OracleRun(cfg, g.lw)
