@@ -62,7 +62,8 @@ __all__ = [
     "attention_probabilities", "attend", "FrameRecord", "SlidingWindow",
     "chunk_step", "absorbed_query", "up_project_output",
     "output_projection", "dense_scalars_per_token", "latent_scalars_per_token",
-    "kv_reduction",
+    "kv_reduction", "softmax_backward", "rope3d_adjoint", "latent_attention_backward",
+    "layer_backward_nonabsorbed",
 ]
 
 
@@ -361,3 +362,107 @@ def up_project_output(o_lat: np.ndarray, w_uv) -> np.ndarray:
 def output_projection(o: np.ndarray, w_o) -> np.ndarray:
     """y = W_O o (reading 7: secondary product)."""
     return np.asarray(o, np.float64) @ np.asarray(w_o, np.float64).T
+
+
+# ---------------------------------------------------------------------------
+# gradients of the attention layer (training use: the pages train the latent students with
+# teacher forcing and distillation through these layers; hyper.ai summary, "Method").  With an
+# upstream gradient g of the output, L = sum g * output; the derivatives below are the
+# textbook ones of softmax attention, taken one step of the forward at a time, in reverse.
+
+def softmax_backward(p: np.ndarray, d_p: np.ndarray) -> np.ndarray:
+    """dL/ds for p = softmax over the last axis of s, given dL/dp:
+    p * (d_p - sum_j p_j d_p_j)."""
+    return p * (d_p - (p * d_p).sum(axis=-1, keepdims=True))
+
+
+def rope3d_adjoint(vec: np.ndarray, pos: np.ndarray, d: Dims) -> np.ndarray:
+    """Transpose of the 3D-RoPE map at positions pos: each pair's rotation by a is orthogonal,
+    so its transpose is the rotation by -a, i.e. the map at the negated positions."""
+    return rope3d(vec, -np.asarray(pos), d)
+
+
+def latent_attention_backward(q: np.ndarray, c_keys: np.ndarray, k_r_keys: np.ndarray,
+                              pos_k: np.ndarray, d_o_lat: np.ndarray, d: Dims):
+    """Gradients of the latent-space attention call.
+
+    Forward (what the attention kernel computes): for head h and query n,
+      K'_m = [c_m || RoPE3D(k_R,m, pos_m)],  s = scale * q[n, h] . K'_m,
+      p = softmax over m,  O_lat[n, h] = sum_m p_m c_m.
+    q [N, H, d_c + d_rope] (positional part already rotated), c_keys [M, d_c], k_r_keys
+    [M, d_rope] (unrotated), pos_k [M, 3], d_o_lat [N, H, d_c] = dL/dO_lat.
+
+    Returns o_lat, lse [H, N], d_q [N, H, D] (w.r.t. q as given), d_c [M, d_c] and d_k_r
+    [M, d_rope] (w.r.t. the unrotated positional keys).  The value of a key is its content
+    latent, so d_c collects both the value gradient and the content part of the key gradient.
+    """
+    q = np.asarray(q, np.float64)
+    c_keys = np.asarray(c_keys, np.float64)
+    d_o_lat = np.asarray(d_o_lat, np.float64)
+    n, n_heads, width = q.shape
+    scale = d.softmax_scale
+    k_full = np.concatenate([c_keys, rope3d(k_r_keys, pos_k, d)], axis=1)     # K' [M, D]
+    o_lat = np.empty((n, n_heads, d.d_c))
+    lse = np.empty((n_heads, n))
+    d_q = np.empty_like(q)
+    d_k_full = np.zeros_like(k_full)
+    d_v = np.zeros_like(c_keys)
+    for h in range(n_heads):
+        s = (q[:, h] @ k_full.T) * scale
+        row_max = s.max(axis=1, keepdims=True)
+        e = np.exp(s - row_max)
+        p = e / e.sum(axis=1, keepdims=True)
+        lse[h] = (row_max + np.log(e.sum(axis=1, keepdims=True)))[:, 0]
+        o_lat[:, h] = p @ c_keys
+        # O_lat = p V (V = c_keys)
+        d_p = d_o_lat[:, h] @ c_keys.T
+        d_v += p.T @ d_o_lat[:, h]
+        # p = softmax(s)
+        d_s = softmax_backward(p, d_p)
+        # s = scale q K'^T
+        d_q[:, h] = scale * (d_s @ k_full)
+        d_k_full += scale * (d_s.T @ q[:, h])
+    d_c = d_v + d_k_full[:, :d.d_c]
+    d_k_r = rope3d_adjoint(d_k_full[:, d.d_c:], pos_k, d)
+    return dict(o_lat=o_lat, lse=lse, d_q=d_q, d_c=d_c, d_k_r=d_k_r)
+
+
+def layer_backward_nonabsorbed(d: Dims, w, c_q: np.ndarray, pos_q: np.ndarray,
+                               c_keys: np.ndarray, k_r_keys: np.ndarray, pos_k: np.ndarray,
+                               d_o: np.ndarray):
+    """Gradients of the non-absorbed layer (per-head keys and values rebuilt from c_KV) w.r.t.
+    the query latent c_Q [N, d_cq], the key latents c_keys [M, d_c] and the unrotated positional
+    keys k_r_keys [M, d_rope], for the upstream gradient d_o [N, H, d_head] of the per-head
+    outputs o_h = sum_m p_m v_m,h.  Returns d_c_q, d_c, d_k_r and o [N, H, d_head]."""
+    scale = d.softmax_scale
+    q_nope, q_r = query_heads(c_q, w.w_uq, w.w_qr)
+    q_rope = rope3d(q_r, pos_q, d)
+    k_nope, v = key_value_heads(c_keys, w.w_uk, w.w_uv)
+    k_rope = rope3d(k_r_keys, pos_k, d)
+    n, n_heads, dh = q_nope.shape
+    d_o = np.asarray(d_o, np.float64)
+    o = np.empty((n, n_heads, dh))
+    d_q_nope = np.empty_like(q_nope)
+    d_q_rope = np.empty_like(q_rope)
+    d_k_nope = np.zeros_like(k_nope)
+    d_v = np.zeros_like(v)
+    d_k_rope = np.zeros_like(k_rope)
+    for h in range(n_heads):
+        p, _ = attention_probabilities(q_nope[:, h], q_rope[:, h], k_nope[:, h], k_rope, scale)
+        o[:, h] = p @ v[:, h]
+        d_p = d_o[:, h] @ v[:, h].T
+        d_v[:, h] = p.T @ d_o[:, h]
+        d_s = softmax_backward(p, d_p)
+        d_q_nope[:, h] = scale * (d_s @ k_nope[:, h])
+        d_q_rope[:, h] = scale * (d_s @ k_rope)
+        d_k_nope[:, h] = scale * (d_s.T @ q_nope[:, h])
+        d_k_rope += scale * (d_s.T @ q_rope[:, h])
+    w_uq, w_uk = np.asarray(w.w_uq, np.float64), np.asarray(w.w_uk, np.float64)
+    w_uv, w_qr = np.asarray(w.w_uv, np.float64), np.asarray(w.w_qr, np.float64)
+    # k_nope_h = W_UK_h c, v_h = W_UV_h c, k_rope = RoPE(k_R)
+    d_c = (np.einsum("hdc,mhd->mc", w_uk, d_k_nope) + np.einsum("hdc,mhd->mc", w_uv, d_v))
+    d_k_r = rope3d_adjoint(d_k_rope, pos_k, d)
+    # q_nope_h = W_UQ_h c_Q, q_rope_h = RoPE(W_QR_h c_Q)
+    d_q_r = rope3d_adjoint(d_q_rope, pos_q, d)
+    d_c_q = (np.einsum("hdk,nhd->nk", w_uq, d_q_nope) + np.einsum("hdk,nhd->nk", w_qr, d_q_r))
+    return dict(d_c_q=d_c_q, d_c=d_c, d_k_r=d_k_r, o=o)

@@ -334,6 +334,93 @@ def test_output_projection_brute_force():
 
 
 # --------------------------------------------------------------------------
+# gradients (training use): pinned to finite differences of the forward, to the non-absorbed
+# chain rule, and to the adjoint property of a rotation
+
+def _latent_forward(q, c, k_r, pos_k, d):
+    """O_lat through the (separately pinned) forward pieces: attention_probabilities with the
+    content latent as both the content key and the value, and the rotated positional key."""
+    n_heads = q.shape[1]
+    keys = np.repeat(c[:, None, :], n_heads, axis=1)
+    return oracle.attend(q[:, :, :d.d_c], q[:, :, d.d_c:], keys, oracle.rope3d(k_r, pos_k, d),
+                         keys, d.softmax_scale, c_keys=c)["o_lat"]
+
+
+def _backward_case(seed=3, n=4, m=6):
+    d = random_dims()
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((n, d.n_heads, d.d_c + d.d_rope))
+    c = rng.standard_normal((m, d.d_c))
+    k_r = rng.standard_normal((m, d.d_rope))
+    pos_k = rng.integers(0, 5, size=(m, 3))
+    g = rng.standard_normal((n, d.n_heads, d.d_c))
+    return d, q, c, k_r, pos_k, g
+
+
+def test_backward_matches_finite_differences():
+    d, q, c, k_r, pos_k, g = _backward_case()
+    res = oracle.latent_attention_backward(q, c, k_r, pos_k, g, d)
+    loss = lambda q_, c_, k_: float((g * _latent_forward(q_, c_, k_, pos_k, d)).sum())
+    eps = 1e-6
+    for name, arr, grad in (("q", q, res["d_q"]), ("c", c, res["d_c"]), ("k_r", k_r, res["d_k_r"])):
+        num = np.zeros_like(arr)
+        for i in np.ndindex(arr.shape):
+            plus, minus = arr.copy(), arr.copy()
+            plus[i] += eps
+            minus[i] -= eps
+            args_p = {"q": (plus, c, k_r), "c": (q, plus, k_r), "k_r": (q, c, plus)}[name]
+            args_m = {"q": (minus, c, k_r), "c": (q, minus, k_r), "k_r": (q, c, minus)}[name]
+            num[i] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8, err_msg=name)
+    np.testing.assert_allclose(res["o_lat"], _latent_forward(q, c, k_r, pos_k, d), atol=1e-12)
+
+
+def test_backward_absorbed_equals_non_absorbed():
+    """The latent-space gradients are those of the layer with per-head keys and values rebuilt
+    from c_KV: w.r.t. c_KV and k_R directly, w.r.t. c_Q through the absorbed query weights."""
+    d = random_dims()
+    rng = np.random.default_rng(11)
+    w = random_weights(d, rng)
+    n, m = 5, 7
+    c_q = rng.standard_normal((n, d.d_cq))
+    pos_q = rng.integers(0, 6, size=(n, 3))
+    c = rng.standard_normal((m, d.d_c))
+    k_r = rng.standard_normal((m, d.d_rope))
+    pos_k = rng.integers(0, 6, size=(m, 3))
+    d_o = rng.standard_normal((n, d.n_heads, d.d_head))
+    ref = oracle.layer_backward_nonabsorbed(d, w, c_q, pos_q, c, k_r, pos_k, d_o)
+    q = oracle.absorbed_query(c_q, w.w_uq, w.w_uk, w.w_qr, pos_q, d)
+    d_o_lat = np.einsum("hdc,nhd->nhc", w.w_uv, d_o)           # o_h = W_UV_h O_lat,h
+    lat = oracle.latent_attention_backward(q, c, k_r, pos_k, d_o_lat, d)
+    np.testing.assert_allclose(lat["d_c"], ref["d_c"], rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(lat["d_k_r"], ref["d_k_r"], rtol=1e-10, atol=1e-10)
+    d_q_lat, d_q_rope = lat["d_q"][..., :d.d_c], lat["d_q"][..., d.d_c:]
+    d_c_q = (np.einsum("hdk,hdc,nhc->nk", w.w_uq, w.w_uk, d_q_lat) +
+             np.einsum("hdk,nhd->nk", w.w_qr, oracle.rope3d_adjoint(d_q_rope, pos_q, d)))
+    np.testing.assert_allclose(d_c_q, ref["d_c_q"], rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(oracle.up_project_output(lat["o_lat"], w.w_uv),
+                               ref["o"].reshape(n, -1), rtol=1e-10, atol=1e-10)
+
+
+def test_rope_adjoint_is_the_transpose():
+    d = random_dims()
+    rng = np.random.default_rng(5)
+    x, y = rng.standard_normal((9, d.d_rope)), rng.standard_normal((9, d.d_rope))
+    pos = rng.integers(-4, 9, size=(9, 3))
+    lhs = (oracle.rope3d(x, pos, d) * y).sum(axis=1)
+    rhs = (x * oracle.rope3d_adjoint(y, pos, d)).sum(axis=1)
+    np.testing.assert_allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+
+
+def test_backward_is_linear_in_the_upstream_gradient():
+    d, q, c, k_r, pos_k, g = _backward_case(seed=8)
+    a = oracle.latent_attention_backward(q, c, k_r, pos_k, g, d)
+    b = oracle.latent_attention_backward(q, c, k_r, pos_k, -2.5 * g, d)
+    for k in ("d_q", "d_c", "d_k_r"):
+        np.testing.assert_allclose(b[k], -2.5 * a[k], rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
 # the pins above catch planted slips
 
 PINS = [test_rope_identity_at_origin, test_rope_preserves_pair_norms,
@@ -343,7 +430,9 @@ PINS = [test_rope_identity_at_origin, test_rope_preserves_pair_norms,
         test_absorbed_form_equals_non_absorbed, test_mha_special_case_matches_library_sdpa,
         test_brute_force_rollout_with_wraparound, test_window_holds_the_last_w_frames,
         test_positions_row_major, test_cache_size_matches_pages,
-        test_output_projection_brute_force]
+        test_output_projection_brute_force, test_backward_matches_finite_differences,
+        test_backward_absorbed_equals_non_absorbed, test_rope_adjoint_is_the_transpose,
+        test_backward_is_linear_in_the_upstream_gradient]
 
 
 def _patch(monkeypatch, name, fn):
@@ -356,6 +445,7 @@ def _mutants():
     orig_rope, orig_angles, orig_attn = M.rope3d, M.rope3d_angles, M.attention_probabilities
     orig_kv, orig_qh, orig_pos = M.key_value_heads, M.query_heads, M.token_positions
     orig_attend = M.attend
+    orig_sbw, orig_lab = M.softmax_backward, M.latent_attention_backward
 
     def rope_flipped(vec, pos, d):
         return orig_rope(vec, -np.asarray(pos), d)
@@ -415,7 +505,32 @@ def _mutants():
     def out_proj_transposed(o, w_o):
         return np.asarray(o, np.float64) @ np.asarray(w_o, np.float64)[:, :np.asarray(o).shape[1]]
 
+    def softmax_bw_no_row_term(p, d_p):
+        return p * d_p
+
+    def rope_adjoint_same_direction(vec, pos, d):
+        return orig_rope(vec, pos, d)
+
+    def backward_value_gradient_dropped(q, c, k_r, pos_k, g, d):
+        res = orig_lab(q, c, k_r, pos_k, g, d)
+        p_t = []
+        for h in range(q.shape[1]):
+            k_full = np.concatenate([c, orig_rope(k_r, pos_k, d)], axis=1)
+            s = q[:, h] @ k_full.T * d.softmax_scale
+            e = np.exp(s - s.max(axis=1, keepdims=True))
+            p_t.append((e / e.sum(axis=1, keepdims=True)).T @ g[:, h])
+        return dict(res, d_c=res["d_c"] - sum(p_t))
+
+    def backward_unscaled_query_gradient(q, c, k_r, pos_k, g, d):
+        res = orig_lab(q, c, k_r, pos_k, g, d)
+        return dict(res, d_q=res["d_q"] / d.softmax_scale)
+
     return {
+        "softmax gradient without the row term": [("softmax_backward", softmax_bw_no_row_term)],
+        "rope adjoint turns the same way": [("rope3d_adjoint", rope_adjoint_same_direction)],
+        "value gradient dropped": [("latent_attention_backward", backward_value_gradient_dropped)],
+        "query gradient without the scale": [("latent_attention_backward",
+                                              backward_unscaled_query_gradient)],
         "rope rotates the wrong way": [("rope3d", rope_flipped)],
         "rope frequency exponent doubled": [("rope3d_angles", angles_wrong_exponent)],
         "rope bands t/h swapped": [("rope3d_angles", angles_bands_swapped)],
