@@ -324,6 +324,39 @@ mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q
                                             float* lse, int32_t* dev_status, void* stream);
 
 /* --------------------------------------------------------------------------------------------
+ * mla_attention_bwd: gradients of mla_attention_fwd without the W_UV epilogue, for training
+ * ([M]: the latent students are trained through these layers).  With G = dL/dO_lat and the
+ * forward's definitions (K'_m = [c_m || RoPE3D(k_R,m)], s = scale q.K'_m, p = exp(s - lse),
+ * O_lat = sum_m p c_m):
+ *   dP = G . c_m,  Delta = G . O_lat,  dS = p (dP - Delta)
+ *   d_q[b, n, h]      = scale sum_m dS K'_m                         (w.r.t. q as given: its
+ *                                                                     positional part rotated)
+ *   d latent of key m = [ sum_{h,n} (p G + scale dS q[:d_c])  ||  RoPE3D^T(scale sum dS q[d_c:]) ]
+ * i.e. w.r.t. the latents as stored (k_R unrotated; the transpose of a rotation is the rotation
+ * by the opposite angle).  Keys are walked as in mla_attention_fwd.
+ *   q, chunk_lat, cache, slot_frame, n_valid_frames, first_frame: as given to the forward
+ *   o_lat     device T [B, n_q, H, d_c]   the forward's latent output (w_uv = NULL)
+ *   lse       device float [B, H, n_q]    the forward's lse
+ *   d_o_lat   device T [B, n_q, H, d_c]   dL/dO_lat
+ *   d_q       device T [B, n_q, H, D]     out
+ *   d_chunk_lat device T [B, n_q, D]      out: gradient of the chunk's latents
+ *   d_cache   device T [B, W*tpf, D]      out: rows 0 .. n_valid_frames*tpf - 1 (the attended
+ *                                         ring slots) are written, the others left untouched;
+ *                                         may be NULL when n_valid_frames == 0
+ *   workspace device scratch of >= mla_attention_bwd_workspace_bytes(cfg, n_valid_frames)
+ *             bytes, 256-byte aligned; contents on entry do not matter
+ * Probabilities are recomputed from q, the keys and lse (fp32).  Errors: MLA_ERR_INVALID_ARG,
+ * MLA_ERR_ALIGNMENT, MLA_ERR_WORKSPACE, MLA_ERR_UNSUPPORTED (d_c + d_rope > 512), MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+size_t mla_attention_bwd_workspace_bytes(const mla_config* cfg, int32_t n_valid_frames);
+mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* chunk_lat,
+                             const void* cache, const int32_t* slot_frame,
+                             int32_t n_valid_frames, int32_t first_frame, const void* o_lat,
+                             const float* lse, const void* d_o_lat, void* d_q,
+                             void* d_chunk_lat, void* d_cache, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------------------------------------------
  * mla_out_proj: value up-projection of latent outputs and the optional output projection
  * ([M]: v_{t,h} is reconstructed from c_KV by W_UV_h; the output projection is the usual
  * attention-layer output map, which the pages do not describe).

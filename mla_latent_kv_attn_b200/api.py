@@ -20,6 +20,7 @@ __all__ = [
     "mla_key_positions", "mla_compose_query_weights", "mla_query_proj", "mla_project_chunk",
     "mla_attention_workspace_bytes", "mla_attention_fwd", "mla_attention_fwd_static_scratch",
     "mla_rotate_ring_keys", "mla_attention_fwd_cached_ring", "mla_attention_uses_tensor_cores",
+    "mla_attention_bwd_workspace_bytes", "mla_attention_bwd",
     "mla_out_proj", "MLAError",
     "MLA_PROJECT", "MLA_APPEND", "MLA_PROJECT_AND_APPEND", "MLA_PATH_AUTO", "MLA_PATH_SIMT",
 ]
@@ -199,6 +200,30 @@ def mla_rotate_ring_keys(c: MLAConfigC, cache, slot_frame, n_valid_frames: int, 
         _ptr(slot_frame, "slot_frame", torch.int32, (B, c.window_frames)), n_valid_frames,
         _ptr(workspace, "workspace"), ws_bytes, _stream(stream))
     _lib.check("mla_rotate_ring_keys", st)
+
+
+def mla_attention_bwd_workspace_bytes(c: MLAConfigC, n_valid_frames: int) -> int:
+    return int(_lib.lib().mla_attention_bwd_workspace_bytes(ctypes.byref(c), n_valid_frames))
+
+
+def mla_attention_bwd(c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_frames: int,
+                      first_frame: int, o_lat, lse, d_o_lat, d_q, d_chunk_lat, d_cache, workspace,
+                      stream=None) -> None:
+    """Gradients of the latent attention call (see include/mla.h)."""
+    tpf, n_q, D = _geom(c)
+    dt = torch_dtype(c)
+    B, H = c.batch, c.n_heads
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib.lib().mla_attention_bwd(
+        ctypes.byref(c), _ptr(q, "q", dt, (B, n_q, H, D)), _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)),
+        _ptr(cache, "cache", dt, (B, c.window_frames * tpf, D)),
+        _ptr(slot_frame, "slot_frame", torch.int32, (B, c.window_frames)), n_valid_frames,
+        first_frame, _ptr(o_lat, "o_lat", dt, (B, n_q, H, c.d_c)),
+        _ptr(lse, "lse", torch.float32, (B, H, n_q)), _ptr(d_o_lat, "d_o_lat", dt, (B, n_q, H, c.d_c)),
+        _ptr(d_q, "d_q", dt, (B, n_q, H, D)), _ptr(d_chunk_lat, "d_chunk_lat", dt, (B, n_q, D)),
+        _ptr(d_cache, "d_cache", dt, (B, c.window_frames * tpf, D)), _ptr(workspace, "workspace"),
+        ws_bytes, _stream(stream))
+    _lib.check("mla_attention_bwd", st)
 
 
 def mla_out_proj(c: MLAConfigC, o_lat, w_uv, o, w_o=None, y=None, stream=None) -> None:

@@ -136,6 +136,24 @@ __device__ __forceinline__ void rope_rotate(float& x0, float& x1, float a) {
   x1 = y1;
 }
 
+// (t, h, w) of key m in the walk order of the attention kernels: ring slots 0 .. nc-1 (their
+// frame from slot_frame), then the chunk's own tokens (frame first_frame + j / tpf).
+__device__ __forceinline__ void key_position(const int32_t* slot_frame, int b, int W, int tpf,
+                                             int frame_w, int nc, int first_frame, int m, int& t,
+                                             int& h, int& w) {
+  int i;
+  if (m < nc) {
+    t = slot_frame[b * W + m / tpf];
+    i = m % tpf;
+  } else {
+    const int j = m - nc;
+    t = first_frame + j / tpf;
+    i = j % tpf;
+  }
+  h = i / frame_w;
+  w = i % frame_w;
+}
+
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int round_up(int a, int b) { return ceil_div(a, b) * b; }
 

@@ -49,6 +49,30 @@ struct KeyWorkspace {
 
 KeyWorkspace key_workspace_layout(const Dims& d, int n_valid);
 
+// Backward of the attention call (attention_bwd.cu).
+struct BwdArgs {
+  const void* q;           // [B, n_q, H, D]
+  const void* chunk_lat;   // [B, n_q, D]
+  const void* cache;       // [B, W*tpf, D]
+  const int32_t* slot_frame;
+  const void* o_lat;       // [B, n_q, H, d_c]
+  const float* lse;        // [B, H, n_q]
+  const void* d_o_lat;     // [B, n_q, H, d_c]
+  void* d_q;               // [B, n_q, H, D]
+  void* d_chunk_lat;       // [B, n_q, D]
+  void* d_cache;           // [B, W*tpf, D]
+};
+
+struct BwdWorkspace {
+  size_t delta_bytes;      // Delta = G . O_lat per (sample, head, row), fp32, then
+  KeyWorkspace keys;       // the rotated positional keys, as in the forward
+  size_t bytes;
+};
+
+BwdWorkspace bwd_workspace_layout(const Dims& d, int n_valid);
+mla_status attention_bwd(const Dims& d, const BwdArgs& a, int n_valid, int first_frame,
+                         void* workspace, cudaStream_t s);
+
 // CUDA-core kernels (simt.cu)
 mla_status gemm_simt(const GemmArgs& g, int dtype, cudaStream_t s);
 mla_status rope3d_inplace(const Dims& d, void* data, int n_samples, int rows, int row_width,

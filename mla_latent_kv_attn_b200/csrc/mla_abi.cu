@@ -424,6 +424,49 @@ mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q
                                       static_cast<cudaStream_t>(stream));
 }
 
+size_t mla_attention_bwd_workspace_bytes(const mla_config* cfg, int32_t n_valid_frames) {
+  if (check_cfg(cfg) != MLA_OK) return 0;
+  const Dims d = dims_of(*cfg);
+  if (n_valid_frames < 0 || n_valid_frames > d.W) return 0;
+  return bwd_workspace_layout(d, n_valid_frames).bytes;
+}
+
+mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* chunk_lat,
+                             const void* cache, const int32_t* slot_frame,
+                             int32_t n_valid_frames, int32_t first_frame, const void* o_lat,
+                             const float* lse, const void* d_o_lat, void* d_q,
+                             void* d_chunk_lat, void* d_cache, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  set_last_error("");
+  MLA_TRY(check_cfg(cfg));
+  const Dims d = dims_of(*cfg);
+  MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
+                d.W);
+  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_ptr(q, "q"));
+  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
+  MLA_TRY(check_ptr(slot_frame, "slot_frame"));
+  MLA_TRY(check_ptr(cache, "cache", n_valid_frames > 0));
+  MLA_TRY(check_ptr(o_lat, "o_lat"));
+  MLA_TRY(check_ptr(lse, "lse"));
+  MLA_TRY(check_ptr(d_o_lat, "d_o_lat"));
+  MLA_TRY(check_ptr(d_q, "d_q"));
+  MLA_TRY(check_ptr(d_chunk_lat, "d_chunk_lat"));
+  MLA_TRY(check_ptr(d_cache, "d_cache", n_valid_frames > 0));
+  const BwdWorkspace w = bwd_workspace_layout(d, n_valid_frames);
+  if (workspace == nullptr || workspace_bytes < w.bytes)
+    MLA_FAIL(MLA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
+             w.bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    MLA_FAIL(MLA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  MLA_TRY(check_ptr(workspace, "workspace"));
+  BwdArgs a{};
+  a.q = q; a.chunk_lat = chunk_lat; a.cache = cache; a.slot_frame = slot_frame; a.o_lat = o_lat;
+  a.lse = lse; a.d_o_lat = d_o_lat; a.d_q = d_q; a.d_chunk_lat = d_chunk_lat; a.d_cache = d_cache;
+  return attention_bwd(d, a, n_valid_frames, first_frame, workspace,
+                       static_cast<cudaStream_t>(stream));
+}
+
 mla_status mla_out_proj(const mla_config* cfg, const void* o_lat, const void* w_uv,
                         const void* w_o, void* o, void* y, void* stream) {
   set_last_error("");

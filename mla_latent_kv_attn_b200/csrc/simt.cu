@@ -201,21 +201,6 @@ mla_status ring_append(const Dims& d, const void* chunk_lat, void* cache, int32_
 // Key positions, in the walk order of the attention kernels.
 // ============================================================================================
 
-__device__ __forceinline__ void key_position(const int32_t* slot_frame, int b, int W, int tpf,
-                                             int frame_w, int nc, int first_frame, int m, int& t,
-                                             int& h, int& w) {
-  int i;
-  if (m < nc) {
-    t = slot_frame[b * W + m / tpf];
-    i = m % tpf;
-  } else {
-    const int j = m - nc;
-    t = first_frame + j / tpf;
-    i = j % tpf;
-  }
-  h = i / frame_w;
-  w = i % frame_w;
-}
 
 namespace {
 

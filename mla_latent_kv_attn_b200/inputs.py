@@ -36,6 +36,9 @@ TID_W_UK = 6
 TID_W_UV = 7
 TID_W_QR = 8
 TID_W_O = 9
+TID_Q = 10          # absorbed queries drawn directly (tests of a single call)
+TID_LATENT = 11     # chunk latents drawn directly
+TID_GRAD = 12       # upstream gradients
 
 
 @dataclasses.dataclass(frozen=True)
@@ -238,6 +241,29 @@ def chunk_x_rows(cfg: MLAConfig, chunk: int, rows: np.ndarray, step: int = 0, la
     full = _normal(cfg, (cfg.n_q, cfg.d_model), 1.0, TID_X, chunk=chunk, step=step,
                    layer=layer, sample=sample)
     return full[np.asarray(rows)]
+
+
+def direct_queries(cfg: MLAConfig, chunk: int, std: float = 0.5, samples=None) -> np.ndarray:
+    """Absorbed queries [B, n_q, H, d_c + d_rope] drawn directly (not projected from x), for
+    tests that feed one call its inputs."""
+    samples = range(cfg.batch) if samples is None else samples
+    return np.stack([_normal(cfg, (cfg.n_q, cfg.n_heads, cfg.d_latent), std, TID_Q, chunk=chunk,
+                             sample=b) for b in samples])
+
+
+def direct_latents(cfg: MLAConfig, chunk: int, samples=None) -> np.ndarray:
+    """Chunk latents [B, n_q, d_c + d_rope] ([c_KV || unrotated k_R]) drawn directly, N(0, 1)."""
+    samples = range(cfg.batch) if samples is None else samples
+    return np.stack([_normal(cfg, (cfg.n_q, cfg.d_latent), 1.0, TID_LATENT, chunk=chunk, sample=b)
+                     for b in samples])
+
+
+def upstream_gradient(cfg: MLAConfig, chunk: int, width: int, std: float = 1.0,
+                      samples=None) -> np.ndarray:
+    """A synthetic upstream gradient [B, n_q, H, width] (training-use tests)."""
+    samples = range(cfg.batch) if samples is None else samples
+    return np.stack([_normal(cfg, (cfg.n_q, cfg.n_heads, width), std, TID_GRAD, chunk=chunk,
+                             sample=b) for b in samples])
 
 
 def sample_rows(n: int, k: int, seed: int = 0, tag: int = 0) -> np.ndarray:

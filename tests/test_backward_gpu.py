@@ -1,0 +1,87 @@
+"""GPU parity of the attention backward (mla_attention_bwd) against the float64 oracle's
+latent_attention_backward, on identical seeded inputs: queries, chunk latents and ring contents
+drawn directly (the ring filled through mla_cache_append so that it wraps), and a seeded upstream
+gradient.  The GPU takes o_lat and lse from its own forward on those inputs; the oracle
+recomputes everything it needs in float64."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_latent_kv_attn_b200 import api, inputs, rollout
+from parity_util import compare, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(cfg, chunk, path=api.MLA_PATH_AUTO, grad_std=1.0):
+    c = api.make_config(cfg, kernel_path=path)
+    dt = api.torch_dtype(c)
+    dev = torch.device("cuda")
+    ring = rollout.Ring(c)
+    d = oracle.dims_from(cfg)
+    windows = [oracle.SlidingWindow(d) for _ in range(cfg.batch)]
+    lat_buf = torch.empty((cfg.batch, cfg.n_q, cfg.d_latent), device=dev, dtype=dt)
+    for ch in range(chunk):                      # earlier chunks enter the ring (it wraps)
+        lat = inputs.direct_latents(cfg, ch)
+        lat_buf.copy_(torch.from_numpy(lat).to(dt))
+        api.mla_cache_append(c, None, None, lat_buf, ring.cache, ring.slot_frame,
+                             cfg.first_frame(ch), api.MLA_APPEND)
+        for b in range(cfg.batch):
+            windows[b].append_chunk(cfg.first_frame(ch), lat[b][:, :cfg.d_c], lat[b][:, cfg.d_c:])
+    first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, chunk)
+    q_np = inputs.direct_queries(cfg, chunk)
+    lat_np = inputs.direct_latents(cfg, chunk)
+    g_np = inputs.upstream_gradient(cfg, chunk, cfg.d_c, std=grad_std)
+    q = torch.from_numpy(q_np).to(device=dev, dtype=dt)
+    lat_buf.copy_(torch.from_numpy(lat_np).to(dt))
+    g = torch.from_numpy(g_np).to(device=dev, dtype=dt)
+    o_lat = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads, cfg.d_c), device=dev, dtype=dt)
+    lse = torch.empty((cfg.batch, cfg.n_heads, cfg.n_q), device=dev, dtype=torch.float32)
+    ws = torch.empty(max(api.mla_attention_workspace_bytes(c, n_valid), 256), device=dev,
+                     dtype=torch.uint8)
+    api.mla_attention_fwd(c, q, lat_buf, ring.cache, ring.slot_frame, n_valid, first, None, o_lat,
+                          lse, ws)
+    d_q = torch.full_like(q, float("nan"))
+    d_lat = torch.full_like(lat_buf, float("nan"))
+    sentinel = 7.0
+    d_cache = torch.full_like(ring.cache, sentinel)
+    bws = torch.empty(api.mla_attention_bwd_workspace_bytes(c, n_valid), device=dev,
+                      dtype=torch.uint8)
+    api.mla_attention_bwd(c, q, lat_buf, ring.cache, ring.slot_frame, n_valid, first, o_lat, lse, g,
+                          d_q, d_lat, d_cache, bws)
+    torch.cuda.synchronize()
+    got = dict(d_q=to_np(d_q), d_lat=to_np(d_lat), d_cache=to_np(d_cache),
+               slot_frame=ring.slot_frame.cpu().numpy())
+    tpf = cfg.tokens_per_frame
+    nc = n_valid * tpf
+    for b in range(cfg.batch):
+        recs = {r.t: r for r in windows[b].frames}
+        slots = got["slot_frame"][b][:n_valid]
+        c_ring = np.concatenate([recs[t].c_kv for t in slots]) if n_valid else np.zeros((0, cfg.d_c))
+        k_ring = np.concatenate([recs[t].k_r for t in slots]) if n_valid else np.zeros((0, cfg.d_rope))
+        pos_ring = oracle.token_positions(list(slots), d)
+        pos_chunk = oracle.token_positions(range(first, first + cfg.chunk_frames), d)
+        ref = oracle.latent_attention_backward(
+            q_np[b], np.concatenate([c_ring, lat_np[b][:, :cfg.d_c]]),
+            np.concatenate([k_ring, lat_np[b][:, cfg.d_c:]]), np.concatenate([pos_ring, pos_chunk]),
+            g_np[b], d)
+        dk = np.concatenate([ref["d_c"], ref["d_k_r"]], axis=1)
+        tag = f"{cfg.name}[b{b}]"
+        compare(tag + ".d_q", got["d_q"][b], ref["d_q"], cfg.dtype)
+        compare(tag + ".d_chunk_lat", got["d_lat"][b], dk[nc:], cfg.dtype)
+        if nc:
+            compare(tag + ".d_cache", got["d_cache"][b][:nc], dk[:nc], cfg.dtype)
+        assert (got["d_cache"][b][nc:] == sentinel).all(), "rows beyond the attended slots changed"
+    return got
+
+
+def test_backward_toy_fp32_wrapped_ring():
+    cfg = inputs.CONFIGS[0]
+    _run(cfg, chunk=3)          # window of 2 frames after 3 one-frame chunks: wrapped
+
+
+@pytest.mark.parametrize("chunk", [0, 3])
+def test_backward_small_frames_bf16(chunk):
+    """Wan widths on 6x10 frames, 12 heads: chunk 0 (no ring) and chunk 3 (ring wrapped)."""
+    _run(inputs.small_bf16_config(), chunk=chunk)
