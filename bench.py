@@ -513,6 +513,76 @@ def run_stack(args, cfg):
     return 0
 
 
+def run_backward(args, cfg):
+    """--backward: the gradient call mla_attention_bwd on the preset's measured chunk (window
+    full), inputs drawn directly (seeded queries, chunk and ring latents, upstream gradient) and
+    the forward's o_lat / lse computed first.  Algorithmic work per (query row, key, head):
+    recomputed scores 2D, dP 2d_c, dq 2D, key gradient 2D, value gradient 2d_c."""
+    import torch
+    from mla_latent_kv_attn_b200 import api, inputs, rollout
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    c = api.make_config(cfg)
+    dt = api.torch_dtype(c)
+    ring = rollout.Ring(c, device=dev)
+    lat = torch.empty((cfg.batch, cfg.n_q, cfg.d_latent), device=dev, dtype=dt)
+    chunk = cfg.measured_chunk
+    for ch in range(chunk):
+        lat.copy_(torch.from_numpy(inputs.direct_latents(cfg, ch)).to(dt))
+        api.mla_cache_append(c, None, None, lat, ring.cache, ring.slot_frame, cfg.first_frame(ch),
+                             api.MLA_APPEND)
+    first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, chunk)
+    q = torch.from_numpy(inputs.direct_queries(cfg, chunk)).to(device=dev, dtype=dt)
+    lat.copy_(torch.from_numpy(inputs.direct_latents(cfg, chunk)).to(dt))
+    g = torch.from_numpy(inputs.upstream_gradient(cfg, chunk, cfg.d_c)).to(device=dev, dtype=dt)
+    o_lat = torch.empty((cfg.batch, cfg.n_q, cfg.n_heads, cfg.d_c), device=dev, dtype=dt)
+    lse = torch.empty((cfg.batch, cfg.n_heads, cfg.n_q), device=dev, dtype=torch.float32)
+    ws = torch.empty(api.mla_attention_workspace_bytes(c, n_valid), device=dev, dtype=torch.uint8)
+    api.mla_attention_fwd(c, q, lat, ring.cache, ring.slot_frame, n_valid, first, None, o_lat, lse, ws)
+    d_q, d_lat, d_cache = torch.empty_like(q), torch.empty_like(lat), torch.empty_like(ring.cache)
+    bws = torch.empty(api.mla_attention_bwd_workspace_bytes(c, n_valid), device=dev,
+                      dtype=torch.uint8)
+    call = lambda: api.mla_attention_bwd(c, q, lat, ring.cache, ring.slot_frame, n_valid, first,
+                                         o_lat, lse, g, d_q, d_lat, d_cache, bws)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    steps = args.steps if args.steps_given else 5
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    with ClockSampler(local) as clk:
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record()
+            call()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    per = 2.0 * (3 * cfg.d_latent + 2 * cfg.d_c)
+    flops = per * cfg.n_q * cfg.keys_per_query(chunk) * cfg.n_heads * cfg.batch
+    peaks, peak_kind = load_peaks()
+    value = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "MLA attention backward TFLOP/s (Wan-1.3B shape)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "call": "mla_attention_bwd", "batch": cfg.batch,
+                   "n_q": cfg.n_q, "keys_per_query": cfg.keys_per_query(chunk),
+                   "flop_per_row_key_head": per,
+                   "l2": "flushed before every call (256 MiB memset outside the event intervals)"},
+        "roofline": {"bound": "tensor", "achieved": value, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": value / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "mla_attention_bwd (" + ("tensor-core" if api.mla_attention_uses_tensor_cores(c, False) and cfg.d_c == 192 and cfg.d_rope == 32 and cfg.n_q % 4 == 0 else "CUDA-core") + " kernels)",
+                     "peak_kind": f"{peak_kind} burst bf16"},
+        "e2e": None, "gpu_launches": 5 * steps, "clocks": clk.summary()}), flush=True)
+    return 0
+
+
 def kernel_sha() -> str:
     import hashlib
     h = hashlib.sha256()
@@ -531,6 +601,8 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=192)
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the attention backward call instead of the forward step")
     ap.add_argument("--d-c", type=int, default=None,
                     help="content-latent width (latent-size ablation shapes; default: the preset's)")
     ap.add_argument("--d-rope", type=int, default=None,
@@ -547,6 +619,8 @@ def main(argv=None):
         cfg = inputs.with_latent_shape(cfg, args.d_c or cfg.d_c, args.d_rope or cfg.d_rope)
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.backward:
+        return run_backward(args, cfg)
     if cfg.n_layers > 1:
         return run_stack(args, cfg)
     return run_ours(args, cfg)

@@ -345,8 +345,13 @@ mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q
  *                                         may be NULL when n_valid_frames == 0
  *   workspace device scratch of >= mla_attention_bwd_workspace_bytes(cfg, n_valid_frames)
  *             bytes, 256-byte aligned; contents on entry do not matter
- * Probabilities are recomputed from q, the keys and lse (fp32).  Errors: MLA_ERR_INVALID_ARG,
- * MLA_ERR_ALIGNMENT, MLA_ERR_WORKSPACE, MLA_ERR_UNSUPPORTED (d_c + d_rope > 512), MLA_ERR_CUDA.
+ *   dev_status device int32 word or NULL, as in mla_attention_fwd (bounded waits of the
+ *             tensor-core kernels)
+ * Probabilities are recomputed from q, the keys and lse.  bf16 with d_c 192, d_rope 32 and n_q a
+ * multiple of 4 runs on the tensor cores (P and dS rounded to bf16 as MMA operands, fp32
+ * accumulation); other shapes, fp32 and MLA_PATH_SIMT on CUDA cores in fp32.  Errors:
+ * MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_WORKSPACE, MLA_ERR_UNSUPPORTED
+ * (d_c + d_rope > 512), MLA_ERR_CUDA.
  * ------------------------------------------------------------------------------------------ */
 size_t mla_attention_bwd_workspace_bytes(const mla_config* cfg, int32_t n_valid_frames);
 mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* chunk_lat,
@@ -354,7 +359,7 @@ mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* c
                              int32_t n_valid_frames, int32_t first_frame, const void* o_lat,
                              const float* lse, const void* d_o_lat, void* d_q,
                              void* d_chunk_lat, void* d_cache, void* workspace,
-                             size_t workspace_bytes, void* stream);
+                             size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /* --------------------------------------------------------------------------------------------
  * mla_out_proj: value up-projection of latent outputs and the optional output projection

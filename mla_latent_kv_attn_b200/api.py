@@ -208,7 +208,7 @@ def mla_attention_bwd_workspace_bytes(c: MLAConfigC, n_valid_frames: int) -> int
 
 def mla_attention_bwd(c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_frames: int,
                       first_frame: int, o_lat, lse, d_o_lat, d_q, d_chunk_lat, d_cache, workspace,
-                      stream=None) -> None:
+                      dev_status=None, stream=None) -> None:
     """Gradients of the latent attention call (see include/mla.h)."""
     tpf, n_q, D = _geom(c)
     dt = torch_dtype(c)
@@ -222,7 +222,7 @@ def mla_attention_bwd(c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_fr
         _ptr(lse, "lse", torch.float32, (B, H, n_q)), _ptr(d_o_lat, "d_o_lat", dt, (B, n_q, H, c.d_c)),
         _ptr(d_q, "d_q", dt, (B, n_q, H, D)), _ptr(d_chunk_lat, "d_chunk_lat", dt, (B, n_q, D)),
         _ptr(d_cache, "d_cache", dt, (B, c.window_frames * tpf, D)), _ptr(workspace, "workspace"),
-        ws_bytes, _stream(stream))
+        ws_bytes, _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     _lib.check("mla_attention_bwd", st)
 
 

@@ -11,7 +11,8 @@
 //   d latent_m = [dV_m + dK'_m[0:d_c]  ||  RoPE3D^T(dK'_m[d_c:])]
 // (the transpose of a rotation is the rotation by the opposite angle).
 //
-// CUDA-core kernels, all fp32 arithmetic, no atomics:
+// CUDA-core kernels (the tensor-core path for the Wan shape is attention_bwd_sm100.cu; both use
+// bwd_delta_kernel), all fp32 arithmetic, no atomics:
 //   bwd_delta_kernel   one warp per (b, n, h): Delta = G . O_lat
 //   bwd_dq_kernel      one warp per (b, h, n): loop over the keys
 //   bwd_dkey_kernel    one warp per (b, key): loop over every head and query row
@@ -193,10 +194,15 @@ __global__ void __launch_bounds__(128)
 }
 
 template <typename T>
-mla_status launch_bwd(const BwdParams& p, cudaStream_t s) {
+mla_status launch_delta(const BwdParams& p, cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(p.B) * p.n_q * p.H;
   bwd_delta_kernel<T><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, s>>>(p);
   MLA_LAUNCH_CHECK("bwd_delta");
+  return MLA_OK;
+}
+
+template <typename T>
+mla_status launch_bwd_simt(const BwdParams& p, cudaStream_t s) {
   dim3 gq(ceil_div(p.n_q, 4), p.H, p.B);
   bwd_dq_kernel<T><<<gq, 128, 0, s>>>(p);
   MLA_LAUNCH_CHECK("bwd_dq");
@@ -212,12 +218,14 @@ BwdWorkspace bwd_workspace_layout(const Dims& d, int n_valid) {
   BwdWorkspace w;
   w.delta_bytes = static_cast<size_t>(round_up(d.B * d.H * d.n_q, 64)) * sizeof(float);
   w.keys = key_workspace_layout(d, n_valid);
-  w.bytes = w.delta_bytes + w.keys.bytes;
+  w.groups = tc_bwd_supported(d) ? bwd_tc_head_groups(d, n_valid) : 0;
+  w.partial_bytes = static_cast<size_t>(w.groups) * d.B * w.keys.rows * d.D * sizeof(float);
+  w.bytes = w.delta_bytes + w.keys.bytes + w.partial_bytes;
   return w;
 }
 
 mla_status attention_bwd(const Dims& d, const BwdArgs& a, int n_valid, int first_frame,
-                         void* workspace, cudaStream_t s) {
+                         void* workspace, int32_t* dev_status, cudaStream_t s) {
   if (d.D > 32 * kLanesMax) MLA_FAIL(MLA_ERR_UNSUPPORTED, "d_c + d_rope above %d", 32 * kLanesMax);
   const BwdWorkspace w = bwd_workspace_layout(d, n_valid);
   float* delta = static_cast<float*>(workspace);
@@ -233,7 +241,14 @@ mla_status attention_bwd(const Dims& d, const BwdArgs& a, int n_valid, int first
   p.tpf = d.tpf; p.frame_w = d.frame_w; p.nc = w.keys.nc; p.nc_pad = w.keys.nc_pad;
   p.rows_ws = w.keys.rows; p.first_frame = first_frame;
   p.scale = d.scale; p.scale_log2 = d.scale * 1.4426950408889634f; p.rope = rope_geom(d);
-  return d.dtype == MLA_FP32 ? launch_bwd<float>(p, s) : launch_bwd<bf16>(p, s);
+  mla_status r = d.dtype == MLA_FP32 ? launch_delta<float>(p, s) : launch_delta<bf16>(p, s);
+  if (r != MLA_OK) return r;
+  if (w.groups > 0) {
+    float* partial = reinterpret_cast<float*>(static_cast<char*>(ws_rope) + w.keys.bytes);
+    return attention_bwd_tc(d, a, n_valid, first_frame, delta, ws_rope, partial, w.groups,
+                            dev_status, s);
+  }
+  return d.dtype == MLA_FP32 ? launch_bwd_simt<float>(p, s) : launch_bwd_simt<bf16>(p, s);
 }
 
 }  // namespace mla

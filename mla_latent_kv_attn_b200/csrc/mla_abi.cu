@@ -436,7 +436,7 @@ mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* c
                              int32_t n_valid_frames, int32_t first_frame, const void* o_lat,
                              const float* lse, const void* d_o_lat, void* d_q,
                              void* d_chunk_lat, void* d_cache, void* workspace,
-                             size_t workspace_bytes, void* stream) {
+                             size_t workspace_bytes, int32_t* dev_status, void* stream) {
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -453,6 +453,7 @@ mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* c
   MLA_TRY(check_ptr(d_q, "d_q"));
   MLA_TRY(check_ptr(d_chunk_lat, "d_chunk_lat"));
   MLA_TRY(check_ptr(d_cache, "d_cache", n_valid_frames > 0));
+  MLA_TRY(check_ptr(dev_status, "dev_status", false));
   const BwdWorkspace w = bwd_workspace_layout(d, n_valid_frames);
   if (workspace == nullptr || workspace_bytes < w.bytes)
     MLA_FAIL(MLA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes,
@@ -463,7 +464,7 @@ mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* c
   BwdArgs a{};
   a.q = q; a.chunk_lat = chunk_lat; a.cache = cache; a.slot_frame = slot_frame; a.o_lat = o_lat;
   a.lse = lse; a.d_o_lat = d_o_lat; a.d_q = d_q; a.d_chunk_lat = d_chunk_lat; a.d_cache = d_cache;
-  return attention_bwd(d, a, n_valid_frames, first_frame, workspace,
+  return attention_bwd(d, a, n_valid_frames, first_frame, workspace, dev_status,
                        static_cast<cudaStream_t>(stream));
 }
 

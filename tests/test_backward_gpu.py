@@ -81,7 +81,10 @@ def test_backward_toy_fp32_wrapped_ring():
     _run(cfg, chunk=3)          # window of 2 frames after 3 one-frame chunks: wrapped
 
 
+@pytest.mark.parametrize("path", ["tc", "simt"])
 @pytest.mark.parametrize("chunk", [0, 3])
-def test_backward_small_frames_bf16(chunk):
-    """Wan widths on 6x10 frames, 12 heads: chunk 0 (no ring) and chunk 3 (ring wrapped)."""
-    _run(inputs.small_bf16_config(), chunk=chunk)
+def test_backward_small_frames_bf16(chunk, path):
+    """Wan widths on 6x10 frames, 12 heads: chunk 0 (no ring) and chunk 3 (ring wrapped), on
+    the tensor-core kernels and on the CUDA-core kernels."""
+    _run(inputs.small_bf16_config(), chunk=chunk,
+         path=api.MLA_PATH_AUTO if path == "tc" else api.MLA_PATH_SIMT)
