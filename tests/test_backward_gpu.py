@@ -88,3 +88,68 @@ def test_backward_small_frames_bf16(chunk, path):
     the tensor-core kernels and on the CUDA-core kernels."""
     _run(inputs.small_bf16_config(), chunk=chunk,
          path=api.MLA_PATH_AUTO if path == "tc" else api.MLA_PATH_SIMT)
+
+
+def test_backward_wan_config1_full_size():
+    """The Wan preset at full size on the tensor-core backward (4680 queries, 14,040 keys, 12
+    heads).  dq on 64 sampled rows against the oracle (rows are independent given the keys); the
+    key gradients through identities that hold at any size, since every row's probabilities sum
+    to one (so every row's dS sums to zero): summed over all keys, the content gradients equal
+    the summed upstream gradient and the positional ones, rotated back to the keys' frames, sum
+    to zero."""
+    cfg = inputs.CONFIGS[1]
+    c = api.make_config(cfg)
+    dt = api.torch_dtype(c)
+    dev = torch.device("cuda")
+    ring = rollout.Ring(c)
+    d = oracle.dims_from(cfg)
+    chunk = cfg.measured_chunk
+    lat_buf = torch.empty((1, cfg.n_q, cfg.d_latent), device=dev, dtype=dt)
+    recs = {}
+    for ch in range(chunk):
+        lat = inputs.direct_latents(cfg, ch)
+        lat_buf.copy_(torch.from_numpy(lat).to(dt))
+        api.mla_cache_append(c, None, None, lat_buf, ring.cache, ring.slot_frame,
+                             cfg.first_frame(ch), api.MLA_APPEND)
+        tpf = cfg.tokens_per_frame
+        for f in range(cfg.chunk_frames):
+            recs[cfg.first_frame(ch) + f] = lat[0][f * tpf:(f + 1) * tpf]
+    first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, chunk)
+    q_np = inputs.direct_queries(cfg, chunk)
+    lat_np = inputs.direct_latents(cfg, chunk)
+    g_np = inputs.upstream_gradient(cfg, chunk, cfg.d_c)
+    q = torch.from_numpy(q_np).to(device=dev, dtype=dt)
+    lat_buf.copy_(torch.from_numpy(lat_np).to(dt))
+    g = torch.from_numpy(g_np).to(device=dev, dtype=dt)
+    o_lat = torch.empty((1, cfg.n_q, cfg.n_heads, cfg.d_c), device=dev, dtype=dt)
+    lse = torch.empty((1, cfg.n_heads, cfg.n_q), device=dev, dtype=torch.float32)
+    ws = torch.empty(api.mla_attention_workspace_bytes(c, n_valid), device=dev, dtype=torch.uint8)
+    api.mla_attention_fwd(c, q, lat_buf, ring.cache, ring.slot_frame, n_valid, first, None, o_lat,
+                          lse, ws)
+    d_q, d_lat, d_cache = torch.empty_like(q), torch.empty_like(lat_buf), torch.empty_like(ring.cache)
+    status = torch.zeros(1, device=dev, dtype=torch.int32)
+    bws = torch.empty(api.mla_attention_bwd_workspace_bytes(c, n_valid), device=dev,
+                      dtype=torch.uint8)
+    api.mla_attention_bwd(c, q, lat_buf, ring.cache, ring.slot_frame, n_valid, first, o_lat, lse, g,
+                          d_q, d_lat, d_cache, bws, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    slots = ring.slot_frame.cpu().numpy()[0][:n_valid]
+    tpf = cfg.tokens_per_frame
+    c_ring = np.concatenate([recs[t][:, :cfg.d_c] for t in slots])
+    k_ring = np.concatenate([recs[t][:, cfg.d_c:] for t in slots])
+    pos_k = np.concatenate([oracle.token_positions(list(slots), d),
+                            oracle.token_positions(range(first, first + cfg.chunk_frames), d)])
+    rows = inputs.sample_rows(cfg.n_q, 64, tag=21)
+    ref = oracle.latent_attention_backward(
+        q_np[0][rows], np.concatenate([c_ring, lat_np[0][:, :cfg.d_c]]),
+        np.concatenate([k_ring, lat_np[0][:, cfg.d_c:]]), pos_k, g_np[0][rows], d)
+    compare("cfg1.d_q", to_np(d_q)[0][rows], ref["d_q"], "bf16")
+    nc = n_valid * tpf
+    grads = np.concatenate([to_np(d_cache)[0][:nc], to_np(d_lat)[0]])       # [keys, D]
+    content_sum = grads[:, :cfg.d_c].sum(axis=0)
+    expect = g_np[0].astype(np.float64).sum(axis=(0, 1))
+    assert np.linalg.norm(content_sum - expect) <= 2e-2 * np.linalg.norm(expect)
+    rope_back = oracle.rope3d(grads[:, cfg.d_c:], pos_k, d).sum(axis=0)
+    scale_ref = np.abs(grads[:, cfg.d_c:]).sum(axis=0)
+    assert (np.abs(rope_back) <= 2e-2 * scale_ref + 1e-3).all()
