@@ -3,25 +3,27 @@
 // products are tcgen05 MMAs with fp32 accumulators in TMEM and bf16 operands (P and dS are
 // rounded to bf16 as MMA operands; the softmax statistics stay fp32).
 //
-// dQ kernel: one CTA per (128-row query tile, head, sample); the key tiles stream through a
-// 2-stage ring.  Per key tile j:
-//   S   = Q' K'_j^T        M128 N128 K224   (A: Q' smem, B: K'_j smem, both K-major)
-//   dP  = G  V_j^T         M128 N128 K192   (A: G smem, B: content blocks of K'_j, K-major)
-//   dS  = scale * P o (dP - Delta), P = exp(S scale - lse)  (softmax warps, bf16 into TMEM)
-//   dQ += dS K'_j          M128 N192 + N32  K128 (A: dS in TMEM, B: K'_j read MN-major)
-// Key kernel: one CTA per (128-key tile, group of heads, sample); for every (head, query tile)
-// of its group:
-//   S^T  = K' Q'^T         M128 N128 K224
-//   dP^T = V G^T           M128 N128 K192
-//   P^T, dS^T (scaled)     softmax warps, one key row per thread, lse/Delta per query column
-//   dL  += P^T G           M128 N192 K128   (value gradient: the value is the content latent)
-//   dL  += dS^T Q'         M128 N192 + N32 K128 (key gradient, content and positional parts)
+// Both kernels own a 128-row tile and stream 64-row sub-tiles of the other side through a ring
+// of shared-memory stages; S and dP of a sub-tile are double-buffered in TMEM, so the softmax of
+// sub-tile i runs while the MMAs of sub-tile i+1 do.
+// dQ kernel: one CTA per (128-row query tile, head, sample); per 64-key sub-tile j:
+//   S_j  = Q' K'_j^T       M128 N64 K224    (A: Q' smem, B: K'_j smem, both K-major)
+//   dP_j = G  V_j^T        M128 N64 K192    (A: G smem, B: content blocks of K'_j, K-major)
+//   dS_j = scale * P o (dP - Delta), P = exp(S scale - lse)    (softmax warps, bf16 into TMEM)
+//   dQ  += dS_j K'_j       M128 N192 + N32 K64 (A: dS in TMEM, B: K'_j read MN-major)
+// Key kernel: one CTA per (128-key tile, group of heads, sample); per (head, 64-query sub-tile):
+//   S^T  = K' Q'_i^T       M128 N64 K224
+//   dP^T = V  G_i^T        M128 N64 K192
+//   P^T, scale * dS^T      softmax warps, one key row per thread, lse/Delta per query column
+//   dL  += P^T G_i         M128 N192 K64    (value gradient: the value is the content latent)
+//   dL  += dS^T Q'_i       M128 N192 + N32 K64 (key gradient, content and positional parts)
 // dL (fp32, 224 wide) goes to a workspace slice per head group; bwd_reduce_kernel sums the
 // groups, maps the positional part back through the transposed rotation and stores bf16.
-// TMEM columns: S [0,128), dP [128,256), accumulator [256,480); P^T / dS are written over the
-// first 64 columns of S and of dP.  Roles (192 threads): warps 0-3 softmax and epilogue (one
-// TMEM lane = one row), warp 4 TMA producer, warp 5 TMEM allocation and the MMA thread.  Every
-// wait is bounded; a wait that runs out writes MLA_ERR_DEVICE_TIMEOUT to dev_status.
+// TMEM columns: S buffers [0,64) [64,128), dP buffers [128,192) [192,256), accumulator
+// [256,480); P / dS (bf16, 32 columns) are written over the first columns of their buffers.
+// Roles (192 threads): warps 0-3 softmax and epilogue (one TMEM lane = one row), warp 4 TMA
+// producer, warp 5 TMEM allocation and the MMA thread.  Every wait is bounded; a wait that runs
+// out writes MLA_ERR_DEVICE_TIMEOUT to dev_status.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -31,25 +33,31 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kR = 128;                     // rows of every tile (queries or keys)
+constexpr int kR = 128;                     // rows of the tile a CTA owns
+constexpr int kS = 64;                      // rows of a streamed sub-tile
 constexpr int kDc = 192, kDr = 32, kD = 224;
-constexpr int kBlk = kR * 128;              // 16 KB: 128 rows x 128 B (64 bf16), 128B swizzle
-constexpr int kRopeBlk = kR * 64;           // 8 KB: 128 rows x 64 B (32 bf16), 64B swizzle
-constexpr int kTileD = 3 * kBlk + kRopeBlk; // 56 KB: a 128 x 224 tile (Q' or K')
-constexpr int kTileG = 3 * kBlk;            // 48 KB: a 128 x 192 tile (G)
+constexpr int kBlkR = kR * 128;             // 16 KB: 128 rows x 128 B (64 bf16), 128B swizzle
+constexpr int kBlkS = kS * 128;             // 8 KB:  64 rows x 128 B
+constexpr int kTileR = 3 * kBlkR + kR * 64; // 56 KB: a 128 x 224 tile (content + 64B-swizzled rope)
+constexpr int kTileGR = 3 * kBlkR;          // 48 KB: a 128 x 192 tile of G
+constexpr int kTileS = 3 * kBlkS + kS * 64; // 28 KB: a 64 x 224 sub-tile
+constexpr int kTileGS = 3 * kBlkS;          // 24 KB: a 64 x 192 sub-tile of G
 constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr int kProducerWarp = 4, kMmaWarp = 5;
 constexpr int kSoftmaxThreads = 128;
-constexpr int kQStages = 2;                 // dQ kernel: K' ring
-constexpr int kSmemQ = kTileD + kTileG + kQStages * kTileD + 1024;
-constexpr int kStats = 2 * kR * 4;          // lse and Delta of a query tile: 1 KB
-constexpr int kSmemK = kTileD + kTileD + kTileG + kStats + 1024;   // K' + one (Q', G) stage
+constexpr int kQStages = 4;                                        // dQ kernel: K' sub-tiles
+constexpr int kSmemQ = kTileR + kTileGR + kQStages * kTileS + 1024;
+constexpr int kKStage = kTileS + kTileGS + 1024;                   // Q' + G sub-tiles + stats
+constexpr int kKStages = 3;
+constexpr int kSmemK = kTileR + kKStages * kKStage + 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdTcParams {
-  int n_q, H, nc, nc_pad, nt_ring, nt, rows_ws, heads_per_group, n_qt;
+  int n_q, H, nc, nc_pad, nt_ring, nt, rows_ws, heads_per_group;
+  int ns_ring, ns;          // dQ kernel: 64-key sub-tiles of the ring, in all
+  int n_qs;                 // key kernel: 64-query sub-tiles per head
   float scale, scale_log2;
   const float* lse;      // [B, H, n_q]
   const float* delta;    // [B, H, n_q]
@@ -64,64 +72,67 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// K-major tile operand (content blocks, 128B swizzle) and its positional block (64B swizzle).
+// Descriptors of a tile's blocks.  K-major (rows = M or N, K = columns): 8-row atoms, SBO 1024
+// (content, 128B swizzle) or 512 (rope, 64B swizzle).  MN-major (N = columns, K = rows): atoms of
+// 64 (content) or 32 (rope) columns x 8 rows; LBO = stride between column blocks, SBO = stride
+// between 8-row groups.
 __device__ __forceinline__ uint64_t kmajor_content(uint32_t a) {
   return smem_desc(a, 16, 1024, kSwizzle128B);
 }
 __device__ __forceinline__ uint64_t kmajor_rope(uint32_t a) {
   return smem_desc(a, 16, 512, kSwizzle64B);
 }
-// The same blocks read MN-major (N = columns of the tile, K = its rows): atoms of 64 (resp. 32)
-// columns x 8 rows; LBO = stride between column blocks, SBO = stride between 8-row groups.
-__device__ __forceinline__ uint64_t mnmajor_content(uint32_t a) {
-  return smem_desc(a, kBlk, 1024, kSwizzle128B);
+__device__ __forceinline__ uint64_t mnmajor_content(uint32_t a, uint32_t blk_bytes) {
+  return smem_desc(a, blk_bytes, 1024, kSwizzle128B);
 }
 __device__ __forceinline__ uint64_t mnmajor_rope(uint32_t a) {
-  return smem_desc(a, kRopeBlk, 512, kSwizzle64B);
+  return smem_desc(a, 4096, 512, kSwizzle64B);
 }
 
-constexpr uint32_t kIdescNN = idesc_bf16_f32(kR, 128, 0, 0);   // S, dP (both K-major)
+constexpr uint32_t kIdescS = idesc_bf16_f32(kR, kS, 0, 0);     // S, dP: M128 N64, K-major
 constexpr uint32_t kIdescC = idesc_bf16_f32(kR, kDc, 0, 1);    // A TMEM, B MN-major, N 192
 constexpr uint32_t kIdescR = idesc_bf16_f32(kR, kDr, 0, 1);    // A TMEM, B MN-major, N 32
-constexpr uint32_t kBlkD = kBlk >> 4;
 
-// D = A B^T over a 224-wide K (12 content k-steps + 2 positional ones); A, B tile bases.
-__device__ __forceinline__ void mma_k224(uint32_t d, uint32_t a_tile, uint32_t b_tile) {
+// D = A B^T over K = 224 (12 content k-steps + 2 positional); a_blk / b_blk: byte stride of the
+// 64-column content blocks of A / B (their rope block follows the third).
+__device__ __forceinline__ void mma_k224(uint32_t d, uint32_t a_tile, uint32_t a_blk,
+                                         uint32_t b_tile, uint32_t b_blk) {
   const uint64_t ac = kmajor_content(a_tile), bc = kmajor_content(b_tile);
-  const uint64_t ar = kmajor_rope(a_tile + 3 * kBlk), br = kmajor_rope(b_tile + 3 * kBlk);
+  const uint64_t ar = kmajor_rope(a_tile + 3 * a_blk), br = kmajor_rope(b_tile + 3 * b_blk);
 #pragma unroll
   for (int blk = 0; blk < 3; ++blk)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_ss(d, ac + (blk * kBlkD + 2 * kk), bc + (blk * kBlkD + 2 * kk), kIdescNN,
+      mma_ss(d, ac + ((blk * a_blk) >> 4) + 2 * kk, bc + ((blk * b_blk) >> 4) + 2 * kk, kIdescS,
              (blk | kk) != 0 ? 1u : 0u);
 #pragma unroll
-  for (int kk = 0; kk < 2; ++kk) mma_ss(d, ar + 2 * kk, br + 2 * kk, kIdescNN, 1u);
+  for (int kk = 0; kk < 2; ++kk) mma_ss(d, ar + 2 * kk, br + 2 * kk, kIdescS, 1u);
 }
 
 // D = A B^T over the 192 content columns only.
-__device__ __forceinline__ void mma_k192(uint32_t d, uint32_t a_tile, uint32_t b_tile) {
+__device__ __forceinline__ void mma_k192(uint32_t d, uint32_t a_tile, uint32_t a_blk,
+                                         uint32_t b_tile, uint32_t b_blk) {
   const uint64_t ac = kmajor_content(a_tile), bc = kmajor_content(b_tile);
 #pragma unroll
   for (int blk = 0; blk < 3; ++blk)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_ss(d, ac + (blk * kBlkD + 2 * kk), bc + (blk * kBlkD + 2 * kk), kIdescNN,
+      mma_ss(d, ac + ((blk * a_blk) >> 4) + 2 * kk, bc + ((blk * b_blk) >> 4) + 2 * kk, kIdescS,
              (blk | kk) != 0 ? 1u : 0u);
 }
 
-// acc[:, 0:192] (+)= A_tmem (128 x 128, bf16) . tile[:, 0:192]; with_rope: also
-// acc[:, 192:224] (+)= A_tmem . tile[:, 192:224].  K = the tile's 128 rows.
-__device__ __forceinline__ void mma_tmem_by_tile(uint32_t acc, uint32_t a_tmem, uint32_t tile,
-                                                 bool with_rope, bool accumulate) {
-  const uint64_t bc = mnmajor_content(tile);
-  const uint64_t br = mnmajor_rope(tile + 3 * kBlk);
+// acc[:, 0:192] (+)= A_tmem (128 x 64, bf16) . sub[:, 0:192]; with_rope: also
+// acc[:, 192:224] (+)= A_tmem . sub[:, 192:224].  K = the 64 rows of the sub-tile.
+__device__ __forceinline__ void mma_tmem_by_sub(uint32_t acc, uint32_t a_tmem, uint32_t sub,
+                                                bool with_rope, bool accumulate) {
+  const uint64_t bc = mnmajor_content(sub, kBlkS);
+  const uint64_t br = mnmajor_rope(sub + 3 * kBlkS);
 #pragma unroll
-  for (int kk = 0; kk < kR / 16; ++kk) {
+  for (int kk = 0; kk < kS / 16; ++kk) {
     // 16 rows further per k-step: 2048 B (content, 128 B rows) and 1024 B (rope, 64 B rows)
     mma_ts(acc, a_tmem + kk * 8, bc + 128 * kk, kIdescC, (accumulate || kk) ? 1u : 0u);
     if (with_rope)
-      mma_ts(acc + kDc, a_tmem + kk * 8, br + 64 * kk, kIdescR, (accumulate || kk) ? 1u : 0u);
+      mma_ts(acc + kDc, a_tmem + kk * 8, br + 64 * kk, kIdescR, 1u);
   }
 }
 
@@ -137,14 +148,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t qg_full;
   __shared__ __align__(8) uint64_t kv_full[kQStages];
   __shared__ __align__(8) uint64_t kv_empty[kQStages];
-  __shared__ __align__(8) uint64_t s_full;       // S and dP of tile j are in TMEM
-  __shared__ __align__(8) uint64_t ds_full;      // the softmax has written dS(j)
-  __shared__ __align__(8) uint64_t dq_done;      // the dQ products of tile j have completed
+  __shared__ __align__(8) uint64_t s_full[2];     // S and dP of sub-tile j in TMEM buffer j&1
+  // the softmax has written dS(j) into buffer j&1; one barrier per buffer, so that a waiter is
+  // never two phases behind (sub-tile j+2 cannot start before the products of j were issued)
+  __shared__ __align__(8) uint64_t ds_full[2];
+  __shared__ __align__(8) uint64_t buf_free[2];   // the dQ products that read buffer b completed
+                                                  // (the epilogue waits for the last of them)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sQ = sbase, sG = sbase + kTileD, sK = sbase + kTileD + kTileG;
+  const uint32_t sQ = sbase, sG = sbase + kTileR, sK = sbase + kTileR + kTileGR;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int q0 = qt * kR;
@@ -157,9 +171,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&kv_full[s]), 1);
       mbar_init(smem_u32(&kv_empty[s]), 1);
     }
-    mbar_init(smem_u32(&s_full), 1);
-    mbar_init(smem_u32(&ds_full), kSoftmaxThreads);
-    mbar_init(smem_u32(&dq_done), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&buf_free[i]), 1);
+    }
+    mbar_init(smem_u32(&ds_full[0]), kSoftmaxThreads);
+    mbar_init(smem_u32(&ds_full[1]), kSoftmaxThreads);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -174,52 +191,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp) {
     if (lane == 0) {
       const uint32_t qb = smem_u32(&qg_full);
-      mbar_arrive_expect_tx(qb, kTileD + kTileG);
-      for (int i = 0; i < 3; ++i) tma_load_4d(sQ + i * kBlk, &tm_q, qb, 64 * i, h, q0, b);
-      tma_load_4d(sQ + 3 * kBlk, &tm_qr, qb, kDc, h, q0, b);
-      for (int i = 0; i < 3; ++i) tma_load_4d(sG + i * kBlk, &tm_g, qb, 64 * i, h, q0, b);
+      mbar_arrive_expect_tx(qb, kTileR + kTileGR);
+      for (int i = 0; i < 3; ++i) tma_load_4d(sQ + i * kBlkR, &tm_q, qb, 64 * i, h, q0, b);
+      tma_load_4d(sQ + 3 * kBlkR, &tm_qr, qb, kDc, h, q0, b);
+      for (int i = 0; i < 3; ++i) tma_load_4d(sG + i * kBlkR, &tm_g, qb, 64 * i, h, q0, b);
       bool ok = true;
-      for (int j = 0; j < p.nt && ok; ++j) {
+      for (int j = 0; j < p.ns && ok; ++j) {
         const int s = j % kQStages;
         ok = mbar_wait_or_abort(smem_u32(&kv_empty[s]), ((j / kQStages) & 1) ^ 1, abort_flag,
                                 p.dev_status);
         if (!ok) break;
-        const uint32_t dst = sK + s * kTileD;
+        const uint32_t dst = sK + s * kTileS;
         const uint32_t fb = smem_u32(&kv_full[s]);
-        mbar_arrive_expect_tx(fb, kTileD);
-        if (j < p.nt_ring) {
-          const int r0 = j * kR;
-          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlk, &tm_cache, fb, 64 * i, r0, b);
-          tma_load_3d(dst + 3 * kBlk, &tm_ws, fb, 0, r0, b);
+        mbar_arrive_expect_tx(fb, kTileS);
+        if (j < p.ns_ring) {
+          const int r0 = j * kS;
+          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlkS, &tm_cache, fb, 64 * i, r0, b);
+          tma_load_3d(dst + 3 * kBlkS, &tm_ws, fb, 0, r0, b);
         } else {
-          const int r0 = (j - p.nt_ring) * kR;
-          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlk, &tm_chunk, fb, 64 * i, r0, b);
-          tma_load_3d(dst + 3 * kBlk, &tm_ws, fb, 0, p.nc_pad + r0, b);
+          const int r0 = (j - p.ns_ring) * kS;
+          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlkS, &tm_chunk, fb, 64 * i, r0, b);
+          tma_load_3d(dst + 3 * kBlkS, &tm_ws, fb, 0, p.nc_pad + r0, b);
         }
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
+      // Order of issue: S/dP(j) into buffer j&1, then the dQ products of sub-tile j-1 (whose dS
+      // the softmax wrote meanwhile), so the softmax of j-1 overlaps the products of j.
       bool ok = mbar_wait_or_abort(smem_u32(&qg_full), 0, abort_flag, p.dev_status);
-      for (int j = 0; j < p.nt && ok; ++j) {
-        const int s = j % kQStages;
-        ok = mbar_wait_or_abort(smem_u32(&kv_full[s]), (j / kQStages) & 1, abort_flag,
-                                p.dev_status);
-        // dS(j-1) sits in the S columns: its dQ products must have read it
-        if (ok && j > 0)
-          ok = mbar_wait_or_abort(smem_u32(&dq_done), (j - 1) & 1, abort_flag, p.dev_status);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kt = sK + s * kTileD;
-        mma_k224(tmem + kColS, sQ, kt);
-        mma_k192(tmem + kColDP, sG, kt);
-        mma_commit(smem_u32(&s_full));
-        ok = mbar_wait_or_abort(smem_u32(&ds_full), j & 1, abort_flag, p.dev_status);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tmem_by_tile(tmem + kColAcc, tmem + kColS, kt, true, j > 0);
-        mma_commit(smem_u32(&kv_empty[s]));
-        mma_commit(smem_u32(&dq_done));
+      for (int j = 0; j <= p.ns && ok; ++j) {
+        if (j < p.ns) {
+          const int s = j % kQStages, buf = j & 1;
+          // S(j) overwrites the buffer whose dS(j-2) the dQ products of j-2 read: those were
+          // issued earlier by this thread, and MMAs of one thread run in issue order
+          ok = mbar_wait_or_abort(smem_u32(&kv_full[s]), (j / kQStages) & 1, abort_flag,
+                                  p.dev_status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kt = sK + s * kTileS;
+          mma_k224(tmem + kColS + 64 * buf, sQ, kBlkR, kt, kBlkS);
+          mma_k192(tmem + kColDP + 64 * buf, sG, kBlkR, kt, kBlkS);
+          mma_commit(smem_u32(&s_full[buf]));
+        }
+        if (j >= 1) {
+          const int jp = j - 1, sp = jp % kQStages, bp = jp & 1;
+          ok = mbar_wait_or_abort(smem_u32(&ds_full[bp]), (jp >> 1) & 1, abort_flag,
+                                  p.dev_status);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tmem_by_sub(tmem + kColAcc, tmem + kColS + 64 * bp, sK + sp * kTileS, true, jp > 0);
+          mma_commit(smem_u32(&kv_empty[sp]));
+          mma_commit(smem_u32(&buf_free[bp]));
+        }
       }
     }
   } else {
@@ -231,49 +255,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t sr = (static_cast<int64_t>(b) * p.H + h) * p.n_q + n;
     const float lse2 = row_ok ? p.lse[sr] * kLog2e : INFINITY;   // invalid rows: p = 0
     const float delta = row_ok ? p.delta[sr] : 0.f;
+    // the dQ positional columns start with the first sub-tile's products, which accumulate:
+    // zero them first (the content columns are initialised by the first product)
+    {
+      uint32_t z[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) z[i] = 0u;
+      tmem_st16(tmem + lane_off + kColAcc + kDc, z);
+      tmem_st16(tmem + lane_off + kColAcc + kDc + 16, z);
+      tmem_wait_st();
+    }
     bool ok = true;
-    for (int j = 0; j < p.nt && ok; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&s_full), j & 1, abort_flag,
-                                                      p.dev_status));
+    for (int j = 0; j < p.ns && ok; ++j) {
+      const int buf = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&s_full[buf]), (j >> 1) & 1,
+                                                      abort_flag, p.dev_status));
       if (!ok) break;
       tc_fence_after();
-      const int valid = j < p.nt_ring ? min(kR, p.nc - j * kR)
-                                      : min(kR, p.n_q - (j - p.nt_ring) * kR);
-      // two halves of 64 keys; dS of half k goes to S columns [32k, 32k + 32), which hold
-      // scores that have been read already
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        uint32_t rs[64], rp[64];
-        tmem_ld64_wait(tmem + lane_off + kColS + 64 * half, rs);
-        tmem_ld64_wait(tmem + lane_off + kColDP + 64 * half, rp);
-        uint32_t w[32];
+      const int valid = j < p.ns_ring ? min(kS, p.nc - j * kS)
+                                      : min(kS, p.n_q - (j - p.ns_ring) * kS);
+      uint32_t rs[64], rp[64];
+      tmem_ld64_wait(tmem + lane_off + kColS + 64 * buf, rs);
+      tmem_ld64_wait(tmem + lane_off + kColDP + 64 * buf, rp);
+      uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float d2[2];
+      for (int i = 0; i < 32; ++i) {
+        float d2[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 2 * i + u;
-            const float pr = 64 * half + c < valid
-                ? fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 - lse2) : 0.f;
-            d2[u] = pr * (__uint_as_float(rp[c]) - delta) * p.scale;
-          }
-          w[i] = pack_bf16x2(d2[0], d2[1]);
+        for (int u = 0; u < 2; ++u) {
+          const int c = 2 * i + u;
+          const float pr = c < valid ? fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 - lse2) : 0.f;
+          d2[u] = pr * (__uint_as_float(rp[c]) - delta) * p.scale;
         }
-#pragma unroll
-        for (int c = 0; c < 32; c += 16) {
-          uint32_t w16[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) w16[i] = w[c + i];
-          tmem_st16(tmem + lane_off + kColS + 32 * half + c, w16);
-        }
-        tmem_wait_st();
+        w[i] = pack_bf16x2(d2[0], d2[1]);
       }
+#pragma unroll
+      for (int c = 0; c < 32; c += 16) {
+        uint32_t w16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w16[i] = w[c + i];
+        tmem_st16(tmem + lane_off + kColS + 64 * buf + c, w16);
+      }
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&ds_full));
+      mbar_arrive(smem_u32(&ds_full[buf]));
     }
+    // the last dQ products completed: buffer (ns-1)&1 was freed for the ((ns-1)>>1)-th time
     if (ok)
-      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&dq_done), (p.nt - 1) & 1,
-                                                      abort_flag, p.dev_status));
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&buf_free[(p.ns - 1) & 1]),
+                                                      ((p.ns - 1) >> 1) & 1, abort_flag,
+                                                      p.dev_status));
     if (ok) {
       tc_fence_after();
       bf16* out = static_cast<bf16*>(p.d_q) + ((static_cast<int64_t>(b) * p.n_q + n) * p.H + h) * kD;
@@ -310,32 +341,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_ws, BwdTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t k_full;
-  __shared__ __align__(8) uint64_t qg_full;     // Q'(i), G(i) landed
-  __shared__ __align__(8) uint64_t qg_empty;    // the products of iteration i have read them
-  __shared__ __align__(8) uint64_t s_full;
-  __shared__ __align__(8) uint64_t ps_full;
-  __shared__ __align__(8) uint64_t acc_done;    // the dL products of iteration i completed
+  __shared__ __align__(8) uint64_t qg_full[kKStages];   // Q'_i, G_i and their stats landed
+  __shared__ __align__(8) uint64_t qg_empty[kKStages];  // the products of sub-tile i read them
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t ps_full[2];   // P^T, dS^T of sub-tile i in buffer i&1
+  __shared__ __align__(8) uint64_t buf_free[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sK = sbase, sQ = sbase + kTileD, sG = sbase + 2 * kTileD;
-  const uint32_t sStats = sG + kTileG;          // lse [128] then Delta [128] of the query tile
-  const float* col_lse = reinterpret_cast<const float*>(smem_raw + (sStats - smem_u32(smem_raw)));
-  const float* col_delta = col_lse + kR;
+  const uint32_t sK = sbase, sStage = sbase + kTileR;
+  // stage layout: Q' sub-tile (28 KB), G sub-tile (24 KB), lse [64] and Delta [64] (512 B)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int kt = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
-  const int n_iter = p.heads_per_group * p.n_qt;
+  const int n_iter = p.heads_per_group * p.n_qs;
   volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
     mbar_init(smem_u32(&k_full), 1);
-    mbar_init(smem_u32(&qg_full), 1);
-    mbar_init(smem_u32(&qg_empty), 1);
-    mbar_init(smem_u32(&s_full), 1);
-    mbar_init(smem_u32(&ps_full), kSoftmaxThreads);
-    mbar_init(smem_u32(&acc_done), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(smem_u32(&qg_full[s]), 1);
+      mbar_init(smem_u32(&qg_empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&buf_free[i]), 1);
+    }
+    mbar_init(smem_u32(&ps_full[0]), kSoftmaxThreads);
+    mbar_init(smem_u32(&ps_full[1]), kSoftmaxThreads);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -350,58 +384,69 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp) {
     if (lane == 0) {
       const uint32_t kb = smem_u32(&k_full);
-      mbar_arrive_expect_tx(kb, kTileD);
+      mbar_arrive_expect_tx(kb, kTileR);
       if (kt < p.nt_ring) {
         const int r0 = kt * kR;
-        for (int i = 0; i < 3; ++i) tma_load_3d(sK + i * kBlk, &tm_cache, kb, 64 * i, r0, b);
-        tma_load_3d(sK + 3 * kBlk, &tm_ws, kb, 0, r0, b);
+        for (int i = 0; i < 3; ++i) tma_load_3d(sK + i * kBlkR, &tm_cache, kb, 64 * i, r0, b);
+        tma_load_3d(sK + 3 * kBlkR, &tm_ws, kb, 0, r0, b);
       } else {
         const int r0 = (kt - p.nt_ring) * kR;
-        for (int i = 0; i < 3; ++i) tma_load_3d(sK + i * kBlk, &tm_chunk, kb, 64 * i, r0, b);
-        tma_load_3d(sK + 3 * kBlk, &tm_ws, kb, 0, p.nc_pad + r0, b);
+        for (int i = 0; i < 3; ++i) tma_load_3d(sK + i * kBlkR, &tm_chunk, kb, 64 * i, r0, b);
+        tma_load_3d(sK + 3 * kBlkR, &tm_ws, kb, 0, p.nc_pad + r0, b);
       }
       bool ok = true;
       for (int it = 0; it < n_iter && ok; ++it) {
-        ok = mbar_wait_or_abort(smem_u32(&qg_empty), (it & 1) ^ 1, abort_flag, p.dev_status);
+        const int s = it % kKStages;
+        ok = mbar_wait_or_abort(smem_u32(&qg_empty[s]), ((it / kKStages) & 1) ^ 1, abort_flag,
+                                p.dev_status);
         if (!ok) break;
-        const int h = grp * p.heads_per_group + it / p.n_qt;
-        const int q0 = (it % p.n_qt) * kR;
-        // column statistics of the query tile: n_q is a multiple of 4, so both the source
-        // (row (b, h) of [B, H, n_q] floats, column q0) and the size are 16-byte multiples
-        const uint32_t stat_bytes = static_cast<uint32_t>(min(kR, p.n_q - q0)) * 4u;
+        const int h = grp * p.heads_per_group + it / p.n_qs;
+        const int q0 = (it % p.n_qs) * kS;
+        // column statistics of the sub-tile: n_q is a multiple of 4, so both the source (row
+        // (b, h) of [B, H, n_q] floats, column q0) and the size are 16-byte multiples
+        const uint32_t stat_bytes = static_cast<uint32_t>(min(kS, p.n_q - q0)) * 4u;
         const int64_t so = (static_cast<int64_t>(b) * p.H + h) * p.n_q + q0;
-        const uint32_t fb = smem_u32(&qg_full);
-        mbar_arrive_expect_tx(fb, kTileD + kTileG + 2 * stat_bytes);
-        for (int i = 0; i < 3; ++i) tma_load_4d(sQ + i * kBlk, &tm_q, fb, 64 * i, h, q0, b);
-        tma_load_4d(sQ + 3 * kBlk, &tm_qr, fb, kDc, h, q0, b);
-        for (int i = 0; i < 3; ++i) tma_load_4d(sG + i * kBlk, &tm_g, fb, 64 * i, h, q0, b);
-        bulk_load(sStats, p.lse + so, stat_bytes, fb);
-        bulk_load(sStats + kR * 4, p.delta + so, stat_bytes, fb);
+        const uint32_t st = sStage + s * kKStage;
+        const uint32_t fb = smem_u32(&qg_full[s]);
+        mbar_arrive_expect_tx(fb, kTileS + kTileGS + 2 * stat_bytes);
+        for (int i = 0; i < 3; ++i) tma_load_4d(st + i * kBlkS, &tm_q, fb, 64 * i, h, q0, b);
+        tma_load_4d(st + 3 * kBlkS, &tm_qr, fb, kDc, h, q0, b);
+        for (int i = 0; i < 3; ++i) tma_load_4d(st + kTileS + i * kBlkS, &tm_g, fb, 64 * i, h, q0, b);
+        bulk_load(st + kTileS + kTileGS, p.lse + so, stat_bytes, fb);
+        bulk_load(st + kTileS + kTileGS + 256, p.delta + so, stat_bytes, fb);
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       bool ok = mbar_wait_or_abort(smem_u32(&k_full), 0, abort_flag, p.dev_status);
-      for (int it = 0; it < n_iter && ok; ++it) {
-        ok = mbar_wait_or_abort(smem_u32(&qg_full), it & 1, abort_flag, p.dev_status);
-        // P^T(it-1) and dS^T(it-1) sit in the S and dP columns until their products completed
-        if (ok && it > 0)
-          ok = mbar_wait_or_abort(smem_u32(&acc_done), (it - 1) & 1, abort_flag, p.dev_status);
-        if (!ok) break;
-        tc_fence_after();
-        mma_k224(tmem + kColS, sK, sQ);
-        mma_k192(tmem + kColDP, sK, sG);
-        mma_commit(smem_u32(&s_full));
-        ok = mbar_wait_or_abort(smem_u32(&ps_full), it & 1, abort_flag, p.dev_status);
-        if (!ok) break;
-        tc_fence_after();
-        // value gradient P^T G into the content columns, then the key gradient dS^T Q'
-        // (the positional accumulator columns get no value term; the softmax warps zeroed them
-        // before their first arrival, so every product into them accumulates)
-        mma_tmem_by_tile(tmem + kColAcc, tmem + kColS, sG, false, it > 0);
-        mma_tmem_by_tile(tmem + kColAcc, tmem + kColDP, sQ, true, true);
-        mma_commit(smem_u32(&qg_empty));
-        mma_commit(smem_u32(&acc_done));
+      for (int it = 0; it <= n_iter && ok; ++it) {
+        if (it < n_iter) {
+          const int s = it % kKStages, buf = it & 1;
+          // S^T / dP^T(it) overwrite the buffers whose P^T / dS^T(it-2) the products of it-2
+          // read: those were issued earlier by this thread, and its MMAs run in issue order
+          ok = mbar_wait_or_abort(smem_u32(&qg_full[s]), (it / kKStages) & 1, abort_flag,
+                                  p.dev_status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t st = sStage + s * kKStage;
+          mma_k224(tmem + kColS + 64 * buf, sK, kBlkR, st, kBlkS);
+          mma_k192(tmem + kColDP + 64 * buf, sK, kBlkR, st + kTileS, kBlkS);
+          mma_commit(smem_u32(&s_full[buf]));
+        }
+        if (it >= 1) {
+          const int ip = it - 1, sp = ip % kKStages, bp = ip & 1;
+          ok = mbar_wait_or_abort(smem_u32(&ps_full[bp]), (ip >> 1) & 1, abort_flag,
+                                  p.dev_status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t st = sStage + sp * kKStage;
+          // value gradient P^T G, then the key gradient dS^T Q' (the positional accumulator
+          // columns, which get no value term, were zeroed by the softmax warps)
+          mma_tmem_by_sub(tmem + kColAcc, tmem + kColS + 64 * bp, st + kTileS, false, ip > 0);
+          mma_tmem_by_sub(tmem + kColAcc, tmem + kColDP + 64 * bp, st, true, true);
+          mma_commit(smem_u32(&qg_empty[sp]));
+          mma_commit(smem_u32(&buf_free[bp]));
+        }
       }
     }
   } else {
@@ -409,7 +454,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const bool key_ok = kt < p.nt_ring ? kt * kR + row < p.nc
                                        : (kt - p.nt_ring) * kR + row < p.n_q;
-    // the positional accumulator columns have no value term: zero them before any product
     {
       uint32_t z[16];
 #pragma unroll
@@ -420,57 +464,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
-      // S^T(it) and dP^T(it), and the column statistics that the bulk copies of qg_full(it)
+      const int s = it % kKStages, buf = it & 1;
+      // S^T and dP^T of sub-tile it, and the column statistics the bulk copies of qg_full
       // brought (observed directly: the copies complete on that barrier)
       ok = __all_sync(0xffffffffu,
-                      mbar_wait_or_abort(smem_u32(&s_full), it & 1, abort_flag, p.dev_status) &&
-                          mbar_wait_or_abort(smem_u32(&qg_full), it & 1, abort_flag, p.dev_status));
+                      mbar_wait_or_abort(smem_u32(&s_full[buf]), (it >> 1) & 1, abort_flag,
+                                         p.dev_status) &&
+                          mbar_wait_or_abort(smem_u32(&qg_full[s]), (it / kKStages) & 1,
+                                             abort_flag, p.dev_status));
       if (!ok) break;
       tc_fence_after();
-      const int q0 = (it % p.n_qt) * kR;
-      const int ncols = min(kR, p.n_q - q0);
-      // two halves of 64 query columns; P^T / dS^T of half k go to columns [32k, 32k + 32) of
-      // S / dP, which hold values that have been read already
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        uint32_t rs[64], rp[64];
-        tmem_ld64_wait(tmem + lane_off + kColS + 64 * half, rs);
-        tmem_ld64_wait(tmem + lane_off + kColDP + 64 * half, rp);
-        uint32_t wp[32], wd[32];
+      const float* col_lse = reinterpret_cast<const float*>(
+          smem_raw + (sStage + s * kKStage + kTileS + kTileGS - smem_u32(smem_raw)));
+      const float* col_delta = col_lse + 64;
+      const int ncols = min(kS, p.n_q - (it % p.n_qs) * kS);
+      uint32_t rs[64], rp[64];
+      tmem_ld64_wait(tmem + lane_off + kColS + 64 * buf, rs);
+      tmem_ld64_wait(tmem + lane_off + kColDP + 64 * buf, rp);
+      uint32_t wp[32], wd[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float pp[2], dd[2];
+      for (int i = 0; i < 32; ++i) {
+        float pp[2], dd[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 64 * half + 2 * i + u;
-            const bool col_ok = key_ok && c < ncols;
-            const float pr = col_ok ? fast_exp2(__uint_as_float(rs[2 * i + u]) * p.scale_log2 -
-                                                col_lse[c] * kLog2e)
-                                    : 0.f;
-            pp[u] = pr;
-            dd[u] = col_ok ? pr * (__uint_as_float(rp[2 * i + u]) - col_delta[c]) * p.scale : 0.f;
-          }
-          wp[i] = pack_bf16x2(pp[0], pp[1]);
-          wd[i] = pack_bf16x2(dd[0], dd[1]);
+        for (int u = 0; u < 2; ++u) {
+          const int c = 2 * i + u;
+          const bool col_ok = key_ok && c < ncols;
+          const float pr = col_ok ? fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 -
+                                              col_lse[c] * kLog2e)
+                                  : 0.f;
+          pp[u] = pr;
+          dd[u] = col_ok ? pr * (__uint_as_float(rp[c]) - col_delta[c]) * p.scale : 0.f;
         }
-#pragma unroll
-        for (int c = 0; c < 32; c += 16) {
-          uint32_t w16[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) w16[i] = wp[c + i];
-          tmem_st16(tmem + lane_off + kColS + 32 * half + c, w16);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) w16[i] = wd[c + i];
-          tmem_st16(tmem + lane_off + kColDP + 32 * half + c, w16);
-        }
-        tmem_wait_st();
+        wp[i] = pack_bf16x2(pp[0], pp[1]);
+        wd[i] = pack_bf16x2(dd[0], dd[1]);
       }
+#pragma unroll
+      for (int c = 0; c < 32; c += 16) {
+        uint32_t w16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w16[i] = wp[c + i];
+        tmem_st16(tmem + lane_off + kColS + 64 * buf + c, w16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w16[i] = wd[c + i];
+        tmem_st16(tmem + lane_off + kColDP + 64 * buf + c, w16);
+      }
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&ps_full));
+      mbar_arrive(smem_u32(&ps_full[buf]));
     }
     if (ok)
-      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&acc_done), (n_iter - 1) & 1,
-                                                      abort_flag, p.dev_status));
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&buf_free[(n_iter - 1) & 1]),
+                                                      ((n_iter - 1) >> 1) & 1, abort_flag,
+                                                      p.dev_status));
     if (ok) {
       tc_fence_after();
       const int prow = kt < p.nt_ring ? kt * kR + row : p.nc_pad + (kt - p.nt_ring) * kR + row;
@@ -556,69 +601,95 @@ bool tc_bwd_supported(const Dims& d) {
          d.n_q % 4 == 0;
 }
 
-mla_status attention_bwd_tc(const Dims& d, const BwdArgs& a, int n_valid, int first_frame,
-                            const float* delta, const void* ws_rope, float* partial, int groups,
-                            int32_t* dev_status, cudaStream_t s) {
-  const KeyWorkspace kw = key_workspace_layout(d, n_valid);
-  CUtensorMap tq, tqr, tg, tcache, tchunk, tws;
+namespace {
+
+// Tensor maps of the backward's operands with row boxes of `rows` (128 for a tile a CTA owns, 64
+// for a streamed sub-tile).
+struct BwdMaps {
+  CUtensorMap q, qr, g, cache, chunk, ws;
+};
+
+mla_status make_bwd_maps(const Dims& d, const BwdArgs& a, const KeyWorkspace& kw,
+                         const void* ws_rope, uint32_t rows, BwdMaps* m) {
   mla_status st;
   {
     const uint64_t dims[4] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.H),
                               static_cast<uint64_t>(d.n_q), static_cast<uint64_t>(d.B)};
     const uint64_t strides[3] = {kD * 2ull, static_cast<uint64_t>(d.H) * kD * 2,
                                  static_cast<uint64_t>(d.n_q) * d.H * kD * 2};
-    const uint32_t box[4] = {64, 1, kR, 1};
-    if ((st = make_tmap_bf16(&tq, a.q, 4, dims, strides, box, 128)) != MLA_OK) return st;
-    const uint32_t box_r[4] = {kDr, 1, kR, 1};
-    if ((st = make_tmap_bf16(&tqr, a.q, 4, dims, strides, box_r, 64)) != MLA_OK) return st;
+    const uint32_t box[4] = {64, 1, rows, 1};
+    if ((st = make_tmap_bf16(&m->q, a.q, 4, dims, strides, box, 128)) != MLA_OK) return st;
+    const uint32_t box_r[4] = {kDr, 1, rows, 1};
+    if ((st = make_tmap_bf16(&m->qr, a.q, 4, dims, strides, box_r, 64)) != MLA_OK) return st;
   }
   {
     const uint64_t dims[4] = {static_cast<uint64_t>(kDc), static_cast<uint64_t>(d.H),
                               static_cast<uint64_t>(d.n_q), static_cast<uint64_t>(d.B)};
     const uint64_t strides[3] = {kDc * 2ull, static_cast<uint64_t>(d.H) * kDc * 2,
                                  static_cast<uint64_t>(d.n_q) * d.H * kDc * 2};
-    const uint32_t box[4] = {64, 1, kR, 1};
-    if ((st = make_tmap_bf16(&tg, a.d_o_lat, 4, dims, strides, box, 128)) != MLA_OK) return st;
+    const uint32_t box[4] = {64, 1, rows, 1};
+    if ((st = make_tmap_bf16(&m->g, a.d_o_lat, 4, dims, strides, box, 128)) != MLA_OK) return st;
   }
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.n_q),
                               static_cast<uint64_t>(d.B)};
     const uint64_t strides[2] = {kD * 2ull, static_cast<uint64_t>(d.n_q) * kD * 2};
-    const uint32_t box[3] = {64, kR, 1};
-    if ((st = make_tmap_bf16(&tchunk, a.chunk_lat, 3, dims, strides, box, 128)) != MLA_OK) return st;
+    const uint32_t box[3] = {64, rows, 1};
+    if ((st = make_tmap_bf16(&m->chunk, a.chunk_lat, 3, dims, strides, box, 128)) != MLA_OK)
+      return st;
   }
   if (kw.nc > 0) {
     const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(kw.nc),
                               static_cast<uint64_t>(d.B)};
     const uint64_t strides[2] = {kD * 2ull, static_cast<uint64_t>(d.W) * d.tpf * kD * 2};
-    const uint32_t box[3] = {64, kR, 1};
-    if ((st = make_tmap_bf16(&tcache, a.cache, 3, dims, strides, box, 128)) != MLA_OK) return st;
+    const uint32_t box[3] = {64, rows, 1};
+    if ((st = make_tmap_bf16(&m->cache, a.cache, 3, dims, strides, box, 128)) != MLA_OK) return st;
   } else {
-    tcache = tchunk;
+    m->cache = m->chunk;   // never read: no ring rows
   }
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(kDr), static_cast<uint64_t>(kw.rows),
                               static_cast<uint64_t>(d.B)};
     const uint64_t strides[2] = {kDr * 2ull, static_cast<uint64_t>(kw.rows) * kDr * 2};
-    const uint32_t box[3] = {kDr, kR, 1};
-    if ((st = make_tmap_bf16(&tws, ws_rope, 3, dims, strides, box, 64)) != MLA_OK) return st;
+    const uint32_t box[3] = {kDr, rows, 1};
+    if ((st = make_tmap_bf16(&m->ws, ws_rope, 3, dims, strides, box, 64)) != MLA_OK) return st;
   }
+  return MLA_OK;
+}
+
+}  // namespace
+
+mla_status attention_bwd_tc(const Dims& d, const BwdArgs& a, int n_valid, int first_frame,
+                            const float* delta, const void* ws_rope, float* partial, int groups,
+                            int32_t* dev_status, cudaStream_t s) {
+  const KeyWorkspace kw = key_workspace_layout(d, n_valid);
+  BwdMaps m128, m64;
+  mla_status st = make_bwd_maps(d, a, kw, ws_rope, kR, &m128);
+  if (st != MLA_OK) return st;
+  if ((st = make_bwd_maps(d, a, kw, ws_rope, kS, &m64)) != MLA_OK) return st;
   BwdTcParams p;
   p.n_q = d.n_q; p.H = d.H; p.nc = kw.nc; p.nc_pad = kw.nc_pad;
   p.nt_ring = ceil_div(kw.nc, kR);
   p.nt = p.nt_ring + ceil_div(d.n_q, kR);
-  p.rows_ws = kw.rows; p.heads_per_group = d.H / groups; p.n_qt = ceil_div(d.n_q, kR);
+  p.ns_ring = ceil_div(kw.nc, kS);
+  p.ns = p.ns_ring + ceil_div(d.n_q, kS);
+  p.n_qs = ceil_div(d.n_q, kS);
+  p.rows_ws = kw.rows; p.heads_per_group = d.H / groups;
   p.scale = d.scale; p.scale_log2 = d.scale * kLog2e;
   p.lse = a.lse; p.delta = delta; p.d_q = a.d_q; p.partial = partial; p.dev_status = dev_status;
   MLA_CUDA_TRY(cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     kSmemQ));
   MLA_CUDA_TRY(cudaFuncSetAttribute(bwd_dkey_tc_kernel,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemK));
+  // dQ kernel: owns a 128-row query tile (Q', G by 128-row boxes), streams 64-key sub-tiles
   dim3 gq(ceil_div(d.n_q, kR), d.H, d.B);
-  bwd_dq_tc_kernel<<<gq, kThreads, kSmemQ, s>>>(tq, tqr, tg, tcache, tchunk, tws, p);
+  bwd_dq_tc_kernel<<<gq, kThreads, kSmemQ, s>>>(m128.q, m128.qr, m128.g, m64.cache, m64.chunk,
+                                                m64.ws, p);
   MLA_LAUNCH_CHECK("bwd_dq_tc");
+  // key kernel: owns a 128-key tile, streams 64-query sub-tiles (Q', G by 64-row boxes)
   dim3 gk(p.nt, groups, d.B);
-  bwd_dkey_tc_kernel<<<gk, kThreads, kSmemK, s>>>(tq, tqr, tg, tcache, tchunk, tws, p);
+  bwd_dkey_tc_kernel<<<gk, kThreads, kSmemK, s>>>(m64.q, m64.qr, m64.g, m128.cache, m128.chunk,
+                                                  m128.ws, p);
   MLA_LAUNCH_CHECK("bwd_dkey_tc");
   const int64_t total = static_cast<int64_t>(d.B) * (kw.nc + d.n_q) * (kD / 2);
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));
