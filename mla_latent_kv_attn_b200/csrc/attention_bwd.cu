@@ -219,8 +219,9 @@ BwdWorkspace bwd_workspace_layout(const Dims& d, int n_valid) {
   w.delta_bytes = static_cast<size_t>(round_up(d.B * d.H * d.n_q, 64)) * sizeof(float);
   w.keys = key_workspace_layout(d, n_valid);
   w.groups = tc_bwd_supported(d) ? bwd_tc_head_groups(d, n_valid) : 0;
+  w.keys_tc_bytes = w.groups > 0 ? static_cast<size_t>(d.B) * w.keys.rows * kBwdKeyWidth * 2 : 0;
   w.partial_bytes = static_cast<size_t>(w.groups) * d.B * w.keys.rows * d.D * sizeof(float);
-  w.bytes = w.delta_bytes + w.keys.bytes + w.partial_bytes;
+  w.bytes = w.delta_bytes + w.keys.bytes + w.keys_tc_bytes + w.partial_bytes;
   return w;
 }
 
@@ -244,9 +245,10 @@ mla_status attention_bwd(const Dims& d, const BwdArgs& a, int n_valid, int first
   mla_status r = d.dtype == MLA_FP32 ? launch_delta<float>(p, s) : launch_delta<bf16>(p, s);
   if (r != MLA_OK) return r;
   if (w.groups > 0) {
-    float* partial = reinterpret_cast<float*>(static_cast<char*>(ws_rope) + w.keys.bytes);
-    return attention_bwd_tc(d, a, n_valid, first_frame, delta, ws_rope, partial, w.groups,
-                            dev_status, s);
+    void* keys_tc = static_cast<char*>(ws_rope) + w.keys.bytes;
+    float* partial = reinterpret_cast<float*>(static_cast<char*>(keys_tc) + w.keys_tc_bytes);
+    return attention_bwd_tc(d, a, n_valid, first_frame, delta, ws_rope, keys_tc, partial,
+                            w.groups, dev_status, s);
   }
   return d.dtype == MLA_FP32 ? launch_bwd_simt<float>(p, s) : launch_bwd_simt<bf16>(p, s);
 }

@@ -6,21 +6,28 @@
 // Both kernels own a 128-row tile and stream 64-row sub-tiles of the other side through a ring
 // of shared-memory stages; S and dP of a sub-tile are double-buffered in TMEM, so the softmax of
 // sub-tile i runs while the MMAs of sub-tile i+1 do.
+// A streamed sub-tile that is read MN-major (K'_j in the dQ kernel, Q'_i in the key kernel) is
+// held 256 columns wide: three 64-column content blocks and a fourth block with the 32
+// positional columns followed by 32 zeros, all with the 128-byte swizzle. Its product is then a
+// single N=256 MMA per k-step (columns 224-255 of the accumulator receive zeros and are never
+// read) instead of an N=192 and a separate, slow, N=32 one. The keys come from a copy the
+// pre-pass bwd_pad_keys_kernel assembles in the workspace; Q'_i's fourth block is a TMA box that
+// runs past the query's 224 columns, which the copy engine fills with zeros.
 // dQ kernel: one CTA per (128-row query tile, head, sample); per 64-key sub-tile j:
 //   S_j  = Q' K'_j^T       M128 N64 K224    (A: Q' smem, B: K'_j smem, both K-major)
 //   dP_j = G  V_j^T        M128 N64 K192    (A: G smem, B: content blocks of K'_j, K-major)
 //   dS_j = scale * P o (dP - Delta), P = exp(S scale - lse)    (softmax warps, bf16 into TMEM)
-//   dQ  += dS_j K'_j       M128 N192 + N32 K64 (A: dS in TMEM, B: K'_j read MN-major)
+//   dQ  += dS_j K'_j       M128 N256 K64    (A: dS in TMEM, B: K'_j read MN-major)
 // Key kernel: one CTA per (128-key tile, group of heads, sample); per (head, 64-query sub-tile):
 //   S^T  = K' Q'_i^T       M128 N64 K224
 //   dP^T = V  G_i^T        M128 N64 K192
 //   P^T, scale * dS^T      softmax warps, one key row per thread, lse/Delta per query column
+//   dL  += dS^T Q'_i       M128 N256 K64    (key gradient, content and positional parts)
 //   dL  += P^T G_i         M128 N192 K64    (value gradient: the value is the content latent)
-//   dL  += dS^T Q'_i       M128 N192 + N32 K64 (key gradient, content and positional parts)
 // dL (fp32, 224 wide) goes to a workspace slice per head group; bwd_reduce_kernel sums the
 // groups, maps the positional part back through the transposed rotation and stores bf16.
 // TMEM columns: S buffers [0,64) [64,128), dP buffers [128,192) [192,256), accumulator
-// [256,480); P / dS (bf16, 32 columns) are written over the first columns of their buffers.
+// [256,512); P / dS (bf16, 32 columns) are written over the first columns of their buffers.
 // Roles (192 threads): warps 0-3 softmax and epilogue (one TMEM lane = one row), warp 4 TMA
 // producer, warp 5 TMEM allocation and the MMA thread.  Every wait is bounded; a wait that runs
 // out writes MLA_ERR_DEVICE_TIMEOUT to dev_status.
@@ -40,18 +47,20 @@ constexpr int kBlkR = kR * 128;             // 16 KB: 128 rows x 128 B (64 bf16)
 constexpr int kBlkS = kS * 128;             // 8 KB:  64 rows x 128 B
 constexpr int kTileR = 3 * kBlkR + kR * 64; // 56 KB: a 128 x 224 tile (content + 64B-swizzled rope)
 constexpr int kTileGR = 3 * kBlkR;          // 48 KB: a 128 x 192 tile of G
-constexpr int kTileS = 3 * kBlkS + kS * 64; // 28 KB: a 64 x 224 sub-tile
+constexpr int kTileS = 4 * kBlkS;           // 32 KB: a 64 x 256 sub-tile (rope block padded)
 constexpr int kTileGS = 3 * kBlkS;          // 24 KB: a 64 x 192 sub-tile of G
 constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr int kProducerWarp = 4, kMmaWarp = 5;
 constexpr int kSoftmaxThreads = 128;
-constexpr int kQStages = 4;                                        // dQ kernel: K' sub-tiles
+constexpr int kQStages = 3;                                        // dQ kernel: K' sub-tiles
 constexpr int kSmemQ = kTileR + kTileGR + kQStages * kTileS + 1024;
-constexpr int kKStage = kTileS + kTileGS + 1024;                   // Q' + G sub-tiles + stats
+constexpr int kKStage = kTileS + kTileGS;                          // key kernel: Q' + G sub-tiles
 constexpr int kKStages = 3;
-constexpr int kSmemK = kTileR + kKStages * kKStage + 1024;
+constexpr int kStatBytes = 2 * kS * 4;                             // lse and Delta of a sub-tile
+constexpr int kSmemK = kTileR + kKStages * (kKStage + kStatBytes) + 1024;
+static_assert(kSmemQ <= 227 * 1024 && kSmemK + 256 <= 227 * 1024, "shared memory");
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdTcParams {
@@ -73,9 +82,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // Descriptors of a tile's blocks.  K-major (rows = M or N, K = columns): 8-row atoms, SBO 1024
-// (content, 128B swizzle) or 512 (rope, 64B swizzle).  MN-major (N = columns, K = rows): atoms of
-// 64 (content) or 32 (rope) columns x 8 rows; LBO = stride between column blocks, SBO = stride
-// between 8-row groups.
+// (128-byte rows, 128B swizzle) or 512 (the 64-byte rope rows, 64B swizzle).  MN-major (N =
+// columns, K = rows): atoms of 64 columns x 8 rows; LBO = stride between column blocks, SBO =
+// stride between 8-row groups.
 __device__ __forceinline__ uint64_t kmajor_content(uint32_t a) {
   return smem_desc(a, 16, 1024, kSwizzle128B);
 }
@@ -85,20 +94,20 @@ __device__ __forceinline__ uint64_t kmajor_rope(uint32_t a) {
 __device__ __forceinline__ uint64_t mnmajor_content(uint32_t a, uint32_t blk_bytes) {
   return smem_desc(a, blk_bytes, 1024, kSwizzle128B);
 }
-__device__ __forceinline__ uint64_t mnmajor_rope(uint32_t a) {
-  return smem_desc(a, 4096, 512, kSwizzle64B);
-}
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(kR, kS, 0, 0);     // S, dP: M128 N64, K-major
 constexpr uint32_t kIdescC = idesc_bf16_f32(kR, kDc, 0, 1);    // A TMEM, B MN-major, N 192
-constexpr uint32_t kIdescR = idesc_bf16_f32(kR, kDr, 0, 1);    // A TMEM, B MN-major, N 32
+constexpr uint32_t kIdescW = idesc_bf16_f32(kR, 256, 0, 1);    // A TMEM, B MN-major, N 256
 
 // D = A B^T over K = 224 (12 content k-steps + 2 positional); a_blk / b_blk: byte stride of the
-// 64-column content blocks of A / B (their rope block follows the third).
-__device__ __forceinline__ void mma_k224(uint32_t d, uint32_t a_tile, uint32_t a_blk,
-                                         uint32_t b_tile, uint32_t b_blk) {
+// 64-column content blocks of A / B. Their rope block follows the third: 64-byte rows with the
+// 64-byte swizzle, or (a_wide / b_wide) a padded 128-byte block like the content ones. Both
+// advance 32 bytes per k-step.
+__device__ __forceinline__ void mma_k224(uint32_t d, uint32_t a_tile, uint32_t a_blk, bool a_wide,
+                                         uint32_t b_tile, uint32_t b_blk, bool b_wide) {
   const uint64_t ac = kmajor_content(a_tile), bc = kmajor_content(b_tile);
-  const uint64_t ar = kmajor_rope(a_tile + 3 * a_blk), br = kmajor_rope(b_tile + 3 * b_blk);
+  const uint64_t ar = a_wide ? kmajor_content(a_tile + 3 * a_blk) : kmajor_rope(a_tile + 3 * a_blk);
+  const uint64_t br = b_wide ? kmajor_content(b_tile + 3 * b_blk) : kmajor_rope(b_tile + 3 * b_blk);
 #pragma unroll
   for (int blk = 0; blk < 3; ++blk)
 #pragma unroll
@@ -121,19 +130,18 @@ __device__ __forceinline__ void mma_k192(uint32_t d, uint32_t a_tile, uint32_t a
              (blk | kk) != 0 ? 1u : 0u);
 }
 
-// acc[:, 0:192] (+)= A_tmem (128 x 64, bf16) . sub[:, 0:192]; with_rope: also
-// acc[:, 192:224] (+)= A_tmem . sub[:, 192:224].  K = the 64 rows of the sub-tile.
+// acc[:, 0:n] (+)= A_tmem (128 x 64, bf16) . sub[:, 0:n], n = 192 (content blocks) or 256 (all
+// four blocks of a padded sub-tile).  K = the 64 rows of the sub-tile; one MMA per k-step, 16
+// rows = 2048 bytes further each.
+template <int kN>
 __device__ __forceinline__ void mma_tmem_by_sub(uint32_t acc, uint32_t a_tmem, uint32_t sub,
-                                                bool with_rope, bool accumulate) {
-  const uint64_t bc = mnmajor_content(sub, kBlkS);
-  const uint64_t br = mnmajor_rope(sub + 3 * kBlkS);
+                                                bool accumulate) {
+  static_assert(kN == kDc || kN == 256, "product width");
+  const uint64_t b = mnmajor_content(sub, kBlkS);
 #pragma unroll
-  for (int kk = 0; kk < kS / 16; ++kk) {
-    // 16 rows further per k-step: 2048 B (content, 128 B rows) and 1024 B (rope, 64 B rows)
-    mma_ts(acc, a_tmem + kk * 8, bc + 128 * kk, kIdescC, (accumulate || kk) ? 1u : 0u);
-    if (with_rope)
-      mma_ts(acc + kDc, a_tmem + kk * 8, br + 64 * kk, kIdescR, 1u);
-  }
+  for (int kk = 0; kk < kS / 16; ++kk)
+    mma_ts(acc, a_tmem + kk * 8, b + 128 * kk, kN == kDc ? kIdescC : kIdescW,
+           (accumulate || kk) ? 1u : 0u);
 }
 
 // -------------------------------------------------------------------------------- dQ kernel
@@ -141,9 +149,7 @@ __device__ __forceinline__ void mma_tmem_by_sub(uint32_t acc, uint32_t a_tmem, u
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                      const __grid_constant__ CUtensorMap tm_g,
-                     const __grid_constant__ CUtensorMap tm_cache,
-                     const __grid_constant__ CUtensorMap tm_chunk,
-                     const __grid_constant__ CUtensorMap tm_ws, BwdTcParams p) {
+                     const __grid_constant__ CUtensorMap tm_keys, BwdTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t qg_full;
   __shared__ __align__(8) uint64_t kv_full[kQStages];
@@ -204,15 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t dst = sK + s * kTileS;
         const uint32_t fb = smem_u32(&kv_full[s]);
         mbar_arrive_expect_tx(fb, kTileS);
-        if (j < p.ns_ring) {
-          const int r0 = j * kS;
-          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlkS, &tm_cache, fb, 64 * i, r0, b);
-          tma_load_3d(dst + 3 * kBlkS, &tm_ws, fb, 0, r0, b);
-        } else {
-          const int r0 = (j - p.ns_ring) * kS;
-          for (int i = 0; i < 3; ++i) tma_load_3d(dst + i * kBlkS, &tm_chunk, fb, 64 * i, r0, b);
-          tma_load_3d(dst + 3 * kBlkS, &tm_ws, fb, 0, p.nc_pad + r0, b);
-        }
+        const int r0 = j < p.ns_ring ? j * kS : p.nc_pad + (j - p.ns_ring) * kS;
+        for (int i = 0; i < 4; ++i) tma_load_3d(dst + i * kBlkS, &tm_keys, fb, 64 * i, r0, b);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -230,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t kt = sK + s * kTileS;
-          mma_k224(tmem + kColS + 64 * buf, sQ, kBlkR, kt, kBlkS);
+          mma_k224(tmem + kColS + 64 * buf, sQ, kBlkR, false, kt, kBlkS, true);
           mma_k192(tmem + kColDP + 64 * buf, sG, kBlkR, kt, kBlkS);
           mma_commit(smem_u32(&s_full[buf]));
         }
@@ -240,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   p.dev_status);
           if (!ok) break;
           tc_fence_after();
-          mma_tmem_by_sub(tmem + kColAcc, tmem + kColS + 64 * bp, sK + sp * kTileS, true, jp > 0);
+          mma_tmem_by_sub<256>(tmem + kColAcc, tmem + kColS + 64 * bp, sK + sp * kTileS, jp > 0);
           mma_commit(smem_u32(&kv_empty[sp]));
           mma_commit(smem_u32(&buf_free[bp]));
         }
@@ -255,16 +254,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t sr = (static_cast<int64_t>(b) * p.H + h) * p.n_q + n;
     const float lse2 = row_ok ? p.lse[sr] * kLog2e : INFINITY;   // invalid rows: p = 0
     const float delta = row_ok ? p.delta[sr] : 0.f;
-    // the dQ positional columns start with the first sub-tile's products, which accumulate:
-    // zero them first (the content columns are initialised by the first product)
-    {
-      uint32_t z[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) z[i] = 0u;
-      tmem_st16(tmem + lane_off + kColAcc + kDc, z);
-      tmem_st16(tmem + lane_off + kColAcc + kDc + 16, z);
-      tmem_wait_st();
-    }
     bool ok = true;
     for (int j = 0; j < p.ns && ok; ++j) {
       const int buf = j & 1;
@@ -334,11 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------------- key kernel
 
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_dkey_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
-                       const __grid_constant__ CUtensorMap tm_g,
-                       const __grid_constant__ CUtensorMap tm_cache,
-                       const __grid_constant__ CUtensorMap tm_chunk,
-                       const __grid_constant__ CUtensorMap tm_ws, BwdTcParams p) {
+    bwd_dkey_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
+                       const __grid_constant__ CUtensorMap tm_keys,
+                       const __grid_constant__ CUtensorMap tm_keys_r, BwdTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t k_full;
   __shared__ __align__(8) uint64_t qg_full[kKStages];   // Q'_i, G_i and their stats landed
@@ -351,7 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sK = sbase, sStage = sbase + kTileR;
-  // stage layout: Q' sub-tile (28 KB), G sub-tile (24 KB), lse [64] and Delta [64] (512 B)
+  const uint32_t sStat = sStage + kKStages * kKStage;
+  // stage s: Q' sub-tile (32 KB, padded rope block) and G sub-tile (24 KB) at sStage + s * kKStage;
+  // their lse [64] and Delta [64] (512 B) at sStat + s * kStatBytes
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int kt = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
   const int n_iter = p.heads_per_group * p.n_qs;
@@ -385,15 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t kb = smem_u32(&k_full);
       mbar_arrive_expect_tx(kb, kTileR);
-      if (kt < p.nt_ring) {
-        const int r0 = kt * kR;
-        for (int i = 0; i < 3; ++i) tma_load_3d(sK + i * kBlkR, &tm_cache, kb, 64 * i, r0, b);
-        tma_load_3d(sK + 3 * kBlkR, &tm_ws, kb, 0, r0, b);
-      } else {
-        const int r0 = (kt - p.nt_ring) * kR;
-        for (int i = 0; i < 3; ++i) tma_load_3d(sK + i * kBlkR, &tm_chunk, kb, 64 * i, r0, b);
-        tma_load_3d(sK + 3 * kBlkR, &tm_ws, kb, 0, p.nc_pad + r0, b);
-      }
+      // the key tile is only read K-major: its rope block keeps 64-byte rows
+      const int r0 = kt < p.nt_ring ? kt * kR : p.nc_pad + (kt - p.nt_ring) * kR;
+      for (int i = 0; i < 3; ++i) tma_load_3d(sK + i * kBlkR, &tm_keys, kb, 64 * i, r0, b);
+      tma_load_3d(sK + 3 * kBlkR, &tm_keys_r, kb, kDc, r0, b);
       bool ok = true;
       for (int it = 0; it < n_iter && ok; ++it) {
         const int s = it % kKStages;
@@ -409,11 +393,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t st = sStage + s * kKStage;
         const uint32_t fb = smem_u32(&qg_full[s]);
         mbar_arrive_expect_tx(fb, kTileS + kTileGS + 2 * stat_bytes);
-        for (int i = 0; i < 3; ++i) tma_load_4d(st + i * kBlkS, &tm_q, fb, 64 * i, h, q0, b);
-        tma_load_4d(st + 3 * kBlkS, &tm_qr, fb, kDc, h, q0, b);
+        // the fourth box covers columns 192-255 of Q': 224-255 lie past the row and are
+        // filled with zeros (the padded rope block); the byte count is the full box
+        for (int i = 0; i < 4; ++i) tma_load_4d(st + i * kBlkS, &tm_q, fb, 64 * i, h, q0, b);
         for (int i = 0; i < 3; ++i) tma_load_4d(st + kTileS + i * kBlkS, &tm_g, fb, 64 * i, h, q0, b);
-        bulk_load(st + kTileS + kTileGS, p.lse + so, stat_bytes, fb);
-        bulk_load(st + kTileS + kTileGS + 256, p.delta + so, stat_bytes, fb);
+        bulk_load(sStat + s * kStatBytes, p.lse + so, stat_bytes, fb);
+        bulk_load(sStat + s * kStatBytes + kS * 4, p.delta + so, stat_bytes, fb);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -429,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = sStage + s * kKStage;
-          mma_k224(tmem + kColS + 64 * buf, sK, kBlkR, st, kBlkS);
+          mma_k224(tmem + kColS + 64 * buf, sK, kBlkR, false, st, kBlkS, true);
           mma_k192(tmem + kColDP + 64 * buf, sK, kBlkR, st + kTileS, kBlkS);
           mma_commit(smem_u32(&s_full[buf]));
         }
@@ -440,10 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = sStage + sp * kKStage;
-          // value gradient P^T G, then the key gradient dS^T Q' (the positional accumulator
-          // columns, which get no value term, were zeroed by the softmax warps)
-          mma_tmem_by_sub(tmem + kColAcc, tmem + kColS + 64 * bp, st + kTileS, false, ip > 0);
-          mma_tmem_by_sub(tmem + kColAcc, tmem + kColDP + 64 * bp, st, true, true);
+          // key gradient dS^T Q' over all 256 columns first (it initialises the accumulator),
+          // then the value gradient P^T G into the content columns
+          mma_tmem_by_sub<256>(tmem + kColAcc, tmem + kColDP + 64 * bp, st, ip > 0);
+          mma_tmem_by_sub<kDc>(tmem + kColAcc, tmem + kColS + 64 * bp, st + kTileS, true);
           mma_commit(smem_u32(&qg_empty[sp]));
           mma_commit(smem_u32(&buf_free[bp]));
         }
@@ -454,14 +439,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const bool key_ok = kt < p.nt_ring ? kt * kR + row < p.nc
                                        : (kt - p.nt_ring) * kR + row < p.n_q;
-    {
-      uint32_t z[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) z[i] = 0u;
-      tmem_st16(tmem + lane_off + kColAcc + kDc, z);
-      tmem_st16(tmem + lane_off + kColAcc + kDc + 16, z);
-      tmem_wait_st();
-    }
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       const int s = it % kKStages, buf = it & 1;
@@ -475,8 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const float* col_lse = reinterpret_cast<const float*>(
-          smem_raw + (sStage + s * kKStage + kTileS + kTileGS - smem_u32(smem_raw)));
-      const float* col_delta = col_lse + 64;
+          smem_raw + (sStat + s * kStatBytes - smem_u32(smem_raw)));
+      const float* col_delta = col_lse + kS;
       const int ncols = min(kS, p.n_q - (it % p.n_qs) * kS);
       uint32_t rs[64], rp[64];
       tmem_ld64_wait(tmem + lane_off + kColS + 64 * buf, rs);
@@ -538,6 +515,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Writes the keys the tensor-core kernels read, row prow of sample b of the key workspace:
+// [content latent (192) | rotated positional key (32) | 32 zeros]; rows past the valid ring
+// keys (ring part [0, nc_pad)) or chunk keys (chunk part from nc_pad on) are zero.  One thread
+// per 16-byte piece (8 bf16, 32 per row).
+__global__ void bwd_pad_keys_kernel(const bf16* __restrict__ cache, const bf16* __restrict__ chunk_lat,
+                                    const bf16* __restrict__ ws_rope, int B, int W, int tpf, int nc,
+                                    int nc_pad, int n_q, int rows_ws, bf16* __restrict__ keys) {
+  constexpr int kPieces = kBwdKeyWidth / 8;
+  const int64_t total = static_cast<int64_t>(B) * rows_ws * kPieces;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int c8 = static_cast<int>(e % kPieces);
+    const int64_t br = e / kPieces;
+    const int prow = static_cast<int>(br % rows_ws), b = static_cast<int>(br / rows_ws);
+    const bool ring = prow < nc_pad;
+    const int m = ring ? prow : prow - nc_pad;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (ring ? m < nc : m < n_q) {
+      if (c8 < kDc / 8) {
+        const bf16* src = ring ? cache + (static_cast<int64_t>(b) * W * tpf + m) * kD
+                               : chunk_lat + (static_cast<int64_t>(b) * n_q + m) * kD;
+        v = *reinterpret_cast<const uint4*>(src + 8 * c8);
+      } else if (c8 < kD / 8) {
+        v = *reinterpret_cast<const uint4*>(ws_rope + br * kDr + 8 * (c8 - kDc / 8));
+      }
+    }
+    *reinterpret_cast<uint4*>(keys + br * kBwdKeyWidth + 8 * c8) = v;
   }
 }
 
@@ -604,13 +611,14 @@ bool tc_bwd_supported(const Dims& d) {
 namespace {
 
 // Tensor maps of the backward's operands with row boxes of `rows` (128 for a tile a CTA owns, 64
-// for a streamed sub-tile).
+// for a streamed sub-tile).  keys / keys_r: the padded key copy, 64-column boxes with the
+// 128-byte swizzle / the 32 positional columns with the 64-byte swizzle.
 struct BwdMaps {
-  CUtensorMap q, qr, g, cache, chunk, ws;
+  CUtensorMap q, qr, g, keys, keys_r;
 };
 
 mla_status make_bwd_maps(const Dims& d, const BwdArgs& a, const KeyWorkspace& kw,
-                         const void* ws_rope, uint32_t rows, BwdMaps* m) {
+                         const void* keys_tc, uint32_t rows, BwdMaps* m) {
   mla_status st;
   {
     const uint64_t dims[4] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.H),
@@ -631,28 +639,15 @@ mla_status make_bwd_maps(const Dims& d, const BwdArgs& a, const KeyWorkspace& kw
     if ((st = make_tmap_bf16(&m->g, a.d_o_lat, 4, dims, strides, box, 128)) != MLA_OK) return st;
   }
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.n_q),
+    const uint64_t dims[3] = {static_cast<uint64_t>(kBwdKeyWidth), static_cast<uint64_t>(kw.rows),
                               static_cast<uint64_t>(d.B)};
-    const uint64_t strides[2] = {kD * 2ull, static_cast<uint64_t>(d.n_q) * kD * 2};
+    const uint64_t strides[2] = {kBwdKeyWidth * 2ull,
+                                 static_cast<uint64_t>(kw.rows) * kBwdKeyWidth * 2};
     const uint32_t box[3] = {64, rows, 1};
-    if ((st = make_tmap_bf16(&m->chunk, a.chunk_lat, 3, dims, strides, box, 128)) != MLA_OK)
+    if ((st = make_tmap_bf16(&m->keys, keys_tc, 3, dims, strides, box, 128)) != MLA_OK) return st;
+    const uint32_t box_r[3] = {kDr, rows, 1};
+    if ((st = make_tmap_bf16(&m->keys_r, keys_tc, 3, dims, strides, box_r, 64)) != MLA_OK)
       return st;
-  }
-  if (kw.nc > 0) {
-    const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(kw.nc),
-                              static_cast<uint64_t>(d.B)};
-    const uint64_t strides[2] = {kD * 2ull, static_cast<uint64_t>(d.W) * d.tpf * kD * 2};
-    const uint32_t box[3] = {64, rows, 1};
-    if ((st = make_tmap_bf16(&m->cache, a.cache, 3, dims, strides, box, 128)) != MLA_OK) return st;
-  } else {
-    m->cache = m->chunk;   // never read: no ring rows
-  }
-  {
-    const uint64_t dims[3] = {static_cast<uint64_t>(kDr), static_cast<uint64_t>(kw.rows),
-                              static_cast<uint64_t>(d.B)};
-    const uint64_t strides[2] = {kDr * 2ull, static_cast<uint64_t>(kw.rows) * kDr * 2};
-    const uint32_t box[3] = {kDr, rows, 1};
-    if ((st = make_tmap_bf16(&m->ws, ws_rope, 3, dims, strides, box, 64)) != MLA_OK) return st;
   }
   return MLA_OK;
 }
@@ -660,13 +655,13 @@ mla_status make_bwd_maps(const Dims& d, const BwdArgs& a, const KeyWorkspace& kw
 }  // namespace
 
 mla_status attention_bwd_tc(const Dims& d, const BwdArgs& a, int n_valid, int first_frame,
-                            const float* delta, const void* ws_rope, float* partial, int groups,
-                            int32_t* dev_status, cudaStream_t s) {
+                            const float* delta, const void* ws_rope, void* keys_tc,
+                            float* partial, int groups, int32_t* dev_status, cudaStream_t s) {
   const KeyWorkspace kw = key_workspace_layout(d, n_valid);
   BwdMaps m128, m64;
-  mla_status st = make_bwd_maps(d, a, kw, ws_rope, kR, &m128);
+  mla_status st = make_bwd_maps(d, a, kw, keys_tc, kR, &m128);
   if (st != MLA_OK) return st;
-  if ((st = make_bwd_maps(d, a, kw, ws_rope, kS, &m64)) != MLA_OK) return st;
+  if ((st = make_bwd_maps(d, a, kw, keys_tc, kS, &m64)) != MLA_OK) return st;
   BwdTcParams p;
   p.n_q = d.n_q; p.H = d.H; p.nc = kw.nc; p.nc_pad = kw.nc_pad;
   p.nt_ring = ceil_div(kw.nc, kR);
@@ -677,19 +672,26 @@ mla_status attention_bwd_tc(const Dims& d, const BwdArgs& a, int n_valid, int fi
   p.rows_ws = kw.rows; p.heads_per_group = d.H / groups;
   p.scale = d.scale; p.scale_log2 = d.scale * kLog2e;
   p.lse = a.lse; p.delta = delta; p.d_q = a.d_q; p.partial = partial; p.dev_status = dev_status;
+  {
+    const int64_t pieces = static_cast<int64_t>(d.B) * kw.rows * (kBwdKeyWidth / 8);
+    const int blocks = static_cast<int>(std::min<int64_t>((pieces + 255) / 256, 148 * 16));
+    bwd_pad_keys_kernel<<<blocks, 256, 0, s>>>(
+        static_cast<const bf16*>(a.cache), static_cast<const bf16*>(a.chunk_lat),
+        static_cast<const bf16*>(ws_rope), d.B, d.W, d.tpf, kw.nc, kw.nc_pad, d.n_q, kw.rows,
+        static_cast<bf16*>(keys_tc));
+    MLA_LAUNCH_CHECK("bwd_pad_keys");
+  }
   MLA_CUDA_TRY(cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     kSmemQ));
   MLA_CUDA_TRY(cudaFuncSetAttribute(bwd_dkey_tc_kernel,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemK));
   // dQ kernel: owns a 128-row query tile (Q', G by 128-row boxes), streams 64-key sub-tiles
   dim3 gq(ceil_div(d.n_q, kR), d.H, d.B);
-  bwd_dq_tc_kernel<<<gq, kThreads, kSmemQ, s>>>(m128.q, m128.qr, m128.g, m64.cache, m64.chunk,
-                                                m64.ws, p);
+  bwd_dq_tc_kernel<<<gq, kThreads, kSmemQ, s>>>(m128.q, m128.qr, m128.g, m64.keys, p);
   MLA_LAUNCH_CHECK("bwd_dq_tc");
   // key kernel: owns a 128-key tile, streams 64-query sub-tiles (Q', G by 64-row boxes)
   dim3 gk(p.nt, groups, d.B);
-  bwd_dkey_tc_kernel<<<gk, kThreads, kSmemK, s>>>(m64.q, m64.qr, m64.g, m128.cache, m128.chunk,
-                                                  m128.ws, p);
+  bwd_dkey_tc_kernel<<<gk, kThreads, kSmemK, s>>>(m64.q, m64.g, m128.keys, m128.keys_r, p);
   MLA_LAUNCH_CHECK("bwd_dkey_tc");
   const int64_t total = static_cast<int64_t>(d.B) * (kw.nc + d.n_q) * (kD / 2);
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));

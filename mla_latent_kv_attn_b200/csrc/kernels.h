@@ -66,9 +66,10 @@ struct BwdArgs {
 struct BwdWorkspace {
   size_t delta_bytes;      // Delta = G . O_lat per (sample, head, row), fp32, then
   KeyWorkspace keys;       // the rotated positional keys, as in the forward, then
-  int groups;              // (tensor-core path) per head group, the keys' fp32 partial
-  size_t partial_bytes;    //   latent gradients [groups, B, keys.rows, D]
-  size_t bytes;
+  int groups;              // (tensor-core path) the keys as the MMAs read them,
+  size_t keys_tc_bytes;    //   [B, keys.rows, 256] bf16 (latent, rotated key, zeros), then per
+  size_t partial_bytes;    //   head group the keys' fp32 partial latent gradients
+  size_t bytes;            //   [groups, B, keys.rows, D]
 };
 
 BwdWorkspace bwd_workspace_layout(const Dims& d, int n_valid);
@@ -77,9 +78,10 @@ mla_status attention_bwd(const Dims& d, const BwdArgs& a, int n_valid, int first
 // tensor-core backward (attention_bwd_sm100.cu)
 bool tc_bwd_supported(const Dims& d);
 int bwd_tc_head_groups(const Dims& d, int n_valid);
+constexpr int kBwdKeyWidth = 256;   // row width of the tensor-core path's key copy
 mla_status attention_bwd_tc(const Dims& d, const BwdArgs& a, int n_valid, int first_frame,
-                            const float* delta, const void* ws_rope, float* partial, int groups,
-                            int32_t* dev_status, cudaStream_t s);
+                            const float* delta, const void* ws_rope, void* keys_tc,
+                            float* partial, int groups, int32_t* dev_status, cudaStream_t s);
 
 // CUDA-core kernels (simt.cu)
 mla_status gemm_simt(const GemmArgs& g, int dtype, cudaStream_t s);
