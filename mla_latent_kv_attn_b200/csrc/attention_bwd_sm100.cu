@@ -4,8 +4,14 @@
 // rounded to bf16 as MMA operands; the softmax statistics stay fp32).
 //
 // Both kernels own a 128-row tile and stream 64-row sub-tiles of the other side through a ring
-// of shared-memory stages; S and dP of a sub-tile are double-buffered in TMEM, so the softmax of
-// sub-tile i runs while the MMAs of sub-tile i+1 do.
+// of shared-memory stages.  The operand a CTA keeps for its whole life (its 128 query rows Q' in
+// the dQ kernel, its 128 keys K' in the key kernel) sits in TMEM as bf16 pairs, so the S and dP
+// MMAs read only their streamed B operand from shared memory: with both operands in shared
+// memory an M128 N64 MMA is bound by shared-memory reads (6 KB per k-step), with A in TMEM it
+// runs at the tensor rate.  The softmax warps load S and dP into registers and release the TMEM
+// buffers at once, so the S/dP MMAs of the next sub-tile overlap the softmax; P and dS go to
+// shared memory (128-byte-swizzled K-major rows, written the way a TMA load would place them)
+// as the A operands of the gradient products.
 // A streamed sub-tile that is read MN-major (K'_j in the dQ kernel, Q'_i in the key kernel) is
 // held 256 columns wide: three 64-column content blocks and a fourth block with the 32
 // positional columns followed by 32 zeros, all with the 128-byte swizzle. Its product is then a
@@ -14,23 +20,22 @@
 // pre-pass bwd_pad_keys_kernel assembles in the workspace; Q'_i's fourth block is a TMA box that
 // runs past the query's 224 columns, which the copy engine fills with zeros.
 // dQ kernel: one CTA per (128-row query tile, head, sample); per 64-key sub-tile j:
-//   S_j  = Q' K'_j^T       M128 N64 K224    (A: Q' smem, B: K'_j smem, both K-major)
+//   S_j  = Q' K'_j^T       M128 N64 K224    (A: Q' in TMEM, B: K'_j smem, K-major)
 //   dP_j = G  V_j^T        M128 N64 K192    (A: G smem, B: content blocks of K'_j, K-major)
-//   dS_j = scale * P o (dP - Delta), P = exp(S scale - lse)    (softmax warps, bf16 into TMEM)
-//   dQ  += dS_j K'_j       M128 N256 K64    (A: dS in TMEM, B: K'_j read MN-major)
+//   dS_j = scale * P o (dP - Delta), P = exp(S scale - lse)    (softmax warps, bf16 to smem)
+//   dQ  += dS_j K'_j       M128 N256 K64    (A: dS smem, B: K'_j read MN-major)
 // Key kernel: one CTA per (128-key tile, group of heads, sample); per (head, 64-query sub-tile):
-//   S^T  = K' Q'_i^T       M128 N64 K224
-//   dP^T = V  G_i^T        M128 N64 K192
-//   P^T, scale * dS^T      softmax warps, one key row per thread, lse/Delta per query column
+//   S^T  = K' Q'_i^T       M128 N64 K224    (A: K' in TMEM)
+//   dP^T = V  G_i^T        M128 N64 K192    (A: the content columns of K' in TMEM)
+//   P^T, scale * dS^T      softmax warps, one half key row per thread, lse/Delta per column
 //   dL  += dS^T Q'_i       M128 N256 K64    (key gradient, content and positional parts)
 //   dL  += P^T G_i         M128 N192 K64    (value gradient: the value is the content latent)
 // dL (fp32, 224 wide) goes to a workspace slice per head group; bwd_reduce_kernel sums the
 // groups, maps the positional part back through the transposed rotation and stores bf16.
-// TMEM columns: S buffers [0,64) [64,128), dP buffers [128,192) [192,256), accumulator
-// [256,512); P / dS (bf16, 32 columns) are written over the first columns of their buffers.
-// Roles (192 threads): warps 0-3 softmax and epilogue (one TMEM lane = one row), warp 4 TMA
-// producer, warp 5 TMEM allocation and the MMA thread.  Every wait is bounded; a wait that runs
-// out writes MLA_ERR_DEVICE_TIMEOUT to dev_status.
+// TMEM columns: resident A operand [0,112), S [128,192), dP [192,256), accumulator [256,512).
+// Roles: softmax / epilogue warps (one TMEM lane = one row), a TMA producer warp, and a warp that
+// allocates TMEM and whose lane 0 issues every MMA.  Every wait is bounded; a wait that runs out
+// writes MLA_ERR_DEVICE_TIMEOUT to dev_status.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -45,22 +50,28 @@ constexpr int kS = 64;                      // rows of a streamed sub-tile
 constexpr int kDc = 192, kDr = 32, kD = 224;
 constexpr int kBlkR = kR * 128;             // 16 KB: 128 rows x 128 B (64 bf16), 128B swizzle
 constexpr int kBlkS = kS * 128;             // 8 KB:  64 rows x 128 B
-constexpr int kTileR = 3 * kBlkR + kR * 64; // 56 KB: a 128 x 224 tile (content + 64B-swizzled rope)
 constexpr int kTileGR = 3 * kBlkR;          // 48 KB: a 128 x 192 tile of G
 constexpr int kTileS = 4 * kBlkS;           // 32 KB: a 64 x 256 sub-tile (rope block padded)
 constexpr int kTileGS = 3 * kBlkS;          // 24 KB: a 64 x 192 sub-tile of G
-constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256;
+constexpr int kOpBytes = kR * 128;          // 16 KB: a 128 x 64 bf16 operand (dS, P) in smem
+constexpr uint32_t kColA = 0, kColS = 128, kColDP = 192, kColAcc = 256;
+constexpr int kAWords = kD / 2;             // 112 TMEM columns of bf16 pairs
 constexpr uint32_t kTmemCols = 512;
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4, kMmaWarp = 5;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kQStages = 3;                                        // dQ kernel: K' sub-tiles
-constexpr int kSmemQ = kTileR + kTileGR + kQStages * kTileS + 1024;
-constexpr int kKStage = kTileS + kTileGS;                          // key kernel: Q' + G sub-tiles
+// dQ kernel: 4 softmax warps, producer, MMA
+constexpr int kSoftmaxQ = 128, kThreadsQ = kSoftmaxQ + 64;
+constexpr int kProducerWarpQ = 4, kMmaWarpQ = 5;
+constexpr int kQStages = 4;                                   // K' sub-tiles in flight
+constexpr int kSmemQ = kTileGR + kQStages * kTileS + 2 * kOpBytes + 1024;
+// key kernel: 8 softmax warps (two per TMEM lane quarter, each half of the columns)
+constexpr int kSoftmaxK = 256, kThreadsK = kSoftmaxK + 64;
+constexpr int kProducerWarpK = 8, kMmaWarpK = 9;
+constexpr int kKStage = kTileS + kTileGS;                     // Q' + G sub-tiles
 constexpr int kKStages = 3;
-constexpr int kStatBytes = 2 * kS * 4;                             // lse and Delta of a sub-tile
-constexpr int kSmemK = kTileR + kKStages * (kKStage + kStatBytes) + 1024;
-static_assert(kSmemQ <= 227 * 1024 && kSmemK + 256 <= 227 * 1024, "shared memory");
+constexpr int kStatBytes = 2 * kS * 4;                        // lse and Delta of a sub-tile
+constexpr int kStatArea = 2048;                               // kKStages * kStatBytes, padded
+constexpr int kSmemK = kKStages * kKStage + kStatArea + 2 * kOpBytes + 1024;
+static_assert(kKStages * kStatBytes <= kStatArea, "stat area");
+static_assert(kSmemQ <= 227 * 1024 && kSmemK <= 227 * 1024, "shared memory");
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdTcParams {
@@ -68,6 +79,8 @@ struct BwdTcParams {
   int ns_ring, ns;          // dQ kernel: 64-key sub-tiles of the ring, in all
   int n_qs;                 // key kernel: 64-query sub-tiles per head
   float scale, scale_log2;
+  const bf16* q;         // [B, n_q, H, D]
+  const bf16* keys;      // [B, rows_ws, 256] padded key copy
   const float* lse;      // [B, H, n_q]
   const float* delta;    // [B, H, n_q]
   void* d_q;             // [B, n_q, H, D] bf16
@@ -81,44 +94,47 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Descriptors of a tile's blocks.  K-major (rows = M or N, K = columns): 8-row atoms, SBO 1024
-// (128-byte rows, 128B swizzle) or 512 (the 64-byte rope rows, 64B swizzle).  MN-major (N =
-// columns, K = rows): atoms of 64 columns x 8 rows; LBO = stride between column blocks, SBO =
-// stride between 8-row groups.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// 16-byte piece `chunk` (0-7) of row `row` of a K-major operand with 128-byte rows and the
+// 128-byte swizzle (a 1024-byte-aligned buffer): the piece index is XORed with the row's position
+// in its 8-row group, as a TMA load with that swizzle places it.
+__device__ __forceinline__ uint32_t swz128(uint32_t buf, int row, int chunk) {
+  return buf + static_cast<uint32_t>(row) * 128u + (static_cast<uint32_t>(chunk ^ (row & 7)) << 4);
+}
+
+// Descriptors of a tile's blocks.  K-major (rows = M or N, K = columns): 8-row atoms of 128-byte
+// rows, SBO 1024.  MN-major (N = columns, K = rows): atoms of 64 columns x 8 rows; LBO = stride
+// between column blocks, SBO = stride between 8-row groups.
 __device__ __forceinline__ uint64_t kmajor_content(uint32_t a) {
   return smem_desc(a, 16, 1024, kSwizzle128B);
-}
-__device__ __forceinline__ uint64_t kmajor_rope(uint32_t a) {
-  return smem_desc(a, 16, 512, kSwizzle64B);
 }
 __device__ __forceinline__ uint64_t mnmajor_content(uint32_t a, uint32_t blk_bytes) {
   return smem_desc(a, blk_bytes, 1024, kSwizzle128B);
 }
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(kR, kS, 0, 0);     // S, dP: M128 N64, K-major
-constexpr uint32_t kIdescC = idesc_bf16_f32(kR, kDc, 0, 1);    // A TMEM, B MN-major, N 192
-constexpr uint32_t kIdescW = idesc_bf16_f32(kR, 256, 0, 1);    // A TMEM, B MN-major, N 256
+constexpr uint32_t kIdescC = idesc_bf16_f32(kR, kDc, 0, 1);    // B MN-major, N 192
+constexpr uint32_t kIdescW = idesc_bf16_f32(kR, 256, 0, 1);    // B MN-major, N 256
 
-// D = A B^T over K = 224 (12 content k-steps + 2 positional); a_blk / b_blk: byte stride of the
-// 64-column content blocks of A / B. Their rope block follows the third: 64-byte rows with the
-// 64-byte swizzle, or (a_wide / b_wide) a padded 128-byte block like the content ones. Both
-// advance 32 bytes per k-step.
-__device__ __forceinline__ void mma_k224(uint32_t d, uint32_t a_tile, uint32_t a_blk, bool a_wide,
-                                         uint32_t b_tile, uint32_t b_blk, bool b_wide) {
-  const uint64_t ac = kmajor_content(a_tile), bc = kmajor_content(b_tile);
-  const uint64_t ar = a_wide ? kmajor_content(a_tile + 3 * a_blk) : kmajor_rope(a_tile + 3 * a_blk);
-  const uint64_t br = b_wide ? kmajor_content(b_tile + 3 * b_blk) : kmajor_rope(b_tile + 3 * b_blk);
+// D = A B^T, A (128 rows) in TMEM as bf16 pairs from column a_tmem (8 columns per k-step), B a
+// K-major sub-tile of 64 rows whose 64-column blocks lie kBlkS apart; kSteps k-steps of 16.
+template <int kSteps>
+__device__ __forceinline__ void mma_tmem_a(uint32_t d, uint32_t a_tmem, uint32_t b_tile) {
+  const uint64_t b = kmajor_content(b_tile);
 #pragma unroll
-  for (int blk = 0; blk < 3; ++blk)
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_ss(d, ac + ((blk * a_blk) >> 4) + 2 * kk, bc + ((blk * b_blk) >> 4) + 2 * kk, kIdescS,
-             (blk | kk) != 0 ? 1u : 0u);
-#pragma unroll
-  for (int kk = 0; kk < 2; ++kk) mma_ss(d, ar + 2 * kk, br + 2 * kk, kIdescS, 1u);
+  for (int kk = 0; kk < kSteps; ++kk)
+    mma_ts(d, a_tmem + 8 * kk, b + (((kk >> 2) * kBlkS) >> 4) + 2 * (kk & 3), kIdescS,
+           kk ? 1u : 0u);
 }
 
-// D = A B^T over the 192 content columns only.
+// D = A B^T over the 192 content columns, both operands K-major in shared memory; a_blk / b_blk:
+// byte stride of the 64-column blocks of A / B.
 __device__ __forceinline__ void mma_k192(uint32_t d, uint32_t a_tile, uint32_t a_blk,
                                          uint32_t b_tile, uint32_t b_blk) {
   const uint64_t ac = kmajor_content(a_tile), bc = kmajor_content(b_tile);
@@ -130,41 +146,55 @@ __device__ __forceinline__ void mma_k192(uint32_t d, uint32_t a_tile, uint32_t a
              (blk | kk) != 0 ? 1u : 0u);
 }
 
-// acc[:, 0:n] (+)= A_tmem (128 x 64, bf16) . sub[:, 0:n], n = 192 (content blocks) or 256 (all
-// four blocks of a padded sub-tile).  K = the 64 rows of the sub-tile; one MMA per k-step, 16
-// rows = 2048 bytes further each.
+// acc[:, 0:kN] (+)= A (128 x 64 bf16, K-major 128-byte swizzled rows in smem) . sub[:, 0:kN],
+// kN = 192 (content blocks) or 256 (all four blocks of a padded sub-tile); K = the 64 rows of the
+// sub-tile, one MMA per k-step (A 32 bytes further, B 16 rows = 2048 bytes further).
 template <int kN>
-__device__ __forceinline__ void mma_tmem_by_sub(uint32_t acc, uint32_t a_tmem, uint32_t sub,
-                                                bool accumulate) {
+__device__ __forceinline__ void mma_op_by_sub(uint32_t acc, uint32_t a_smem, uint32_t sub,
+                                              bool accumulate) {
   static_assert(kN == kDc || kN == 256, "product width");
+  const uint64_t a = kmajor_content(a_smem);
   const uint64_t b = mnmajor_content(sub, kBlkS);
 #pragma unroll
   for (int kk = 0; kk < kS / 16; ++kk)
-    mma_ts(acc, a_tmem + kk * 8, b + 128 * kk, kN == kDc ? kIdescC : kIdescW,
+    mma_ss(acc, a + 2 * kk, b + 128 * kk, kN == kDc ? kIdescC : kIdescW,
            (accumulate || kk) ? 1u : 0u);
+}
+
+// Writes `nwords` bf16 pairs of a global row (16-byte aligned; nullptr: zeros) into this thread's
+// TMEM lane from column taddr on, 16 columns at a time.
+__device__ __forceinline__ void row_to_tmem(uint32_t taddr, const bf16* src, int nwords) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  for (int c = 0; c < nwords; c += 16) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = src != nullptr ? s4[c / 4 + i] : make_uint4(0u, 0u, 0u, 0u);
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+    tmem_st16(taddr + c, w);
+  }
 }
 
 // -------------------------------------------------------------------------------- dQ kernel
 
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
-                     const __grid_constant__ CUtensorMap tm_g,
+__global__ void __launch_bounds__(kThreadsQ, 1)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_g,
                      const __grid_constant__ CUtensorMap tm_keys, BwdTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t qg_full;
+  __shared__ __align__(8) uint64_t g_full;      // G landed
+  __shared__ __align__(8) uint64_t a_ready;     // the softmax warps wrote Q' into TMEM
   __shared__ __align__(8) uint64_t kv_full[kQStages];
   __shared__ __align__(8) uint64_t kv_empty[kQStages];
-  __shared__ __align__(8) uint64_t s_full[2];     // S and dP of sub-tile j in TMEM buffer j&1
-  // the softmax has written dS(j) into buffer j&1; one barrier per buffer, so that a waiter is
-  // never two phases behind (sub-tile j+2 cannot start before the products of j were issued)
-  __shared__ __align__(8) uint64_t ds_full[2];
-  __shared__ __align__(8) uint64_t buf_free[2];   // the dQ products that read buffer b completed
-                                                  // (the epilogue waits for the last of them)
+  __shared__ __align__(8) uint64_t sdp_full;    // S(j), dP(j) complete in TMEM
+  __shared__ __align__(8) uint64_t sdp_free;    // the softmax warps loaded S(j), dP(j)
+  __shared__ __align__(8) uint64_t ds_full[2];  // dS(j) written to buffer j&1
+  __shared__ __align__(8) uint64_t ds_free[2];  // the products that read buffer b completed
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sQ = sbase, sG = sbase + kTileR, sK = sbase + kTileR + kTileGR;
+  const uint32_t sG = sbase, sK = sG + kTileGR, sDS = sK + kQStages * kTileS;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int q0 = qt * kR;
@@ -172,20 +202,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
-    mbar_init(smem_u32(&qg_full), 1);
+    mbar_init(smem_u32(&g_full), 1);
+    mbar_init(smem_u32(&a_ready), kSoftmaxQ);
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(smem_u32(&kv_full[s]), 1);
       mbar_init(smem_u32(&kv_empty[s]), 1);
     }
+    mbar_init(smem_u32(&sdp_full), 1);
+    mbar_init(smem_u32(&sdp_free), kSoftmaxQ);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&buf_free[i]), 1);
+      mbar_init(smem_u32(&ds_full[i]), kSoftmaxQ);
+      mbar_init(smem_u32(&ds_free[i]), 1);
     }
-    mbar_init(smem_u32(&ds_full[0]), kSoftmaxThreads);
-    mbar_init(smem_u32(&ds_full[1]), kSoftmaxThreads);
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarpQ) {
     tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
     tmem_relinquish();
   }
@@ -194,13 +225,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == kProducerWarp) {
+  if (warp == kProducerWarpQ) {
     if (lane == 0) {
-      const uint32_t qb = smem_u32(&qg_full);
-      mbar_arrive_expect_tx(qb, kTileR + kTileGR);
-      for (int i = 0; i < 3; ++i) tma_load_4d(sQ + i * kBlkR, &tm_q, qb, 64 * i, h, q0, b);
-      tma_load_4d(sQ + 3 * kBlkR, &tm_qr, qb, kDc, h, q0, b);
-      for (int i = 0; i < 3; ++i) tma_load_4d(sG + i * kBlkR, &tm_g, qb, 64 * i, h, q0, b);
+      const uint32_t gb = smem_u32(&g_full);
+      mbar_arrive_expect_tx(gb, kTileGR);
+      for (int i = 0; i < 3; ++i) tma_load_4d(sG + i * kBlkR, &tm_g, gb, 64 * i, h, q0, b);
       bool ok = true;
       for (int j = 0; j < p.ns && ok; ++j) {
         const int s = j % kQStages;
@@ -214,24 +243,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) tma_load_3d(dst + i * kBlkS, &tm_keys, fb, 64 * i, r0, b);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarpQ) {
     if (lane == 0) {
-      // Order of issue: S/dP(j) into buffer j&1, then the dQ products of sub-tile j-1 (whose dS
-      // the softmax wrote meanwhile), so the softmax of j-1 overlaps the products of j.
-      bool ok = mbar_wait_or_abort(smem_u32(&qg_full), 0, abort_flag, p.dev_status);
+      // Order of issue: S/dP(j) once the softmax has loaded S/dP(j-1), then the dQ products of
+      // sub-tile j-1 once its dS is in shared memory.
+      bool ok = mbar_wait_or_abort(smem_u32(&a_ready), 0, abort_flag, p.dev_status) &&
+                mbar_wait_or_abort(smem_u32(&g_full), 0, abort_flag, p.dev_status);
       for (int j = 0; j <= p.ns && ok; ++j) {
         if (j < p.ns) {
-          const int s = j % kQStages, buf = j & 1;
-          // S(j) overwrites the buffer whose dS(j-2) the dQ products of j-2 read: those were
-          // issued earlier by this thread, and MMAs of one thread run in issue order
+          const int s = j % kQStages;
           ok = mbar_wait_or_abort(smem_u32(&kv_full[s]), (j / kQStages) & 1, abort_flag,
-                                  p.dev_status);
+                                  p.dev_status) &&
+               (j == 0 || mbar_wait_or_abort(smem_u32(&sdp_free), (j - 1) & 1, abort_flag,
+                                             p.dev_status));
           if (!ok) break;
           tc_fence_after();
           const uint32_t kt = sK + s * kTileS;
-          mma_k224(tmem + kColS + 64 * buf, sQ, kBlkR, false, kt, kBlkS, true);
-          mma_k192(tmem + kColDP + 64 * buf, sG, kBlkR, kt, kBlkS);
-          mma_commit(smem_u32(&s_full[buf]));
+          mma_tmem_a<kD / 16>(tmem + kColS, tmem + kColA, kt);
+          mma_k192(tmem + kColDP, sG, kBlkR, kt, kBlkS);
+          mma_commit(smem_u32(&sdp_full));
         }
         if (j >= 1) {
           const int jp = j - 1, sp = jp % kQStages, bp = jp & 1;
@@ -239,9 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   p.dev_status);
           if (!ok) break;
           tc_fence_after();
-          mma_tmem_by_sub<256>(tmem + kColAcc, tmem + kColS + 64 * bp, sK + sp * kTileS, jp > 0);
+          mma_op_by_sub<256>(tmem + kColAcc, sDS + bp * kOpBytes, sK + sp * kTileS, jp > 0);
           mma_commit(smem_u32(&kv_empty[sp]));
-          mma_commit(smem_u32(&buf_free[bp]));
+          mma_commit(smem_u32(&ds_free[bp]));
         }
       }
     }
@@ -254,18 +284,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t sr = (static_cast<int64_t>(b) * p.H + h) * p.n_q + n;
     const float lse2 = row_ok ? p.lse[sr] * kLog2e : INFINITY;   // invalid rows: p = 0
     const float delta = row_ok ? p.delta[sr] : 0.f;
+    row_to_tmem(tmem + lane_off + kColA,
+                row_ok ? p.q + ((static_cast<int64_t>(b) * p.n_q + n) * p.H + h) * kD : nullptr,
+                kAWords);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(smem_u32(&a_ready));
     bool ok = true;
     for (int j = 0; j < p.ns && ok; ++j) {
       const int buf = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&s_full[buf]), (j >> 1) & 1,
-                                                      abort_flag, p.dev_status));
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&sdp_full), j & 1, abort_flag,
+                                                      p.dev_status));
       if (!ok) break;
       tc_fence_after();
       const int valid = j < p.ns_ring ? min(kS, p.nc - j * kS)
                                       : min(kS, p.n_q - (j - p.ns_ring) * kS);
       uint32_t rs[64], rp[64];
-      tmem_ld64_wait(tmem + lane_off + kColS + 64 * buf, rs);
-      tmem_ld64_wait(tmem + lane_off + kColDP + 64 * buf, rp);
+      tmem_ld64_wait(tmem + lane_off + kColS, rs);
+      tmem_ld64_wait(tmem + lane_off + kColDP, rp);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sdp_free));
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -278,20 +316,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         w[i] = pack_bf16x2(d2[0], d2[1]);
       }
+      // buffer j&1 was last read by the products of sub-tile j-2
+      if (j >= 2)
+        ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&ds_free[buf]),
+                                                        ((j >> 1) & 1) ^ 1, abort_flag,
+                                                        p.dev_status));
+      if (!ok) break;
+      const uint32_t dsb = sDS + buf * kOpBytes;
 #pragma unroll
-      for (int c = 0; c < 32; c += 16) {
-        uint32_t w16[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w16[i] = w[c + i];
-        tmem_st16(tmem + lane_off + kColS + 64 * buf + c, w16);
-      }
-      tmem_wait_st();
-      tc_fence_before();
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(swz128(dsb, row, c), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      fence_proxy_async_smem();
       mbar_arrive(smem_u32(&ds_full[buf]));
     }
     // the last dQ products completed: buffer (ns-1)&1 was freed for the ((ns-1)>>1)-th time
     if (ok)
-      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&buf_free[(p.ns - 1) & 1]),
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&ds_free[(p.ns - 1) & 1]),
                                                       ((p.ns - 1) >> 1) & 1, abort_flag,
                                                       p.dev_status));
     if (ok) {
@@ -314,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarpQ) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -322,25 +362,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------------------- key kernel
 
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_dkey_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
-                       const __grid_constant__ CUtensorMap tm_keys,
-                       const __grid_constant__ CUtensorMap tm_keys_r, BwdTcParams p) {
+__global__ void __launch_bounds__(kThreadsK, 1)
+    bwd_dkey_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_g, BwdTcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t k_full;
+  __shared__ __align__(8) uint64_t a_ready;              // the key tile is in TMEM
   __shared__ __align__(8) uint64_t qg_full[kKStages];   // Q'_i, G_i and their stats landed
   __shared__ __align__(8) uint64_t qg_empty[kKStages];  // the products of sub-tile i read them
-  __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ __align__(8) uint64_t ps_full[2];   // P^T, dS^T of sub-tile i in buffer i&1
-  __shared__ __align__(8) uint64_t buf_free[2];
+  __shared__ __align__(8) uint64_t sdp_full;            // S^T, dP^T of sub-tile i complete
+  __shared__ __align__(8) uint64_t sdp_free;            // the softmax warps loaded them
+  __shared__ __align__(8) uint64_t pds_full;            // P^T, dS^T of sub-tile i in smem
+  __shared__ __align__(8) uint64_t pds_free;            // the products that read them completed
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sK = sbase, sStage = sbase + kTileR;
-  const uint32_t sStat = sStage + kKStages * kKStage;
   // stage s: Q' sub-tile (32 KB, padded rope block) and G sub-tile (24 KB) at sStage + s * kKStage;
-  // their lse [64] and Delta [64] (512 B) at sStat + s * kStatBytes
+  // their lse [64] and Delta [64] (512 B) at sStat + s * kStatBytes; then the P^T and dS^T operands
+  const uint32_t sStage = sbase;
+  const uint32_t sStat = sStage + kKStages * kKStage;
+  const uint32_t sP = sStat + kStatArea, sDS = sP + kOpBytes;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int kt = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
   const int n_iter = p.heads_per_group * p.n_qs;
@@ -348,20 +389,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
-    mbar_init(smem_u32(&k_full), 1);
+    mbar_init(smem_u32(&a_ready), kSoftmaxK);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(smem_u32(&qg_full[s]), 1);
       mbar_init(smem_u32(&qg_empty[s]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&buf_free[i]), 1);
-    }
-    mbar_init(smem_u32(&ps_full[0]), kSoftmaxThreads);
-    mbar_init(smem_u32(&ps_full[1]), kSoftmaxThreads);
+    mbar_init(smem_u32(&sdp_full), 1);
+    mbar_init(smem_u32(&sdp_free), kSoftmaxK);
+    mbar_init(smem_u32(&pds_full), kSoftmaxK);
+    mbar_init(smem_u32(&pds_free), 1);
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarpK) {
     tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
     tmem_relinquish();
   }
@@ -370,14 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == kProducerWarp) {
+  if (warp == kProducerWarpK) {
     if (lane == 0) {
-      const uint32_t kb = smem_u32(&k_full);
-      mbar_arrive_expect_tx(kb, kTileR);
-      // the key tile is only read K-major: its rope block keeps 64-byte rows
-      const int r0 = kt < p.nt_ring ? kt * kR : p.nc_pad + (kt - p.nt_ring) * kR;
-      for (int i = 0; i < 3; ++i) tma_load_3d(sK + i * kBlkR, &tm_keys, kb, 64 * i, r0, b);
-      tma_load_3d(sK + 3 * kBlkR, &tm_keys_r, kb, kDc, r0, b);
       bool ok = true;
       for (int it = 0; it < n_iter && ok; ++it) {
         const int s = it % kKStages;
@@ -401,66 +434,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(sStat + s * kStatBytes + kS * 4, p.delta + so, stat_bytes, fb);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarpK) {
     if (lane == 0) {
-      bool ok = mbar_wait_or_abort(smem_u32(&k_full), 0, abort_flag, p.dev_status);
+      bool ok = mbar_wait_or_abort(smem_u32(&a_ready), 0, abort_flag, p.dev_status);
       for (int it = 0; it <= n_iter && ok; ++it) {
         if (it < n_iter) {
-          const int s = it % kKStages, buf = it & 1;
-          // S^T / dP^T(it) overwrite the buffers whose P^T / dS^T(it-2) the products of it-2
-          // read: those were issued earlier by this thread, and its MMAs run in issue order
+          const int s = it % kKStages;
           ok = mbar_wait_or_abort(smem_u32(&qg_full[s]), (it / kKStages) & 1, abort_flag,
-                                  p.dev_status);
+                                  p.dev_status) &&
+               (it == 0 || mbar_wait_or_abort(smem_u32(&sdp_free), (it - 1) & 1, abort_flag,
+                                              p.dev_status));
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = sStage + s * kKStage;
-          mma_k224(tmem + kColS + 64 * buf, sK, kBlkR, false, st, kBlkS, true);
-          mma_k192(tmem + kColDP + 64 * buf, sK, kBlkR, st + kTileS, kBlkS);
-          mma_commit(smem_u32(&s_full[buf]));
+          mma_tmem_a<kD / 16>(tmem + kColS, tmem + kColA, st);
+          mma_tmem_a<kDc / 16>(tmem + kColDP, tmem + kColA, st + kTileS);
+          mma_commit(smem_u32(&sdp_full));
         }
         if (it >= 1) {
-          const int ip = it - 1, sp = ip % kKStages, bp = ip & 1;
-          ok = mbar_wait_or_abort(smem_u32(&ps_full[bp]), (ip >> 1) & 1, abort_flag,
-                                  p.dev_status);
+          const int ip = it - 1, sp = ip % kKStages;
+          ok = mbar_wait_or_abort(smem_u32(&pds_full), ip & 1, abort_flag, p.dev_status);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t st = sStage + sp * kKStage;
+          const uint32_t stp = sStage + sp * kKStage;
           // key gradient dS^T Q' over all 256 columns first (it initialises the accumulator),
           // then the value gradient P^T G into the content columns
-          mma_tmem_by_sub<256>(tmem + kColAcc, tmem + kColDP + 64 * bp, st, ip > 0);
-          mma_tmem_by_sub<kDc>(tmem + kColAcc, tmem + kColS + 64 * bp, st + kTileS, true);
+          mma_op_by_sub<256>(tmem + kColAcc, sDS, stp, ip > 0);
+          mma_op_by_sub<kDc>(tmem + kColAcc, sP, stp + kTileS, true);
           mma_commit(smem_u32(&qg_empty[sp]));
-          mma_commit(smem_u32(&buf_free[bp]));
+          mma_commit(smem_u32(&pds_free));
         }
       }
     }
   } else {
-    const int row = warp * 32 + lane;           // key row of the tile
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // softmax warps: warps w and w + 4 share TMEM lanes 32 (w % 4) ...; each takes half of the
+    // columns (ch = 0: sub-tile columns 0-31, 1: 32-63)
+    const int quad = warp & 3, ch = warp >> 2;
+    const int row = quad * 32 + lane;           // key row of the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const bool key_ok = kt < p.nt_ring ? kt * kR + row < p.nc
                                        : (kt - p.nt_ring) * kR + row < p.n_q;
+    const int prow = kt < p.nt_ring ? kt * kR + row : p.nc_pad + (kt - p.nt_ring) * kR + row;
+    {
+      // the key row into TMEM (bf16 pairs 0-63 by the first half, 64-111 by the second); rows
+      // past the valid keys are zero in the padded copy
+      const bf16* src = p.keys + (static_cast<int64_t>(b) * p.rows_ws + prow) * kBwdKeyWidth;
+      row_to_tmem(tmem + lane_off + kColA + 64 * ch, src + 128 * ch, ch == 0 ? 64 : kAWords - 64);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&a_ready));
+    }
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
-      const int s = it % kKStages, buf = it & 1;
+      const int s = it % kKStages;
       // S^T and dP^T of sub-tile it, and the column statistics the bulk copies of qg_full
       // brought (observed directly: the copies complete on that barrier)
       ok = __all_sync(0xffffffffu,
-                      mbar_wait_or_abort(smem_u32(&s_full[buf]), (it >> 1) & 1, abort_flag,
+                      mbar_wait_or_abort(smem_u32(&sdp_full), it & 1, abort_flag,
                                          p.dev_status) &&
                           mbar_wait_or_abort(smem_u32(&qg_full[s]), (it / kKStages) & 1,
                                              abort_flag, p.dev_status));
       if (!ok) break;
       tc_fence_after();
+      uint32_t rs[32], rp[32];
+      tmem_ld32_wait(tmem + lane_off + kColS + 32 * ch, rs);
+      tmem_ld32_wait(tmem + lane_off + kColDP + 32 * ch, rp);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sdp_free));
       const float* col_lse = reinterpret_cast<const float*>(
-          smem_raw + (sStat + s * kStatBytes - smem_u32(smem_raw)));
+          smem_raw + (sStat + s * kStatBytes - smem_u32(smem_raw))) + 32 * ch;
       const float* col_delta = col_lse + kS;
-      const int ncols = min(kS, p.n_q - (it % p.n_qs) * kS);
-      uint32_t rs[64], rp[64];
-      tmem_ld64_wait(tmem + lane_off + kColS + 64 * buf, rs);
-      tmem_ld64_wait(tmem + lane_off + kColDP + 64 * buf, rp);
-      uint32_t wp[32], wd[32];
+      const int ncols = min(kS, p.n_q - (it % p.n_qs) * kS) - 32 * ch;
+      uint32_t wp[16], wd[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         float pp[2], dd[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -475,31 +522,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         wp[i] = pack_bf16x2(pp[0], pp[1]);
         wd[i] = pack_bf16x2(dd[0], dd[1]);
       }
+      // the operands of sub-tile it-1 were read by its products
+      if (it >= 1)
+        ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&pds_free), (it - 1) & 1,
+                                                        abort_flag, p.dev_status));
+      if (!ok) break;
 #pragma unroll
-      for (int c = 0; c < 32; c += 16) {
-        uint32_t w16[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w16[i] = wp[c + i];
-        tmem_st16(tmem + lane_off + kColS + 64 * buf + c, w16);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w16[i] = wd[c + i];
-        tmem_st16(tmem + lane_off + kColDP + 64 * buf + c, w16);
+      for (int c = 0; c < 4; ++c) {
+        st_shared_v4(swz128(sP, row, 4 * ch + c), wp[4 * c], wp[4 * c + 1], wp[4 * c + 2], wp[4 * c + 3]);
+        st_shared_v4(swz128(sDS, row, 4 * ch + c), wd[4 * c], wd[4 * c + 1], wd[4 * c + 2], wd[4 * c + 3]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&ps_full[buf]));
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&pds_full));
     }
     if (ok)
-      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&buf_free[(n_iter - 1) & 1]),
-                                                      ((n_iter - 1) >> 1) & 1, abort_flag,
-                                                      p.dev_status));
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&pds_free), (n_iter - 1) & 1,
+                                                      abort_flag, p.dev_status));
     if (ok) {
       tc_fence_after();
-      const int prow = kt < p.nt_ring ? kt * kR + row : p.nc_pad + (kt - p.nt_ring) * kR + row;
       float* out = p.partial +
                    ((static_cast<int64_t>(grp) * gridDim.z + b) * p.rows_ws + prow) * kD;
+      // columns [0, 128) by the first half, [128, 224) by the second
 #pragma unroll 1
-      for (int c = 0; c < kD; c += 32) {
+      for (int c = 128 * ch; c < (ch == 0 ? 128 : kD); c += 32) {
         uint32_t r[32];
         tmem_ld32_wait(tmem + lane_off + kColAcc + c, r);
         float4* d4 = reinterpret_cast<float4*>(out + c);
@@ -512,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarpK) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -611,10 +656,10 @@ bool tc_bwd_supported(const Dims& d) {
 namespace {
 
 // Tensor maps of the backward's operands with row boxes of `rows` (128 for a tile a CTA owns, 64
-// for a streamed sub-tile).  keys / keys_r: the padded key copy, 64-column boxes with the
-// 128-byte swizzle / the 32 positional columns with the 64-byte swizzle.
+// for a streamed sub-tile), all with 64-column boxes and the 128-byte swizzle; keys: the padded
+// key copy.
 struct BwdMaps {
-  CUtensorMap q, qr, g, keys, keys_r;
+  CUtensorMap q, g, keys;
 };
 
 mla_status make_bwd_maps(const Dims& d, const BwdArgs& a, const KeyWorkspace& kw,
@@ -627,8 +672,6 @@ mla_status make_bwd_maps(const Dims& d, const BwdArgs& a, const KeyWorkspace& kw
                                  static_cast<uint64_t>(d.n_q) * d.H * kD * 2};
     const uint32_t box[4] = {64, 1, rows, 1};
     if ((st = make_tmap_bf16(&m->q, a.q, 4, dims, strides, box, 128)) != MLA_OK) return st;
-    const uint32_t box_r[4] = {kDr, 1, rows, 1};
-    if ((st = make_tmap_bf16(&m->qr, a.q, 4, dims, strides, box_r, 64)) != MLA_OK) return st;
   }
   {
     const uint64_t dims[4] = {static_cast<uint64_t>(kDc), static_cast<uint64_t>(d.H),
@@ -645,9 +688,6 @@ mla_status make_bwd_maps(const Dims& d, const BwdArgs& a, const KeyWorkspace& kw
                                  static_cast<uint64_t>(kw.rows) * kBwdKeyWidth * 2};
     const uint32_t box[3] = {64, rows, 1};
     if ((st = make_tmap_bf16(&m->keys, keys_tc, 3, dims, strides, box, 128)) != MLA_OK) return st;
-    const uint32_t box_r[3] = {kDr, rows, 1};
-    if ((st = make_tmap_bf16(&m->keys_r, keys_tc, 3, dims, strides, box_r, 64)) != MLA_OK)
-      return st;
   }
   return MLA_OK;
 }
@@ -671,6 +711,7 @@ mla_status attention_bwd_tc(const Dims& d, const BwdArgs& a, int n_valid, int fi
   p.n_qs = ceil_div(d.n_q, kS);
   p.rows_ws = kw.rows; p.heads_per_group = d.H / groups;
   p.scale = d.scale; p.scale_log2 = d.scale * kLog2e;
+  p.q = static_cast<const bf16*>(a.q); p.keys = static_cast<const bf16*>(keys_tc);
   p.lse = a.lse; p.delta = delta; p.d_q = a.d_q; p.partial = partial; p.dev_status = dev_status;
   {
     const int64_t pieces = static_cast<int64_t>(d.B) * kw.rows * (kBwdKeyWidth / 8);
@@ -685,13 +726,15 @@ mla_status attention_bwd_tc(const Dims& d, const BwdArgs& a, int n_valid, int fi
                                     kSmemQ));
   MLA_CUDA_TRY(cudaFuncSetAttribute(bwd_dkey_tc_kernel,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemK));
-  // dQ kernel: owns a 128-row query tile (Q', G by 128-row boxes), streams 64-key sub-tiles
+  // dQ kernel: owns a 128-row query tile (Q' copied into TMEM by its threads, G by 128-row
+  // boxes), streams 64-key sub-tiles
   dim3 gq(ceil_div(d.n_q, kR), d.H, d.B);
-  bwd_dq_tc_kernel<<<gq, kThreads, kSmemQ, s>>>(m128.q, m128.qr, m128.g, m64.keys, p);
+  bwd_dq_tc_kernel<<<gq, kThreadsQ, kSmemQ, s>>>(m128.g, m64.keys, p);
   MLA_LAUNCH_CHECK("bwd_dq_tc");
-  // key kernel: owns a 128-key tile, streams 64-query sub-tiles (Q', G by 64-row boxes)
+  // key kernel: owns a 128-key tile (copied into TMEM by its threads), streams 64-query
+  // sub-tiles (Q', G by 64-row boxes)
   dim3 gk(p.nt, groups, d.B);
-  bwd_dkey_tc_kernel<<<gk, kThreads, kSmemK, s>>>(m64.q, m64.g, m128.keys, m128.keys_r, p);
+  bwd_dkey_tc_kernel<<<gk, kThreadsK, kSmemK, s>>>(m64.q, m64.g, p);
   MLA_LAUNCH_CHECK("bwd_dkey_tc");
   const int64_t total = static_cast<int64_t>(d.B) * (kw.nc + d.n_q) * (kD / 2);
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));
