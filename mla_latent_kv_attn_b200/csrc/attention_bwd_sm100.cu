@@ -65,13 +65,14 @@ constexpr int kSmemQ = kTileGR + kQStages * kTileS + 2 * kOpBytes + 1024;
 // key kernel: 8 softmax warps (two per TMEM lane quarter, each half of the columns)
 constexpr int kSoftmaxK = 256, kThreadsK = kSoftmaxK + 64;
 constexpr int kProducerWarpK = 8, kMmaWarpK = 9;
-constexpr int kKStage = kTileS + kTileGS;                     // Q' + G sub-tiles
+// a key-kernel stage stacks a Q' sub-tile over a G sub-tile: block i (64 columns) holds 128
+// rows, Q' rows 0-63 then G rows 0-63; the G half of block 3 (past G's 192 columns) is zero
+constexpr int kBlkQG = 2 * kBlkS;                             // 16 KB
+constexpr int kKStage = 4 * kBlkQG;                           // 64 KB
 constexpr int kKStages = 3;
 constexpr int kStatBytes = 2 * kS * 4;                        // lse and Delta of a sub-tile
-constexpr int kStatArea = 2048;                               // kKStages * kStatBytes, padded
-constexpr int kSmemK = kKStages * kKStage + kStatArea + 2 * kOpBytes + 1024;
-static_assert(kKStages * kStatBytes <= kStatArea, "stat area");
-static_assert(kSmemQ <= 227 * 1024 && kSmemK <= 227 * 1024, "shared memory");
+constexpr int kSmemK = kKStages * kKStage + 2 * kOpBytes + kKStages * kStatBytes + 1024;
+static_assert(kSmemQ <= 227 * 1024 && kSmemK + 256 <= 227 * 1024, "shared memory");
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdTcParams {
@@ -119,42 +120,56 @@ __device__ __forceinline__ uint64_t mnmajor_content(uint32_t a, uint32_t blk_byt
 }
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(kR, kS, 0, 0);     // S, dP: M128 N64, K-major
+constexpr uint32_t kIdescSD = idesc_bf16_f32(kR, 2 * kS, 0, 0); // [S | dP]: M128 N128, K-major
 constexpr uint32_t kIdescC = idesc_bf16_f32(kR, kDc, 0, 1);    // B MN-major, N 192
 constexpr uint32_t kIdescW = idesc_bf16_f32(kR, 256, 0, 1);    // B MN-major, N 256
 
-// D = A B^T, A (128 rows) in TMEM as bf16 pairs from column a_tmem (8 columns per k-step), B a
-// K-major sub-tile of 64 rows whose 64-column blocks lie kBlkS apart; kSteps k-steps of 16.
-template <int kSteps>
-__device__ __forceinline__ void mma_tmem_a(uint32_t d, uint32_t a_tmem, uint32_t b_tile) {
-  const uint64_t b = kmajor_content(b_tile);
+// S = A_S B_S^T over K 224 (A in TMEM from column a_tmem) and dP = A_dP B_dP^T over the 192
+// content columns (A in TMEM from the same column when kDpTmem, else a K-major 128-row tile in
+// shared memory at dp_smem, blocks kBlkR apart); B_S / B_dP: K-major 64-row sub-tiles, blocks
+// kBlkS apart.  The k-steps of the two are issued alternately: the accumulations are
+// independent, so an MMA need not wait for the accumulator write of its own predecessor.
+template <bool kDpTmem>
+__device__ __forceinline__ void mma_s_dp(uint32_t s_acc, uint32_t dp_acc, uint32_t a_tmem,
+                                         uint32_t dp_smem, uint32_t bs_tile, uint32_t bdp_tile) {
+  const uint64_t bs = kmajor_content(bs_tile), bd = kmajor_content(bdp_tile);
+  const uint64_t ad = kmajor_content(dp_smem);
 #pragma unroll
-  for (int kk = 0; kk < kSteps; ++kk)
-    mma_ts(d, a_tmem + 8 * kk, b + (((kk >> 2) * kBlkS) >> 4) + 2 * (kk & 3), kIdescS,
+  for (int kk = 0; kk < kD / 16; ++kk) {
+    const uint32_t off = (((kk >> 2) * kBlkS) >> 4) + 2 * (kk & 3);
+    mma_ts(s_acc, a_tmem + 8 * kk, bs + off, kIdescS, kk ? 1u : 0u);
+    if (kk < kDc / 16) {
+      if (kDpTmem)
+        mma_ts(dp_acc, a_tmem + 8 * kk, bd + off, kIdescS, kk ? 1u : 0u);
+      else
+        mma_ss(dp_acc, ad + (((kk >> 2) * kBlkR) >> 4) + 2 * (kk & 3), bd + off, kIdescS,
+               kk ? 1u : 0u);
+    }
+  }
+}
+
+// [S | dP] = A [Q'_i ; G'_i]^T in one N=128 MMA chain over K 224: A (the key tile) in TMEM from
+// column a_tmem, B a stacked stage (blocks kBlkQG apart).  G'_i is G_i with 32 zero columns
+// appended, so the second half of the result is V G_i^T: the content columns of the key tile
+// times G_i (the positional part meets the zeros).
+__device__ __forceinline__ void mma_s_dp_stacked(uint32_t d, uint32_t a_tmem, uint32_t stage) {
+  const uint64_t b = kmajor_content(stage);
+#pragma unroll
+  for (int kk = 0; kk < kD / 16; ++kk)
+    mma_ts(d, a_tmem + 8 * kk, b + (((kk >> 2) * kBlkQG) >> 4) + 2 * (kk & 3), kIdescSD,
            kk ? 1u : 0u);
 }
 
-// D = A B^T over the 192 content columns, both operands K-major in shared memory; a_blk / b_blk:
-// byte stride of the 64-column blocks of A / B.
-__device__ __forceinline__ void mma_k192(uint32_t d, uint32_t a_tile, uint32_t a_blk,
-                                         uint32_t b_tile, uint32_t b_blk) {
-  const uint64_t ac = kmajor_content(a_tile), bc = kmajor_content(b_tile);
-#pragma unroll
-  for (int blk = 0; blk < 3; ++blk)
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_ss(d, ac + ((blk * a_blk) >> 4) + 2 * kk, bc + ((blk * b_blk) >> 4) + 2 * kk, kIdescS,
-             (blk | kk) != 0 ? 1u : 0u);
-}
-
 // acc[:, 0:kN] (+)= A (128 x 64 bf16, K-major 128-byte swizzled rows in smem) . sub[:, 0:kN],
-// kN = 192 (content blocks) or 256 (all four blocks of a padded sub-tile); K = the 64 rows of the
-// sub-tile, one MMA per k-step (A 32 bytes further, B 16 rows = 2048 bytes further).
+// kN = 192 (content blocks) or 256 (all four blocks of a padded sub-tile), the sub-tile's
+// 64-column blocks blk_bytes apart; K = its 64 rows, one MMA per k-step (A 32 bytes further, B
+// 16 rows = 2048 bytes further).
 template <int kN>
 __device__ __forceinline__ void mma_op_by_sub(uint32_t acc, uint32_t a_smem, uint32_t sub,
-                                              bool accumulate) {
+                                              uint32_t blk_bytes, bool accumulate) {
   static_assert(kN == kDc || kN == 256, "product width");
   const uint64_t a = kmajor_content(a_smem);
-  const uint64_t b = mnmajor_content(sub, kBlkS);
+  const uint64_t b = mnmajor_content(sub, blk_bytes);
 #pragma unroll
   for (int kk = 0; kk < kS / 16; ++kk)
     mma_ss(acc, a + 2 * kk, b + 128 * kk, kN == kDc ? kIdescC : kIdescW,
@@ -259,8 +274,7 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t kt = sK + s * kTileS;
-          mma_tmem_a<kD / 16>(tmem + kColS, tmem + kColA, kt);
-          mma_k192(tmem + kColDP, sG, kBlkR, kt, kBlkS);
+          mma_s_dp<false>(tmem + kColS, tmem + kColDP, tmem + kColA, sG, kt, kt);
           mma_commit(smem_u32(&sdp_full));
         }
         if (j >= 1) {
@@ -269,7 +283,8 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
                                   p.dev_status);
           if (!ok) break;
           tc_fence_after();
-          mma_op_by_sub<256>(tmem + kColAcc, sDS + bp * kOpBytes, sK + sp * kTileS, jp > 0);
+          mma_op_by_sub<256>(tmem + kColAcc, sDS + bp * kOpBytes, sK + sp * kTileS, kBlkS,
+                             jp > 0);
           mma_commit(smem_u32(&kv_empty[sp]));
           mma_commit(smem_u32(&ds_free[bp]));
         }
@@ -377,11 +392,11 @@ __global__ void __launch_bounds__(kThreadsK, 1)
   __shared__ int abort_sh;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  // stage s: Q' sub-tile (32 KB, padded rope block) and G sub-tile (24 KB) at sStage + s * kKStage;
-  // their lse [64] and Delta [64] (512 B) at sStat + s * kStatBytes; then the P^T and dS^T operands
+  // stage s (64 KB, Q' sub-tile stacked over G, see kBlkQG) at sStage + s * kKStage; then the P^T
+  // and dS^T operands; then lse [64] and Delta [64] (512 B) of stage s at sStat + s * kStatBytes
   const uint32_t sStage = sbase;
-  const uint32_t sStat = sStage + kKStages * kKStage;
-  const uint32_t sP = sStat + kStatArea, sDS = sP + kOpBytes;
+  const uint32_t sP = sStage + kKStages * kKStage, sDS = sP + kOpBytes;
+  const uint32_t sStat = sDS + kOpBytes;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int kt = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
   const int n_iter = p.heads_per_group * p.n_qs;
@@ -400,6 +415,12 @@ __global__ void __launch_bounds__(kThreadsK, 1)
     mbar_init(smem_u32(&pds_free), 1);
     fence_barrier_init();
   }
+  // the G half of every stage's fourth block stays zero (no load writes it)
+  for (int i = threadIdx.x; i < kKStages * kBlkS / 16; i += kThreadsK) {
+    const int s = i / (kBlkS / 16), o = i % (kBlkS / 16);
+    st_shared_v4(sStage + s * kKStage + 3 * kBlkQG + kBlkS + 16 * o, 0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
   if (warp == kMmaWarpK) {
     tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
     tmem_relinquish();
@@ -428,8 +449,9 @@ __global__ void __launch_bounds__(kThreadsK, 1)
         mbar_arrive_expect_tx(fb, kTileS + kTileGS + 2 * stat_bytes);
         // the fourth box covers columns 192-255 of Q': 224-255 lie past the row and are
         // filled with zeros (the padded rope block); the byte count is the full box
-        for (int i = 0; i < 4; ++i) tma_load_4d(st + i * kBlkS, &tm_q, fb, 64 * i, h, q0, b);
-        for (int i = 0; i < 3; ++i) tma_load_4d(st + kTileS + i * kBlkS, &tm_g, fb, 64 * i, h, q0, b);
+        for (int i = 0; i < 4; ++i) tma_load_4d(st + i * kBlkQG, &tm_q, fb, 64 * i, h, q0, b);
+        for (int i = 0; i < 3; ++i)
+          tma_load_4d(st + i * kBlkQG + kBlkS, &tm_g, fb, 64 * i, h, q0, b);
         bulk_load(sStat + s * kStatBytes, p.lse + so, stat_bytes, fb);
         bulk_load(sStat + s * kStatBytes + kS * 4, p.delta + so, stat_bytes, fb);
       }
@@ -447,8 +469,7 @@ __global__ void __launch_bounds__(kThreadsK, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t st = sStage + s * kKStage;
-          mma_tmem_a<kD / 16>(tmem + kColS, tmem + kColA, st);
-          mma_tmem_a<kDc / 16>(tmem + kColDP, tmem + kColA, st + kTileS);
+          mma_s_dp_stacked(tmem + kColS, tmem + kColA, st);
           mma_commit(smem_u32(&sdp_full));
         }
         if (it >= 1) {
@@ -459,8 +480,8 @@ __global__ void __launch_bounds__(kThreadsK, 1)
           const uint32_t stp = sStage + sp * kKStage;
           // key gradient dS^T Q' over all 256 columns first (it initialises the accumulator),
           // then the value gradient P^T G into the content columns
-          mma_op_by_sub<256>(tmem + kColAcc, sDS, stp, ip > 0);
-          mma_op_by_sub<kDc>(tmem + kColAcc, sP, stp + kTileS, true);
+          mma_op_by_sub<256>(tmem + kColAcc, sDS, stp, kBlkQG, ip > 0);
+          mma_op_by_sub<kDc>(tmem + kColAcc, sP, stp + kBlkS, kBlkQG, true);
           mma_commit(smem_u32(&qg_empty[sp]));
           mma_commit(smem_u32(&pds_free));
         }
@@ -501,9 +522,17 @@ __global__ void __launch_bounds__(kThreadsK, 1)
       tmem_ld32_wait(tmem + lane_off + kColDP + 32 * ch, rp);
       tc_fence_before();
       mbar_arrive(smem_u32(&sdp_free));
-      const float* col_lse = reinterpret_cast<const float*>(
-          smem_raw + (sStat + s * kStatBytes - smem_u32(smem_raw))) + 32 * ch;
-      const float* col_delta = col_lse + kS;
+      const float4* col_lse = reinterpret_cast<const float4*>(
+          smem_raw + (sStat + s * kStatBytes - smem_u32(smem_raw))) + 8 * ch;
+      const float4* col_delta = col_lse + kS / 4;
+      float nl[32], dl[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 l = col_lse[i], d = col_delta[i];
+        nl[4 * i] = -l.x * kLog2e; nl[4 * i + 1] = -l.y * kLog2e;
+        nl[4 * i + 2] = -l.z * kLog2e; nl[4 * i + 3] = -l.w * kLog2e;
+        dl[4 * i] = d.x; dl[4 * i + 1] = d.y; dl[4 * i + 2] = d.z; dl[4 * i + 3] = d.w;
+      }
       const int ncols = min(kS, p.n_q - (it % p.n_qs) * kS) - 32 * ch;
       uint32_t wp[16], wd[16];
 #pragma unroll
@@ -513,11 +542,10 @@ __global__ void __launch_bounds__(kThreadsK, 1)
         for (int u = 0; u < 2; ++u) {
           const int c = 2 * i + u;
           const bool col_ok = key_ok && c < ncols;
-          const float pr = col_ok ? fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 -
-                                              col_lse[c] * kLog2e)
+          const float pr = col_ok ? fast_exp2(fmaf(__uint_as_float(rs[c]), p.scale_log2, nl[c]))
                                   : 0.f;
           pp[u] = pr;
-          dd[u] = col_ok ? pr * (__uint_as_float(rp[c]) - col_delta[c]) * p.scale : 0.f;
+          dd[u] = col_ok ? pr * (__uint_as_float(rp[c]) - dl[c]) * p.scale : 0.f;
         }
         wp[i] = pack_bf16x2(pp[0], pp[1]);
         wd[i] = pack_bf16x2(dd[0], dd[1]);
