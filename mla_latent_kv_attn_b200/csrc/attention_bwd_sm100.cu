@@ -319,17 +319,29 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
       tmem_ld64_wait(tmem + lane_off + kColDP, rp);
       tc_fence_before();
       mbar_arrive(smem_u32(&sdp_free));
+      // pairs of columns on the packed fp32 pipe: x = S scale log2(e) - lse log2(e),
+      // dS = exp2(x) (dP scale - Delta scale); columns past the valid keys get P = 0
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(-lse2, -lse2);
+      const uint64_t dsc2 = f2_pack(p.scale, p.scale);
+      const uint64_t nd2 = f2_pack(-delta * p.scale, -delta * p.scale);
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        float d2[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = 2 * i + u;
-          const float pr = c < valid ? fast_exp2(__uint_as_float(rs[c]) * p.scale_log2 - lse2) : 0.f;
-          d2[u] = pr * (__uint_as_float(rp[c]) - delta) * p.scale;
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * i]), __uint_as_float(rs[2 * i + 1])), sc2,
+                         nl2),
+                  x0, x1);
+        float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        if (valid < kS) {
+          p0 = 2 * i < valid ? p0 : 0.f;
+          p1 = 2 * i + 1 < valid ? p1 : 0.f;
         }
-        w[i] = pack_bf16x2(d2[0], d2[1]);
+        float d0, d1;
+        f2_unpack(f2_mul(f2_fma(f2_pack(__uint_as_float(rp[2 * i]), __uint_as_float(rp[2 * i + 1])),
+                                dsc2, nd2),
+                         f2_pack(p0, p1)),
+                  d0, d1);
+        w[i] = pack_bf16x2(d0, d1);
       }
       // buffer j&1 was last read by the products of sub-tile j-2
       if (j >= 2)
@@ -522,33 +534,44 @@ __global__ void __launch_bounds__(kThreadsK, 1)
       tmem_ld32_wait(tmem + lane_off + kColDP + 32 * ch, rp);
       tc_fence_before();
       mbar_arrive(smem_u32(&sdp_free));
+      // column statistics as packed pairs: -lse log2(e) and -Delta scale
       const float4* col_lse = reinterpret_cast<const float4*>(
           smem_raw + (sStat + s * kStatBytes - smem_u32(smem_raw))) + 8 * ch;
       const float4* col_delta = col_lse + kS / 4;
-      float nl[32], dl[32];
+      const uint64_t nlog2e2 = f2_pack(-kLog2e, -kLog2e), nsc2 = f2_pack(-p.scale, -p.scale);
+      uint64_t nl2[16], nd2[16];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float4 l = col_lse[i], d = col_delta[i];
-        nl[4 * i] = -l.x * kLog2e; nl[4 * i + 1] = -l.y * kLog2e;
-        nl[4 * i + 2] = -l.z * kLog2e; nl[4 * i + 3] = -l.w * kLog2e;
-        dl[4 * i] = d.x; dl[4 * i + 1] = d.y; dl[4 * i + 2] = d.z; dl[4 * i + 3] = d.w;
+        nl2[2 * i] = f2_mul(f2_pack(l.x, l.y), nlog2e2);
+        nl2[2 * i + 1] = f2_mul(f2_pack(l.z, l.w), nlog2e2);
+        nd2[2 * i] = f2_mul(f2_pack(d.x, d.y), nsc2);
+        nd2[2 * i + 1] = f2_mul(f2_pack(d.z, d.w), nsc2);
       }
+      // pairs of columns on the packed fp32 pipe; past the valid queries (or for a key row
+      // past the valid keys) P and dS are 0, whatever the stale statistics there hold
       const int ncols = min(kS, p.n_q - (it % p.n_qs) * kS) - 32 * ch;
+      const bool full = key_ok && ncols >= 32;
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), dsc2 = f2_pack(p.scale, p.scale);
       uint32_t wp[16], wd[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        float pp[2], dd[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = 2 * i + u;
-          const bool col_ok = key_ok && c < ncols;
-          const float pr = col_ok ? fast_exp2(fmaf(__uint_as_float(rs[c]), p.scale_log2, nl[c]))
-                                  : 0.f;
-          pp[u] = pr;
-          dd[u] = col_ok ? pr * (__uint_as_float(rp[c]) - dl[c]) * p.scale : 0.f;
+        float x0, x1, d0, d1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * i]), __uint_as_float(rs[2 * i + 1])), sc2,
+                         nl2[i]),
+                  x0, x1);
+        float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        f2_unpack(f2_mul(f2_fma(f2_pack(__uint_as_float(rp[2 * i]), __uint_as_float(rp[2 * i + 1])),
+                                dsc2, nd2[i]),
+                         f2_pack(p0, p1)),
+                  d0, d1);
+        if (!full) {
+          const bool ok0 = key_ok && 2 * i < ncols, ok1 = key_ok && 2 * i + 1 < ncols;
+          p0 = ok0 ? p0 : 0.f; d0 = ok0 ? d0 : 0.f;
+          p1 = ok1 ? p1 : 0.f; d1 = ok1 ? d1 : 0.f;
         }
-        wp[i] = pack_bf16x2(pp[0], pp[1]);
-        wd[i] = pack_bf16x2(dd[0], dd[1]);
+        wp[i] = pack_bf16x2(p0, p1);
+        wd[i] = pack_bf16x2(d0, d1);
       }
       // the operands of sub-tile it-1 were read by its products
       if (it >= 1)

@@ -100,26 +100,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return y;
 }
 
-// Packed pairs of fp32 (sm_100 FFMA2 / FADD2: two lanes of fp32 arithmetic per instruction).
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
 // 2^x on the FMA pipe, for a pair of arguments in packed form, so that part of the softmax's
 // exponentials bypass the MUFU unit (which otherwise sets the softmax's pace).  x = n + f with
 // n = rint(x) and f in [-1/2, 1/2]; 2^f by the degree-3 polynomial interpolating 2^f at the four
