@@ -11,19 +11,21 @@
 // runs at the tensor rate.  The softmax warps load S and dP into registers and release the TMEM
 // buffers at once, so the S/dP MMAs of the next sub-tile overlap the softmax; P and dS go to
 // shared memory (128-byte-swizzled K-major rows, written the way a TMA load would place them)
-// as the A operands of the gradient products.
+// as the A operands of the key kernel's gradient products; the dQ kernel keeps dS in TMEM,
+// in the 32 columns its N=224 accumulator leaves free.
 // A streamed sub-tile that is read MN-major (K'_j in the dQ kernel, Q'_i in the key kernel) is
 // held 256 columns wide: three 64-column content blocks and a fourth block with the 32
 // positional columns followed by 32 zeros, all with the 128-byte swizzle. Its product is then a
-// single N=256 MMA per k-step (columns 224-255 of the accumulator receive zeros and are never
-// read) instead of an N=192 and a separate, slow, N=32 one. The keys come from a copy the
+// single MMA per k-step instead of an N=192 and a separate, slow, N=32 one: N=256 in the key
+// kernel (columns 224-255 of its accumulator receive zeros and are never read), N=224 in the
+// dQ kernel (the zero half of the fourth block is not read). The keys come from a copy the
 // pre-pass bwd_pad_keys_kernel assembles in the workspace; Q'_i's fourth block is a TMA box that
 // runs past the query's 224 columns, which the copy engine fills with zeros.
 // dQ kernel: one CTA per (128-row query tile, head, sample); per 64-key sub-tile j:
 //   S_j  = Q' K'_j^T       M128 N64 K224    (A: Q' in TMEM, B: K'_j smem, K-major)
 //   dP_j = G  V_j^T        M128 N64 K192    (A: G smem, B: content blocks of K'_j, K-major)
-//   dS_j = scale * P o (dP - Delta), P = exp(S scale - lse)    (softmax warps, bf16 to smem)
-//   dQ  += dS_j K'_j       M128 N256 K64    (A: dS smem, B: K'_j read MN-major)
+//   dS_j = scale * P o (dP - Delta), P = exp(S scale - lse)    (softmax warps, bf16 to TMEM)
+//   dQ  += dS_j K'_j       M128 N224 K64    (A: dS in TMEM, B: K'_j read MN-major)
 // Key kernel: one CTA per (128-key tile, group of heads, sample); per (head, 64-query sub-tile):
 //   S^T  = K' Q'_i^T       M128 N64 K224    (A: K' in TMEM)
 //   dP^T = V  G_i^T        M128 N64 K192    (A: the content columns of K' in TMEM)
@@ -32,7 +34,8 @@
 //   dL  += P^T G_i         M128 N192 K64    (value gradient: the value is the content latent)
 // dL (fp32, 224 wide) goes to a workspace slice per head group; bwd_reduce_kernel sums the
 // groups, maps the positional part back through the transposed rotation and stores bf16.
-// TMEM columns: resident A operand [0,112), S [128,192), dP [192,256), accumulator [256,512).
+// TMEM columns: resident A operand [0,112), S [128,192), dP [192,256), accumulator [256,512)
+// (dQ kernel: [256,480), then dS [480,512)).
 // Roles: softmax / epilogue warps (one TMEM lane = one row), a TMA producer warp, and a warp that
 // allocates TMEM and whose lane 0 issues every MMA.  Every wait is bounded; a wait that runs out
 // writes MLA_ERR_DEVICE_TIMEOUT to dev_status.
@@ -55,13 +58,15 @@ constexpr int kTileS = 4 * kBlkS;           // 32 KB: a 64 x 256 sub-tile (rope 
 constexpr int kTileGS = 3 * kBlkS;          // 24 KB: a 64 x 192 sub-tile of G
 constexpr int kOpBytes = kR * 128;          // 16 KB: a 128 x 64 bf16 operand (dS, P) in smem
 constexpr uint32_t kColA = 0, kColS = 128, kColDP = 192, kColAcc = 256;
+constexpr uint32_t kColDS = kColAcc + kD;   // dQ kernel: dS (bf16 pairs, 32 columns) after an
+                                            // accumulator of N = 224
 constexpr int kAWords = kD / 2;             // 112 TMEM columns of bf16 pairs
 constexpr uint32_t kTmemCols = 512;
 // dQ kernel: 4 softmax warps, producer, MMA
 constexpr int kSoftmaxQ = 128, kThreadsQ = kSoftmaxQ + 64;
 constexpr int kProducerWarpQ = 4, kMmaWarpQ = 5;
-constexpr int kQStages = 4;                                   // K' sub-tiles in flight
-constexpr int kSmemQ = kTileGR + kQStages * kTileS + 2 * kOpBytes + 1024;
+constexpr int kQStages = 5;                                   // K' sub-tiles in flight
+constexpr int kSmemQ = kTileGR + kQStages * kTileS + 1024;
 // key kernel: 8 softmax warps (two per TMEM lane quarter, each half of the columns)
 constexpr int kSoftmaxK = 256, kThreadsK = kSoftmaxK + 64;
 constexpr int kProducerWarpK = 8, kMmaWarpK = 9;
@@ -123,6 +128,7 @@ constexpr uint32_t kIdescS = idesc_bf16_f32(kR, kS, 0, 0);     // S, dP: M128 N6
 constexpr uint32_t kIdescSD = idesc_bf16_f32(kR, 2 * kS, 0, 0); // [S | dP]: M128 N128, K-major
 constexpr uint32_t kIdescC = idesc_bf16_f32(kR, kDc, 0, 1);    // B MN-major, N 192
 constexpr uint32_t kIdescW = idesc_bf16_f32(kR, 256, 0, 1);    // B MN-major, N 256
+constexpr uint32_t kIdescD = idesc_bf16_f32(kR, kD, 0, 1);     // B MN-major, N 224
 
 // S = A_S B_S^T over K 224 (A in TMEM from column a_tmem) and dP = A_dP B_dP^T over the 192
 // content columns (A in TMEM from the same column when kDpTmem, else a K-major 128-row tile in
@@ -176,6 +182,17 @@ __device__ __forceinline__ void mma_op_by_sub(uint32_t acc, uint32_t a_smem, uin
            (accumulate || kk) ? 1u : 0u);
 }
 
+// acc[:, 0:224] (+)= A (128 x 64 bf16, pairs in TMEM from column a_tmem, 8 columns per k-step)
+// . sub[:, 0:224], sub a padded sub-tile read MN-major (blocks kBlkS apart; the fourth block's
+// zero half is not read).  K = its 64 rows.
+__device__ __forceinline__ void mma_tmem_by_sub224(uint32_t acc, uint32_t a_tmem, uint32_t sub,
+                                                   bool accumulate) {
+  const uint64_t b = mnmajor_content(sub, kBlkS);
+#pragma unroll
+  for (int kk = 0; kk < kS / 16; ++kk)
+    mma_ts(acc, a_tmem + 8 * kk, b + 128 * kk, kIdescD, (accumulate || kk) ? 1u : 0u);
+}
+
 // Writes `nwords` bf16 pairs of a global row (16-byte aligned; nullptr: zeros) into this thread's
 // TMEM lane from column taddr on, 16 columns at a time.
 __device__ __forceinline__ void row_to_tmem(uint32_t taddr, const bf16* src, int nwords) {
@@ -203,13 +220,13 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
   __shared__ __align__(8) uint64_t kv_empty[kQStages];
   __shared__ __align__(8) uint64_t sdp_full;    // S(j), dP(j) complete in TMEM
   __shared__ __align__(8) uint64_t sdp_free;    // the softmax warps loaded S(j), dP(j)
-  __shared__ __align__(8) uint64_t ds_full[2];  // dS(j) written to buffer j&1
-  __shared__ __align__(8) uint64_t ds_free[2];  // the products that read buffer b completed
+  __shared__ __align__(8) uint64_t ds_full;     // dS(j) written to TMEM
+  __shared__ __align__(8) uint64_t ds_free;     // the products that read it completed
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sG = sbase, sK = sG + kTileGR, sDS = sK + kQStages * kTileS;
+  const uint32_t sG = sbase, sK = sG + kTileGR;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int q0 = qt * kR;
@@ -225,10 +242,8 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
     }
     mbar_init(smem_u32(&sdp_full), 1);
     mbar_init(smem_u32(&sdp_free), kSoftmaxQ);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&ds_full[i]), kSoftmaxQ);
-      mbar_init(smem_u32(&ds_free[i]), 1);
-    }
+    mbar_init(smem_u32(&ds_full), kSoftmaxQ);
+    mbar_init(smem_u32(&ds_free), 1);
     fence_barrier_init();
   }
   if (warp == kMmaWarpQ) {
@@ -261,7 +276,7 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
   } else if (warp == kMmaWarpQ) {
     if (lane == 0) {
       // Order of issue: S/dP(j) once the softmax has loaded S/dP(j-1), then the dQ products of
-      // sub-tile j-1 once its dS is in shared memory.
+      // sub-tile j-1 once its dS is in TMEM.
       bool ok = mbar_wait_or_abort(smem_u32(&a_ready), 0, abort_flag, p.dev_status) &&
                 mbar_wait_or_abort(smem_u32(&g_full), 0, abort_flag, p.dev_status);
       for (int j = 0; j <= p.ns && ok; ++j) {
@@ -278,15 +293,13 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
           mma_commit(smem_u32(&sdp_full));
         }
         if (j >= 1) {
-          const int jp = j - 1, sp = jp % kQStages, bp = jp & 1;
-          ok = mbar_wait_or_abort(smem_u32(&ds_full[bp]), (jp >> 1) & 1, abort_flag,
-                                  p.dev_status);
+          const int jp = j - 1, sp = jp % kQStages;
+          ok = mbar_wait_or_abort(smem_u32(&ds_full), jp & 1, abort_flag, p.dev_status);
           if (!ok) break;
           tc_fence_after();
-          mma_op_by_sub<256>(tmem + kColAcc, sDS + bp * kOpBytes, sK + sp * kTileS, kBlkS,
-                             jp > 0);
+          mma_tmem_by_sub224(tmem + kColAcc, tmem + kColDS, sK + sp * kTileS, jp > 0);
           mma_commit(smem_u32(&kv_empty[sp]));
-          mma_commit(smem_u32(&ds_free[bp]));
+          mma_commit(smem_u32(&ds_free));
         }
       }
     }
@@ -307,7 +320,6 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
     mbar_arrive(smem_u32(&a_ready));
     bool ok = true;
     for (int j = 0; j < p.ns && ok; ++j) {
-      const int buf = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&sdp_full), j & 1, abort_flag,
                                                       p.dev_status));
       if (!ok) break;
@@ -343,24 +355,28 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
                   d0, d1);
         w[i] = pack_bf16x2(d0, d1);
       }
-      // buffer j&1 was last read by the products of sub-tile j-2
-      if (j >= 2)
-        ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&ds_free[buf]),
-                                                        ((j >> 1) & 1) ^ 1, abort_flag,
-                                                        p.dev_status));
+      // the dS columns were last read by the products of sub-tile j-1
+      if (j >= 1)
+        ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&ds_free), (j - 1) & 1,
+                                                        abort_flag, p.dev_status));
       if (!ok) break;
-      const uint32_t dsb = sDS + buf * kOpBytes;
+      {
+        uint32_t w16[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_shared_v4(swz128(dsb, row, c), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&ds_full[buf]));
+        for (int i = 0; i < 16; ++i) w16[i] = w[i];
+        tmem_st16(tmem + lane_off + kColDS, w16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w16[i] = w[16 + i];
+        tmem_st16(tmem + lane_off + kColDS + 16, w16);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ds_full));
     }
-    // the last dQ products completed: buffer (ns-1)&1 was freed for the ((ns-1)>>1)-th time
+    // the last dQ products completed: the (ns-1)-th completion of ds_free
     if (ok)
-      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&ds_free[(p.ns - 1) & 1]),
-                                                      ((p.ns - 1) >> 1) & 1, abort_flag,
-                                                      p.dev_status));
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&ds_free), (p.ns - 1) & 1,
+                                                      abort_flag, p.dev_status));
     if (ok) {
       tc_fence_after();
       bf16* out = static_cast<bf16*>(p.d_q) + ((static_cast<int64_t>(b) * p.n_q + n) * p.H + h) * kD;
