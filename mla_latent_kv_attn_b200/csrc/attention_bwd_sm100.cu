@@ -130,27 +130,21 @@ constexpr uint32_t kIdescC = idesc_bf16_f32(kR, kDc, 0, 1);    // B MN-major, N 
 constexpr uint32_t kIdescW = idesc_bf16_f32(kR, 256, 0, 1);    // B MN-major, N 256
 constexpr uint32_t kIdescD = idesc_bf16_f32(kR, kD, 0, 1);     // B MN-major, N 224
 
-// S = A_S B_S^T over K 224 (A in TMEM from column a_tmem) and dP = A_dP B_dP^T over the 192
-// content columns (A in TMEM from the same column when kDpTmem, else a K-major 128-row tile in
-// shared memory at dp_smem, blocks kBlkR apart); B_S / B_dP: K-major 64-row sub-tiles, blocks
-// kBlkS apart.  The k-steps of the two are issued alternately: the accumulations are
-// independent, so an MMA need not wait for the accumulator write of its own predecessor.
-template <bool kDpTmem>
+// dQ kernel: S = Q' K'_j^T over K 224 (Q' in TMEM from column a_tmem) and dP = G V_j^T over the
+// 192 content columns (G a K-major 128-row tile in shared memory, blocks kBlkR apart); K'_j a
+// K-major 64-row sub-tile, blocks kBlkS apart.  Both are N=64 chains, at the ~45-cycle floor an
+// M128 K16 instruction has for N <= 64 (32 cycles of work); their k-steps are issued alternately
+// (a probe found no difference from issuing one chain after the other).
 __device__ __forceinline__ void mma_s_dp(uint32_t s_acc, uint32_t dp_acc, uint32_t a_tmem,
-                                         uint32_t dp_smem, uint32_t bs_tile, uint32_t bdp_tile) {
-  const uint64_t bs = kmajor_content(bs_tile), bd = kmajor_content(bdp_tile);
-  const uint64_t ad = kmajor_content(dp_smem);
+                                         uint32_t g_smem, uint32_t k_tile) {
+  const uint64_t bk = kmajor_content(k_tile), ag = kmajor_content(g_smem);
 #pragma unroll
   for (int kk = 0; kk < kD / 16; ++kk) {
     const uint32_t off = (((kk >> 2) * kBlkS) >> 4) + 2 * (kk & 3);
-    mma_ts(s_acc, a_tmem + 8 * kk, bs + off, kIdescS, kk ? 1u : 0u);
-    if (kk < kDc / 16) {
-      if (kDpTmem)
-        mma_ts(dp_acc, a_tmem + 8 * kk, bd + off, kIdescS, kk ? 1u : 0u);
-      else
-        mma_ss(dp_acc, ad + (((kk >> 2) * kBlkR) >> 4) + 2 * (kk & 3), bd + off, kIdescS,
-               kk ? 1u : 0u);
-    }
+    mma_ts(s_acc, a_tmem + 8 * kk, bk + off, kIdescS, kk ? 1u : 0u);
+    if (kk < kDc / 16)
+      mma_ss(dp_acc, ag + (((kk >> 2) * kBlkR) >> 4) + 2 * (kk & 3), bk + off, kIdescS,
+             kk ? 1u : 0u);
   }
 }
 
@@ -289,7 +283,7 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t kt = sK + s * kTileS;
-          mma_s_dp<false>(tmem + kColS, tmem + kColDP, tmem + kColA, sG, kt, kt);
+          mma_s_dp(tmem + kColS, tmem + kColDP, tmem + kColA, sG, kt);
           mma_commit(smem_u32(&sdp_full));
         }
         if (j >= 1) {
