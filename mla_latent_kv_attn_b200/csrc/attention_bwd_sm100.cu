@@ -250,22 +250,26 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
   const uint32_t tmem = tmem_base_sh;
 
   if (warp == kProducerWarpQ) {
+    // one copy per lane (lanes 0-3: the four 64-column blocks), so that a stage's copies go out
+    // at once rather than one after another from a single thread; lane 0 waits and arms
     if (lane == 0) {
       const uint32_t gb = smem_u32(&g_full);
       mbar_arrive_expect_tx(gb, kTileGR);
       for (int i = 0; i < 3; ++i) tma_load_4d(sG + i * kBlkR, &tm_g, gb, 64 * i, h, q0, b);
-      bool ok = true;
-      for (int j = 0; j < p.ns && ok; ++j) {
-        const int s = j % kQStages;
-        ok = mbar_wait_or_abort(smem_u32(&kv_empty[s]), ((j / kQStages) & 1) ^ 1, abort_flag,
-                                p.dev_status);
-        if (!ok) break;
-        const uint32_t dst = sK + s * kTileS;
-        const uint32_t fb = smem_u32(&kv_full[s]);
-        mbar_arrive_expect_tx(fb, kTileS);
-        const int r0 = j < p.ns_ring ? j * kS : p.nc_pad + (j - p.ns_ring) * kS;
-        for (int i = 0; i < 4; ++i) tma_load_3d(dst + i * kBlkS, &tm_keys, fb, 64 * i, r0, b);
-      }
+    }
+    bool ok = true;
+    for (int j = 0; j < p.ns && ok; ++j) {
+      const int s = j % kQStages;
+      ok = __all_sync(0xffffffffu, lane != 0 || mbar_wait_or_abort(smem_u32(&kv_empty[s]),
+                                                                   ((j / kQStages) & 1) ^ 1,
+                                                                   abort_flag, p.dev_status));
+      if (!ok) break;
+      const uint32_t dst = sK + s * kTileS;
+      const uint32_t fb = smem_u32(&kv_full[s]);
+      if (lane == 0) mbar_arrive_expect_tx(fb, kTileS);
+      __syncwarp();
+      const int r0 = j < p.ns_ring ? j * kS : p.nc_pad + (j - p.ns_ring) * kS;
+      if (lane < 4) tma_load_3d(dst + lane * kBlkS, &tm_keys, fb, 64 * lane, r0, b);
     }
   } else if (warp == kMmaWarpQ) {
     if (lane == 0) {
@@ -453,30 +457,37 @@ __global__ void __launch_bounds__(kThreadsK, 1)
   const uint32_t tmem = tmem_base_sh;
 
   if (warp == kProducerWarpK) {
-    if (lane == 0) {
-      bool ok = true;
-      for (int it = 0; it < n_iter && ok; ++it) {
-        const int s = it % kKStages;
-        ok = mbar_wait_or_abort(smem_u32(&qg_empty[s]), ((it / kKStages) & 1) ^ 1, abort_flag,
-                                p.dev_status);
-        if (!ok) break;
-        const int h = grp * p.heads_per_group + it / p.n_qs;
-        const int q0 = (it % p.n_qs) * kS;
-        // column statistics of the sub-tile: n_q is a multiple of 4, so both the source (row
-        // (b, h) of [B, H, n_q] floats, column q0) and the size are 16-byte multiples
-        const uint32_t stat_bytes = static_cast<uint32_t>(min(kS, p.n_q - q0)) * 4u;
-        const int64_t so = (static_cast<int64_t>(b) * p.H + h) * p.n_q + q0;
-        const uint32_t st = sStage + s * kKStage;
-        const uint32_t fb = smem_u32(&qg_full[s]);
-        mbar_arrive_expect_tx(fb, kTileS + kTileGS + 2 * stat_bytes);
-        // the fourth box covers columns 192-255 of Q': 224-255 lie past the row and are
-        // filled with zeros (the padded rope block); the byte count is the full box
-        for (int i = 0; i < 4; ++i) tma_load_4d(st + i * kBlkQG, &tm_q, fb, 64 * i, h, q0, b);
-        for (int i = 0; i < 3; ++i)
-          tma_load_4d(st + i * kBlkQG + kBlkS, &tm_g, fb, 64 * i, h, q0, b);
+    // A stage's nine copies go out from nine lanes at once: issued one after another from a
+    // single thread they take ~500 cycles, which adds to the load latency this kernel is
+    // bound by.  Lane 0 waits for the stage and arms its barrier.
+    bool ok = true;
+    for (int it = 0; it < n_iter && ok; ++it) {
+      const int s = it % kKStages;
+      ok = __all_sync(0xffffffffu, lane != 0 || mbar_wait_or_abort(smem_u32(&qg_empty[s]),
+                                                                   ((it / kKStages) & 1) ^ 1,
+                                                                   abort_flag, p.dev_status));
+      if (!ok) break;
+      const int h = grp * p.heads_per_group + it / p.n_qs;
+      const int q0 = (it % p.n_qs) * kS;
+      // column statistics of the sub-tile: n_q is a multiple of 4, so both the source (row
+      // (b, h) of [B, H, n_q] floats, column q0) and the size are 16-byte multiples
+      const uint32_t stat_bytes = static_cast<uint32_t>(min(kS, p.n_q - q0)) * 4u;
+      const int64_t so = (static_cast<int64_t>(b) * p.H + h) * p.n_q + q0;
+      const uint32_t st = sStage + s * kKStage;
+      const uint32_t fb = smem_u32(&qg_full[s]);
+      if (lane == 0) mbar_arrive_expect_tx(fb, kTileS + kTileGS + 2 * stat_bytes);
+      __syncwarp();
+      // lanes 0-3: the four Q' boxes (the fourth covers columns 192-255: 224-255 lie past the
+      // row and are filled with zeros, the padded rope block; the byte count is the full box);
+      // lanes 4-6: the three G boxes; lanes 7, 8: lse and Delta
+      if (lane < 4)
+        tma_load_4d(st + lane * kBlkQG, &tm_q, fb, 64 * lane, h, q0, b);
+      else if (lane < 7)
+        tma_load_4d(st + (lane - 4) * kBlkQG + kBlkS, &tm_g, fb, 64 * (lane - 4), h, q0, b);
+      else if (lane == 7)
         bulk_load(sStat + s * kStatBytes, p.lse + so, stat_bytes, fb);
+      else if (lane == 8)
         bulk_load(sStat + s * kStatBytes + kS * 4, p.delta + so, stat_bytes, fb);
-      }
     }
   } else if (warp == kMmaWarpK) {
     if (lane == 0) {
