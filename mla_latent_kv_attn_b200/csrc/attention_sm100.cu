@@ -12,20 +12,25 @@
 //              domain with lazy rescaling of O (only when the running max grows by > 8);
 //              write P (bf16) into its TMEM buffer; final 1/l,
 //              optional W_UV epilogue, stores and lse.
-//   warp 4     TMA producer: Q tile once, then 128-key K' tiles into a 3-stage ring: three
-//              128x64 (128B-swizzled) content blocks from the ring/chunk latents and one 128x32
+//              Before the loop they copy their query row into TMEM (DC <= 192, below).
+//   warp 4     TMA producer: 128-key K' tiles into a 4-stage ring: three 128x64
+//              (128B-swizzled) content blocks from the ring/chunk latents and one 128x32
 //              (64B-swizzled) block of pre-rotated positional keys; then the W_UV_h tile.
 //   warps 5, 6 TMEM allocation (warp 5); one thread of warp 5 issues the QK products, one of
 //              warp 6 the PV products and the epilogue (two issuers keep the pipe fed):
-//                S_j   = Q K'_j^T          M=128, N=128, K=224 (12 SW128 + 2 SW64 k-steps)
+//                S_j   = Q K'_j^T          M=128, N=128, K=224 (12 SW128 + 2 SW64 k-steps),
+//                                          Q from TMEM
 //                O    += P_j V_j           M=128, N=192, K=128; P from TMEM, V = content
 //                                          blocks of the same stage read MN-major
 //                o     = O_lat W_UV_h^T    M=128, N=128, K=192 (epilogue, O_lat bf16 in smem)
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+DC), P [256+DC,+64); the epilogue result
-// reuses S0.  P has its own buffer so that a QK may overwrite an S buffer as soon as the
-// softmax has loaded it, instead of after the PV that reads its P.  With DC = 256 O fills the
-// rest of TMEM: P(j) is then written into S buffer j&1 and QK(j+2) waits for PV(j).
-// Stages of the K' ring: as many as shared memory holds, up to 4 (3 from D = 224 up).
+// TMEM columns: S [0,128), Q [128,128+D/2) as bf16 pairs, O [256,256+DC), P [256+DC,+64); the
+// epilogue result reuses S.  With Q in TMEM the QK products read only K' from shared memory
+// (with Q there too, its 4 KB per k-step doubled the operand traffic of QK), and the Q tile's
+// shared memory holds a fourth K' stage.  One S buffer suffices: the softmax loads S(j) into
+// registers and frees the buffer at once, so QK(j+1) overlaps the softmax of j; P has its own
+// buffer for the same reason.
+// With DC = 256 O and P leave no room for Q: Q stays in shared memory, there are two S buffers,
+// P(j) is written into S buffer j&1 and QK(j+2) waits for PV(j).
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -67,18 +72,26 @@ struct AttnShape {
   static constexpr int kRopeKSteps = DR / 16;
   static constexpr int kQTile = kCBlk * kQBlk + kBM * kRopeBytes;
   static constexpr int kKTile = kCBlk * kKBlk + kBN * kRopeBytes;
-  static constexpr int kFit = (kSmemMax - 1024 - kQTile) / kKTile;
-  static constexpr int kStages = kFit < 4 ? kFit : (D >= 224 ? 3 : 4);
-  static_assert(kStages >= 1, "the Q tile and one K' stage must fit in shared memory");
-  static constexpr int kSmem = kQTile + kStages * kKTile + 1024;
-  static_assert(kKTile >= kCBlk * kQBlk, "the W_UV tile is loaded into one K' stage");
   // P (kBN/2 columns of packed bf16) gets its own TMEM columns after O when they fit; with a
   // 256-wide O it is written into the S buffer it came from instead.
   static constexpr bool kAliasP = kColO + DC + kBN / 2 > kTmemCols;
   static constexpr uint32_t kColP = kAliasP ? 0u : kColO + DC;
+  // When P has its own columns, the query tile lives in TMEM (bf16 pairs, D/2 columns from
+  // kColS, written by the softmax threads) in place of the second S buffer: QK reads only K'
+  // from shared memory, and the tile's shared memory becomes one more K' stage.
+  static constexpr bool kQTmem = !kAliasP && D / 2 <= 128;
+  static constexpr int kQWords = (D / 2 + 15) / 16 * 16;    // TMEM columns written (zero tail)
+  static constexpr int kQSmem = kQTmem ? 0 : kQTile;
+  static constexpr int kFit = (kSmemMax - 1024 - kQSmem) / kKTile;
+  static constexpr int kStages = kFit < 4 ? kFit : 4;
+  // (with Q in TMEM, W_UV and O_lat take two different stages after the loop)
+  static_assert(kStages >= (kQTmem ? 2 : 1), "too few K' stages fit in shared memory");
+  static constexpr int kSmem = kQSmem + kStages * kKTile + 1024;
+  static_assert(kKTile >= kCBlk * kQBlk, "the W_UV tile (and O_lat) go into K' stages");
 };
 
 struct AttnParams {
+  const bf16* q;        // [B, n_q, H, D] (read by the softmax threads when Q lives in TMEM)
   int n_q, H, nc, nc_pad, nt_ring, nt;
   float scale_log2;
   int has_w_uv;
@@ -181,8 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kKTile = Sh::kKTile;
   constexpr bool kAliasP = Sh::kAliasP;
   constexpr uint32_t kColP = Sh::kColP;
+  constexpr bool kQTmem = Sh::kQTmem;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full;
+  __shared__ __align__(8) uint64_t q_full;   // the Q tile landed (TMA) or is in TMEM (softmax)
   __shared__ __align__(8) uint64_t kv_full[kStages];
   __shared__ __align__(8) uint64_t kv_empty[kStages];
   __shared__ __align__(8) uint64_t s_full[2];
@@ -197,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_sh;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sQ = sbase;
+  const uint32_t sQ = sbase;                     // (the Q tile, when it is in shared memory)
+  const uint32_t sK0 = sbase + Sh::kQSmem;       // K' stage 0
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int q0 = qt * kBM;
@@ -205,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
-    mbar_init(smem_u32(&q_full), 1);
+    mbar_init(smem_u32(&q_full), kQTmem ? kSoftmaxThreads : 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&kv_full[s]), 1);
       mbar_init(smem_u32(&kv_empty[s]), 1);
@@ -236,19 +251,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_chunk);
       tma_prefetch_desc(&tm_ws);
-      const uint32_t qb = smem_u32(&q_full);
-      mbar_arrive_expect_tx(qb, kQTile);
-      for (int i = 0; i < kCBlk; ++i) tma_load_4d(sQ + i * kQBlk, &tm_q, qb, 64 * i, h, q0, b);
-      tma_load_4d(sQ + kCBlk * kQBlk, &tm_qr, qb, kDc, h, q0, b);
+      if constexpr (!kQTmem) {
+        tma_prefetch_desc(&tm_q);
+        const uint32_t qb = smem_u32(&q_full);
+        mbar_arrive_expect_tx(qb, kQTile);
+        for (int i = 0; i < kCBlk; ++i) tma_load_4d(sQ + i * kQBlk, &tm_q, qb, 64 * i, h, q0, b);
+        tma_load_4d(sQ + kCBlk * kQBlk, &tm_qr, qb, kDc, h, q0, b);
+      }
       bool ok = true;
       for (int j = 0; j < p.nt && ok; ++j) {
         const int s = j % kStages;
         ok = wait_bar(smem_u32(&kv_empty[s]), ((j / kStages) & 1) ^ 1, abort_flag, p.dev_status);
         if (!ok) break;
-        const uint32_t dst = sbase + kQTile + s * kKTile;
+        const uint32_t dst = sK0 + s * kKTile;
         const uint32_t fb = smem_u32(&kv_full[s]);
         mbar_arrive_expect_tx(fb, kKTile);
         if (j < p.nt_ring) {
@@ -268,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t wb = smem_u32(&w_full);
           mbar_arrive_expect_tx(wb, kCBlk * kQBlk);
           for (int i = 0; i < kCBlk; ++i)
-            tma_load_2d(sbase + kQTile + s * kKTile + i * kQBlk, &tm_wuv, wb, 64 * i, h * kDh);
+            tma_load_2d(sK0 + s * kKTile + i * kQBlk, &tm_wuv, wb, 64 * i, h * kDh);
         }
       }
     }
@@ -279,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // it, so the pipe only stays busy if some thread is always issuing; with two issuers one
     // waits on a barrier while the other feeds the pipe.  Order between the two streams is
     // explicit: QK(j) overwrites the S/P buffer that PV(j-2) reads, so it waits for PV(j-2).
+    // With Q in TMEM there is one S buffer, which QK(j) takes once the softmax has loaded S(j-1).
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDc, 0, 1);
@@ -289,16 +307,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kQBlkD = kQBlk >> 4, kKBlkD = kKBlk >> 4, kKTileD = kKTile >> 4;
       const uint64_t q_c = smem_desc(sQ, 16, 1024, kSwizzle128B);
       const uint64_t q_r = smem_desc(sQ + kCBlk * kQBlk, 16, Sh::kRopeSbo, Sh::kRopeSwz);
-      const uint64_t k_c0 = smem_desc(sbase + kQTile, 16, 1024, kSwizzle128B);
-      const uint64_t k_r0 = smem_desc(sbase + kQTile + kCBlk * kKBlk, 16, Sh::kRopeSbo, Sh::kRopeSwz);
-      const uint64_t v_0 = smem_desc(sbase + kQTile, kKBlk, 1024, kSwizzle128B);
+      const uint64_t k_c0 = smem_desc(sK0, 16, 1024, kSwizzle128B);
+      const uint64_t k_r0 = smem_desc(sK0 + kCBlk * kKBlk, 16, Sh::kRopeSbo, Sh::kRopeSwz);
+      const uint64_t v_0 = smem_desc(sK0, kKBlk, 1024, kSwizzle128B);
       bool ok = true;
       if (warp == kQkWarp) {
         ok = wait_bar(smem_u32(&q_full), 0, abort_flag, p.dev_status);
         for (int j = 0; j < p.nt && ok; ++j) {
           const int s = j % kStages;
           ok = wait_bar(smem_u32(&kv_full[s]), (j / kStages) & 1, abort_flag, p.dev_status);
-          if (ok && j >= 2) {
+          if constexpr (kQTmem) {    // the softmax has loaded S(j-1) out of the one buffer
+            if (ok && j >= 1)
+              ok = wait_bar(smem_u32(&s_free[0]), (j - 1) & 1, abort_flag, p.dev_status);
+          } else if (ok && j >= 2) {
             if constexpr (kAliasP)   // PV(j-2) has read P(j-2) out of the buffer this QK overwrites
               ok = wait_bar(smem_u32(&pv_buf_done[j & 1]), ((j - 2) >> 1) & 1, abort_flag,
                             p.dev_status);
@@ -309,17 +330,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint64_t kc = k_c0 + static_cast<uint32_t>(s) * kKTileD;
           const uint64_t kr = k_r0 + static_cast<uint32_t>(s) * kKTileD;
-          const uint32_t d = tmem + (j & 1) * kColS;
+          if constexpr (kQTmem) {
+            // A = Q from TMEM: 8 columns (16 bf16) per k-step, content then positional
+            const uint32_t qa = tmem + kColS;
 #pragma unroll
-          for (int blk = 0; blk < kCBlk; ++blk)
+            for (int blk = 0; blk < kCBlk; ++blk)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ss(d, q_c + (blk * kQBlkD + 2 * kk), kc + (blk * kKBlkD + 2 * kk), idesc_qk,
-                     (blk | kk) != 0 ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ts(tmem, qa + 8 * (4 * blk + kk), kc + (blk * kKBlkD + 2 * kk), idesc_qk,
+                       (blk | kk) != 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < Sh::kRopeKSteps; ++kk)
-            mma_ss(d, q_r + 2 * kk, kr + 2 * kk, idesc_qk, 1u);
-          mma_commit(smem_u32(&s_full[j & 1]));
+            for (int kk = 0; kk < Sh::kRopeKSteps; ++kk)
+              mma_ts(tmem, qa + 8 * (4 * kCBlk + kk), kr + 2 * kk, idesc_qk, 1u);
+            mma_commit(smem_u32(&s_full[0]));
+          } else {
+            const uint32_t d = tmem + (j & 1) * kColS;
+#pragma unroll
+            for (int blk = 0; blk < kCBlk; ++blk)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss(d, q_c + (blk * kQBlkD + 2 * kk), kc + (blk * kKBlkD + 2 * kk), idesc_qk,
+                       (blk | kk) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < Sh::kRopeKSteps; ++kk)
+              mma_ss(d, q_r + 2 * kk, kr + 2 * kk, idesc_qk, 1u);
+            mma_commit(smem_u32(&s_full[j & 1]));
+          }
         }
       } else {
         for (int j = 0; j < p.nt && ok; ++j) {
@@ -342,13 +378,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                wait_bar(smem_u32(&olat_full), 0, abort_flag, p.dev_status);
           if (ok) {
             tc_fence_after();
-            const uint64_t w_c = smem_desc(sbase + kQTile + (p.nt % kStages) * kKTile, 16, 1024,
+            const uint64_t w_c = smem_desc(sK0 + (p.nt % kStages) * kKTile, 16, 1024,
                                            kSwizzle128B);
+            // O_lat: in the dead Q tile, or (Q in TMEM) in the stage after W_UV's
+            const uint64_t o_c =
+                kQTmem ? smem_desc(sK0 + ((p.nt + 1) % kStages) * kKTile, 16, 1024, kSwizzle128B)
+                       : q_c;
 #pragma unroll
             for (int blk = 0; blk < kCBlk; ++blk)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tmem, q_c + (blk * kQBlkD + 2 * kk), w_c + (blk * kQBlkD + 2 * kk), idesc_uv,
+                mma_ss(tmem, o_c + (blk * kQBlkD + 2 * kk), w_c + (blk * kQBlkD + 2 * kk), idesc_uv,
                        (blk | kk) != 0 ? 1u : 0u);
             mma_commit(smem_u32(&epi_done));
           }
@@ -360,25 +400,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = warp * 32 + lane;                 // TMEM lane and query row in the tile
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int n = q0 + row;
+    if constexpr (kQTmem) {
+      // this row of the query tile into TMEM, bf16 pairs from column kColS (zeros past D/2
+      // and for rows past n_q); the QK issuer waits for all 128 rows on q_full
+      const uint4* src = n < p.n_q ? reinterpret_cast<const uint4*>(
+                                         p.q + ((static_cast<int64_t>(b) * p.n_q + n) * p.H + h) * Sh::D)
+                                   : nullptr;
+#pragma unroll 1
+      for (int c = 0; c < Sh::kQWords; c += 16) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int u = c / 4 + i;                 // 16-byte piece of the row (8 bf16)
+          const uint4 v = src != nullptr && u < Sh::D / 8 ? src[u] : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+        tmem_st16(tmem + lane_off + kColS + c, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&q_full));
+    }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < p.nt; ++j) {
+      // S buffer and phase: one buffer with Q in TMEM, else two used in turn
+      const int sb = kQTmem ? 0 : (j & 1);
+      const uint32_t sphase = kQTmem ? (j & 1) : ((j >> 1) & 1);
       ok = __all_sync(0xffffffffu,
-                      wait_bar(smem_u32(&s_full[j & 1]), (j >> 1) & 1, abort_flag, p.dev_status));
+                      wait_bar(smem_u32(&s_full[sb]), sphase, abort_flag, p.dev_status));
       if (!ok) break;
       tc_fence_after();
       float s[kBN];
       {
         uint32_t r[kBN];
-        tmem_ld128_wait(tmem + lane_off + (j & 1) * kColS, r);
+        tmem_ld128_wait(tmem + lane_off + sb * kColS, r);
 #pragma unroll
         for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
       }
-      // S(j) is in registers: its TMEM buffer may take QK(j+2) now (with P in its own buffer;
-      // an aliased P keeps the buffer until PV(j) has read it).
+      // S(j) is in registers: its TMEM buffer may take the next QK now (with P in its own
+      // buffer; an aliased P keeps the buffer until PV(j) has read it).
       if constexpr (!kAliasP) {
         tc_fence_before();
-        mbar_arrive(smem_u32(&s_free[j & 1]));
+        mbar_arrive(smem_u32(&s_free[sb]));
       }
       const int valid = j < p.nt_ring ? min(kBN, p.nc - j * kBN)
                                       : min(kBN, p.n_q - (j - p.nt_ring) * kBN);
@@ -476,8 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // O_lat (bf16) -> shared memory, 128B-swizzled K-major, over the dead Q tile.
-        uint8_t* qsm = smem_raw + (sQ - smem_u32(smem_raw));
+        // O_lat (bf16) -> shared memory, 128B-swizzled K-major, over the dead Q tile (or, with
+        // Q in TMEM, into the K' stage after the one W_UV went to: all stages are free now).
+        const uint32_t so = kQTmem ? sK0 + ((p.nt + 1) % kStages) * kKTile : sQ;
+        uint8_t* qsm = smem_raw + (so - smem_u32(smem_raw));
 #pragma unroll 1
         for (int c = 0; c < kDc; c += 32) {
           uint32_t r[32];
@@ -580,6 +646,7 @@ mla_status attention_tc_impl(const Dims& d, const AttnArgs& a, int n_valid, cuda
     twuv = tchunk;    // never read
   }
   AttnParams p;
+  p.q = static_cast<const bf16*>(a.q);
   p.n_q = d.n_q; p.H = d.H; p.nc = kw.nc; p.nc_pad = kw.nc_pad;
   p.nt_ring = ceil_div(kw.nc, kBN);
   p.nt = p.nt_ring + ceil_div(d.n_q, kBN);
