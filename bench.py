@@ -380,7 +380,8 @@ def run_ours(args, cfg):
     tr_path = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tr_path):
         tr = json.load(open(tr_path))
-        if tr.get("kernel_sha") == kernel_sha():
+        # counters taken on this workload, from the kernel source as it is now
+        if tr.get("kernel_sha") == kernel_sha() and tr.get("workload") == cfg.name:
             traffic = tr.get("bytes_per_launch")
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
