@@ -6,10 +6,12 @@
 // Both kernels own a 128-row tile and stream 64-row sub-tiles of the other side through a ring
 // of shared-memory stages.  The operand a CTA keeps for its whole life (its 128 query rows Q' in
 // the dQ kernel, its 128 keys K' in the key kernel) sits in TMEM as bf16 pairs, so the S and dP
-// MMAs read only their streamed B operand from shared memory: with both operands in shared
-// memory an M128 N64 MMA is bound by shared-memory reads (6 KB per k-step), with A in TMEM it
-// runs at the tensor rate.  The softmax warps load S and dP into registers and release the TMEM
-// buffers at once, so the S/dP MMAs of the next sub-tile overlap the softmax; P and dS go to
+// MMAs read only their streamed B operand from shared memory.  (Measured on this part: an M128
+// K16 MMA with N <= 64 costs ~45 cycles with A in TMEM and ~48 with A in shared memory, against
+// 32 cycles of work, whatever else is in flight; N = 128 and 256 run at the full rate.  Hence the
+// key kernel computes S and dP as one N=128 product, below.)  The softmax warps load S and dP
+// into registers and release the TMEM buffers at once, so the S/dP MMAs of the next sub-tile
+// overlap the softmax; P and dS go to
 // shared memory (128-byte-swizzled K-major rows, written the way a TMA load would place them)
 // as the A operands of the key kernel's gradient products; the dQ kernel keeps dS in TMEM,
 // in the 32 columns its N=224 accumulator leaves free.
@@ -27,8 +29,9 @@
 //   dS_j = scale * P o (dP - Delta), P = exp(S scale - lse)    (softmax warps, bf16 to TMEM)
 //   dQ  += dS_j K'_j       M128 N224 K64    (A: dS in TMEM, B: K'_j read MN-major)
 // Key kernel: one CTA per (128-key tile, group of heads, sample); per (head, 64-query sub-tile):
-//   S^T  = K' Q'_i^T       M128 N64 K224    (A: K' in TMEM)
-//   dP^T = V  G_i^T        M128 N64 K192    (A: the content columns of K' in TMEM)
+//   [S^T | dP^T] = K' [Q'_i ; G_i 0]^T   M128 N128 K224 (A: K' in TMEM; B: the stage stacks the
+//                          Q' sub-tile over G with zeros in its positional columns, so the second
+//                          half is V G_i^T)
 //   P^T, scale * dS^T      softmax warps, one half key row per thread, lse/Delta per column
 //   dL  += dS^T Q'_i       M128 N256 K64    (key gradient, content and positional parts)
 //   dL  += P^T G_i         M128 N192 K64    (value gradient: the value is the content latent)
