@@ -246,15 +246,15 @@ __global__ void rope_keys_kernel(const T* __restrict__ cache, const T* __restric
                                  int B, int W, int D, int d_c, int n_pairs, int n_q, int nc,
                                  int nc_pad, int rows_ws, int row_begin, int row_end,
                                  int first_frame, RopeGeom g) {
-  // rows [row_begin, row_end) of every sample's rows_ws workspace rows
+  // rows [row_begin, row_end) of every sample's rows_ws workspace rows, one thread per pair
+  // (32-bit index arithmetic: B * span * n_pairs stays far below 2^31)
   const int span = row_end - row_begin;
-  const int64_t total = static_cast<int64_t>(B) * span * n_pairs;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int pair = static_cast<int>(e % n_pairs);
-    const int64_t rs = e / n_pairs;
-    const int r = row_begin + static_cast<int>(rs % span);
-    const int b = static_cast<int>(rs / span);
+  const int total = B * span * n_pairs;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const int pair = e % n_pairs;
+    const int rs = e / n_pairs;
+    const int r = row_begin + rs % span;
+    const int b = rs / span;
     const int64_t rr = static_cast<int64_t>(b) * rows_ws + r;
     T* dst = ws + rr * (2 * n_pairs) + 2 * pair;
     const T* src = nullptr;
@@ -300,6 +300,8 @@ mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_l
   const int row_begin = part == kRopeKeysChunk ? k.nc_pad : 0;
   const int row_end = part == kRopeKeysRing ? k.nc_pad : k.rows;
   if (row_end <= row_begin) return MLA_OK;
+  if (static_cast<int64_t>(d.B) * (row_end - row_begin) * (d.d_rope / 2) >= (int64_t{1} << 31))
+    MLA_FAIL(MLA_ERR_UNSUPPORTED, "too many rotated keys for one launch");
   const int64_t total = static_cast<int64_t>(d.B) * (row_end - row_begin) * n_pairs;
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));
   const RopeGeom g = rope_geom(d);
