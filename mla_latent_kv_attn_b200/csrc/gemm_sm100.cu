@@ -5,20 +5,22 @@
 //
 // Persistent: a grid of at most one CTA per SM walks the 128 x BN output tiles (tile index
 // n-fastest, so CTAs working at the same time share the A rows through L2), each CTA taking
-// every gridDim.x-th tile.  Roles (192 threads):
+// every gridDim.x-th tile.  Roles (320 threads):
 //   warp 0     TMA producer: 128x64 (A) and BNx64 (B) K-slices into a ring of 128B-swizzled
 //              buffers as deep as shared memory allows (4 to 8 stages); the ring runs on across
 //              tile boundaries.
 //   warp 1     allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) into one of two
 //              TMEM accumulators (tiles alternate), committing each stage back to the producer
 //              and each finished accumulator to the epilogue.
-//   warps 2-5  epilogue: drain an accumulator (one TMEM lane = one output row per thread) 32
-//              columns at a time, optionally rotate the positional-query columns (the last
-//              d_rope columns of every head block: 3D-RoPE),
-//              write bf16 into a 64B-swizzled 128x32 staging buffer (two, alternating) that one
-//              thread stores with a TMA bulk-tensor store (whole lines, out-of-range rows and
-//              columns clipped), and hand the accumulator back; this overlaps the MMAs of the
-//              CTA's next tile.  Outputs whose strides TMA cannot take are stored row by row.
+//   warps 2-9  epilogue, two groups of four warps (each group one TMEM lane = one output row per
+//              thread, group g taking the 32-column chunks 2k + g): drain an accumulator,
+//              optionally rotate the positional-query columns (the last d_rope columns of every
+//              head block: 3D-RoPE), write bf16 into a 64B-swizzled 128x32 staging buffer (two
+//              per group, alternating) that one thread of the group stores with a TMA
+//              bulk-tensor store (whole lines, out-of-range rows and columns clipped), and hand
+//              the accumulator back; this overlaps the MMAs of the CTA's next tile.  Outputs whose
+//              strides TMA cannot take are stored row by row.  (With one group, one warp per
+//              sub-partition, the drain took longer than the next tile's main loop.)
 // Before the first K-slice of a tile the producer asks L2 for its share of the tile's A panel
 // (when the panel is one contiguous range) with one bulk prefetch, so the panel streams from HBM
 // in long runs instead of one 128-byte piece per row and K-slice.
@@ -35,13 +37,15 @@ using namespace sm100;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;          // one 128-byte swizzle atom of bf16 per row
-constexpr int kThreads = 192;    // 6 warps
-constexpr int kEpiThreads = 128;
+constexpr int kThreads = 320;    // 10 warps
+constexpr int kEpiThreads = 256; // two groups of four warps, each group all 128 TMEM lanes
+constexpr int kEpiGroupThreads = 128;
 
 constexpr int kMaxStages = 8;
 constexpr int kEpiCols = 32;                       // columns per staged store
 constexpr int kStageOut = kBM * kEpiCols * 2;      // 8 KB: one 128 x 32 bf16 staging buffer
-constexpr int kSmemBudget = 220 * 1024 - 2 * kStageOut;   // what the operand ring may use
+constexpr int kStagingBufs = 4;                    // two per epilogue group
+constexpr int kSmemBudget = 220 * 1024 - kStagingBufs * kStageOut;   // for the operand ring
 
 template <int BN>
 struct GemmCfg {
@@ -51,7 +55,7 @@ struct GemmCfg {
   // As many stages as fit: the loads in flight per SM must cover the L2/HBM latency.
   static constexpr int kStages = kSmemBudget / kStage < kMaxStages ? kSmemBudget / kStage : kMaxStages;
   static constexpr int kOut = kStages * kStage;          // staging buffers after the ring
-  static constexpr int kSmem = kOut + 2 * kStageOut + 1024;  // + slack to align to 1024 B
+  static constexpr int kSmem = kOut + kStagingBufs * kStageOut + 1024;  // + slack to align
   // two accumulators, each starting on a power-of-two column
   static constexpr int kAccStride = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
   static constexpr int kTmemCols = 2 * kAccStride;
@@ -215,11 +219,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // epilogue warps 2..5 cover TMEM lane quadrants 2, 3, 0, 1
+    // epilogue warps 2..9: group 0 = warps 2..5, group 1 = warps 6..9, each covering TMEM lane
+    // quadrants 2, 3, 0, 1; group g drains the 32-column chunks 2k + g of every tile (two
+    // groups, because one warp per sub-partition leaves the TMEM loads' latency exposed)
     const int quad = warp & 3;
+    const int grp = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
-    const bool leader = threadIdx.x == 64;   // issues and waits for the TMA stores
-    const uint32_t out_base = base + Cfg::kOut;
+    const bool leader = threadIdx.x == 64 + kEpiGroupThreads * grp;   // issues the TMA stores
+    const uint32_t out_base = base + Cfg::kOut + grp * 2 * kStageOut;
     const bool vec_ok = ((reinterpret_cast<uintptr_t>(p.C) & 15u) == 0) && (p.c_sm % 8 == 0) &&
                         (p.c_batch % 8 == 0) &&
                         (p.n_split == 0 || (((reinterpret_cast<uintptr_t>(p.C2) & 15u) == 0) &&
@@ -244,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t tacc = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::kAccStride;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += kEpiCols, ++chunk) {
+      for (int c0 = kEpiCols * grp; c0 < BN; c0 += 2 * kEpiCols, ++chunk) {
         const int n = n0 + c0;
         if (n >= p.N) break;                   // uniform over the CTA
         uint32_t r[32];
@@ -272,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t buf = out_base + (chunk & 1) * kStageOut;
           // the store that last read this buffer (two chunks ago) has finished reading it
           if (leader) bulk_wait_group_read<1>();
-          named_bar_sync(1, kEpiThreads);
+          named_bar_sync(1 + grp, kEpiGroupThreads);
           // row `row` is 64 B: four 16-byte pieces, piece j at j ^ ((row / 2) mod 4) (64B swizzle)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          : "memory");
           }
           fence_proxy_async_smem();
-          named_bar_sync(1, kEpiThreads);
+          named_bar_sync(1 + grp, kEpiGroupThreads);
           if (leader) {
             const CUtensorMap* map = second ? &tmC2 : &tmC;
             const int col = second ? n - p.n_split : n;
