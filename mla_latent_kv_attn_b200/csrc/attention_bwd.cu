@@ -82,7 +82,23 @@ __global__ void __launch_bounds__(128)
   const T* o = static_cast<const T*>(p.o_lat) + idx * p.d_c;
   const T* g = static_cast<const T*>(p.d_o_lat) + idx * p.d_c;
   float acc = 0.f;
-  for (int c = lane; c < p.d_c; c += 32) acc = fmaf(Elem<T>::to_f(o[c]), Elem<T>::to_f(g[c]), acc);
+  if (sizeof(T) == 2 && p.d_c % 8 == 0) {
+    // bf16 rows of a multiple of 8: 16-byte pieces, one per lane (a row starts 16-byte aligned:
+    // d_c * 2 bytes is a multiple of 16)
+    for (int c8 = lane; c8 < p.d_c / 8; c8 += 32) {
+      const uint4 ov = reinterpret_cast<const uint4*>(o)[c8];
+      const uint4 gv = reinterpret_cast<const uint4*>(g)[c8];
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[i]));
+        const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[i]));
+        acc = fmaf(of.x, gf.x, fmaf(of.y, gf.y, acc));
+      }
+    }
+  } else {
+    for (int c = lane; c < p.d_c; c += 32) acc = fmaf(Elem<T>::to_f(o[c]), Elem<T>::to_f(g[c]), acc);
+  }
   acc = warp_sum(acc);
   if (lane == 0)
     p.delta[(static_cast<int64_t>(b) * p.H + h) * p.n_q + n] = acc;

@@ -684,9 +684,10 @@ __global__ void bwd_reduce_kernel(const float* __restrict__ partial, int groups,
     const int prow = m < nc ? m : nc_pad + (m - nc);
     float x0 = 0.f, x1 = 0.f;
     for (int gi = 0; gi < groups; ++gi) {
-      const float* src = partial + ((static_cast<int64_t>(gi) * B + b) * rows_ws + prow) * kD + 2 * pr;
-      x0 += src[0];
-      x1 += src[1];
+      const float2 v = *reinterpret_cast<const float2*>(
+          partial + ((static_cast<int64_t>(gi) * B + b) * rows_ws + prow) * kD + 2 * pr);
+      x0 += v.x;
+      x1 += v.y;
     }
     if (2 * pr >= kDc) {
       int t, hh, ww;
