@@ -174,6 +174,31 @@ __device__ __forceinline__ float softmax_exp_row(const float (&s)[kKeyTile], flo
   return l0 + l1;
 }
 
+// A query row into this thread's TMEM lane from column taddr on, as bf16 pairs (zeros past D/2
+// and for row == nullptr).  All of the row's 16-byte pieces are loaded before the first store,
+// so the row costs one global-load round trip instead of one per 16 columns.  Not inlined: with
+// the unrolled loads in the kernel body the compiler's register allocation for the main loop
+// changed and the kernel ran 3-4 % slower; as a separate function it is 1 % faster.
+template <int D, int kQWords>
+__device__ __noinline__ void copy_q_row(uint32_t taddr, const bf16* row) {
+  const uint4* src = reinterpret_cast<const uint4*>(row);
+  constexpr int kPieces = kQWords / 4;
+  uint4 v[kPieces];
+#pragma unroll
+  for (int u = 0; u < kPieces; ++u)
+    v[u] = src != nullptr && u < D / 8 ? src[u] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int c = 0; c < kQWords; c += 16) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 x = v[c / 4 + i];
+      w[4 * i] = x.x; w[4 * i + 1] = x.y; w[4 * i + 2] = x.z; w[4 * i + 3] = x.w;
+    }
+    tmem_st16(taddr + c, w);
+  }
+}
+
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          int32_t* dev_status) {
   return mbar_wait_or_abort(bar, parity, abort_flag, dev_status);
@@ -403,20 +428,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (kQTmem) {
       // this row of the query tile into TMEM, bf16 pairs from column kColS (zeros past D/2
       // and for rows past n_q); the QK issuer waits for all 128 rows on q_full
-      const uint4* src = n < p.n_q ? reinterpret_cast<const uint4*>(
-                                         p.q + ((static_cast<int64_t>(b) * p.n_q + n) * p.H + h) * Sh::D)
-                                   : nullptr;
-#pragma unroll 1
-      for (int c = 0; c < Sh::kQWords; c += 16) {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int u = c / 4 + i;                 // 16-byte piece of the row (8 bf16)
-          const uint4 v = src != nullptr && u < Sh::D / 8 ? src[u] : make_uint4(0u, 0u, 0u, 0u);
-          w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-        }
-        tmem_st16(tmem + lane_off + kColS + c, w);
-      }
+      copy_q_row<Sh::D, Sh::kQWords>(tmem + lane_off + kColS,
+                                     n < p.n_q ? p.q + ((static_cast<int64_t>(b) * p.n_q + n) * p.H + h) * Sh::D
+                                               : nullptr);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&q_full));
