@@ -84,10 +84,6 @@ class MLAConfig:
         """Cached scalars per token: content latent plus positional key."""
         return self.d_c + self.d_rope
 
-    @property
-    def cache_tokens(self) -> int:
-        return self.window_frames * self.tokens_per_frame
-
     def first_frame(self, chunk: int) -> int:
         return chunk * self.chunk_frames
 
@@ -233,14 +229,6 @@ def chunk_x(cfg: MLAConfig, chunk: int, step: int = 0, layer: int = 0,
     samples = range(cfg.batch) if samples is None else samples
     return np.stack([_normal(cfg, (cfg.n_q, cfg.d_model), 1.0, TID_X, chunk=chunk, step=step,
                              layer=layer, sample=b) for b in samples])
-
-
-def chunk_x_rows(cfg: MLAConfig, chunk: int, rows: np.ndarray, step: int = 0, layer: int = 0,
-                 sample: int = 0) -> np.ndarray:
-    """Selected rows of one sample's chunk_x (draws the whole stream, keeps rows)."""
-    full = _normal(cfg, (cfg.n_q, cfg.d_model), 1.0, TID_X, chunk=chunk, step=step,
-                   layer=layer, sample=sample)
-    return full[np.asarray(rows)]
 
 
 def direct_queries(cfg: MLAConfig, chunk: int, std: float = 0.5, samples=None) -> np.ndarray:
