@@ -101,6 +101,45 @@ def test_workspace_size():
         assert api.mla_attention_workspace_bytes(c, cfg.window_frames + 1) == 0
 
 
+def _bwd_head_groups(cfg, n_valid):
+    """The key-gradient kernel's head-group count: the divisor g of H whose (key tile, group,
+    sample) CTAs fill whole waves of 148 SMs best, the fewest on ties."""
+    nc = n_valid * cfg.tokens_per_frame
+    tiles = (-(-nc // 128) + -(-cfg.n_q // 128)) * cfg.batch
+    best, best_eff = 1, -1.0
+    for g in range(1, cfg.n_heads + 1):
+        if cfg.n_heads % g:
+            continue
+        ctas = tiles * g
+        eff = ctas / (-(-ctas // 148) * 148)
+        if eff > best_eff + 1e-9:
+            best, best_eff = g, eff
+    return best
+
+
+def test_backward_workspace_size():
+    """Delta, the rotated keys, and (tensor-core path: bf16, d_c 192, d_rope 32, n_q % 4 == 0)
+    the 256-wide padded key copy plus the head groups' fp32 partial key gradients."""
+    cases = [(inputs.CONFIGS[0], api.MLA_PATH_AUTO, False),      # fp32: CUDA cores
+             (inputs.CONFIGS[1], api.MLA_PATH_AUTO, True),       # the Wan preset: tensor cores
+             (inputs.CONFIGS[1], api.MLA_PATH_SIMT, False),      # forced onto CUDA cores
+             (inputs.small_bf16_config(), api.MLA_PATH_AUTO, True)]
+    for cfg, path, tc in cases:
+        c = api.make_config(cfg, kernel_path=path)
+        es = 4 if cfg.dtype == "fp32" else 2
+        for n_valid in (0, 1, cfg.window_frames):
+            nc = n_valid * cfg.tokens_per_frame
+            rows = -(-nc // 128) * 128 + -(-cfg.n_q // 128) * 128
+            delta = -(-(cfg.batch * cfg.n_heads * cfg.n_q) // 64) * 64 * 4
+            keys = cfg.batch * rows * cfg.d_rope * es
+            expect = delta + keys
+            if tc:
+                groups = _bwd_head_groups(cfg, n_valid)
+                expect += cfg.batch * rows * 256 * 2
+                expect += groups * cfg.batch * rows * cfg.d_latent * 4
+            assert api.mla_attention_bwd_workspace_bytes(c, n_valid) == expect, (cfg.name, path, n_valid)
+
+
 def test_schedule_matches_oracle_window():
     """The driver's (first_frame, n_valid) per chunk equals the oracle's window contents."""
     import numpy as np
