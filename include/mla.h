@@ -48,7 +48,7 @@ extern "C" {
 typedef enum mla_status {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = 1,    /* a null pointer, a bad size or an inconsistent configuration */
-  MLA_ERR_UNSUPPORTED = 2,    /* a valid request this build does not implement */
+  MLA_ERR_UNSUPPORTED = 2,    /* a valid request the library does not implement */
   MLA_ERR_ALIGNMENT = 3,      /* a pointer that is not 16-byte aligned */
   MLA_ERR_CUDA = 4,           /* a CUDA runtime or driver call failed */
   MLA_ERR_DEVICE_TIMEOUT = 5, /* value a kernel writes to dev_status when a bounded wait ran out */
