@@ -31,7 +31,10 @@
  *
  * Token order.  A chunk holds chunk_frames latent frames of frame_h x frame_w tokens; tokens
  * are ordered by frame, then row h, then column w.  Positions used by 3D-RoPE are
- * (t, h, w) = (absolute latent-frame index since the rollout began, row, column).
+ * (t, h, w) = (absolute latent-frame index since the rollout began, row, column).  Frame
+ * indices are int32: every entry point that takes first_frame rejects, with
+ * MLA_ERR_INVALID_ARG, a first_frame below 0 or one with first_frame + chunk_frames above
+ * INT32_MAX (mla_rope3d without a frame table: + rows_per_sample / tpf).
  */
 #ifndef MLA_LATENT_KV_ATTN_H_
 #define MLA_LATENT_KV_ATTN_H_

@@ -52,6 +52,16 @@ mla_status check_cfg(const mla_config* cfg) {
   return MLA_OK;
 }
 
+// Frame indices are first_frame + (frame within the chunk) in int32; the chunk's exclusive end
+// first_frame + frames must fit as well.
+mla_status check_first_frame(int32_t first_frame, int64_t frames) {
+  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_CHECK_ARG(int64_t{first_frame} + frames <= INT32_MAX,
+                "first_frame (%d) + %lld frames overflows the int32 frame index", first_frame,
+                static_cast<long long>(frames));
+  return MLA_OK;
+}
+
 // Rejects null, misaligned, host-only or other-device pointers before anything is launched.
 mla_status check_ptr(const void* p, const char* name, bool required = true) {
   if (p == nullptr) {
@@ -159,7 +169,7 @@ mla_status attention_entry(const mla_config* cfg, const void* q, const void* chu
   const Dims d = dims_of(*cfg);
   MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
                 d.W);
-  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_first_frame(first_frame, d.C));
   MLA_TRY(check_ptr(q, "q"));
   MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
   MLA_TRY(check_ptr(slot_frame, "slot_frame"));
@@ -213,8 +223,8 @@ mla_status mla_cache_append(const mla_config* cfg, const void* x, const void* w_
   MLA_TRY(check_cfg(cfg));
   MLA_CHECK_ARG(mode == MLA_PROJECT || mode == MLA_APPEND || mode == MLA_PROJECT_AND_APPEND,
                 "unknown mode %d", mode);
-  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
   const Dims d = dims_of(*cfg);
+  MLA_TRY(check_first_frame(first_frame, d.C));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
   if (mode & MLA_PROJECT) {
@@ -224,7 +234,6 @@ mla_status mla_cache_append(const mla_config* cfg, const void* x, const void* w_
   if (mode & MLA_APPEND) {
     MLA_TRY(check_ptr(cache, "cache"));
     MLA_TRY(check_ptr(slot_frame, "slot_frame"));
-    MLA_CHECK_ARG(first_frame <= INT32_MAX - d.C, "first_frame too large");
   }
   if (mode & MLA_PROJECT)
     MLA_TRY(gemm(d, x, d.d_model, 0, w_dkv_kr, d.d_model, 0, chunk_lat, d.D, 0, d.B * d.n_q, d.D,
@@ -247,7 +256,7 @@ mla_status mla_rope3d(const mla_config* cfg, void* data, int32_t n_samples,
                                   row_width,
                 "rotated vectors reach beyond row_width");
   MLA_CHECK_ARG(int64_t{n_samples} * rows_per_sample * row_width < kMaxElems, "array too large");
-  MLA_CHECK_ARG(frame_table != nullptr || first_frame >= 0, "first_frame must be >= 0");
+  if (frame_table == nullptr) MLA_TRY(check_first_frame(first_frame, rows_per_sample / d.tpf));
   if (int64_t{n_samples} * rows_per_sample * n_vec == 0) return MLA_OK;
   MLA_TRY(check_ptr(data, "data"));
   if (frame_table != nullptr) {
@@ -267,7 +276,7 @@ mla_status mla_key_positions(const mla_config* cfg, const int32_t* slot_frame,
   const Dims d = dims_of(*cfg);
   MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
                 d.W);
-  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_first_frame(first_frame, d.C));
   MLA_TRY(check_ptr(slot_frame, "slot_frame"));
   MLA_TRY(check_ptr(pos_out, "pos_out"));
   return key_positions(d, slot_frame, n_valid_frames, first_frame, pos_out,
@@ -303,7 +312,7 @@ mla_status mla_query_proj(const mla_config* cfg, const void* x, const void* w_dq
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
-  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_first_frame(first_frame, d.C));
   MLA_TRY(check_ptr(x, "x"));
   MLA_TRY(check_ptr(w_dq, "w_dq"));
   MLA_TRY(check_ptr(w_qcat, "w_qcat"));
@@ -321,7 +330,7 @@ mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
-  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_first_frame(first_frame, d.C));
   MLA_TRY(check_ptr(x, "x"));
   MLA_TRY(check_ptr(w_x, "w_x"));
   MLA_TRY(check_ptr(w_qcat, "w_qcat"));
@@ -408,7 +417,7 @@ mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q
   const Dims d = dims_of(*cfg);
   MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
                 d.W);
-  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_first_frame(first_frame, d.C));
   MLA_TRY(check_ptr(q, "q"));
   MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
   MLA_TRY(check_ptr(slot_frame, "slot_frame"));
@@ -442,7 +451,7 @@ mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* c
   const Dims d = dims_of(*cfg);
   MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
                 d.W);
-  MLA_CHECK_ARG(first_frame >= 0, "first_frame must be >= 0");
+  MLA_TRY(check_first_frame(first_frame, d.C));
   MLA_TRY(check_ptr(q, "q"));
   MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
   MLA_TRY(check_ptr(slot_frame, "slot_frame"));

@@ -88,6 +88,26 @@ def test_null_pointers_rejected_without_a_device():
     assert st == _lib.MLA_ERR_INVALID_ARG
 
 
+def test_frame_index_overflow_rejected_without_a_device():
+    c = api.make_config(inputs.CONFIGS[1])              # chunk_frames 3
+    lib = _lib.lib()
+    top = 2**31 - 1
+    for ff in (top, top - 2, -1):
+        st = lib.mla_cache_append(ctypes.byref(c), None, None, None, None, None, ff, 3, None)
+        assert st == _lib.MLA_ERR_INVALID_ARG and "first_frame" in _lib.last_error()
+        st = lib.mla_attention_fwd(ctypes.byref(c), None, None, None, None, 0, ff, None, None,
+                                   None, None, 0, None, None)
+        assert st == _lib.MLA_ERR_INVALID_ARG and "first_frame" in _lib.last_error()
+        st = lib.mla_query_proj(ctypes.byref(c), None, None, None, None, None, ff, None)
+        assert st == _lib.MLA_ERR_INVALID_ARG and "first_frame" in _lib.last_error()
+        st = lib.mla_key_positions(ctypes.byref(c), None, 0, ff, None, None)
+        assert st == _lib.MLA_ERR_INVALID_ARG and "first_frame" in _lib.last_error()
+    # the largest chunk start whose last frame still fits passes the frame check and then
+    # fails on the first null pointer
+    st = lib.mla_cache_append(ctypes.byref(c), None, None, None, None, None, top - 3, 3, None)
+    assert st == _lib.MLA_ERR_INVALID_ARG and "chunk_lat is null" in _lib.last_error()
+
+
 def test_workspace_size():
     for i in (0, 1, 2, 3):
         cfg = inputs.CONFIGS[i]
