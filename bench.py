@@ -65,46 +65,81 @@ REASON_BITS = {
 
 
 class ClockSampler:
-    """nvidia-smi sampled every 10 ms while the timed region runs.  The SM clock reported is the
-    median over the samples taken under load (GPU utilisation >= 50 %), since the B200 lowers its
-    clock under a sustained tensor load (power cap) and idle samples would hide that."""
+    """nvidia-smi sampled every 10 ms around the timed region.  The SM clock reported is the
+    median over the samples stamped inside the timed region (begin() .. end(); by default the
+    with-block), since the B200 lowers its clock under a sustained tensor load (power cap) and
+    idle samples would hide that.  When no sample falls inside (a region shorter than the
+    sampling interval), samples with GPU utilisation >= 50 % are used, then all samples.
+    Two pollers run: one with nvidia-smi's timestamp field and one without it, so that a
+    nvidia-smi that refuses the first query still leaves the unstamped samples."""
+
+    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,utilization.gpu"
 
     def __init__(self, index: int):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.procs = []
+        self.lines = {"stamped": [], "plain": []}
+        self.t_begin = None
+        self.t_end = None
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index),
-                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                 "utilization.gpu",
-                 "--format=csv,noheader,nounits", "-lms", "10"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        for kind, query in (("stamped", "timestamp," + self.FIELDS), ("plain", self.FIELDS)):
+            try:
+                proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + query,
+                     "--format=csv,noheader,nounits", "-lms", "10"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except (OSError, FileNotFoundError):
+                continue
+            thread = threading.Thread(target=self._read, args=(proc, self.lines[kind]),
+                                      daemon=True)
+            thread.start()
+            self.procs.append((proc, thread))
+        self.t_begin = time.time()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def begin(self):
+        self.t_begin = time.time()
+
+    def end(self):
+        self.t_end = time.time()
+
+    @staticmethod
+    def _read(proc, out):
+        for line in proc.stdout:
+            out.append(line.strip())
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self.t_end is None:
+            self.t_end = time.time()
+        for proc, thread in self.procs:
+            proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.thread.join(timeout=2)
+                proc.kill()
+            thread.join(timeout=2)
 
-    def summary(self):
+    @staticmethod
+    def _stamp(text: str):
+        """nvidia-smi's local-time stamp ("2026/12/02 17:05:01.123") as seconds since the epoch."""
+        import datetime
+        try:
+            return datetime.datetime.strptime(text, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
+
+    @staticmethod
+    def _parse(lines, stamped: bool):
         rows = []
-        for ln in self.lines:
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
+            ts = None
+            if stamped:
+                if len(parts) < 6:
+                    continue
+                ts = ClockSampler._stamp(parts[0])
+                parts = parts[1:]
             if len(parts) < 5:
                 continue
             try:
@@ -113,20 +148,29 @@ class ClockSampler:
                 util = float(parts[4])
             except ValueError:
                 continue
-            rows.append((s, m, pw, bits, util))
+            rows.append((ts, s, m, pw, bits, util))
+        return rows
+
+    def summary(self):
+        rows = self._parse(self.lines["stamped"], True) or self._parse(self.lines["plain"], False)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        loaded = [r for r in rows if r[4] >= 50.0]
-        use = loaded if loaded else rows
+        inside = []
+        if self.t_begin is not None and self.t_end is not None:
+            inside = [r for r in rows if r[0] is not None and self.t_begin <= r[0] <= self.t_end]
+        loaded = [r for r in rows if r[5] >= 50.0]
+        use = inside or loaded or rows
         reasons = set()
         for r in use:
             for bit, name in REASON_BITS.items():
-                if r[3] & bit and name != "gpu_idle":
+                if r[4] & bit and name != "gpu_idle":
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(r[0] for r in use),
-                "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
-                "samples": len(rows), "samples_under_load": len(loaded),
-                "power_w_max": max(r[2] for r in rows)}
+        return {"sm_mhz": statistics.median(r[1] for r in use),
+                "sm_max_mhz": max(r[2] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_in_timed_region": len(inside),
+                "samples_under_load": len(loaded),
+                "from": "timed region" if inside else "utilisation >= 50 %" if loaded else "all samples",
+                "power_w_max": max(r[3] for r in rows)}
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -301,12 +345,14 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         time.sleep(0.25)
+        clk.begin()
         for i in range(args.steps):
             flush.zero_()
             ev_s[i].record(stream)
             graphs[args.warmup + i].replay()
             ev_e[i].record(stream)
         torch.cuda.synchronize()
+        clk.end()
         time.sleep(0.25)
     if world > 1:
         dist.barrier()

@@ -73,3 +73,39 @@ def test_device_arm_without_a_gpu_fails_instead_of_falling_back():
     r = _bench("--steps", "1", "--warmup", "3", "--no-cpu-baseline", timeout=300)
     assert r.returncode != 0
     assert _json_lines(r.stdout) == []
+
+
+def test_clock_summary_uses_the_samples_stamped_inside_the_timed_region():
+    import datetime
+    sys.path.insert(0, ROOT)
+    import bench
+    t0 = datetime.datetime(2026, 1, 2, 3, 4, 5, 0)
+
+    def stamp(ms):
+        return (t0 + datetime.timedelta(milliseconds=ms)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+
+    clk = bench.ClockSampler(0)
+    # idle before and after (1965 MHz, 0 % busy), power-capped inside (1600-1700 MHz)
+    clk.lines["stamped"] = (
+        [f"{stamp(ms)}, 1965, 1965, 200.0, 0x0000000000000001, 0" for ms in (0, 10, 20)] +
+        [f"{stamp(ms)}, {mhz}, 1965, 990.0, 0x0000000000000004, 0"
+         for ms, mhz in ((40, 1600), (50, 1650), (60, 1700))] +
+        [f"{stamp(ms)}, 1965, 1965, 210.0, 0x0000000000000001, 0" for ms in (90, 100)])
+    clk.lines["plain"] = ["1965, 1965, 200.0, 0x0000000000000001, 0"]
+    clk.t_begin = (t0 + datetime.timedelta(milliseconds=35)).timestamp()
+    clk.t_end = (t0 + datetime.timedelta(milliseconds=65)).timestamp()
+    s = clk.summary()
+    assert s["sm_mhz"] == 1650 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+    assert s["samples"] == 8 and s["samples_in_timed_region"] == 3 and s["from"] == "timed region"
+    assert s["power_w_max"] == 990.0
+    # a region between two samples falls back to busy samples, then to all of them
+    clk.t_begin = clk.t_end = (t0 + datetime.timedelta(milliseconds=75)).timestamp()
+    s = clk.summary()
+    assert s["from"] == "all samples" and s["samples_in_timed_region"] == 0
+    # without stamped samples the unstamped poller's are used
+    clk.lines["stamped"] = []
+    clk.lines["plain"] = ["1700, 1965, 900.0, 0x0000000000000004, 80",
+                          "1965, 1965, 200.0, 0x0000000000000001, 0"]
+    s = clk.summary()
+    assert s["sm_mhz"] == 1700 and s["from"] == "utilisation >= 50 %" and s["samples"] == 2
