@@ -72,6 +72,22 @@ def test_oversized_workload_is_rejected():
         api.mla_config_check(c)
 
 
+def test_largest_accepted_batch_is_the_int32_element_limit():
+    # Wan preset: the largest array per sample is Q' = n_q * H * (d_c + d_rope) = 12,579,840
+    # elements; every array must hold fewer than 2^31 - 1 elements
+    cfg = inputs.CONFIGS[1]
+    per_sample = cfg.n_q * cfg.n_heads * (cfg.d_c + cfg.d_rope)
+    assert per_sample == 12_579_840
+    top = (2**31 - 2) // per_sample
+    assert top == 170
+    c = api.make_config(cfg, batch=top)
+    api.mla_config_check(c)
+    c = api.make_config(cfg, batch=top + 1)
+    with pytest.raises(api.MLAError) as e:
+        api.mla_config_check(c)
+    assert e.value.status == _lib.MLA_ERR_INVALID_ARG and "2^31" in _lib.last_error()
+
+
 def test_null_pointers_rejected_without_a_device():
     c = api.make_config(inputs.CONFIGS[1])
     lib = _lib.lib()
