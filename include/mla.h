@@ -19,7 +19,9 @@
  *   device, 16-byte aligned, to a dense row-major array of the stated shape.  "T" is the
  *   configuration's element type: bfloat16 (MLA_BF16) or float32 (MLA_FP32).
  * - The caller owns every buffer.  The library never allocates device memory, never
- *   synchronises the device or a stream, and keeps no pointer after a call returns.
+ *   synchronises the device or a stream, and keeps no pointer after a call returns.  The one
+ *   exception is mla_attention_fwd_static_scratch: it uses a fixed array built into the library
+ *   (reserved on every device that loads it) and keeps that array's device address (below).
  * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All work is
  *   enqueued on it, asynchronously.
  * - Arguments are checked on the host before anything is launched.  A rejected call returns a
@@ -27,7 +29,9 @@
  *   mla_last_error() then describes the problem.  A launch that fails returns MLA_ERR_CUDA.
  * - Errors that only the device can see (a bounded wait inside a kernel that ran out) are
  *   written to the optional `dev_status` word (see mla_attention_fwd); kernels never trap.
- * - Entry points are thread-safe; mla_last_error() is per host thread.
+ * - Entry points are thread-safe; mla_last_error() is per host thread.  Again the exception is
+ *   mla_attention_fwd_static_scratch: its calls share one array per device, so calls whose work
+ *   overlaps on the GPU race (below).
  *
  * Token order.  A chunk holds chunk_frames latent frames of frame_h x frame_w tokens; tokens
  * are ordered by frame, then row h, then column w.  Positions used by 3D-RoPE are
@@ -303,18 +307,19 @@ mla_status mla_attention_fwd_cached_ring(const mla_config* cfg, const void* q,
 /* --------------------------------------------------------------------------------------------
  * mla_attention_fwd_static_scratch: mla_attention_fwd without the workspace arguments, for
  * callers that cannot allocate device memory.  The paper has no counterpart to this call; it
- * exists for deployment.  Some callers have no way to hand the library a scratch buffer: code
- * that issues its work while a stream is being captured into a CUDA graph (cudaMalloc is not
- * allowed there), plugins whose host framework gives them only their input and output buffers,
- * and services that forbid device allocation after start-up.  This call keeps its scratch (the
- * rotated positional keys of the attended keys) in a fixed 16 MiB array compiled into the
- * library, and calls no cudaMalloc, cudaFree or other allocating routine.
+ * exists for deployment.  Some callers have no way to hand the library a scratch buffer:
+ * plugins whose host framework gives them only their input and output buffers, and services
+ * that forbid device allocation after start-up.  This call keeps its scratch (the rotated
+ * positional keys of the attended keys) in a fixed 16 MiB array compiled into the library, and
+ * calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Arguments, results and errors are those of mla_attention_fwd.  A call whose scratch,
  *     mla_attention_workspace_bytes(cfg, n_valid_frames), exceeds 16 MiB (16777216 bytes) is
  *     rejected with MLA_ERR_WORKSPACE before anything is launched.
  *   - Every device that loads the library keeps those 16 MiB reserved until the process exits.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
- *     that device current); make that first call before any stream capture begins.
+ *   - The first call in a CUDA context (normally: the first call on a device) looks up the
+ *     array's device address with cudaGetSymbolAddress, with that device current, and caches it
+ *     for that context; make that first call before any stream capture begins.  A device reset
+ *     or another context gives a new context, whose first call looks the address up again.
  *   - All calls share the one array per device.  Calls whose kernels overlap on the GPU (on
  *     different streams, or from different host threads) race on it and give wrong results;
  *     order them on one stream.  Each call rewrites every part of the array it reads, so what an
@@ -387,6 +392,29 @@ mla_status mla_out_proj(const mla_config* cfg, const void* o_lat, const void* w_
  * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
  * ------------------------------------------------------------------------------------------ */
 mla_status mla_selftest_wait_timeout(int32_t* dev_status, int32_t limit_us, void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * Self-tests of the library's own approximations (for tests only).  Each evaluates, on the
+ * device, the very function the kernels use, so that a test can hold it to its error bound.
+ * All arrays are device memory, 4-byte aligned; n >= 0 elements.  Errors: MLA_ERR_INVALID_ARG,
+ * MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ *
+ * mla_selftest_exp2: for every x[i] (float): y_poly[i] = the softmax's FMA-pipe 2^x (degree-3
+ *   interpolant of 2^f at the Chebyshev nodes of [-1/2, 1/2], f = x - rint(x), scaled by 2^rint(x)
+ *   through the exponent field; arguments below -125 are clamped to -125), evaluated in pairs as
+ *   the softmax does; y_sfu[i] = the SFU's ex2.approx.ftz(x); y_exp2f[i] = CUDA's exp2f(x).
+ * mla_selftest_sincos: sin and cos of angle[i] as 3D-RoPE computes them (reduction by 2 pi in two
+ *   float constants, then the hardware sine/cosine on [-pi, pi]).
+ * mla_selftest_rope_angles: for positions pos[i] = (t, h, w) (device int32 [n, 3]) and every
+ *   rotary pair j of cfg ([M] 3D-RoPE, reading of mla_config): angle[i, j] (float [n, d_rope/2])
+ *   as the kernels compute it, and its sine and cosine (sin_out, cos_out, float [n, d_rope/2]).
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_selftest_exp2(const float* x, float* y_poly, float* y_sfu, float* y_exp2f,
+                             int32_t n, void* stream);
+mla_status mla_selftest_sincos(const float* angle, float* sin_out, float* cos_out, int32_t n,
+                               void* stream);
+mla_status mla_selftest_rope_angles(const mla_config* cfg, const int32_t* pos, int32_t n,
+                                    float* angle, float* sin_out, float* cos_out, void* stream);
 
 #ifdef __cplusplus
 }

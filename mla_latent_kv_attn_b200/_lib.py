@@ -75,6 +75,9 @@ SIGNATURES = {
     "mla_attention_fwd_static_scratch": (c_int32, [_CFG, _P, _P, _P, _P, c_int32, c_int32, _P,
                                                    _P, _P, _P, _P]),
     "mla_selftest_wait_timeout": (c_int32, [_P, c_int32, _P]),
+    "mla_selftest_exp2": (c_int32, [_P, _P, _P, _P, c_int32, _P]),
+    "mla_selftest_sincos": (c_int32, [_P, _P, _P, c_int32, _P]),
+    "mla_selftest_rope_angles": (c_int32, [_CFG, _P, c_int32, _P, _P, _P, _P]),
 }
 
 _lib = None

@@ -42,6 +42,7 @@
 // Roles: softmax / epilogue warps (one TMEM lane = one row), a TMA producer warp, and a warp that
 // allocates TMEM and whose lane 0 issues every MMA.  Every wait is bounded; a wait that runs out
 // writes MLA_ERR_DEVICE_TIMEOUT to dev_status.
+#include "exp2.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -96,12 +97,6 @@ struct BwdTcParams {
   float* partial;        // [groups, B, rows_ws, D] fp32
   int32_t* dev_status;
 };
-
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {

@@ -1,8 +1,8 @@
 """The allocation-free attention entry point agrees with the regular one.
 
-Some callers cannot call cudaMalloc: work issued while a stream is being captured into a CUDA
-graph, plugins whose host framework hands them only their own input and output buffers, and
-services that forbid device allocation once they are running.  For them the library offers
+Some callers cannot call cudaMalloc: plugins whose host framework hands them only their own
+input and output buffers, and services that forbid device allocation once they are running.
+For them the library offers
 mla_attention_fwd_static_scratch, which keeps the attention scratch (the rotated positional
 keys) in a 16 MiB array built into the library instead of a caller-provided workspace.
 
