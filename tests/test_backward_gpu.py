@@ -92,18 +92,23 @@ def test_backward_small_frames_bf16(chunk, path):
 
 def test_backward_wan_config1_full_size():
     """The Wan preset at full size on the tensor-core backward (4680 queries, 14,040 keys, 12
-    heads).  dq on 64 sampled rows against the oracle (rows are independent given the keys); the
-    key gradients through identities that hold at any size, since every row's probabilities sum
-    to one (so every row's dS sums to zero): summed over all keys, the content gradients equal
-    the summed upstream gradient and the positional ones, rotated back to the keys' frames, sum
-    to zero."""
+    heads, the launch grid and head-group split of the benchmark workload), one chunk after the
+    window filled so that the ring has wrapped (slots 3..5 hold the oldest frames, 0..2 the
+    newest).  Every gradient is compared element by element with the float64 oracle, which
+    evaluates all rows and keys: d_q of every query row, and the latent gradient of every
+    attended key (ring keys from the oldest and newest slots, the ragged last ring tile, every
+    chunk key).  Besides, two identities that hold at any size, since every row's
+    probabilities sum to one (so every row's dS sums to zero): summed over all keys, the content
+    gradients equal the summed upstream gradient and the positional ones, rotated back to the
+    keys' frames, sum to zero."""
     cfg = inputs.CONFIGS[1]
     c = api.make_config(cfg)
     dt = api.torch_dtype(c)
     dev = torch.device("cuda")
     ring = rollout.Ring(c)
     d = oracle.dims_from(cfg)
-    chunk = cfg.measured_chunk
+    chunk = cfg.measured_chunk + 1
+    tpf = cfg.tokens_per_frame
     lat_buf = torch.empty((1, cfg.n_q, cfg.d_latent), device=dev, dtype=dt)
     recs = {}
     for ch in range(chunk):
@@ -111,7 +116,6 @@ def test_backward_wan_config1_full_size():
         lat_buf.copy_(torch.from_numpy(lat).to(dt))
         api.mla_cache_append(c, None, None, lat_buf, ring.cache, ring.slot_frame,
                              cfg.first_frame(ch), api.MLA_APPEND)
-        tpf = cfg.tokens_per_frame
         for f in range(cfg.chunk_frames):
             recs[cfg.first_frame(ch) + f] = lat[0][f * tpf:(f + 1) * tpf]
     first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, chunk)
@@ -126,7 +130,9 @@ def test_backward_wan_config1_full_size():
     ws = torch.empty(api.mla_attention_workspace_bytes(c, n_valid), device=dev, dtype=torch.uint8)
     api.mla_attention_fwd(c, q, lat_buf, ring.cache, ring.slot_frame, n_valid, first, None, o_lat,
                           lse, ws)
-    d_q, d_lat, d_cache = torch.empty_like(q), torch.empty_like(lat_buf), torch.empty_like(ring.cache)
+    d_q = torch.full_like(q, float("nan"))
+    d_lat = torch.full_like(lat_buf, float("nan"))
+    d_cache = torch.full_like(ring.cache, float("nan"))
     status = torch.zeros(1, device=dev, dtype=torch.int32)
     bws = torch.empty(api.mla_attention_bwd_workspace_bytes(c, n_valid), device=dev,
                       dtype=torch.uint8)
@@ -135,18 +141,30 @@ def test_backward_wan_config1_full_size():
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     slots = ring.slot_frame.cpu().numpy()[0][:n_valid]
-    tpf = cfg.tokens_per_frame
+    assert list(slots) == [first - cfg.window_frames + (s - first) % cfg.window_frames
+                           for s in range(cfg.window_frames)], "ring has not wrapped"
     c_ring = np.concatenate([recs[t][:, :cfg.d_c] for t in slots])
     k_ring = np.concatenate([recs[t][:, cfg.d_c:] for t in slots])
     pos_k = np.concatenate([oracle.token_positions(list(slots), d),
                             oracle.token_positions(range(first, first + cfg.chunk_frames), d)])
-    rows = inputs.sample_rows(cfg.n_q, 64, tag=21)
     ref = oracle.latent_attention_backward(
-        q_np[0][rows], np.concatenate([c_ring, lat_np[0][:, :cfg.d_c]]),
-        np.concatenate([k_ring, lat_np[0][:, cfg.d_c:]]), pos_k, g_np[0][rows], d)
-    compare("cfg1.d_q", to_np(d_q)[0][rows], ref["d_q"], "bf16")
+        q_np[0], np.concatenate([c_ring, lat_np[0][:, :cfg.d_c]]),
+        np.concatenate([k_ring, lat_np[0][:, cfg.d_c:]]), pos_k, g_np[0], d)
     nc = n_valid * tpf
-    grads = np.concatenate([to_np(d_cache)[0][:nc], to_np(d_lat)[0]])       # [keys, D]
+    dk = np.concatenate([ref["d_c"], ref["d_k_r"]], axis=1)              # [keys, D]
+    got_dq, got_cache, got_lat = to_np(d_q)[0], to_np(d_cache)[0], to_np(d_lat)[0]
+    compare("cfg1.d_q", got_dq, ref["d_q"], "bf16")
+    compare("cfg1.d_cache", got_cache[:nc], dk[:nc], "bf16")
+    compare("cfg1.d_chunk_lat", got_lat, dk[nc:], "bf16")
+    # the oldest and newest ring frames and the chunk's last (ragged) key tile on their own
+    oldest, newest = int(np.argmin(slots)), int(np.argmax(slots))
+    for name, lo, hi in (("oldest", oldest * tpf, (oldest + 1) * tpf),
+                         ("newest", newest * tpf, (newest + 1) * tpf),
+                         ("ring tail tile", nc - nc % 128, nc)):
+        compare(f"cfg1.d_cache[{name}]", got_cache[lo:hi], dk[lo:hi], "bf16")
+    compare("cfg1.d_chunk_lat[tail tile]", got_lat[cfg.n_q - cfg.n_q % 128:],
+            dk[nc + cfg.n_q - cfg.n_q % 128:], "bf16")
+    grads = np.concatenate([got_cache[:nc], got_lat])
     content_sum = grads[:, :cfg.d_c].sum(axis=0)
     expect = g_np[0].astype(np.float64).sum(axis=(0, 1))
     assert np.linalg.norm(content_sum - expect) <= 2e-2 * np.linalg.norm(expect)

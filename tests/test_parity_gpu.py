@@ -92,24 +92,36 @@ def test_wan_config1_sampled_rows():
 
 
 def test_wan_config3_batch8_sampled_rows():
-    """Config 3: 8 independent samples, window 9 frames, chunk 3 frames."""
+    """Config 3: 8 independent samples, window 9 frames, chunk 3 frames; 512 sampled rows of
+    every sample (every 128-row query tile holds some), then the append and every sample's ring
+    (slots bit-exact, contents within tolerance)."""
     cfg = inputs.CONFIGS[3]
     g, o = prefilled(cfg, api.MLA_PATH_AUTO, cfg.measured_chunk)
+    check_ring(cfg, g, o)
     ch = cfg.measured_chunk
     x = inputs.chunk_x(cfg, ch)
-    rows = inputs.sample_rows(cfg.n_q, 48, tag=3)
+    rows = inputs.sample_rows(cfg.n_q, 512, tag=3)
+    assert len(set(rows // 128)) == -(-cfg.n_q // 128)
+    pos = g.key_positions(ch)
+    for b in range(cfg.batch):
+        np.testing.assert_array_equal(pos[b], expected_key_positions(cfg, o.windows[b], cfg.first_frame(ch)))
     check_chunk("cfg3", cfg, g.attend(ch, x), o.step(ch, x, rows), rows)
+    g.append(ch)
+    check_ring(cfg, g, o)
 
 
 def test_wan_config2_long_rollout_sampled():
     """Config 2: 80 chunks, window 21 frames; temporal positions reach t = 239 and the ring
-    wraps every 7 chunks.  Every chunk runs the whole path on the GPU; the oracle evaluates
-    sampled rows at chunks while the window fills, across wraps and at the end."""
+    wraps every 7 chunks.  Every chunk runs the whole path on the GPU.  The oracle evaluates 512
+    sampled rows (every query tile holds some) with all heads at chunks 0-8 (the window fills,
+    then the first wraps) and 76-79 (t up to 239), with the key positions; after every chunk's
+    append the whole ring is compared (slots bit-exact, contents within tolerance)."""
     cfg = inputs.CONFIGS[2]
     g = GpuRun(cfg, api.MLA_PATH_AUTO)
     o = OracleRun(cfg, g.lw)
-    checked = {0, 1, 6, 7, 8, 40, 78, 79}
-    rows = inputs.sample_rows(cfg.n_q, 32, tag=2)
+    checked = set(range(9)) | set(range(76, 80))
+    rows = inputs.sample_rows(cfg.n_q, 512, tag=2)
+    assert len(set(rows // 128)) == -(-cfg.n_q // 128)
     for ch in range(cfg.n_chunks):
         x = inputs.chunk_x(cfg, ch)
         if ch in checked:
@@ -121,7 +133,7 @@ def test_wan_config2_long_rollout_sampled():
             g.attend(ch, x, want_latent=False)
             o.prefill(ch, x)
         g.append(ch)
-    check_ring(cfg, g, o)
+        check_ring(cfg, g, o)
     assert int(g.ring.slot_frame.max()) == 239
 
 
@@ -360,7 +372,7 @@ def test_wan_config4_thirty_layer_stack():
     appends its last step's latents.  All 1200 attention calls run on the GPU through
     rollout.LayerStack (ring keys rotated once per chunk and layer, cached-ring attention).  The oracle checks
     sampled rows of layer 29 at the last chunk (steps 0 and 3, ring wrapped, 23,400 keys) and of
-    layer 0 at chunks 0 and 1, plus both layers' ring slots."""
+    layer 0 at chunks 0 and 1 (256 sampled rows, both samples), plus both layers' ring slots."""
     import os
     from concurrent.futures import ThreadPoolExecutor
 
@@ -376,7 +388,7 @@ def test_wan_config4_thirty_layer_stack():
     checks = {(cfg.n_chunks - 1, 0, 29), (cfg.n_chunks - 1, last, 29), (0, 0, 0), (0, last, 0),
               (1, last, 0)}
     history = {29: range(cfg.n_chunks), 0: range(2)}
-    rows = inputs.sample_rows(cfg.n_q, 24, tag=4)
+    rows = inputs.sample_rows(cfg.n_q, 256, tag=4)
     order = [(ch, s, l) for ch in range(cfg.n_chunks) for s in range(cfg.n_steps)
              for l in range(cfg.n_layers)]
     kept, gpu_out = {}, {}
