@@ -275,6 +275,108 @@ def max_over_ranks(value: float, device=None) -> float:
 
 # --------------------------------------------------------------------------- GPU path
 
+def probe_sm_clock(stream, spin_us: int = 200):
+    """Launches the library's clock probe (one warp per SM reads the SM cycle counter against
+    the global timer while spinning spin_us) on `stream`; returns a function that, after the
+    stream has run it, gives the median SM clock in MHz over the SMs."""
+    import torch
+    from mla_latent_kv_attn_b200 import _lib
+    n = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    out = torch.zeros((n, 4), dtype=torch.int64, device="cuda")
+    st = _lib.lib().mla_probe_sm_clock(out.data_ptr(), n, spin_us, stream.cuda_stream)
+    if st != 0:
+        raise RuntimeError("mla_probe_sm_clock: " + _lib.last_error())
+
+    def result():
+        v = out.cpu().numpy().astype(np.float64)
+        mhz = 1000.0 * v[:, 1] / np.maximum(v[:, 2], 1.0)
+        return float(np.median(mhz))
+    return result
+
+
+def time_calls(fn, flush, stream, reps: int):
+    """Mean device time (ms) of fn() over reps launches, each after an L2 flush that lies
+    outside its CUDA-event interval."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for _ in range(3):
+        flush.zero_()
+        fn()
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+
+def bandwidth_entry(nbytes: float, ms: float, hbm_gbs: float, workload: str, **extra):
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    d = {"bytes": int(nbytes), "us": 1e3 * ms, "gbs": gbs, "frac": gbs / hbm_gbs,
+         "workload": workload}
+    d.update(extra)
+    return d
+
+
+def measure_bandwidth(cfg, flush, stream, hbm_gbs: float, reps: int = 20):
+    """The memory-bound calls of the path, each timed alone with CUDA events (L2 flushed before
+    every launch), at the benchmark workload and at a batch whose arrays exceed the 126 MB L2:
+    achieved GB/s = the call's algorithmic bytes / its time, against the measured HBM copy
+    bandwidth.  Algorithmic bytes: ring append 2 * D * sizeof(T) per chunk token (read the chunk
+    latent, write the ring row); ring-key rotation 2 * d_rope * sizeof(T) per ring key (read k_R,
+    write the rotated key); query RoPE 2 * d_rope * sizeof(T) per (token, head); KV
+    down-projection x + [W_down^KV; W_R^K] read, [c_KV || k_R] written once."""
+    import torch
+    from mla_latent_kv_attn_b200 import api, rollout
+    res = {}
+    for tag, batch in (("bench", cfg.batch), ("large", 32)):
+        c = api.make_config(cfg, batch=batch)
+        dt = api.torch_dtype(c)
+        es = 2 if dt == torch.bfloat16 else 4
+        tpf, n_q, D = cfg.tokens_per_frame, cfg.n_q, cfg.d_latent
+        W = cfg.window_frames
+        ring = rollout.Ring(c)
+        lat = torch.randn((batch, n_q, D), device="cuda").to(dt)
+        first = W * 4            # a chunk whose frames wrap into a full ring
+        for ch in range(W // cfg.chunk_frames):
+            api.mla_cache_append(c, None, None, lat, ring.cache, ring.slot_frame,
+                                 ch * cfg.chunk_frames, api.MLA_APPEND)
+        wl = f"{cfg.name}, batch {batch}"
+        ms = time_calls(lambda: api.mla_cache_append(c, None, None, lat, ring.cache,
+                                                     ring.slot_frame, first, api.MLA_APPEND),
+                        flush, stream, reps)
+        res[f"ring_append_{tag}"] = bandwidth_entry(2.0 * batch * n_q * D * es, ms, hbm_gbs, wl,
+                                                    kernel="ring_append_kernel")
+        ws = torch.empty(api.mla_attention_workspace_bytes(c, W), device="cuda", dtype=torch.uint8)
+        ms = time_calls(lambda: api.mla_rotate_ring_keys(c, ring.cache, ring.slot_frame, W, ws),
+                        flush, stream, reps)
+        res[f"rope_ring_keys_{tag}"] = bandwidth_entry(2.0 * batch * W * tpf * cfg.d_rope * es, ms,
+                                                       hbm_gbs, wl, kernel="rope_keys_vec_kernel")
+        q = torch.randn((batch, n_q, cfg.n_heads, D), device="cuda").to(dt)
+        ms = time_calls(lambda: api.mla_rope3d(c, q, n_vec=cfg.n_heads, col_offset=cfg.d_c,
+                                               vec_stride=D, first_frame=first),
+                        flush, stream, reps)
+        res[f"rope_query_{tag}"] = bandwidth_entry(2.0 * batch * n_q * cfg.n_heads * cfg.d_rope * es,
+                                                   ms, hbm_gbs, wl, kernel="rope3d_kernel")
+        if tag == "bench" or batch * n_q * cfg.d_model * es <= 2 ** 30:
+            x = torch.randn((batch, n_q, cfg.d_model), device="cuda").to(dt)
+            wkv = torch.randn((D, cfg.d_model), device="cuda").to(dt)
+            ms = time_calls(lambda: api.mla_cache_append(c, x, wkv, lat, None, None, first,
+                                                         api.MLA_PROJECT),
+                            flush, stream, reps)
+            nbytes = (batch * n_q * cfg.d_model + D * cfg.d_model + batch * n_q * D) * es
+            flops = 2.0 * batch * n_q * cfg.d_model * D
+            res[f"kv_down_projection_{tag}"] = bandwidth_entry(
+                nbytes, ms, hbm_gbs, wl, kernel="gemm_tc_kernel", tflops=flops / (ms * 1e-3) / 1e12)
+            del x, wkv
+        del ring, lat, ws, q
+        torch.cuda.empty_cache()
+    return res
+
+
+
 def run_ours(args, cfg):
     import torch
     import torch.distributed as dist
@@ -351,6 +453,9 @@ def run_ours(args, cfg):
             ev_s[i].record(stream)
             graphs[args.warmup + i].replay()
             ev_e[i].record(stream)
+        # the SM clock read on the device right after the last timed step (nvidia-smi's samples
+        # are 10 ms apart, longer than a short timed region)
+        clock_after = probe_sm_clock(stream)
         torch.cuda.synchronize()
         clk.end()
         time.sleep(0.25)
@@ -358,6 +463,9 @@ def run_ours(args, cfg):
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(ev_s, ev_e)]
     attn_ms = [graphs[args.warmup + i].attention_ms() for i in range(args.steps)]
+    proj_ms = [graphs[args.warmup + i].projection_ms() for i in range(args.steps)]
+    app_ms = [graphs[args.warmup + i].append_ms() for i in range(args.steps)]
+    sm_mhz_device = clock_after()
     total_ms = max_over_ranks(sum(step_ms), device=dev)
     status = int(buf.dev_status.item())
     if status != 0:
@@ -415,6 +523,21 @@ def run_ours(args, cfg):
         dist.barrier()
 
     peaks, peak_kind = load_peaks()
+    bandwidth = measure_bandwidth(cfg, flush, stream, peaks["hbm_gbs"]) if not args.no_bandwidth \
+        else None
+    if bandwidth is not None:
+        # the step's own append and projections, timed inside the step graphs
+        es = 2
+        app_bytes = 2.0 * cfg.batch * cfg.n_q * cfg.d_latent * es
+        bandwidth["ring_append_in_step"] = bandwidth_entry(
+            app_bytes, statistics.mean(app_ms), peaks["hbm_gbs"], cfg.name,
+            kernel="ring_append_kernel (inside the step graph)")
+        n_x = cfg.d_cq + cfg.d_latent
+        proj_flops = 2.0 * cfg.batch * cfg.n_q * (cfg.d_model * n_x + cfg.d_cq * cfg.n_heads * cfg.d_latent)
+        bandwidth["projections_in_step"] = {
+            "us": 1e3 * statistics.mean(proj_ms), "tflops": proj_flops / (statistics.mean(proj_ms) * 1e-3) / 1e12,
+            "kernel": "gemm_tc_kernel x2 (x-projection c_Q || [c_KV || k_R], then Q' with RoPE)",
+            "workload": cfg.name}
     n_units_all = world * cfg.batch
     ms_per_step = total_ms / args.steps
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
@@ -456,8 +579,12 @@ def run_ours(args, cfg):
                 "serial_value": world * flops_step * args.steps / (ser_ms * 1e-3) / 1e12,
                 "serial_ms_per_step": ser_ms / args.steps},
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "clocks": dict(clk.summary(), sm_mhz_device=sm_mhz_device,
+                       sm_mhz_device_method="mla_probe_sm_clock right after the last timed step: "
+                                            "median over SMs of cycles / global-timer ns"),
+        "bandwidth": bandwidth,
     }
+    result["roofline"]["sm_mhz"] = sm_mhz_device
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, dt, n = OracleSample(cfg)(args.cpu_rows)
         result["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s",
@@ -630,10 +757,24 @@ def run_backward(args, cfg):
     return 0
 
 
+def run_bandwidth_only(args, cfg):
+    """--bandwidth-only: the stand-alone timing of the memory-bound calls (measure_bandwidth) and
+    nothing else, one JSON object; used to profile those kernels on their own."""
+    import torch
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    peaks, _ = load_peaks()
+    reps = args.steps if args.steps_given else 20
+    bw = measure_bandwidth(cfg, flush, torch.cuda.current_stream(), peaks["hbm_gbs"], reps=reps)
+    print(json.dumps({"bandwidth": bw, "hbm_gbs": peaks["hbm_gbs"], "reps": reps}), flush=True)
+    return 0
+
+
 def kernel_sha() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("attention_sm100.cu", "sm100.cuh", "common.cuh", "kernels.h"):
+    for f in ("attention_sm100.cu", "sm100.cuh", "common.cuh", "kernels.h", "exp2.cuh"):
         h.update(open(os.path.join(ROOT, "mla_latent_kv_attn_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -648,6 +789,10 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=192)
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bandwidth", action="store_true",
+                    help="skip the stand-alone timing of the memory-bound calls")
+    ap.add_argument("--bandwidth-only", action="store_true",
+                    help="only time the memory-bound calls (append, RoPE, KV down-projection)")
     ap.add_argument("--backward", action="store_true",
                     help="time the attention backward call instead of the forward step")
     ap.add_argument("--d-c", type=int, default=None,
@@ -666,6 +811,8 @@ def main(argv=None):
         cfg = inputs.with_latent_shape(cfg, args.d_c or cfg.d_c, args.d_rope or cfg.d_rope)
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.bandwidth_only:
+        return run_bandwidth_only(args, cfg)
     if args.backward:
         return run_backward(args, cfg)
     if cfg.n_layers > 1:

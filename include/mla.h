@@ -416,6 +416,19 @@ mla_status mla_selftest_sincos(const float* angle, float* sin_out, float* cos_ou
 mla_status mla_selftest_rope_angles(const mla_config* cfg, const int32_t* pos, int32_t n,
                                     float* angle, float* sin_out, float* cos_out, void* stream);
 
+/* --------------------------------------------------------------------------------------------
+ * mla_probe_sm_clock: measures the SM clock on the device, for reports of achieved throughput
+ * (it reads counters only and changes no setting).  Launches n_ctas CTAs of one warp (one per
+ * SM when n_ctas <= the SM count and nothing else runs); thread 0 of each reads its SM's cycle
+ * counter and the global nanosecond timer, spins on the timer for spin_us microseconds and
+ * reads both again.  out (device uint64 [n_ctas, 4]) receives, per CTA: the SM id, the cycles
+ * and the nanoseconds elapsed, 0; the SM clock in MHz is 1000 * cycles / nanoseconds.
+ * 1 <= n_ctas <= 4096, 1 <= spin_us <= 1e5.  Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT,
+ * MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_probe_sm_clock(unsigned long long* out, int32_t n_ctas, int32_t spin_us,
+                              void* stream);
+
 #ifdef __cplusplus
 }
 #endif

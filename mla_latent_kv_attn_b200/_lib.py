@@ -78,6 +78,7 @@ SIGNATURES = {
     "mla_selftest_exp2": (c_int32, [_P, _P, _P, _P, c_int32, _P]),
     "mla_selftest_sincos": (c_int32, [_P, _P, _P, c_int32, _P]),
     "mla_selftest_rope_angles": (c_int32, [_CFG, _P, c_int32, _P, _P, _P, _P]),
+    "mla_probe_sm_clock": (c_int32, [_P, c_int32, c_int32, _P]),
 }
 
 _lib = None

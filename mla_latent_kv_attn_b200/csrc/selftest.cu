@@ -63,6 +63,27 @@ __global__ void rope_selftest_kernel(const int32_t* pos, int n, int n_pairs, Rop
   rope_sincos(a, &s[e], &c[e]);
 }
 
+// One CTA per SM: thread 0 reads the SM's cycle counter and the global nanosecond timer, spins
+// on the timer for spin_ns, and reads both again: out[4 * cta] = {smid, cycles, ns, 0}.
+__global__ void sm_clock_probe_kernel(unsigned long long* out, long long spin_ns) {
+  if (threadIdx.x != 0) return;
+  unsigned long long g0, g1, smid;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g0));
+  const long long c0 = clock64();
+  do {
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g1));
+  } while (static_cast<long long>(g1 - g0) < spin_ns);
+  const long long c1 = clock64();
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g1));
+  unsigned int id;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(id));
+  smid = id;
+  out[4 * blockIdx.x + 0] = smid;
+  out[4 * blockIdx.x + 1] = static_cast<unsigned long long>(c1 - c0);
+  out[4 * blockIdx.x + 2] = g1 - g0;
+  out[4 * blockIdx.x + 3] = 0ull;
+}
+
 mla_status check_device_word(const void* p, const char* name) {
   if (p == nullptr) MLA_FAIL(MLA_ERR_INVALID_ARG, "%s is null", name);
   if ((reinterpret_cast<uintptr_t>(p) & 3u) != 0)
@@ -160,5 +181,20 @@ extern "C" mla_status mla_selftest_wait_timeout(int32_t* dev_status, int32_t lim
   const long long limit = static_cast<long long>(khz) * limit_us / 1000;
   bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev_status, limit);
   MLA_LAUNCH_CHECK("bounded_wait_selftest");
+  return MLA_OK;
+}
+
+extern "C" mla_status mla_probe_sm_clock(unsigned long long* out, int32_t n_ctas, int32_t spin_us,
+                                         void* stream) {
+  using namespace mla;
+  set_last_error("");
+  MLA_CHECK_ARG(n_ctas > 0 && n_ctas <= 4096, "n_ctas must be in [1, 4096]");
+  MLA_CHECK_ARG(spin_us > 0 && spin_us <= 100000, "spin_us must be in (0, 1e5]");
+  MLA_SELFTEST_TRY(check_device_word(out, "out"));
+  if ((reinterpret_cast<uintptr_t>(out) & 7u) != 0)
+    MLA_FAIL(MLA_ERR_ALIGNMENT, "out is not 8-byte aligned");
+  sm_clock_probe_kernel<<<n_ctas, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      out, static_cast<long long>(spin_us) * 1000);
+  MLA_LAUNCH_CHECK("sm_clock_probe");
   return MLA_OK;
 }

@@ -280,6 +280,56 @@ __global__ void rope_keys_kernel(const T* __restrict__ cache, const T* __restric
   }
 }
 
+// The same rows with 16-byte vectors: one thread per 16-byte piece of a rotated key (4 bf16
+// pairs or 2 fp32 pairs), one 16-byte load and one 16-byte store each; the piece's position is
+// computed once for its pairs.  Needs d_c, d_rope and D at whole 16-byte multiples (host check).
+template <typename T>
+__global__ void __launch_bounds__(256)
+    rope_keys_vec_kernel(const T* __restrict__ cache, const T* __restrict__ chunk_lat,
+                         const int32_t* __restrict__ slot_frame, T* __restrict__ ws, int B, int W,
+                         int D, int d_c, int d_rope, int n_q, int nc, int nc_pad, int rows_ws,
+                         int row_begin, int row_end, int first_frame, RopeGeom g) {
+  constexpr int kPer = 16 / sizeof(T);          // elements per piece
+  const int pieces = d_rope / kPer;             // pieces per row
+  const int span = row_end - row_begin;
+  const int total = B * span * pieces;          // < 2^31 (host check)
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const int piece = e % pieces;
+    const int rs = e / pieces;
+    const int r = row_begin + rs % span;
+    const int b = rs / span;
+    uint4* dst = reinterpret_cast<uint4*>(ws + (static_cast<int64_t>(b) * rows_ws + r) * d_rope +
+                                          piece * kPer);
+    const T* src = nullptr;
+    int m = -1;
+    if (r < nc) {
+      m = r;
+      src = cache + (static_cast<int64_t>(b) * W * g.tpf + r) * D;
+    } else if (r >= nc_pad && r - nc_pad < n_q) {
+      m = nc + (r - nc_pad);
+      src = chunk_lat + (static_cast<int64_t>(b) * n_q + (r - nc_pad)) * D;
+    }
+    if (src == nullptr) {
+      *dst = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint4 raw = *reinterpret_cast<const uint4*>(src + d_c + piece * kPer);
+    int t, h, w;
+    key_position(slot_frame, b, W, g.tpf, g.frame_w, nc, first_frame, m, t, h, w);
+    const T* in = reinterpret_cast<const T*>(&raw);
+    uint4 outv;
+    T* out = reinterpret_cast<T*>(&outv);
+#pragma unroll
+    for (int i = 0; i < kPer; i += 2) {
+      float x0 = Elem<T>::to_f(in[i]), x1 = Elem<T>::to_f(in[i + 1]);
+      rope_rotate(x0, x1, rope_angle(g, (piece * kPer + i) / 2, t, h, w));
+      out[i] = Elem<T>::from_f(x0);
+      out[i + 1] = Elem<T>::from_f(x1);
+    }
+    *dst = outv;
+  }
+}
+
 }  // namespace
 
 KeyWorkspace key_workspace_layout(const Dims& d, int n_valid) {
@@ -305,6 +355,26 @@ mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_l
   const int64_t total = static_cast<int64_t>(d.B) * (row_end - row_begin) * n_pairs;
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));
   const RopeGeom g = rope_geom(d);
+  const size_t es = dtype_size(d.dtype);
+  const bool vec = (d.d_c * es) % 16 == 0 && (d.d_rope * es) % 16 == 0 && (d.D * es) % 16 == 0 &&
+                   aligned16(cache) && aligned16(chunk_lat) && aligned16(ws);
+  if (vec) {
+    const int64_t vtotal = static_cast<int64_t>(d.B) * (row_end - row_begin) *
+                           (d.d_rope * static_cast<int64_t>(es) / 16);
+    const int vblocks = static_cast<int>(std::min<int64_t>((vtotal + 255) / 256, 148 * 16));
+    if (d.dtype == MLA_FP32)
+      rope_keys_vec_kernel<float><<<vblocks, 256, 0, s>>>(
+          static_cast<const float*>(cache), static_cast<const float*>(chunk_lat), slot_frame,
+          static_cast<float*>(ws), d.B, d.W, d.D, d.d_c, d.d_rope, d.n_q, k.nc, k.nc_pad, k.rows,
+          row_begin, row_end, first_frame, g);
+    else
+      rope_keys_vec_kernel<bf16><<<vblocks, 256, 0, s>>>(
+          static_cast<const bf16*>(cache), static_cast<const bf16*>(chunk_lat), slot_frame,
+          static_cast<bf16*>(ws), d.B, d.W, d.D, d.d_c, d.d_rope, d.n_q, k.nc, k.nc_pad, k.rows,
+          row_begin, row_end, first_frame, g);
+    MLA_LAUNCH_CHECK("rope_keys_vec");
+    return MLA_OK;
+  }
   if (d.dtype == MLA_FP32)
     rope_keys_kernel<float><<<blocks, 256, 0, s>>>(
         static_cast<const float*>(cache), static_cast<const float*>(chunk_lat), slot_frame,

@@ -210,8 +210,10 @@ class ChunkGraph:
     frames, ring slots), so each chunk index gets its own graph; capturing is host-side work
     that can run ahead of the device, and a replay launches the chunk's kernels back to back
     without per-kernel host overhead.  Buffers, ring and weights are bound at capture time and
-    must stay alive and in place while the graph is used.  `events=True` also records a pair of
-    timing events around the attention call inside the graph (attn_start / attn_end).
+    must stay alive and in place while the graph is used.  `events=True` also records timing
+    events inside the graph around each of the chunk's three calls: the projections
+    (proj_start .. attn_start), the attention call (attn_start .. attn_end) and the append
+    (attn_end .. append_end).
     """
 
     def __init__(self, c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
@@ -221,12 +223,14 @@ class ChunkGraph:
         x = buf.x if x is None else x
         # external events: recorded by the graph at replay time (a plain event recorded during
         # capture only orders the graph's nodes and cannot be timed)
-        self.attn_start = torch.cuda.Event(enable_timing=True, external=True) if events else None
-        self.attn_end = torch.cuda.Event(enable_timing=True, external=True) if events else None
+        mk = lambda: torch.cuda.Event(enable_timing=True, external=True) if events else None
+        self.proj_start, self.attn_start, self.attn_end, self.append_end = mk(), mk(), mk(), mk()
         self.graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.graph(self.graph, stream=side, capture_error_mode="relaxed"):
+            if events:
+                self.proj_start.record()
             api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
             if events:
                 self.attn_start.record()
@@ -238,6 +242,8 @@ class ChunkGraph:
                 self.attn_end.record()
             api.mla_cache_append(c, None, None, buf.chunk_lat, ring.cache, ring.slot_frame,
                                  first, MLA_APPEND)
+            if events:
+                self.append_end.record()
         torch.cuda.current_stream().wait_stream(side)
         self.out = out
 
@@ -247,6 +253,12 @@ class ChunkGraph:
 
     def attention_ms(self) -> float:
         return self.attn_start.elapsed_time(self.attn_end)
+
+    def projection_ms(self) -> float:
+        return self.proj_start.elapsed_time(self.attn_start)
+
+    def append_ms(self) -> float:
+        return self.attn_end.elapsed_time(self.append_end)
 
 
 class LayerStack:
