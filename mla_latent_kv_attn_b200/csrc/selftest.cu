@@ -70,9 +70,11 @@ __global__ void sm_clock_probe_kernel(unsigned long long* out, long long spin_ns
   unsigned long long g0, g1, smid;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g0));
   const long long c0 = clock64();
-  do {
+  // bounded: at most 2^30 polls however the timer behaves
+  for (long long it = 0; it < (1LL << 30); ++it) {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g1));
-  } while (static_cast<long long>(g1 - g0) < spin_ns);
+    if (static_cast<long long>(g1 - g0) >= spin_ns) break;
+  }
   const long long c1 = clock64();
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g1));
   unsigned int id;
