@@ -391,7 +391,7 @@ def run_ours(args, cfg):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    c = api.make_config(cfg)
+    c = api.make_config(cfg, kernel_path=kernel_path(args))
     lw = inputs.layer_weights(cfg)
     w = rollout.upload_weights(c, lw, device=dev)
     ring = rollout.Ring(c, device=dev)
@@ -568,7 +568,9 @@ def run_ours(args, cfg):
         "attention_call_ms": attn_avg_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "mla_attention_fwd (rotated-key pre-pass + attention_tc_kernel)",
+                     "kernel": "mla_attention_fwd (rotated-key pre-pass + " +
+                               ("attention_pair_kernel" if args.kernel_path == "auto" and cfg.n_heads % 2 == 0
+                                and cfg.d_c in (128, 192) else "attention_tc_kernel") + ")",
                      "peak_kind": f"{peak_kind} burst bf16",
                      "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
         "e2e": {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12,
@@ -757,6 +759,11 @@ def run_backward(args, cfg):
     return 0
 
 
+def kernel_path(args) -> int:
+    from mla_latent_kv_attn_b200 import api
+    return {"auto": api.MLA_PATH_AUTO, "single": api.MLA_PATH_TC_SINGLE}[args.kernel_path]
+
+
 def run_bandwidth_only(args, cfg):
     """--bandwidth-only: the stand-alone timing of the memory-bound calls (measure_bandwidth) and
     nothing else, one JSON object; used to profile those kernels on their own."""
@@ -774,7 +781,8 @@ def run_bandwidth_only(args, cfg):
 def kernel_sha() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("attention_sm100.cu", "sm100.cuh", "common.cuh", "kernels.h", "exp2.cuh"):
+    for f in ("attention_sm100.cu", "attention_pair_sm100.cu", "sm100.cuh", "common.cuh",
+              "kernels.h", "exp2.cuh"):
         h.update(open(os.path.join(ROOT, "mla_latent_kv_attn_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -791,6 +799,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bandwidth", action="store_true",
                     help="skip the stand-alone timing of the memory-bound calls")
+    ap.add_argument("--kernel-path", choices=("auto", "single"), default="auto",
+                    help="attention kernel: auto (CTA pairs where the shape allows) or single "
+                         "(one CTA per head and query tile)")
     ap.add_argument("--bandwidth-only", action="store_true",
                     help="only time the memory-bound calls (append, RoPE, KV down-projection)")
     ap.add_argument("--backward", action="store_true",

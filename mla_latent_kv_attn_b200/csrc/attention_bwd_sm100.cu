@@ -720,7 +720,7 @@ int bwd_tc_head_groups(const Dims& d, int n_valid) {
 
 bool tc_bwd_supported(const Dims& d) {
   // n_q a multiple of 4: the key kernel copies a query tile's lse / Delta with 16-byte bulk copies
-  return d.dtype == MLA_BF16 && d.path == MLA_PATH_AUTO && d.d_c == kDc && d.d_rope == kDr &&
+  return d.dtype == MLA_BF16 && d.path != MLA_PATH_SIMT && d.d_c == kDc && d.d_rope == kDr &&
          d.n_q % 4 == 0;
 }
 

@@ -122,9 +122,7 @@ mla_status attention_fwd_static_scratch(const Dims& d, const AttnArgs& args,
   if (st != MLA_OK) return st;
   AttnArgs a = args;
   a.ws = ws;
-  if (d.dtype == MLA_BF16 && d.path == MLA_PATH_AUTO && tc_attention_supported(d, a.w_uv != nullptr))
-    return attention_tc(d, a, n_valid, s);
-  return attention_simt(d, a, n_valid, s);
+  return attention_dispatch(d, a, n_valid, s);
 }
 
 }  // namespace mla

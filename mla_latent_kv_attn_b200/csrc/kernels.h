@@ -140,6 +140,12 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s);
 
 bool tc_attention_supported(const Dims& d, bool has_w_uv);
 mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
+// CTA-pair tensor-core attention (attention_pair_sm100.cu): pairs of heads share each key tile.
+bool tc_attention_pair_supported(const Dims& d, bool has_w_uv);
+mla_status attention_tc_pair(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
+// The attention kernel a configuration gets (pair, single-CTA tensor-core or CUDA-core), given a
+// workspace that already holds the rotated keys.
+mla_status attention_dispatch(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
 
 // Attention with the scratch held in the library's built-in device array
 // (attention_static_ws.cu); args.ws is ignored.

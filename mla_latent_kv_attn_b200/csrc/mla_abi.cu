@@ -39,7 +39,8 @@ mla_status check_cfg(const mla_config* cfg) {
                 "chunk_frames (%d) must not exceed window_frames (%d)", c.chunk_frames,
                 c.window_frames);
   MLA_CHECK_ARG(c.dtype == MLA_BF16 || c.dtype == MLA_FP32, "unknown dtype %d", c.dtype);
-  MLA_CHECK_ARG(c.kernel_path == MLA_PATH_AUTO || c.kernel_path == MLA_PATH_SIMT,
+  MLA_CHECK_ARG(c.kernel_path == MLA_PATH_AUTO || c.kernel_path == MLA_PATH_SIMT ||
+                    c.kernel_path == MLA_PATH_TC_SINGLE,
                 "unknown kernel_path %d", c.kernel_path);
   const int64_t tpf = int64_t{c.frame_h} * c.frame_w;
   const int64_t D = int64_t{c.d_c} + c.d_rope;
@@ -91,7 +92,7 @@ mla_status check_ptr(const void* p, const char* name, bool required = true) {
     if (_s != MLA_OK) return _s;    \
   } while (0)
 
-bool use_tc(const Dims& d) { return d.dtype == MLA_BF16 && d.path == MLA_PATH_AUTO; }
+bool use_tc(const Dims& d) { return d.dtype == MLA_BF16 && d.path != MLA_PATH_SIMT; }
 
 // C[z](m, n) = sum_k A[z](m, k) B[z](n, k) with K contiguous in A and B; C row-major.
 mla_status gemm(const Dims& d, const void* A, int64_t a_sm, int64_t a_batch, const void* B,
@@ -185,12 +186,21 @@ mla_status attention_entry(const mla_config* cfg, const void* q, const void* chu
   AttnArgs a{};
   a.q = q; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = workspace; a.w_uv = w_uv;
   a.out = out; a.lse = lse; a.dev_status = dev_status;
-  if (use_tc(d) && tc_attention_supported(d, w_uv != nullptr))
-    return attention_tc(d, a, n_valid_frames, s);
-  return attention_simt(d, a, n_valid_frames, s);
+  return attention_dispatch(d, a, n_valid_frames, s);
 }
 
 }  // namespace
+
+mla_status attention_dispatch(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
+  const bool has_w_uv = a.w_uv != nullptr;
+  if (use_tc(d) && tc_attention_supported(d, has_w_uv)) {
+    if (d.path == MLA_PATH_AUTO && tc_attention_pair_supported(d, has_w_uv))
+      return attention_tc_pair(d, a, n_valid, s);
+    return attention_tc(d, a, n_valid, s);
+  }
+  return attention_simt(d, a, n_valid, s);
+}
+
 }  // namespace mla
 
 using namespace mla;

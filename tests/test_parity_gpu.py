@@ -16,7 +16,9 @@ from parity_util import (GpuRun, OracleRun, check_chunk, check_ring, compare,
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"tc": api.MLA_PATH_AUTO, "simt": api.MLA_PATH_SIMT}
+# "tc": the default path (CTA-pair attention where the shape allows); "tc1": tensor cores with
+# one CTA per head and query tile; "simt": CUDA cores
+PATHS = {"tc": api.MLA_PATH_AUTO, "tc1": api.MLA_PATH_TC_SINGLE, "simt": api.MLA_PATH_SIMT}
 
 
 def full_rollout(cfg, path, rows=None, check_positions=True):
@@ -53,15 +55,19 @@ def test_small_frames_bf16_rollout(path):
 LATENT_SHAPES = [(dc, dr) for dc in (128, 192, 256) for dr in (16, 32, 64)]
 
 
+@pytest.mark.parametrize("path", ["tc", "tc1"])
 @pytest.mark.parametrize("d_c,d_rope", LATENT_SHAPES)
-def test_latent_shape_sweep_tensor_cores_match_oracle(d_c, d_rope):
+def test_latent_shape_sweep_tensor_cores_match_oracle(d_c, d_rope, path):
     """The latent-size ablation shapes (d_c in {128, 192, 256} x d_rope in {16, 32, 64}) run on
-    the tensor-core kernels and match the oracle over a 4-chunk rollout whose ring wraps."""
+    the tensor-core kernels (the CTA-pair kernel for d_c 128 and 192 on the default path, and
+    the one-CTA kernel) and match the oracle over a 4-chunk rollout whose ring wraps."""
+    if path == "tc1" and d_c == 256:
+        pytest.skip("d_c 256 always runs the one-CTA kernel (covered by the default path)")
     cfg = inputs.with_latent_shape(inputs.small_bf16_config(), d_c, d_rope)
-    c = api.make_config(cfg)
+    c = api.make_config(cfg, kernel_path=PATHS[path])
     assert api.mla_attention_uses_tensor_cores(c, True)
     assert api.mla_attention_uses_tensor_cores(c, False)
-    report = full_rollout(cfg, api.MLA_PATH_AUTO)
+    report = full_rollout(cfg, PATHS[path])
     worst = max(v[1] for k, v in report.items() if k.endswith(".o"))
     assert worst <= 5e-3
 
@@ -135,6 +141,23 @@ def test_wan_config2_long_rollout_sampled():
         g.append(ch)
         check_ring(cfg, g, o)
     assert int(g.ring.slot_frame.max()) == 239
+
+
+def test_pair_and_single_cta_attention_agree_on_config1():
+    """Diagnostic cross-check on every row, head and output of config 1: the CTA-pair kernel
+    against the one-CTA tensor-core kernel (same operands, same fp32 accumulation; only the
+    order of the MMA pipeline's additions may differ, so a last-place bf16 difference at most)."""
+    cfg = inputs.CONFIGS[1]
+    outs = []
+    for path in (api.MLA_PATH_AUTO, api.MLA_PATH_TC_SINGLE):
+        g, _ = prefilled(cfg, path, cfg.measured_chunk)
+        outs.append(g.attend(cfg.measured_chunk, inputs.chunk_x(cfg, cfg.measured_chunk)))
+    for k in ("o", "o_lat", "lse"):
+        a, b = outs[0][k], outs[1][k]
+        err = np.abs(a - b)
+        assert np.isfinite(a).all(), k
+        assert err.max() <= 2 * 2.0 ** -8 * max(1.0, np.abs(b).max()), (k, err.max())
+        assert np.linalg.norm(a - b) / np.linalg.norm(b) <= 1e-3, k
 
 
 def test_tensor_core_and_cuda_core_paths_agree_on_config1():
