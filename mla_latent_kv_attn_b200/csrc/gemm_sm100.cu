@@ -25,7 +25,8 @@
 // (when the panel is one contiguous range) with one bulk prefetch, so the panel streams from HBM
 // in long runs instead of one 128-byte piece per row and K-slice.
 // Optionally the columns n >= n_split go to a second output C2 (column n - n_split): one GEMM
-// over [W_1; W_2] then writes x W_1^T and x W_2^T to their own arrays.
+// over [W_1; W_2] then writes x W_1^T and x W_2^T to their own arrays.  Optionally every output
+// row is also stored into a ring of frames (the fused down-projection and cache append).
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -79,6 +80,9 @@ struct GemmParams {
   int epilogue;
   int rope_D, rope_dr, rope_n_q, rope_first_frame;
   RopeGeom rope;
+  bf16* ring;                // ring append (see TcGemmArgs), or null
+  int32_t* slot_frame;
+  int ring_W, ring_tpf, ring_n_q, ring_first, ring_B;
 };
 
 __device__ __forceinline__ void store_row32(bf16* dst, const float* v, int valid, bool vec_ok) {
@@ -231,6 +235,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (p.c_batch % 8 == 0) &&
                         (p.n_split == 0 || (((reinterpret_cast<uintptr_t>(p.C2) & 15u) == 0) &&
                                             (p.c2_sm % 8 == 0) && (p.c2_batch % 8 == 0)));
+    if (p.ring != nullptr && blockIdx.x == 0 && threadIdx.x == 64) {
+      // the appended frames' slots: frame first + j of every sample lands in slot (first+j) mod W
+      const int frames = p.ring_n_q / p.ring_tpf;
+      for (int e = 0; e < p.ring_B * frames; ++e) {
+        const int f = p.ring_first + e % frames;
+        p.slot_frame[(e / frames) * p.ring_W + f % p.ring_W] = f;
+      }
+    }
+    const bool ring_vec = p.ring != nullptr && ((reinterpret_cast<uintptr_t>(p.ring) & 15u) == 0) &&
+                          (p.N % 8 == 0);
     int lt = 0, chunk = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
       const int acc = lt & 1;
@@ -275,6 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const bool second = p.n_split > 0 && n >= p.n_split;
+        if (p.ring != nullptr && m < p.M) {
+          // the same row into its ring slot (whole frames wrap; row width N)
+          const int bs = m / p.ring_n_q, r = m % p.ring_n_q;
+          const int slot = (p.ring_first + r / p.ring_tpf) % p.ring_W;
+          bf16* rrow = p.ring + (static_cast<int64_t>(bs) * p.ring_W * p.ring_tpf +
+                                 static_cast<int64_t>(slot) * p.ring_tpf + r % p.ring_tpf) * p.N;
+          store_row32(rrow + n, v, p.N - n, ring_vec);
+        }
         if (p.tma_store) {
           const uint32_t buf = out_base + (chunk & 1) * kStageOut;
           // the store that last read this buffer (two chunks ago) has finished reading it
@@ -393,6 +415,9 @@ mla_status launch_gemm(const TcGemmArgs& g, cudaStream_t s) {
   p.rope_first_frame = g.rope_first_frame; p.rope = g.rope;
   p.A = g.A; p.a_sm = g.a_sm;
   p.prefetch_a = (g.batch == 1 && g.a_sm == g.K) ? 1 : 0;
+  p.ring = static_cast<bf16*>(g.ring); p.slot_frame = g.slot_frame;
+  p.ring_W = g.ring_W; p.ring_tpf = g.ring_tpf; p.ring_n_q = g.ring_n_q;
+  p.ring_first = g.ring_first; p.ring_B = g.ring_B;
   // output maps: 32 x 128 boxes, 64B swizzle (the staging layout)
   CUtensorMap tc, tc2;
   p.tma_store = tma_storable(g.C, g.c_sm, g.c_batch, g.batch) &&
@@ -432,6 +457,11 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s) {
   if (g.M == 0 || g.N == 0) return MLA_OK;
   if (g.n_split != 0 && (g.n_split % 32 != 0 || g.n_split >= g.N || g.C2 == nullptr))
     MLA_FAIL(MLA_ERR_INVALID_ARG, "GEMM column split must be a multiple of 32 inside N");
+  if (g.ring != nullptr &&
+      (g.batch != 1 || g.n_split != 0 || g.slot_frame == nullptr || g.ring_W <= 0 ||
+       g.ring_tpf <= 0 || g.ring_n_q % g.ring_tpf != 0 ||
+       static_cast<int64_t>(g.ring_B) * g.ring_n_q != g.M))
+    MLA_FAIL(MLA_ERR_INVALID_ARG, "GEMM ring epilogue: inconsistent ring geometry");
   if (g.epilogue == kEpiRopeQ &&
       (g.rope_D <= 0 || g.N % g.rope_D != 0 || g.rope_dr % 2 != 0 || g.rope_dr > g.rope_D ||
        g.rope_dr / 2 > kMaxRopePairs))

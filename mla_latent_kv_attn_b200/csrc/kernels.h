@@ -133,6 +133,13 @@ struct TcGemmArgs {
   // last rope_dr columns are rotated.
   int rope_D, rope_dr, rope_n_q, rope_first_frame;
   RopeGeom rope;
+  // Optional ring append from the epilogue (batch 1, n_split 0): row m = chunk token
+  // (sample m / ring_n_q, frame j, token i) is also stored to ring row
+  // ((ring_first + j) mod ring_W) * ring_tpf + i of its sample (row width N), and slot_frame of
+  // every appended frame is set.
+  void* ring;
+  int32_t* slot_frame;
+  int ring_W, ring_tpf, ring_n_q, ring_first, ring_B;
 };
 
 bool tc_gemm_supported(int M, int N, int K, int64_t a_sm, int64_t b_sn);

@@ -245,8 +245,23 @@ mla_status mla_cache_append(const mla_config* cfg, const void* x, const void* w_
     MLA_TRY(check_ptr(cache, "cache"));
     MLA_TRY(check_ptr(slot_frame, "slot_frame"));
   }
+  const int M = d.B * d.n_q;
+  if (mode == MLA_PROJECT_AND_APPEND && use_tc(d) &&
+      tc_gemm_supported(M, d.D, d.d_model, d.d_model, d.d_model)) {
+    // one kernel: the GEMM's epilogue stores every row to chunk_lat and to its ring slot
+    TcGemmArgs g{};
+    g.A = x; g.a_sm = d.d_model; g.a_batch = 0;
+    g.B = w_dkv_kr; g.b_sn = d.d_model; g.b_batch = 0;
+    g.C = chunk_lat; g.c_sm = d.D; g.c_batch = 0;
+    g.M = M; g.N = d.D; g.K = d.d_model; g.batch = 1;
+    g.epilogue = kEpiStore;
+    g.ring = cache; g.slot_frame = slot_frame;
+    g.ring_W = d.W; g.ring_tpf = d.tpf; g.ring_n_q = d.n_q; g.ring_first = first_frame;
+    g.ring_B = d.B;
+    return gemm_tc(g, s);
+  }
   if (mode & MLA_PROJECT)
-    MLA_TRY(gemm(d, x, d.d_model, 0, w_dkv_kr, d.d_model, 0, chunk_lat, d.D, 0, d.B * d.n_q, d.D,
+    MLA_TRY(gemm(d, x, d.d_model, 0, w_dkv_kr, d.d_model, 0, chunk_lat, d.D, 0, M, d.D,
                  d.d_model, 1, s));
   if (mode & MLA_APPEND) MLA_TRY(ring_append(d, chunk_lat, cache, slot_frame, first_frame, s));
   return MLA_OK;

@@ -212,6 +212,32 @@ def test_project_chunk_matches_separate_projections(cfg_id, path):
         compare("fused.q", fused["q"][bi][rows], q_ref, cfg.dtype)
 
 
+@pytest.mark.parametrize("cfg_id", ["small", "3"])
+def test_fused_project_and_append_matches_separate_calls(cfg_id):
+    """mla_cache_append(MLA_PROJECT_AND_APPEND) on the tensor cores stores every projected row
+    to its ring slot from the GEMM's epilogue; the ring, slot_frame and chunk latents are
+    bit-identical to MLA_PROJECT followed by MLA_APPEND, over chunks whose frames wrap the ring
+    (and, for the small frames, wrap inside a chunk)."""
+    cfg = inputs.small_bf16_config() if cfg_id == "small" else inputs.CONFIGS[3]
+    a, b = GpuRun(cfg), GpuRun(cfg)
+    n = cfg.n_chunks if cfg_id == "small" else cfg.window_frames // cfg.chunk_frames + 2
+    for ch in range(n):
+        x = inputs.chunk_x(cfg, ch)
+        first = cfg.first_frame(ch)
+        a.load_x(x)
+        b.load_x(x)
+        api.mla_cache_append(a.c, a.buf.x, a.w.w_dkv_kr, a.buf.chunk_lat, a.ring.cache,
+                             a.ring.slot_frame, first, api.MLA_PROJECT_AND_APPEND)
+        api.mla_cache_append(b.c, b.buf.x, b.w.w_dkv_kr, b.buf.chunk_lat, b.ring.cache,
+                             b.ring.slot_frame, first, api.MLA_PROJECT)
+        api.mla_cache_append(b.c, None, None, b.buf.chunk_lat, b.ring.cache, b.ring.slot_frame,
+                             first, api.MLA_APPEND)
+        torch.cuda.synchronize()
+        assert torch.equal(a.buf.chunk_lat, b.buf.chunk_lat), ch
+        assert torch.equal(a.ring.slot_frame, b.ring.slot_frame), ch
+        assert torch.equal(a.ring.cache, b.ring.cache), ch
+
+
 def test_host_streamer_matches_serial_rollout():
     """rollout.HostStreamer (pinned host tokens in, output out, copies overlapped with the
     neighbouring chunks' compute) gives bit-identical outputs to run_chunk one chunk at a time."""
