@@ -44,8 +44,14 @@ def headers():
     return hs + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 
 
+def extra_flags():
+    """MLA_NVTX=1 in the environment builds NVTX ranges around every C-ABI call (for profilers;
+    off by default)."""
+    return ["-DMLA_NVTX"] if os.environ.get("MLA_NVTX") == "1" else []
+
+
 def _compile(src: str, obj: str, ptxas_verbose: bool) -> str:
-    cmd = [nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
+    cmd = [nvcc(), *ARCH, *FLAGS, *extra_flags(), "-c", src, "-o", obj]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,6 +62,13 @@ def _compile(src: str, obj: str, ptxas_verbose: bool) -> str:
 
 def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:
     os.makedirs(BUILD, exist_ok=True)
+    # objects built with other flags (e.g. NVTX on/off) are rebuilt
+    stamp = os.path.join(BUILD, "flags.txt")
+    flags = " ".join(ARCH + FLAGS + extra_flags())
+    if not os.path.exists(stamp) or open(stamp).read() != flags:
+        force = True
+        with open(stamp, "w") as f:
+            f.write(flags)
     hdr_time = max(os.path.getmtime(h) for h in headers())
     jobs = []
     objs = []

@@ -49,6 +49,23 @@ void set_last_error(const std::string& msg);  // per host thread (mla_abi.cu)
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// ---- NVTX ranges (built in only with -DMLA_NVTX; header-only NVTX 3, no link dependency) -----
+
+#ifdef MLA_NVTX
+}  // namespace mla
+#include <nvtx3/nvToolsExt.h>
+namespace mla {
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+#define MLA_NVTX_RANGE(name) ::mla::NvtxRange mla_nvtx_range_(name)
+#else
+#define MLA_NVTX_RANGE(name) \
+  do {                       \
+  } while (0)
+#endif
+
 // ---- element types ---------------------------------------------------------------------------
 
 using bf16 = __nv_bfloat16;

@@ -224,11 +224,15 @@ const char* mla_last_error(void) { return g_last_error.c_str(); }
 
 int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
 
-mla_status mla_config_check(const mla_config* cfg) { return check_cfg(cfg); }
+mla_status mla_config_check(const mla_config* cfg) {
+  MLA_NVTX_RANGE("mla_config_check");
+  return check_cfg(cfg);
+}
 
 mla_status mla_cache_append(const mla_config* cfg, const void* x, const void* w_dkv_kr,
                             void* chunk_lat, void* cache, int32_t* slot_frame,
                             int32_t first_frame, int32_t mode, void* stream) {
+  MLA_NVTX_RANGE("mla_cache_append");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   MLA_CHECK_ARG(mode == MLA_PROJECT || mode == MLA_APPEND || mode == MLA_PROJECT_AND_APPEND,
@@ -271,6 +275,7 @@ mla_status mla_rope3d(const mla_config* cfg, void* data, int32_t n_samples,
                       int32_t rows_per_sample, int32_t row_width, int32_t col_offset,
                       int32_t n_vec, int32_t vec_stride, const int32_t* frame_table,
                       int32_t frame_table_stride, int32_t first_frame, void* stream) {
+  MLA_NVTX_RANGE("mla_rope3d");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -296,6 +301,7 @@ mla_status mla_rope3d(const mla_config* cfg, void* data, int32_t n_samples,
 mla_status mla_key_positions(const mla_config* cfg, const int32_t* slot_frame,
                              int32_t n_valid_frames, int32_t first_frame, int32_t* pos_out,
                              void* stream) {
+  MLA_NVTX_RANGE("mla_key_positions");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -310,6 +316,7 @@ mla_status mla_key_positions(const mla_config* cfg, const int32_t* slot_frame,
 
 mla_status mla_compose_query_weights(const mla_config* cfg, const void* w_uq, const void* w_uk,
                                      const void* w_qr, void* w_qcat, void* stream) {
+  MLA_NVTX_RANGE("mla_compose_query_weights");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -334,6 +341,7 @@ mla_status mla_compose_query_weights(const mla_config* cfg, const void* w_uq, co
 mla_status mla_query_proj(const mla_config* cfg, const void* x, const void* w_dq,
                           const void* w_qcat, void* c_q, void* q, int32_t first_frame,
                           void* stream) {
+  MLA_NVTX_RANGE("mla_query_proj");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -352,6 +360,7 @@ mla_status mla_query_proj(const mla_config* cfg, const void* x, const void* w_dq
 mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w_x,
                              const void* w_qcat, void* c_q, void* q, void* chunk_lat,
                              int32_t first_frame, void* stream) {
+  MLA_NVTX_RANGE("mla_project_chunk");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -402,6 +411,7 @@ mla_status mla_attention_fwd(const mla_config* cfg, const void* q, const void* c
                              int32_t n_valid_frames, int32_t first_frame, const void* w_uv,
                              void* out, float* lse, void* workspace, size_t workspace_bytes,
                              int32_t* dev_status, void* stream) {
+  MLA_NVTX_RANGE("mla_attention_fwd");
   return attention_entry(cfg, q, chunk_lat, cache, slot_frame, n_valid_frames, first_frame, w_uv,
                          out, lse, workspace, workspace_bytes, dev_status, stream, kRopeKeysAll);
 }
@@ -412,6 +422,7 @@ mla_status mla_attention_fwd_cached_ring(const mla_config* cfg, const void* q,
                                          int32_t first_frame, const void* w_uv, void* out,
                                          float* lse, void* workspace, size_t workspace_bytes,
                                          int32_t* dev_status, void* stream) {
+  MLA_NVTX_RANGE("mla_attention_fwd_cached_ring");
   return attention_entry(cfg, q, chunk_lat, cache, slot_frame, n_valid_frames, first_frame, w_uv,
                          out, lse, workspace, workspace_bytes, dev_status, stream,
                          kRopeKeysChunk);
@@ -420,6 +431,7 @@ mla_status mla_attention_fwd_cached_ring(const mla_config* cfg, const void* q,
 mla_status mla_rotate_ring_keys(const mla_config* cfg, const void* cache,
                                 const int32_t* slot_frame, int32_t n_valid_frames,
                                 void* workspace, size_t workspace_bytes, void* stream) {
+  MLA_NVTX_RANGE("mla_rotate_ring_keys");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -437,6 +449,7 @@ mla_status mla_attention_fwd_static_scratch(const mla_config* cfg, const void* q
                                             const int32_t* slot_frame, int32_t n_valid_frames,
                                             int32_t first_frame, const void* w_uv, void* out,
                                             float* lse, int32_t* dev_status, void* stream) {
+  MLA_NVTX_RANGE("mla_attention_fwd_static_scratch");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -471,6 +484,7 @@ mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* c
                              const float* lse, const void* d_o_lat, void* d_q,
                              void* d_chunk_lat, void* d_cache, void* workspace,
                              size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  MLA_NVTX_RANGE("mla_attention_bwd");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
@@ -504,6 +518,7 @@ mla_status mla_attention_bwd(const mla_config* cfg, const void* q, const void* c
 
 mla_status mla_out_proj(const mla_config* cfg, const void* o_lat, const void* w_uv,
                         const void* w_o, void* o, void* y, void* stream) {
+  MLA_NVTX_RANGE("mla_out_proj");
   set_last_error("");
   MLA_TRY(check_cfg(cfg));
   const Dims d = dims_of(*cfg);
