@@ -355,7 +355,8 @@ def measure_bandwidth(cfg, flush, stream, hbm_gbs: float, reps: int = 20):
         res[f"rope_ring_keys_{tag}"] = bandwidth_entry(2.0 * batch * W * tpf * cfg.d_rope * es, ms,
                                                        hbm_gbs, wl, kernel="rope_keys_vec_kernel")
         q = torch.randn((batch, n_q, cfg.n_heads, D), device="cuda").to(dt)
-        ms = time_calls(lambda: api.mla_rope3d(c, q, n_vec=cfg.n_heads, col_offset=cfg.d_c,
+        q3 = q.view(batch, n_q, cfg.n_heads * D)
+        ms = time_calls(lambda: api.mla_rope3d(c, q3, n_vec=cfg.n_heads, col_offset=cfg.d_c,
                                                vec_stride=D, first_frame=first),
                         flush, stream, reps)
         res[f"rope_query_{tag}"] = bandwidth_entry(2.0 * batch * n_q * cfg.n_heads * cfg.d_rope * es,
@@ -371,7 +372,7 @@ def measure_bandwidth(cfg, flush, stream, hbm_gbs: float, reps: int = 20):
             res[f"kv_down_projection_{tag}"] = bandwidth_entry(
                 nbytes, ms, hbm_gbs, wl, kernel="gemm_tc_kernel", tflops=flops / (ms * 1e-3) / 1e12)
             del x, wkv
-        del ring, lat, ws, q
+        del ring, lat, ws, q, q3
         torch.cuda.empty_cache()
     return res
 
@@ -525,19 +526,19 @@ def run_ours(args, cfg):
     peaks, peak_kind = load_peaks()
     bandwidth = measure_bandwidth(cfg, flush, stream, peaks["hbm_gbs"]) if not args.no_bandwidth \
         else None
-    if bandwidth is not None:
-        # the step's own append and projections, timed inside the step graphs
-        es = 2
-        app_bytes = 2.0 * cfg.batch * cfg.n_q * cfg.d_latent * es
-        bandwidth["ring_append_in_step"] = bandwidth_entry(
-            app_bytes, statistics.mean(app_ms), peaks["hbm_gbs"], cfg.name,
-            kernel="ring_append_kernel (inside the step graph)")
-        n_x = cfg.d_cq + cfg.d_latent
-        proj_flops = 2.0 * cfg.batch * cfg.n_q * (cfg.d_model * n_x + cfg.d_cq * cfg.n_heads * cfg.d_latent)
-        bandwidth["projections_in_step"] = {
-            "us": 1e3 * statistics.mean(proj_ms), "tflops": proj_flops / (statistics.mean(proj_ms) * 1e-3) / 1e12,
-            "kernel": "gemm_tc_kernel x2 (x-projection c_Q || [c_KV || k_R], then Q' with RoPE)",
-            "workload": cfg.name}
+    # the step's three calls, timed by events inside the step graphs (means over the timed steps)
+    n_x = cfg.d_cq + cfg.d_latent
+    proj_flops = 2.0 * cfg.batch * cfg.n_q * (cfg.d_model * n_x + cfg.d_cq * cfg.n_heads * cfg.d_latent)
+    app_bytes = 2.0 * cfg.batch * cfg.n_q * cfg.d_latent * 2
+    step_breakdown = {
+        "projections_us": 1e3 * statistics.mean(proj_ms),
+        "projections_tflops": proj_flops / (statistics.mean(proj_ms) * 1e-3) / 1e12,
+        "attention_call_us": 1e3 * statistics.mean(attn_ms),
+        "append_us": 1e3 * statistics.mean(app_ms),
+        "append_gbs": app_bytes / (statistics.mean(app_ms) * 1e-3) / 1e9,
+        "step_us": 1e3 * statistics.mean(step_ms),
+        "calls": "mla_project_chunk (x-projection GEMM, Q' GEMM + RoPE) | mla_attention_fwd "
+                 "(rotated-key pre-pass + attention) | mla_cache_append(MLA_APPEND)"}
     n_units_all = world * cfg.batch
     ms_per_step = total_ms / args.steps
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
@@ -584,6 +585,7 @@ def run_ours(args, cfg):
         "clocks": dict(clk.summary(), sm_mhz_device=sm_mhz_device,
                        sm_mhz_device_method="mla_probe_sm_clock right after the last timed step: "
                                             "median over SMs of cycles / global-timer ns"),
+        "step_breakdown": step_breakdown,
         "bandwidth": bandwidth,
     }
     result["roofline"]["sm_mhz"] = sm_mhz_device
