@@ -122,9 +122,12 @@ __device__ __forceinline__ float pair_exp_row(const float (&s)[kBN], float scale
   return l0 + l1;
 }
 
+// Waits use the default acquire (CTA scope) whoever arrives: the data behind every per-tile
+// barrier is TMEM or TMA-written shared memory, ordered by tcgen05 fences and the async proxy;
+// the one hand-off of generic shared-memory writes (O_lat) is released at cluster scope.
 __device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                       int32_t* dev_status) {
-  return mbar_wait_cluster_or_abort(bar, parity, abort_flag, dev_status);
+  return mbar_wait_or_abort(bar, parity, abort_flag, dev_status);
 }
 
 template <int DC, int DR>
@@ -295,7 +298,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (ok && p.has_w_uv) {
           ok = pwait(smem_u32(&w_full), 0, abort_flag, p.dev_status) &&
-               pwait(smem_u32(&olat_full), 0, abort_flag, p.dev_status);
+               mbar_wait_cluster_or_abort(smem_u32(&olat_full), 0, abort_flag, p.dev_status);
           if (ok) {
             tc_fence_after();
             const uint64_t o_c = smem_desc(sQ, 16, 1024, kSwizzle128B);     // O_lat over Q
@@ -317,8 +320,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int row = warp * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int n = q0 + row;
-    const uint32_t s_free_l[2] = {map_to_cta(smem_u32(&s_free[0]), 0),
-                                  map_to_cta(smem_u32(&s_free[1]), 0)};
+    const uint32_t s_free_l0 = map_to_cta(smem_u32(&s_free[0]), 0);
+    const uint32_t s_free_l1 = map_to_cta(smem_u32(&s_free[1]), 0);
     const uint32_t p_full_l = map_to_cta(smem_u32(&p_full), 0);
     const uint32_t olat_full_l = map_to_cta(smem_u32(&olat_full), 0);
     float m_run = -INFINITY, l_run = 0.f;
@@ -339,7 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // S(j) is in registers: one arrival per warp frees its buffer for QK(j+2)
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(s_free_l[sb]);
+      if (lane == 0) mbar_arrive_remote(sb ? s_free_l1 : s_free_l0);
       const int valid = j < p.nt_ring ? min(kBN, p.nc - j * kBN)
                                       : min(kBN, p.n_q - (j - p.nt_ring) * kBN);
       if (valid < kBN) {
@@ -400,7 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(p_full_l);
+      if (lane == 0) mbar_arrive_remote(p_full_l);
     }
     if (ok)
       ok = __all_sync(0xffffffffu, pwait(smem_u32(&pv_done), (p.nt - 1) & 1, abort_flag, p.dev_status));

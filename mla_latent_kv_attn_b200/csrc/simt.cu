@@ -130,6 +130,57 @@ __global__ void rope3d_kernel(T* data, int n_samples, int rows, int row_width, i
   }
 }
 
+// One thread per rotated vector (d_rope values, whole 16-byte pieces): every piece is loaded
+// before the first is rotated and stored, and the row's position is computed once.
+template <typename T, int kPieces>
+__global__ void __launch_bounds__(256)
+    rope3d_vec_kernel(T* data, int n_samples, int rows, int row_width, int col_offset, int n_vec,
+                      int vec_stride, const int32_t* frame_table, int frame_table_stride,
+                      int first_frame, RopeGeom g) {
+  constexpr int kPer = 16 / sizeof(T);
+  const int64_t total = static_cast<int64_t>(n_samples) * rows * n_vec;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int v = static_cast<int>(e % n_vec);
+    const int64_t rr = e / n_vec;                  // sample * rows + row
+    const int r = static_cast<int>(rr % rows);
+    const int smp = static_cast<int>(rr / rows);
+    const int fi = r / g.tpf, i = r % g.tpf;
+    const int t = frame_table ? frame_table[static_cast<int64_t>(smp) * frame_table_stride + fi]
+                              : first_frame + fi;
+    if (t < 0) continue;
+    uint4* p = reinterpret_cast<uint4*>(data + rr * row_width + col_offset +
+                                        static_cast<int64_t>(v) * vec_stride);
+    uint4 raw[kPieces];
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) raw[k] = p[k];
+    const int h = i / g.frame_w, w = i % g.frame_w;
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) {
+      T* x = reinterpret_cast<T*>(&raw[k]);
+#pragma unroll
+      for (int q = 0; q < kPer; q += 2) {
+        float x0 = Elem<T>::to_f(x[q]), x1 = Elem<T>::to_f(x[q + 1]);
+        rope_rotate(x0, x1, rope_angle(g, (k * kPer + q) / 2, t, h, w));
+        x[q] = Elem<T>::from_f(x0);
+        x[q + 1] = Elem<T>::from_f(x1);
+      }
+      p[k] = raw[k];
+    }
+  }
+}
+
+template <typename T, int kPieces>
+void launch_rope3d_vec(T* data, int n_samples, int rows, int row_width, int col_offset, int n_vec,
+                       int vec_stride, const int32_t* frame_table, int frame_table_stride,
+                       int first_frame, const RopeGeom& g, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(n_samples) * rows * n_vec;
+  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));
+  rope3d_vec_kernel<T, kPieces><<<blocks, 256, 0, s>>>(data, n_samples, rows, row_width,
+                                                       col_offset, n_vec, vec_stride, frame_table,
+                                                       frame_table_stride, first_frame, g);
+}
+
 }  // namespace
 
 mla_status rope3d_inplace(const Dims& d, void* data, int n_samples, int rows, int row_width,
@@ -141,6 +192,27 @@ mla_status rope3d_inplace(const Dims& d, void* data, int n_samples, int rows, in
   const int threads = 256;
   const int blocks = static_cast<int>(std::min<int64_t>((total + threads - 1) / threads, 148 * 16));
   const RopeGeom g = rope_geom(d);
+  const int es = static_cast<int>(dtype_size(d.dtype));
+  const int pieces = d.d_rope * es / 16;
+  if (aligned16(data) && (d.d_rope * es) % 16 == 0 && (col_offset * es) % 16 == 0 &&
+      (vec_stride * es) % 16 == 0 && (static_cast<int64_t>(row_width) * es) % 16 == 0 &&
+      (pieces == 2 || pieces == 4 || pieces == 8)) {
+#define MLA_ROPE_VEC(T, P)                                                                      \
+  launch_rope3d_vec<T, P>(static_cast<T*>(data), n_samples, rows, row_width, col_offset, n_vec, \
+                          vec_stride, frame_table, frame_table_stride, first_frame, g, s)
+    if (d.dtype == MLA_FP32) {
+      if (pieces == 2) MLA_ROPE_VEC(float, 2);
+      else if (pieces == 4) MLA_ROPE_VEC(float, 4);
+      else MLA_ROPE_VEC(float, 8);
+    } else {
+      if (pieces == 2) MLA_ROPE_VEC(bf16, 2);
+      else if (pieces == 4) MLA_ROPE_VEC(bf16, 4);
+      else MLA_ROPE_VEC(bf16, 8);
+    }
+#undef MLA_ROPE_VEC
+    MLA_LAUNCH_CHECK("rope3d_vec");
+    return MLA_OK;
+  }
   if (d.dtype == MLA_FP32)
     rope3d_kernel<float><<<blocks, threads, 0, s>>>(static_cast<float*>(data), n_samples, rows,
                                                     row_width, col_offset, n_vec, vec_stride,
@@ -280,26 +352,23 @@ __global__ void rope_keys_kernel(const T* __restrict__ cache, const T* __restric
   }
 }
 
-// The same rows with 16-byte vectors: one thread per 16-byte piece of a rotated key (4 bf16
-// pairs or 2 fp32 pairs), one 16-byte load and one 16-byte store each; the piece's position is
-// computed once for its pairs.  Needs d_c, d_rope and D at whole 16-byte multiples (host check).
-template <typename T>
+// The same rows with 16-byte vectors: one thread per rotated key (kPieces 16-byte pieces of
+// d_rope values); every piece is loaded before the first is rotated and stored, and the key's
+// position is computed once.  Needs d_c, d_rope and D at whole 16-byte multiples (host check).
+template <typename T, int kPieces>
 __global__ void __launch_bounds__(256)
     rope_keys_vec_kernel(const T* __restrict__ cache, const T* __restrict__ chunk_lat,
                          const int32_t* __restrict__ slot_frame, T* __restrict__ ws, int B, int W,
-                         int D, int d_c, int d_rope, int n_q, int nc, int nc_pad, int rows_ws,
-                         int row_begin, int row_end, int first_frame, RopeGeom g) {
+                         int D, int d_c, int n_q, int nc, int nc_pad, int rows_ws, int row_begin,
+                         int row_end, int first_frame, RopeGeom g) {
   constexpr int kPer = 16 / sizeof(T);          // elements per piece
-  const int pieces = d_rope / kPer;             // pieces per row
+  constexpr int kDr = kPieces * kPer;
   const int span = row_end - row_begin;
-  const int total = B * span * pieces;          // < 2^31 (host check)
+  const int total = B * span;                   // < 2^31 (host check)
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-    const int piece = e % pieces;
-    const int rs = e / pieces;
-    const int r = row_begin + rs % span;
-    const int b = rs / span;
-    uint4* dst = reinterpret_cast<uint4*>(ws + (static_cast<int64_t>(b) * rows_ws + r) * d_rope +
-                                          piece * kPer);
+    const int r = row_begin + e % span;
+    const int b = e / span;
+    uint4* dst = reinterpret_cast<uint4*>(ws + (static_cast<int64_t>(b) * rows_ws + r) * kDr);
     const T* src = nullptr;
     int m = -1;
     if (r < nc) {
@@ -310,23 +379,28 @@ __global__ void __launch_bounds__(256)
       src = chunk_lat + (static_cast<int64_t>(b) * n_q + (r - nc_pad)) * D;
     }
     if (src == nullptr) {
-      *dst = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int k = 0; k < kPieces; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
       continue;
     }
-    const uint4 raw = *reinterpret_cast<const uint4*>(src + d_c + piece * kPer);
+    uint4 raw[kPieces];
+    const uint4* s4 = reinterpret_cast<const uint4*>(src + d_c);
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) raw[k] = s4[k];
     int t, h, w;
     key_position(slot_frame, b, W, g.tpf, g.frame_w, nc, first_frame, m, t, h, w);
-    const T* in = reinterpret_cast<const T*>(&raw);
-    uint4 outv;
-    T* out = reinterpret_cast<T*>(&outv);
 #pragma unroll
-    for (int i = 0; i < kPer; i += 2) {
-      float x0 = Elem<T>::to_f(in[i]), x1 = Elem<T>::to_f(in[i + 1]);
-      rope_rotate(x0, x1, rope_angle(g, (piece * kPer + i) / 2, t, h, w));
-      out[i] = Elem<T>::from_f(x0);
-      out[i + 1] = Elem<T>::from_f(x1);
+    for (int k = 0; k < kPieces; ++k) {
+      T* x = reinterpret_cast<T*>(&raw[k]);
+#pragma unroll
+      for (int q = 0; q < kPer; q += 2) {
+        float x0 = Elem<T>::to_f(x[q]), x1 = Elem<T>::to_f(x[q + 1]);
+        rope_rotate(x0, x1, rope_angle(g, (k * kPer + q) / 2, t, h, w));
+        x[q] = Elem<T>::from_f(x0);
+        x[q + 1] = Elem<T>::from_f(x1);
+      }
+      dst[k] = raw[k];
     }
-    *dst = outv;
   }
 }
 
@@ -358,20 +432,25 @@ mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_l
   const size_t es = dtype_size(d.dtype);
   const bool vec = (d.d_c * es) % 16 == 0 && (d.d_rope * es) % 16 == 0 && (d.D * es) % 16 == 0 &&
                    aligned16(cache) && aligned16(chunk_lat) && aligned16(ws);
-  if (vec) {
-    const int64_t vtotal = static_cast<int64_t>(d.B) * (row_end - row_begin) *
-                           (d.d_rope * static_cast<int64_t>(es) / 16);
+  const int pieces = d.d_rope * static_cast<int>(es) / 16;
+  if (vec && (pieces == 2 || pieces == 4 || pieces == 8)) {
+    const int64_t vtotal = static_cast<int64_t>(d.B) * (row_end - row_begin);
     const int vblocks = static_cast<int>(std::min<int64_t>((vtotal + 255) / 256, 148 * 16));
-    if (d.dtype == MLA_FP32)
-      rope_keys_vec_kernel<float><<<vblocks, 256, 0, s>>>(
-          static_cast<const float*>(cache), static_cast<const float*>(chunk_lat), slot_frame,
-          static_cast<float*>(ws), d.B, d.W, d.D, d.d_c, d.d_rope, d.n_q, k.nc, k.nc_pad, k.rows,
-          row_begin, row_end, first_frame, g);
-    else
-      rope_keys_vec_kernel<bf16><<<vblocks, 256, 0, s>>>(
-          static_cast<const bf16*>(cache), static_cast<const bf16*>(chunk_lat), slot_frame,
-          static_cast<bf16*>(ws), d.B, d.W, d.D, d.d_c, d.d_rope, d.n_q, k.nc, k.nc_pad, k.rows,
-          row_begin, row_end, first_frame, g);
+#define MLA_KEYS_VEC(T, P)                                                                       \
+  rope_keys_vec_kernel<T, P><<<vblocks, 256, 0, s>>>(                                          \
+      static_cast<const T*>(cache), static_cast<const T*>(chunk_lat), slot_frame,               \
+      static_cast<T*>(ws), d.B, d.W, d.D, d.d_c, d.n_q, k.nc, k.nc_pad, k.rows, row_begin,      \
+      row_end, first_frame, g)
+    if (d.dtype == MLA_FP32) {
+      if (pieces == 2) MLA_KEYS_VEC(float, 2);
+      else if (pieces == 4) MLA_KEYS_VEC(float, 4);
+      else MLA_KEYS_VEC(float, 8);
+    } else {
+      if (pieces == 2) MLA_KEYS_VEC(bf16, 2);
+      else if (pieces == 4) MLA_KEYS_VEC(bf16, 4);
+      else MLA_KEYS_VEC(bf16, 8);
+    }
+#undef MLA_KEYS_VEC
     MLA_LAUNCH_CHECK("rope_keys_vec");
     return MLA_OK;
   }

@@ -345,7 +345,15 @@ __device__ __forceinline__ uint32_t map_to_cta(uint32_t addr, uint32_t rank) {
 }
 
 // Arrives on an mbarrier that may live in another CTA of the cluster (cluster-window address),
-// releasing this thread's prior writes at cluster scope.
+// with the default release semantics at CTA scope: enough to order this thread's tcgen05
+// operations (behind tcgen05.fence::before_thread_sync) for a thread of the other CTA, and no
+// memory fence.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// The same, releasing this thread's prior memory writes at cluster scope (a fence: use it off
+// the hot path, e.g. for shared-memory data that the other CTA's MMA reads).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
