@@ -21,11 +21,17 @@
 // buffers QK(j+1) never waits for the softmax to have loaded S(j); the softmax of tile j and the
 // products of neighbouring tiles overlap.
 //
-// Roles (224 threads per CTA, the same in both CTAs except that only the even CTA issues MMAs):
+// The key halves and the value halves travel in two rings of their own: a key stage is refilled
+// as soon as QK of its tile has completed, a full PV earlier than a shared stage would be, so
+// the load latency of the next key tiles stays off the critical path with three stages each.
+//
+// Roles (256 threads per CTA, the same in both CTAs except that only the even CTA issues MMAs):
 //   warps 0-3  softmax of the CTA's own 128 rows (one TMEM lane each): as in attention_sm100.cu
-//   warp 4     TMA producer of the CTA's halves; completion is counted on the even CTA's barriers
+//   warp 4     TMA producer of the query tile and key halves (then the W_UV tile); completion is
+//              counted on the even CTA's barriers
 //   warp 5     TMEM allocation (both CTAs, collectively); in the even CTA one thread issues QK
 //   warp 6     in the even CTA one thread issues PV and the W_UV epilogue
+//   warp 7     TMA producer of the value halves
 // Barriers that a thread of either CTA arrives on live in the even CTA (counts: one TMA arrival,
 // or one arrival per softmax warp of both CTAs); barriers the tensor cores signal exist in both
 // CTAs and receive the pair MMAs' commits by cluster multicast.  Every wait is bounded.
@@ -44,10 +50,11 @@ constexpr int kBN = kKeyTile;      // keys per tile (both CTAs)
 constexpr int kHalfN = kBN / 2;    // keys per CTA in the QK operand
 constexpr int kDh = 128;           // head width of the W_UV epilogue
 constexpr int kSoftmaxWarps = 4;
-constexpr int kProducerWarp = 4;
+constexpr int kProducerWarp = 4;   // query tile, key halves (and the W_UV tile)
 constexpr int kQkWarp = 5;
 constexpr int kPvWarp = 6;
-constexpr int kThreads = 224;
+constexpr int kVProducerWarp = 7;  // value halves
+constexpr int kThreads = 256;
 constexpr int kSmemMax = 227 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint16_t kBothCtas = 0x3;
@@ -67,21 +74,24 @@ struct PairShape {
   // query tile: kCBlk blocks of 128 rows x 128 B (128B swizzle), then 128 rows of DR values
   static constexpr int kQBlk = kBM * 128;
   static constexpr int kQTile = kCBlk * kQBlk + kBM * kRopeBytes;
-  // stage: the CTA's 64 keys for QK (kCBlk blocks of 64 rows x 128 B, then 64 rope rows), then
-  // the CTA's DC/2 value columns of all 128 keys (DC/64 blocks of 128 rows x 64 B, 64B swizzle)
+  // Two rings of the same depth, filled and freed independently:
+  //   key stage:   the CTA's 64 keys for QK (kCBlk blocks of 64 rows x 128 B, then 64 rope
+  //                rows); free once QK of its tile has completed
+  //   value stage: the CTA's DC/2 value columns of all 128 keys (DC/64 blocks of 128 rows x
+  //                64 B, 64B swizzle); free once PV of its tile has completed
   static constexpr int kOwnBlk = kHalfN * 128;
   static constexpr int kOwn = kCBlk * kOwnBlk + kHalfN * kRopeBytes;
   static constexpr int kVBlk = kBN * 64;
   static constexpr int kVCols = DC / 2;
   static constexpr int kVBlocks = kVCols / 32;
-  static constexpr int kStage = kOwn + kVBlocks * kVBlk;
-  static constexpr int kFit = (kSmemMax - 1024 - kQTile) / kStage;
+  static constexpr int kVStage = kVBlocks * kVBlk;
+  static constexpr int kFit = (kSmemMax - 1024 - kQTile) / (kOwn + kVStage);
   static constexpr int kStages = kFit < 4 ? kFit : 4;
   static_assert(kStages >= 2, "too few stages fit in shared memory");
-  static_assert(kOwn % 1024 == 0 && kStage % 1024 == 0, "stage regions must stay 1 KB aligned");
-  static constexpr int kSmem = kQTile + kStages * kStage + 1024;
+  static_assert(kOwn % 1024 == 0 && kVStage % 1024 == 0, "stage regions must stay 1 KB aligned");
+  static constexpr int kSmem = kQTile + kStages * (kOwn + kVStage) + 1024;
   static constexpr int kWTile = kCBlk * kQBlk;              // W_UV_h: 128 rows x DC
-  static_assert(kWTile <= kStage, "the W_UV tile goes into stage 0");
+  static_assert(kWTile <= kStages * kOwn, "the W_UV tile goes into the key ring");
   static constexpr uint32_t kColO = 256;
   static constexpr uint32_t kColP = kColO + DC;
   static_assert(kColP + kBN / 2 <= kTmemCols, "TMEM: S0, S1, O and P must fit");
@@ -146,8 +156,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   constexpr uint32_t kColO = Sh::kColO, kColP = Sh::kColP;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full;            // even CTA: both query tiles landed
-  __shared__ __align__(8) uint64_t kv_full[kStages];  // even CTA: both halves of a stage landed
-  __shared__ __align__(8) uint64_t kv_empty[kStages]; // both: PV of the stage's tile done
+  __shared__ __align__(8) uint64_t k_full[kStages];   // even CTA: both CTAs' key halves landed
+  __shared__ __align__(8) uint64_t k_empty[kStages];  // both: QK of the stage's tile done
+  __shared__ __align__(8) uint64_t v_full[kStages];   // even CTA: both CTAs' value halves landed
+  __shared__ __align__(8) uint64_t v_empty[kStages];  // both: PV of the stage's tile done
   __shared__ __align__(8) uint64_t s_full[2];         // both: S buffer written
   __shared__ __align__(8) uint64_t s_free[2];         // even CTA: 8 softmax warps loaded it
   __shared__ __align__(8) uint64_t p_full;            // even CTA: 8 softmax warps wrote P
@@ -160,7 +172,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = sbase;
-  const uint32_t sK0 = sbase + Sh::kQTile;
+  const uint32_t sK0 = sbase + Sh::kQTile;                       // key ring
+  const uint32_t sV0 = sK0 + kStages * Sh::kOwn;                  // value ring
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -172,8 +185,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     abort_sh = 0;
     mbar_init(smem_u32(&q_full), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&kv_full[s]), 1);
-      mbar_init(smem_u32(&kv_empty[s]), 1);
+      mbar_init(smem_u32(&k_full[s]), 1);
+      mbar_init(smem_u32(&k_empty[s]), 1);
+      mbar_init(smem_u32(&v_full[s]), 1);
+      mbar_init(smem_u32(&v_empty[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
@@ -197,10 +212,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = tmem_base_sh;
 
   if (warp == kProducerWarp) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer: Q, keys
     if (lane == 0) {
       tma_prefetch_desc(&tm_chunk_k);
-      tma_prefetch_desc(&tm_chunk_v);
       tma_prefetch_desc(&tm_ws);
       tma_prefetch_desc(&tm_q);
       // completions are counted on the even CTA's barriers
@@ -212,27 +226,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int j = 0; j < p.nt && ok; ++j) {
         const int s = j % kStages;
-        ok = pwait(smem_u32(&kv_empty[s]), ((j / kStages) & 1) ^ 1, abort_flag, p.dev_status);
+        ok = pwait(smem_u32(&k_empty[s]), ((j / kStages) & 1) ^ 1, abort_flag, p.dev_status);
         if (!ok) break;
-        const uint32_t own = sK0 + s * Sh::kStage;
-        const uint32_t vreg = own + Sh::kOwn;
-        const uint32_t fb = map_to_cta(smem_u32(&kv_full[s]), 0);
-        if (leader) mbar_arrive_expect_tx(smem_u32(&kv_full[s]), 2 * Sh::kStage);
+        const uint32_t own = sK0 + s * Sh::kOwn;
+        const uint32_t fb = map_to_cta(smem_u32(&k_full[s]), 0);
+        if (leader) mbar_arrive_expect_tx(smem_u32(&k_full[s]), 2 * Sh::kOwn);
         const bool ring = j < p.nt_ring;
         const int r0 = ring ? j * kBN : (j - p.nt_ring) * kBN;       // tile's first key row
         const int rk = r0 + kHalfN * static_cast<int>(rank);          // this CTA's QK keys
         const CUtensorMap* mk = ring ? &tm_cache_k : &tm_chunk_k;
-        const CUtensorMap* mv = ring ? &tm_cache_v : &tm_chunk_v;
         for (int i = 0; i < kCBlk; ++i) tma_load_3d_pair(own + i * Sh::kOwnBlk, mk, fb, 64 * i, rk, b);
         tma_load_3d_pair(own + kCBlk * Sh::kOwnBlk, &tm_ws, fb, 0, ring ? rk : p.nc_pad + rk, b);
-        for (int i = 0; i < Sh::kVBlocks; ++i)
-          tma_load_3d_pair(vreg + i * Sh::kVBlk, mv, fb, Sh::kVCols * static_cast<int>(rank) + 32 * i,
-                           r0, b);
       }
       if (ok && p.has_w_uv) {
-        // W_UV of this CTA's head into stage 0 once every stage is free
+        // W_UV of this CTA's head into the key ring once every key stage is free
         for (int jj = p.nt; jj < p.nt + kStages && ok; ++jj)
-          ok = pwait(smem_u32(&kv_empty[jj % kStages]), ((jj / kStages) & 1) ^ 1, abort_flag,
+          ok = pwait(smem_u32(&k_empty[jj % kStages]), ((jj / kStages) & 1) ^ 1, abort_flag,
                      p.dev_status);
         if (ok) {
           const uint32_t wb = map_to_cta(smem_u32(&w_full), 0);
@@ -240,6 +249,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int i = 0; i < kCBlk; ++i)
             tma_load_2d_pair(sK0 + i * Sh::kQBlk, &tm_wuv, wb, 64 * i, h * kDh);
         }
+      }
+    }
+  } else if (warp == kVProducerWarp) {
+    // ------------------------------------------------------------------ TMA producer: values
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_chunk_v);
+      bool ok = true;
+      for (int j = 0; j < p.nt && ok; ++j) {
+        const int s = j % kStages;
+        ok = pwait(smem_u32(&v_empty[s]), ((j / kStages) & 1) ^ 1, abort_flag, p.dev_status);
+        if (!ok) break;
+        const uint32_t vreg = sV0 + s * Sh::kVStage;
+        const uint32_t fb = map_to_cta(smem_u32(&v_full[s]), 0);
+        if (leader) mbar_arrive_expect_tx(smem_u32(&v_full[s]), 2 * Sh::kVStage);
+        const bool ring = j < p.nt_ring;
+        const int r0 = ring ? j * kBN : (j - p.nt_ring) * kBN;
+        const CUtensorMap* mv = ring ? &tm_cache_v : &tm_chunk_v;
+        for (int i = 0; i < Sh::kVBlocks; ++i)
+          tma_load_3d_pair(vreg + i * Sh::kVBlk, mv, fb, Sh::kVCols * static_cast<int>(rank) + 32 * i,
+                           r0, b);
       }
     }
   } else if (warp == kQkWarp || warp == kPvWarp) {
@@ -253,22 +282,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint64_t q_r = smem_desc(sQ + kCBlk * Sh::kQBlk, 16, Sh::kRopeSbo, Sh::kRopeSwz);
       const uint64_t k_c0 = smem_desc(sK0, 16, 1024, kSwizzle128B);
       const uint64_t k_r0 = smem_desc(sK0 + kCBlk * Sh::kOwnBlk, 16, Sh::kRopeSbo, Sh::kRopeSwz);
-      const uint64_t v_0 = smem_desc(sK0 + Sh::kOwn, Sh::kVBlk, 512, kSwizzle64B);
-      constexpr uint32_t kStageD = Sh::kStage >> 4;
+      const uint64_t v_0 = smem_desc(sV0, Sh::kVBlk, 512, kSwizzle64B);
+      constexpr uint32_t kOwnD = Sh::kOwn >> 4, kVStageD = Sh::kVStage >> 4;
       bool ok = true;
       if (warp == kQkWarp) {
         ok = pwait(smem_u32(&q_full), 0, abort_flag, p.dev_status);
         for (int j = 0; j < p.nt && ok; ++j) {
           const int s = j % kStages;
-          ok = pwait(smem_u32(&kv_full[s]), (j / kStages) & 1, abort_flag, p.dev_status);
+          ok = pwait(smem_u32(&k_full[s]), (j / kStages) & 1, abort_flag, p.dev_status);
           // S buffer j&1 was loaded by both CTAs' softmax warps (tile j-2)
           if (ok && j >= 2)
             ok = pwait(smem_u32(&s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.dev_status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t d = tmem + (j & 1) * kBN;
-          const uint64_t kc = k_c0 + static_cast<uint32_t>(s) * kStageD;
-          const uint64_t kr = k_r0 + static_cast<uint32_t>(s) * kStageD;
+          const uint64_t kc = k_c0 + static_cast<uint32_t>(s) * kOwnD;
+          const uint64_t kr = k_r0 + static_cast<uint32_t>(s) * kOwnD;
 #pragma unroll
           for (int blk = 0; blk < kCBlk; ++blk)
 #pragma unroll
@@ -280,20 +309,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < Sh::kRopeKSteps; ++kk)
             mma_ss_pair(d, q_r + 2 * kk, kr + 2 * kk, idesc_qk, 1u);
           mma_commit_pair(smem_u32(&s_full[j & 1]), kBothCtas);
+          mma_commit_pair(smem_u32(&k_empty[s]), kBothCtas);
         }
       } else {
         for (int j = 0; j < p.nt && ok; ++j) {
-          ok = pwait(smem_u32(&p_full), j & 1, abort_flag, p.dev_status);
+          const int s = j % kStages;
+          ok = pwait(smem_u32(&v_full[s]), (j / kStages) & 1, abort_flag, p.dev_status) &&
+               pwait(smem_u32(&p_full), j & 1, abort_flag, p.dev_status);
           if (!ok) break;
           tc_fence_after();
-          const int s = j % kStages;
-          const uint64_t vd = v_0 + static_cast<uint32_t>(s) * kStageD;
+          const uint64_t vd = v_0 + static_cast<uint32_t>(s) * kVStageD;
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
             // keys kk*16 .. +15: 16 rows of 64 B further per step (1024 B = 64 units)
             mma_ts_pair(tmem + kColO, tmem + kColP + kk * 8, vd + 64 * kk, idesc_pv,
                         (j | kk) != 0 ? 1u : 0u);
-          mma_commit_pair(smem_u32(&kv_empty[s]), kBothCtas);
+          mma_commit_pair(smem_u32(&v_empty[s]), kBothCtas);
           mma_commit_pair(smem_u32(&pv_done), kBothCtas);
         }
         if (ok && p.has_w_uv) {
@@ -302,7 +333,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (ok) {
             tc_fence_after();
             const uint64_t o_c = smem_desc(sQ, 16, 1024, kSwizzle128B);     // O_lat over Q
-            const uint64_t w_c = smem_desc(sK0, 16, 1024, kSwizzle128B);    // W_UV in stage 0
+            const uint64_t w_c = smem_desc(sK0, 16, 1024, kSwizzle128B);    // W_UV: key ring
 #pragma unroll
             for (int blk = 0; blk < kCBlk; ++blk)
 #pragma unroll
