@@ -140,6 +140,23 @@ __device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, volatile in
   return mbar_wait_or_abort(bar, parity, abort_flag, dev_status);
 }
 
+// Bounded wait until a shared counter written by another thread of the CTA reaches `target`.
+__device__ __forceinline__ bool wait_count_at_least(const int* counter, int target,
+                                                    volatile int* abort_flag, int32_t* dev_status) {
+  const volatile int* c = counter;
+  if (*c >= target) return true;
+  const long long start = clock64();
+  while (true) {
+    if (*c >= target) return true;
+    if (*abort_flag) return false;
+    if (clock64() - start > kWaitLimitCycles) {
+      *abort_flag = 1;
+      if (dev_status != nullptr) atomicExch(dev_status, static_cast<int32_t>(MLA_ERR_DEVICE_TIMEOUT));
+      return false;
+    }
+  }
+}
+
 template <int DC, int DR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attention_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -164,6 +181,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t s_free[2];         // even CTA: 8 softmax warps loaded it
   __shared__ __align__(8) uint64_t p_full;            // even CTA: 8 softmax warps wrote P
   __shared__ __align__(8) uint64_t pv_done;           // both: PV(j) done (O and P free)
+  __shared__ int pv_issued_sh;                        // even CTA: PV tiles handed to the pipe
   __shared__ __align__(8) uint64_t w_full;            // even CTA: both W_UV tiles landed
   __shared__ __align__(8) uint64_t olat_full;         // even CTA: 8 softmax warps wrote O_lat
   __shared__ __align__(8) uint64_t epi_done;          // both: epilogue product done
@@ -196,6 +214,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&p_full), 2 * kSoftmaxWarps);
     mbar_init(smem_u32(&pv_done), 1);
+    pv_issued_sh = 0;
     mbar_init(smem_u32(&w_full), 1);
     mbar_init(smem_u32(&olat_full), 2 * kSoftmaxWarps);
     mbar_init(smem_u32(&epi_done), 1);
@@ -290,9 +309,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int j = 0; j < p.nt && ok; ++j) {
           const int s = j % kStages;
           ok = pwait(smem_u32(&k_full[s]), (j / kStages) & 1, abort_flag, p.dev_status);
-          // S buffer j&1 was loaded by both CTAs' softmax warps (tile j-2)
+          // S buffer j&1 was loaded by both CTAs' softmax warps (tile j-2), and PV(j-2) is
+          // already in the pipe: the pipe runs QK(j-1), PV(j-2), QK(j), PV(j-1), ... in that
+          // order (MMAs execute in issue order; a QK issuer running further ahead would queue
+          // PV behind later QKs and hold up the softmax, which needs PV(j-1) before writing P)
           if (ok && j >= 2)
-            ok = pwait(smem_u32(&s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.dev_status);
+            ok = pwait(smem_u32(&s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.dev_status) &&
+                 wait_count_at_least(&pv_issued_sh, j - 1, abort_flag, p.dev_status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t d = tmem + (j & 1) * kBN;
@@ -326,6 +349,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         (j | kk) != 0 ? 1u : 0u);
           mma_commit_pair(smem_u32(&v_empty[s]), kBothCtas);
           mma_commit_pair(smem_u32(&pv_done), kBothCtas);
+          // a count, not a barrier phase: the QK issuer may look only after several PV tiles
+          __threadfence_block();
+          *reinterpret_cast<volatile int*>(&pv_issued_sh) = j + 1;
         }
         if (ok && p.has_w_uv) {
           ok = pwait(smem_u32(&w_full), 0, abort_flag, p.dev_status) &&
