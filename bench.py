@@ -570,7 +570,7 @@ def run_ours(args, cfg):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "mla_attention_fwd (rotated-key pre-pass + " +
-                               ("attention_pair_kernel" if args.kernel_path == "auto" and cfg.n_heads % 2 == 0
+                               ("attention_pair_kernel" if args.kernel_path == "pair" and cfg.n_heads % 2 == 0
                                 and cfg.d_c in (128, 192) else "attention_tc_kernel") + ")",
                      "peak_kind": f"{peak_kind} burst bf16",
                      "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
@@ -763,7 +763,7 @@ def run_backward(args, cfg):
 
 def kernel_path(args) -> int:
     from mla_latent_kv_attn_b200 import api
-    return {"auto": api.MLA_PATH_AUTO, "single": api.MLA_PATH_TC_SINGLE}[args.kernel_path]
+    return {"auto": api.MLA_PATH_AUTO, "pair": api.MLA_PATH_TC_PAIR}[args.kernel_path]
 
 
 def run_bandwidth_only(args, cfg):
@@ -801,9 +801,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bandwidth", action="store_true",
                     help="skip the stand-alone timing of the memory-bound calls")
-    ap.add_argument("--kernel-path", choices=("auto", "single"), default="auto",
-                    help="attention kernel: auto (CTA pairs where the shape allows) or single "
-                         "(one CTA per head and query tile)")
+    ap.add_argument("--kernel-path", choices=("auto", "pair"), default="auto",
+                    help="attention kernel: auto (one CTA per head and query tile) or pair (the "
+                         "CTA-pair kernel, for comparison)")
     ap.add_argument("--bandwidth-only", action="store_true",
                     help="only time the memory-bound calls (append, RoPE, KV down-projection)")
     ap.add_argument("--backward", action="store_true",

@@ -66,15 +66,18 @@ typedef enum mla_dtype { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype;
 
 /* Which kernels serve a call.  MLA_PATH_AUTO picks the tensor-core (tcgen05/TMA) kernels when
  * the shape allows (bf16; for attention d_c in {128, 192, 256}, d_rope in {16, 32, 64} and,
- * with the W_UV epilogue, d_head = 128) and the CUDA-core kernels otherwise; for attention with
- * an even head count and d_c in {128, 192} it runs the CTA-pair kernel, in which two CTAs
- * (two heads of one query tile) share every key tile.  MLA_PATH_TC_SINGLE is AUTO without the
- * CTA-pair kernel (one CTA per head and query tile; for cross-checks).  MLA_PATH_SIMT forces the
- * CUDA-core kernels (every dtype and shape; slow but simple, used as a cross-check). */
+ * with the W_UV epilogue, d_head = 128) and the CUDA-core kernels otherwise; attention runs one
+ * CTA per head and query tile.  MLA_PATH_TC_SINGLE is the same choice (kept for callers that
+ * name it).  MLA_PATH_TC_PAIR runs attention, for an even head count and d_c in {128, 192}, on
+ * the CTA-pair kernel instead, in which two CTAs (two heads of one query tile) execute every MMA
+ * together and share each key tile (correct, but slower than the one-CTA kernel on this part;
+ * for measurements); other calls as AUTO.  MLA_PATH_SIMT forces the CUDA-core kernels (every
+ * dtype and shape; slow but simple, used as a cross-check). */
 typedef enum mla_kernel_path {
   MLA_PATH_AUTO = 0,
   MLA_PATH_SIMT = 1,
-  MLA_PATH_TC_SINGLE = 2
+  MLA_PATH_TC_SINGLE = 2,
+  MLA_PATH_TC_PAIR = 3
 } mla_kernel_path;
 
 /* Layer shape, frame geometry and rollout geometry ([M], [F1]).

@@ -26,6 +26,7 @@ MLA_FP32 = 1
 MLA_PATH_AUTO = 0
 MLA_PATH_SIMT = 1
 MLA_PATH_TC_SINGLE = 2
+MLA_PATH_TC_PAIR = 3
 
 MLA_PROJECT = 1
 MLA_APPEND = 2

@@ -13,7 +13,7 @@ import torch
 
 from . import _lib
 from ._lib import (MLA_APPEND, MLA_BF16, MLA_FP32, MLA_PATH_AUTO, MLA_PATH_SIMT,
-                   MLA_PATH_TC_SINGLE, MLA_PROJECT, MLA_PROJECT_AND_APPEND, MLAConfigC, MLAError)
+                   MLA_PATH_TC_PAIR, MLA_PATH_TC_SINGLE, MLA_PROJECT, MLA_PROJECT_AND_APPEND, MLAConfigC, MLAError)
 
 __all__ = [
     "make_config", "torch_dtype", "mla_config_check", "mla_cache_append", "mla_rope3d",
@@ -23,7 +23,7 @@ __all__ = [
     "mla_attention_bwd_workspace_bytes", "mla_attention_bwd",
     "mla_out_proj", "MLAError",
     "MLA_PROJECT", "MLA_APPEND", "MLA_PROJECT_AND_APPEND", "MLA_PATH_AUTO", "MLA_PATH_SIMT",
-    "MLA_PATH_TC_SINGLE",
+    "MLA_PATH_TC_SINGLE", "MLA_PATH_TC_PAIR",
 ]
 
 

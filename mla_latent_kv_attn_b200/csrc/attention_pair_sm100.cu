@@ -17,10 +17,9 @@
 //
 // Per CTA and key tile that is 28 KB of keys and 24 KB of values (52 KB) instead of one 56 KB
 // tile read twice by the tensor core, so the query tile stays in shared memory and TMEM has
-// room for two S buffers: S0 [0,128), S1 [128,256), O [256,256+DC).  P(j) (bf16 pairs) goes into
-// the first 64 columns of the S buffer it came from, so the softmax writes P(j) without waiting
-// for PV(j-1) (only a rescale of O waits for it), and QK(j+2) reuses the buffer once PV(j) has
-// read P(j).
+// room for two S buffers: S0 [0,128), S1 [128,256), O [256,256+DC), P [256+DC, +64).  With two S
+// buffers QK(j+1) never waits for the softmax to have loaded S(j); the softmax of tile j and the
+// products of neighbouring tiles overlap.
 //
 // The key halves and the value halves travel in two rings of their own: a key stage is refilled
 // as soon as QK of its tile has completed, a full PV earlier than a shared stage would be, so
@@ -94,7 +93,8 @@ struct PairShape {
   static constexpr int kWTile = kCBlk * kQBlk;              // W_UV_h: 128 rows x DC
   static_assert(kWTile <= kStages * kOwn, "the W_UV tile goes into the key ring");
   static constexpr uint32_t kColO = 256;
-  static_assert(kColO + DC <= kTmemCols, "TMEM: S0, S1 and O must fit");
+  static constexpr uint32_t kColP = kColO + DC;
+  static_assert(kColP + kBN / 2 <= kTmemCols, "TMEM: S0, S1, O and P must fit");
 };
 
 struct PairParams {
@@ -153,7 +153,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   using Sh = PairShape<DC, DR>;
   constexpr int kCBlk = Sh::kCBlk;
   constexpr int kStages = Sh::kStages;
-  constexpr uint32_t kColO = Sh::kColO;
+  constexpr uint32_t kColO = Sh::kColO, kColP = Sh::kColP;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full;            // even CTA: both query tiles landed
   __shared__ __align__(8) uint64_t k_full[kStages];   // even CTA: both CTAs' key halves landed
@@ -161,9 +161,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t v_full[kStages];   // even CTA: both CTAs' value halves landed
   __shared__ __align__(8) uint64_t v_empty[kStages];  // both: PV of the stage's tile done
   __shared__ __align__(8) uint64_t s_full[2];         // both: S buffer written
+  __shared__ __align__(8) uint64_t s_free[2];         // even CTA: 8 softmax warps loaded it
   __shared__ __align__(8) uint64_t p_full;            // even CTA: 8 softmax warps wrote P
-  __shared__ __align__(8) uint64_t pv_buf_done[2];    // even CTA: PV read P out of S buffer b
-  __shared__ __align__(8) uint64_t pv_done;           // both: PV(j) done (O may be rescaled)
+  __shared__ __align__(8) uint64_t pv_done;           // both: PV(j) done (O and P free)
   __shared__ __align__(8) uint64_t w_full;            // even CTA: both W_UV tiles landed
   __shared__ __align__(8) uint64_t olat_full;         // even CTA: 8 softmax warps wrote O_lat
   __shared__ __align__(8) uint64_t epi_done;          // both: epilogue product done
@@ -192,7 +192,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&pv_buf_done[i]), 1);
+      mbar_init(smem_u32(&s_free[i]), 2 * kSoftmaxWarps);
     }
     mbar_init(smem_u32(&p_full), 2 * kSoftmaxWarps);
     mbar_init(smem_u32(&pv_done), 1);
@@ -290,9 +290,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int j = 0; j < p.nt && ok; ++j) {
           const int s = j % kStages;
           ok = pwait(smem_u32(&k_full[s]), (j / kStages) & 1, abort_flag, p.dev_status);
-          // S buffer j&1 held P(j-2): PV(j-2) has read it (and so the softmax had loaded S(j-2))
+          // S buffer j&1 was loaded by both CTAs' softmax warps (tile j-2)
           if (ok && j >= 2)
-            ok = pwait(smem_u32(&pv_buf_done[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.dev_status);
+            ok = pwait(smem_u32(&s_free[j & 1]), ((j - 2) >> 1) & 1, abort_flag, p.dev_status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t d = tmem + (j & 1) * kBN;
@@ -321,12 +321,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint64_t vd = v_0 + static_cast<uint32_t>(s) * kVStageD;
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            // P(j) is bf16 pairs in S buffer j&1; keys kk*16 .. +15: 16 rows of 64 B further
-            // per step (1024 B = 64 units)
-            mma_ts_pair(tmem + kColO, tmem + (j & 1) * kBN + kk * 8, vd + 64 * kk, idesc_pv,
+            // keys kk*16 .. +15: 16 rows of 64 B further per step (1024 B = 64 units)
+            mma_ts_pair(tmem + kColO, tmem + kColP + kk * 8, vd + 64 * kk, idesc_pv,
                         (j | kk) != 0 ? 1u : 0u);
           mma_commit_pair(smem_u32(&v_empty[s]), kBothCtas);
-          mma_commit_pair(smem_u32(&pv_buf_done[j & 1]), 0x1);
           mma_commit_pair(smem_u32(&pv_done), kBothCtas);
         }
         if (ok && p.has_w_uv) {
@@ -353,6 +351,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int row = warp * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int n = q0 + row;
+    const uint32_t s_free_l0 = map_to_cta(smem_u32(&s_free[0]), 0);
+    const uint32_t s_free_l1 = map_to_cta(smem_u32(&s_free[1]), 0);
     const uint32_t p_full_l = map_to_cta(smem_u32(&p_full), 0);
     const uint32_t olat_full_l = map_to_cta(smem_u32(&olat_full), 0);
     float m_run = -INFINITY, l_run = 0.f;
@@ -370,6 +370,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
       }
+      // S(j) is in registers: one arrival per warp frees its buffer for QK(j+2)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(sb ? s_free_l1 : s_free_l0);
       const int valid = j < p.nt_ring ? min(kBN, p.nc - j * kBN)
                                       : min(kBN, p.n_q - (j - p.nt_ring) * kBN);
       if (valid < kBN) {
@@ -404,9 +408,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t w[kBN / 2];
       if (valid == kBN) l_run += pair_exp_row<true>(s, p.scale_log2, m_run, w);
       else l_run += pair_exp_row<false>(s, p.scale_log2, m_run, w);
-      // O may be rescaled only once PV(j-1) has completed; P(j) goes into the S buffer it
-      // came from, which nothing else reads or writes until PV(j) has read it
-      if (j > 0 && rescale) {
+      // P and O are free once PV(j-1) has completed
+      if (j > 0) {
         ok = __all_sync(0xffffffffu, pwait(smem_u32(&pv_done), (j - 1) & 1, abort_flag, p.dev_status));
         if (!ok) break;
         tc_fence_after();
@@ -426,7 +429,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t w16[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) w16[i] = w[c + i];
-        tmem_st16(tmem + lane_off + sb * kBN + c, w16);
+        tmem_st16(tmem + lane_off + kColP + c, w16);
       }
       tmem_wait_st();
       tc_fence_before();

@@ -40,7 +40,7 @@ mla_status check_cfg(const mla_config* cfg) {
                 c.window_frames);
   MLA_CHECK_ARG(c.dtype == MLA_BF16 || c.dtype == MLA_FP32, "unknown dtype %d", c.dtype);
   MLA_CHECK_ARG(c.kernel_path == MLA_PATH_AUTO || c.kernel_path == MLA_PATH_SIMT ||
-                    c.kernel_path == MLA_PATH_TC_SINGLE,
+                    c.kernel_path == MLA_PATH_TC_SINGLE || c.kernel_path == MLA_PATH_TC_PAIR,
                 "unknown kernel_path %d", c.kernel_path);
   const int64_t tpf = int64_t{c.frame_h} * c.frame_w;
   const int64_t D = int64_t{c.d_c} + c.d_rope;
@@ -194,7 +194,7 @@ mla_status attention_entry(const mla_config* cfg, const void* q, const void* chu
 mla_status attention_dispatch(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
   const bool has_w_uv = a.w_uv != nullptr;
   if (use_tc(d) && tc_attention_supported(d, has_w_uv)) {
-    if (d.path == MLA_PATH_AUTO && tc_attention_pair_supported(d, has_w_uv))
+    if (d.path == MLA_PATH_TC_PAIR && tc_attention_pair_supported(d, has_w_uv))
       return attention_tc_pair(d, a, n_valid, s);
     return attention_tc(d, a, n_valid, s);
   }

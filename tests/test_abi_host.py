@@ -54,7 +54,7 @@ def test_presets_are_valid_configs(i):
 
 @pytest.mark.parametrize("field,value", [
     ("d_rope", 30), ("chunk_frames", 7), ("dtype", 5), ("batch", 0), ("rope_base", 1.0),
-    ("softmax_scale", -1.0), ("kernel_path", 3), ("frame_w", 0),
+    ("softmax_scale", -1.0), ("kernel_path", 4), ("frame_w", 0),
 ])
 def test_bad_configs_are_rejected(field, value):
     c = api.make_config(inputs.CONFIGS[1])

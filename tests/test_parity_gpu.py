@@ -16,9 +16,9 @@ from parity_util import (GpuRun, OracleRun, check_chunk, check_ring, compare,
 
 pytestmark = pytest.mark.gpu
 
-# "tc": the default path (CTA-pair attention where the shape allows); "tc1": tensor cores with
-# one CTA per head and query tile; "simt": CUDA cores
-PATHS = {"tc": api.MLA_PATH_AUTO, "tc1": api.MLA_PATH_TC_SINGLE, "simt": api.MLA_PATH_SIMT}
+# "tc": the default path (tensor cores, one CTA per head and query tile); "pair": the CTA-pair
+# attention kernel; "simt": CUDA cores
+PATHS = {"tc": api.MLA_PATH_AUTO, "pair": api.MLA_PATH_TC_PAIR, "simt": api.MLA_PATH_SIMT}
 
 
 def full_rollout(cfg, path, rows=None, check_positions=True):
@@ -55,14 +55,14 @@ def test_small_frames_bf16_rollout(path):
 LATENT_SHAPES = [(dc, dr) for dc in (128, 192, 256) for dr in (16, 32, 64)]
 
 
-@pytest.mark.parametrize("path", ["tc", "tc1"])
+@pytest.mark.parametrize("path", ["tc", "pair"])
 @pytest.mark.parametrize("d_c,d_rope", LATENT_SHAPES)
 def test_latent_shape_sweep_tensor_cores_match_oracle(d_c, d_rope, path):
     """The latent-size ablation shapes (d_c in {128, 192, 256} x d_rope in {16, 32, 64}) run on
-    the tensor-core kernels (the CTA-pair kernel for d_c 128 and 192 on the default path, and
-    the one-CTA kernel) and match the oracle over a 4-chunk rollout whose ring wraps."""
-    if path == "tc1" and d_c == 256:
-        pytest.skip("d_c 256 always runs the one-CTA kernel (covered by the default path)")
+    the tensor-core kernels (the one-CTA kernel on the default path, and the CTA-pair kernel for
+    d_c 128 and 192) and match the oracle over a 4-chunk rollout whose ring wraps."""
+    if path == "pair" and d_c == 256:
+        pytest.skip("d_c 256 has no CTA-pair kernel (no TMEM room for two S buffers)")
     cfg = inputs.with_latent_shape(inputs.small_bf16_config(), d_c, d_rope)
     c = api.make_config(cfg, kernel_path=PATHS[path])
     assert api.mla_attention_uses_tensor_cores(c, True)
@@ -149,7 +149,7 @@ def test_pair_and_single_cta_attention_agree_on_config1():
     order of the MMA pipeline's additions may differ, so a last-place bf16 difference at most)."""
     cfg = inputs.CONFIGS[1]
     outs = []
-    for path in (api.MLA_PATH_AUTO, api.MLA_PATH_TC_SINGLE):
+    for path in (api.MLA_PATH_TC_PAIR, api.MLA_PATH_AUTO):
         g, _ = prefilled(cfg, path, cfg.measured_chunk)
         outs.append(g.attend(cfg.measured_chunk, inputs.chunk_x(cfg, cfg.measured_chunk)))
     for k in ("o", "o_lat", "lse"):
