@@ -59,7 +59,11 @@ typedef enum mla_status {
   MLA_ERR_ALIGNMENT = 3,      /* a pointer that is not 16-byte aligned */
   MLA_ERR_CUDA = 4,           /* a CUDA runtime or driver call failed */
   MLA_ERR_DEVICE_TIMEOUT = 5, /* value a kernel writes to dev_status when a bounded wait ran out */
-  MLA_ERR_WORKSPACE = 6       /* workspace missing or smaller than required */
+  MLA_ERR_WORKSPACE = 6,      /* workspace missing or smaller than required */
+  MLA_ERR_DEVICE_CHECK = 7    /* value a kernel of the MLA_DEBUG build writes to dev_status when
+                                 an input's contents break the call's contract (a ring slot whose
+                                 frame is empty or outside the chunk's window); the release build
+                                 does not make these checks */
 } mla_status;
 
 typedef enum mla_dtype { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype;

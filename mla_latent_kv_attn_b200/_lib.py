@@ -11,6 +11,8 @@ import threading
 from ctypes import c_float, c_int32, c_size_t, c_void_p, POINTER
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_b200.so")
+# the same library built with MLA_DEBUG (device-side contract checks; see include/mla.h)
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_b200_debug.so")
 
 # mla_status codes (include/mla.h)
 MLA_OK = 0
@@ -20,6 +22,7 @@ MLA_ERR_ALIGNMENT = 3
 MLA_ERR_CUDA = 4
 MLA_ERR_DEVICE_TIMEOUT = 5
 MLA_ERR_WORKSPACE = 6
+MLA_ERR_DEVICE_CHECK = 7
 
 MLA_BF16 = 0
 MLA_FP32 = 1

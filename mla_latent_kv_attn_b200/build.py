@@ -22,6 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmla_b200.so")
+DEBUG_LIB = os.path.join(PKG, "libmla_b200_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
@@ -44,14 +45,15 @@ def headers():
     return hs + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 
 
-def extra_flags():
+def extra_flags(debug: bool = False):
     """MLA_NVTX=1 in the environment builds NVTX ranges around every C-ABI call (for profilers;
-    off by default)."""
-    return ["-DMLA_NVTX"] if os.environ.get("MLA_NVTX") == "1" else []
+    off by default); debug builds add the device-side contract checks (MLA_DEBUG)."""
+    f = ["-DMLA_NVTX"] if os.environ.get("MLA_NVTX") == "1" else []
+    return f + (["-DMLA_DEBUG"] if debug else [])
 
 
-def _compile(src: str, obj: str, ptxas_verbose: bool) -> str:
-    cmd = [nvcc(), *ARCH, *FLAGS, *extra_flags(), "-c", src, "-o", obj]
+def _compile(src: str, obj: str, ptxas_verbose: bool, debug: bool = False) -> str:
+    cmd = [nvcc(), *ARCH, *FLAGS, *extra_flags(debug), "-c", src, "-o", obj]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -60,11 +62,15 @@ def _compile(src: str, obj: str, ptxas_verbose: bool) -> str:
     return r.stdout + r.stderr
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True,
+          debug: bool = False) -> str:
+    """Builds libmla_b200.so (or, with debug, libmla_b200_debug.so from objects of its own)."""
+    build_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib_path = DEBUG_LIB if debug else LIB
+    os.makedirs(build_dir, exist_ok=True)
     # objects built with other flags (e.g. NVTX on/off) are rebuilt
-    stamp = os.path.join(BUILD, "flags.txt")
-    flags = " ".join(ARCH + FLAGS + extra_flags())
+    stamp = os.path.join(build_dir, "flags.txt")
+    flags = " ".join(ARCH + FLAGS + extra_flags(debug))
     if not os.path.exists(stamp) or open(stamp).read() != flags:
         force = True
         with open(stamp, "w") as f:
@@ -73,7 +79,7 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
     jobs = []
     objs = []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         stale = (force or ptxas_verbose or not os.path.exists(obj)
                  or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr_time))
@@ -82,12 +88,12 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
     logs = []
     if jobs:
         with cf.ThreadPoolExecutor(max_workers=min(8, len(jobs))) as ex:
-            futs = [ex.submit(_compile, s, o, ptxas_verbose) for s, o in jobs]
+            futs = [ex.submit(_compile, s, o, ptxas_verbose, debug) for s, o in jobs]
             for f in futs:
                 logs.append(f.result())
-    if jobs or force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(
+    if jobs or force or not os.path.exists(lib_path) or os.path.getmtime(lib_path) < max(
             os.path.getmtime(o) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", LIB, *objs, "-cudart",
+        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", lib_path, *objs, "-cudart",
                "static", "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map")]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -95,16 +101,20 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
     log = "".join(logs)
     if not quiet and log:
         print(log)
-    return LIB
+    return lib_path
 
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--debug", action="store_true",
+                    help="also build libmla_b200_debug.so (device-side contract checks)")
     a = ap.parse_args(argv)
     path = build(force=a.force, ptxas_verbose=a.verbose_ptxas, quiet=False)
     print(path)
+    if a.debug:
+        print(build(force=a.force, ptxas_verbose=a.verbose_ptxas, quiet=False, debug=True))
     return 0
 
 

@@ -248,7 +248,7 @@ mla_status attention_bwd(const Dims& d, const BwdArgs& a, int n_valid, int first
   float* delta = static_cast<float*>(workspace);
   void* ws_rope = static_cast<char*>(workspace) + w.delta_bytes;
   const mla_status st = build_rope_keys(d, a.cache, a.chunk_lat, a.slot_frame, n_valid,
-                                       first_frame, ws_rope, s);
+                                       first_frame, ws_rope, s, kRopeKeysAll, dev_status, 1);
   if (st != MLA_OK) return st;
   BwdParams p;
   p.q = a.q; p.chunk_lat = a.chunk_lat; p.cache = a.cache; p.slot_frame = a.slot_frame;

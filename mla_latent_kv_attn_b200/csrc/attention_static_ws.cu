@@ -118,7 +118,8 @@ mla_status attention_fwd_static_scratch(const Dims& d, const AttnArgs& args,
   if (st != MLA_OK) return st;
   // Every row of the scratch that the attention kernels read is rewritten here (padding rows
   // with zeros), so what an earlier call left behind never matters.
-  st = build_rope_keys(d, args.cache, args.chunk_lat, slot_frame, n_valid, first_frame, ws, s);
+  st = build_rope_keys(d, args.cache, args.chunk_lat, slot_frame, n_valid, first_frame, ws, s,
+                       kRopeKeysAll, args.dev_status, 1);
   if (st != MLA_OK) return st;
   AttnArgs a = args;
   a.ws = ws;

@@ -171,6 +171,18 @@ __device__ __forceinline__ void key_position(const int32_t* slot_frame, int b, i
   w = i % frame_w;
 }
 
+// Device-side contract checks of the MLA_DEBUG build: a failed check writes
+// MLA_ERR_DEVICE_CHECK to the caller's status word (if given) and the kernel carries on; nothing
+// traps.  In the release build the check compiles to nothing.
+__device__ __forceinline__ void debug_check(bool ok, int32_t* dev_status) {
+#ifdef MLA_DEBUG
+  if (!ok && dev_status != nullptr) atomicExch(dev_status, static_cast<int32_t>(MLA_ERR_DEVICE_CHECK));
+#else
+  (void)ok;
+  (void)dev_status;
+#endif
+}
+
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int round_up(int a, int b) { return ceil_div(a, b) * b; }
 

@@ -95,9 +95,13 @@ mla_status key_positions(const Dims& d, const int32_t* slot_frame, int n_valid, 
 // Which rows of the rotated-key workspace build_rope_keys writes: all, the ring part (rows
 // [0, nc_pad)) or the chunk part (rows [nc_pad, rows)).
 enum RopeKeysPart : int { kRopeKeysAll = 0, kRopeKeysRing = 1, kRopeKeysChunk = 2 };
+// dev_status (optional): with MLA_DEBUG builds the kernel checks that every attended ring slot
+// holds a frame (t >= 0) and, with check_window, one of the chunk's window
+// (first_frame - W <= t < first_frame), writing MLA_ERR_DEVICE_CHECK there otherwise.
 mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_lat,
                            const int32_t* slot_frame, int n_valid, int first_frame, void* ws,
-                           cudaStream_t s, int part = kRopeKeysAll);
+                           cudaStream_t s, int part = kRopeKeysAll, int32_t* dev_status = nullptr,
+                           int check_window = 0);
 mla_status attention_simt(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
 mla_status copy_rows(int dtype, const void* src, int64_t src_stride, void* dst,
                      int64_t dst_stride, int rows, int cols, int64_t src_batch,

@@ -182,7 +182,7 @@ mla_status attention_entry(const mla_config* cfg, const void* q, const void* chu
   MLA_TRY(check_workspace(d, n_valid_frames, workspace, workspace_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   MLA_TRY(build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid_frames, first_frame, workspace, s,
-                          rope_part));
+                          rope_part, dev_status, 1));
   AttnArgs a{};
   a.q = q; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = workspace; a.w_uv = w_uv;
   a.out = out; a.lse = lse; a.dev_status = dev_status;
@@ -216,6 +216,7 @@ const char* mla_status_string(int32_t status) {
     case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
     case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
     case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK";
     default: return "MLA_ERR_UNKNOWN";
   }
 }

@@ -317,7 +317,8 @@ __global__ void rope_keys_kernel(const T* __restrict__ cache, const T* __restric
                                  const int32_t* __restrict__ slot_frame, T* __restrict__ ws,
                                  int B, int W, int D, int d_c, int n_pairs, int n_q, int nc,
                                  int nc_pad, int rows_ws, int row_begin, int row_end,
-                                 int first_frame, RopeGeom g) {
+                                 int first_frame, RopeGeom g, int32_t* dev_status,
+                                 int check_window) {
   // rows [row_begin, row_end) of every sample's rows_ws workspace rows, one thread per pair
   // (32-bit index arithmetic: B * span * n_pairs stays far below 2^31)
   const int span = row_end - row_begin;
@@ -345,6 +346,8 @@ __global__ void rope_keys_kernel(const T* __restrict__ cache, const T* __restric
     }
     int t, h, w;
     key_position(slot_frame, b, W, g.tpf, g.frame_w, nc, first_frame, m, t, h, w);
+    if (m < nc)
+      debug_check(t >= 0 && (!check_window || (t < first_frame && t >= first_frame - W)), dev_status);
     float x0 = Elem<T>::to_f(src[0]), x1 = Elem<T>::to_f(src[1]);
     rope_rotate(x0, x1, rope_angle(g, pair, t, h, w));
     dst[0] = Elem<T>::from_f(x0);
@@ -360,7 +363,8 @@ __global__ void __launch_bounds__(256)
     rope_keys_vec_kernel(const T* __restrict__ cache, const T* __restrict__ chunk_lat,
                          const int32_t* __restrict__ slot_frame, T* __restrict__ ws, int B, int W,
                          int D, int d_c, int n_q, int nc, int nc_pad, int rows_ws, int row_begin,
-                         int row_end, int first_frame, RopeGeom g) {
+                         int row_end, int first_frame, RopeGeom g, int32_t* dev_status,
+                         int check_window) {
   constexpr int kPer = 16 / sizeof(T);          // elements per piece
   constexpr int kDr = kPieces * kPer;
   const int span = row_end - row_begin;
@@ -389,6 +393,8 @@ __global__ void __launch_bounds__(256)
     for (int k = 0; k < kPieces; ++k) raw[k] = s4[k];
     int t, h, w;
     key_position(slot_frame, b, W, g.tpf, g.frame_w, nc, first_frame, m, t, h, w);
+    if (m < nc)
+      debug_check(t >= 0 && (!check_window || (t < first_frame && t >= first_frame - W)), dev_status);
 #pragma unroll
     for (int k = 0; k < kPieces; ++k) {
       T* x = reinterpret_cast<T*>(&raw[k]);
@@ -417,7 +423,7 @@ KeyWorkspace key_workspace_layout(const Dims& d, int n_valid) {
 
 mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_lat,
                            const int32_t* slot_frame, int n_valid, int first_frame, void* ws,
-                           cudaStream_t s, int part) {
+                           cudaStream_t s, int part, int32_t* dev_status, int check_window) {
   const KeyWorkspace k = key_workspace_layout(d, n_valid);
   const int n_pairs = d.d_rope / 2;
   // the ring part is rows [0, nc_pad) (its padding rows included), the chunk part the rest
@@ -440,7 +446,7 @@ mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_l
   rope_keys_vec_kernel<T, P><<<vblocks, 256, 0, s>>>(                                          \
       static_cast<const T*>(cache), static_cast<const T*>(chunk_lat), slot_frame,               \
       static_cast<T*>(ws), d.B, d.W, d.D, d.d_c, d.n_q, k.nc, k.nc_pad, k.rows, row_begin,      \
-      row_end, first_frame, g)
+      row_end, first_frame, g, dev_status, check_window)
     if (d.dtype == MLA_FP32) {
       if (pieces == 2) MLA_KEYS_VEC(float, 2);
       else if (pieces == 4) MLA_KEYS_VEC(float, 4);
@@ -458,12 +464,12 @@ mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_l
     rope_keys_kernel<float><<<blocks, 256, 0, s>>>(
         static_cast<const float*>(cache), static_cast<const float*>(chunk_lat), slot_frame,
         static_cast<float*>(ws), d.B, d.W, d.D, d.d_c, n_pairs, d.n_q, k.nc, k.nc_pad, k.rows,
-        row_begin, row_end, first_frame, g);
+        row_begin, row_end, first_frame, g, dev_status, check_window);
   else
     rope_keys_kernel<bf16><<<blocks, 256, 0, s>>>(
         static_cast<const bf16*>(cache), static_cast<const bf16*>(chunk_lat), slot_frame,
         static_cast<bf16*>(ws), d.B, d.W, d.D, d.d_c, n_pairs, d.n_q, k.nc, k.nc_pad, k.rows,
-        row_begin, row_end, first_frame, g);
+        row_begin, row_end, first_frame, g, dev_status, check_window);
   MLA_LAUNCH_CHECK("rope_keys");
   return MLA_OK;
 }
