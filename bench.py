@@ -673,10 +673,14 @@ def run_stack(args, cfg):
         "query_tokens_per_s": world * cfg.batch * cfg.n_q * cfg.n_chunks * cfg.n_steps *
                               cfg.n_layers * steps / (total_ms * 1e-3),
         "pct_of_bf16_peak": 100.0 * value / peaks["bf16_tflops"],
-        "roofline": {"bound": "tensor", "achieved": value, "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": value / peaks["bf16_tflops"], "traffic": None,
+        # a rollout is seconds of back-to-back tensor work under the 1 kW cap: the sustained
+        # figure is its peak (the burst one is reported beside it)
+        "roofline": {"bound": "tensor", "achieved": value,
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": value / peaks["bf16_tflops_sustained"], "traffic": None,
                      "kernel": "whole rollout (attention flops / all kernels' time)",
-                     "peak_kind": f"{peak_kind} burst bf16"},
+                     "peak_kind": f"{peak_kind} sustained bf16",
+                     "frac_of_burst": value / peaks["bf16_tflops"]},
         "e2e": None,
         # per call: x-projection GEMM, Q' GEMM, chunk-key rotation, attention; per chunk and
         # layer: the ring-key rotation (chunks with a non-empty window) and the append
