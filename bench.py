@@ -652,6 +652,7 @@ def run_stack(args, cfg):
             for g in graphs:
                 g.replay()
             ev[i][1].record(stream)
+        clock_after = probe_sm_clock(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -686,7 +687,7 @@ def run_stack(args, cfg):
         # layer: the ring-key rotation (chunks with a non-empty window) and the append
         "gpu_launches": steps * (calls * 4 + cfg.n_layers * (
             cfg.n_chunks + sum(1 for ch in range(cfg.n_chunks) if cfg.valid_frames(ch) > 0))),
-        "clocks": clk.summary(),
+        "clocks": dict(clk.summary(), sm_mhz_device=clock_after()),
     }
     if rank == 0:
         print(json.dumps(result), flush=True)
@@ -742,6 +743,7 @@ def run_backward(args, cfg):
             ev[i][0].record()
             call()
             ev[i][1].record()
+        clock_after = probe_sm_clock(torch.cuda.current_stream())
         torch.cuda.synchronize()
     ms = sum(a.elapsed_time(b) for a, b in ev) / steps
     per = 2.0 * (3 * cfg.d_latent + 2 * cfg.d_c)
@@ -761,7 +763,8 @@ def run_backward(args, cfg):
                      "unit": "TFLOP/s", "frac": value / peaks["bf16_tflops"], "traffic": None,
                      "kernel": "mla_attention_bwd (" + ("tensor-core" if api.mla_attention_uses_tensor_cores(c, False) and cfg.d_c == 192 and cfg.d_rope == 32 and cfg.n_q % 4 == 0 else "CUDA-core") + " kernels)",
                      "peak_kind": f"{peak_kind} burst bf16"},
-        "e2e": None, "gpu_launches": 5 * steps, "clocks": clk.summary()}), flush=True)
+        "e2e": None, "gpu_launches": 5 * steps,
+        "clocks": dict(clk.summary(), sm_mhz_device=clock_after())}), flush=True)
     return 0
 
 
