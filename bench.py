@@ -407,8 +407,11 @@ def run_ours(args, cfg):
         rollout.prefill_chunk(c, w, ring, buf, ch)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 5   # x GEMM (c_Q || chunk latents), Q' GEMM+RoPE, rope-key pre-pass,
-                            # attention (+W_UV), ring append
+    # the query heads formed inside the attention kernel where the shape allows
+    fused_q = rollout.fused_query_supported(c) and not args.unfused_query
+    # x GEMM (c_Q || chunk latents), [Q' GEMM + RoPE,] rope-key pre-pass, attention (+W_UV),
+    # ring append
+    launches_per_step = 4 if fused_q else 5
 
     first_chunk = cfg.measured_chunk
     flops_step = cfg.attention_flops(first_chunk)   # same for every later chunk (window full)
@@ -417,11 +420,19 @@ def run_ours(args, cfg):
         ch = first_chunk + i
         x = pool[i % n_pool] if x is None else x
         first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, ch)
-        api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
+        if fused_q:
+            api.mla_project_latents(c, x, w.w_x, buf.c_q, buf.chunk_lat)
+        else:
+            api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
         if ev is not None:
             ev[0].record(stream)
-        api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid,
-                              first, w.w_uv, buf.o, buf.lse, buf.workspace, buf.dev_status)
+        if fused_q:
+            api.mla_attention_fwd_from_cq(c, buf.c_q, w.w_qcat, buf.chunk_lat, ring.cache,
+                                          ring.slot_frame, n_valid, first, w.w_uv, buf.o, buf.lse,
+                                          buf.workspace, buf.dev_status)
+        else:
+            api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid,
+                                  first, w.w_uv, buf.o, buf.lse, buf.workspace, buf.dev_status)
         if ev is not None:
             ev[1].record(stream)
         api.mla_cache_append(c, None, None, buf.chunk_lat, ring.cache, ring.slot_frame, first,
@@ -430,7 +441,8 @@ def run_ours(args, cfg):
     # Each step is one CUDA graph (rollout.ChunkGraph): the chunk's five kernels replay back to
     # back without per-launch host overhead.  Graphs are captured before the timed region (host
     # set-up, like encoding a plan); capturing launches nothing.
-    graphs = [rollout.ChunkGraph(c, w, ring, buf, first_chunk + i, x=pool[i % n_pool], events=True)
+    graphs = [rollout.ChunkGraph(c, w, ring, buf, first_chunk + i, x=pool[i % n_pool], events=True,
+                                 fused_q=fused_q)
               for i in range(args.warmup + args.steps)]
     # warm-up
     for i in range(args.warmup):
@@ -486,7 +498,7 @@ def run_ours(args, cfg):
     streamer = rollout.HostStreamer(c, w, ring, device=dev, compute_stream=stream)
     for i in range(args.warmup):          # warm the streamer's own buffers and streams
         flush.zero_()
-        streamer.submit(first_chunk + base + i, x_host[i % n_pool], o_host[i % 2])
+        streamer.submit(first_chunk + base + i, x_host[i % n_pool], o_host[i % 2], fused_q=fused_q)
     streamer.finish()
     torch.cuda.synchronize()
     base += args.warmup
@@ -498,7 +510,8 @@ def run_ours(args, cfg):
     streamer.begin(e2e_a)
     for i in range(args.steps):
         flush.zero_()
-        streamer.submit(first_chunk + base + i, x_host[(base + i) % n_pool], o_host[i % 2])
+        streamer.submit(first_chunk + base + i, x_host[(base + i) % n_pool], o_host[i % 2],
+                        fused_q=fused_q)
     streamer.finish()
     e2e_b.record(stream)
     torch.cuda.synchronize()
@@ -537,8 +550,11 @@ def run_ours(args, cfg):
         "append_us": 1e3 * statistics.mean(app_ms),
         "append_gbs": app_bytes / (statistics.mean(app_ms) * 1e-3) / 1e9,
         "step_us": 1e3 * statistics.mean(step_ms),
-        "calls": "mla_project_chunk (x-projection GEMM, Q' GEMM + RoPE) | mla_attention_fwd "
-                 "(rotated-key pre-pass + attention) | mla_cache_append(MLA_APPEND)"}
+        "calls": ("mla_project_latents (x-projection GEMM) | mla_attention_fwd_from_cq "
+                  "(rotated-key pre-pass + attention with the query heads formed inside it) | "
+                  "mla_cache_append(MLA_APPEND)") if fused_q else
+                 ("mla_project_chunk (x-projection GEMM, Q' GEMM + RoPE) | mla_attention_fwd "
+                  "(rotated-key pre-pass + attention) | mla_cache_append(MLA_APPEND)")}
     n_units_all = world * cfg.batch
     ms_per_step = total_ms / args.steps
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
@@ -569,7 +585,8 @@ def run_ours(args, cfg):
         "attention_call_ms": attn_avg_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "mla_attention_fwd (rotated-key pre-pass + " +
+                     "kernel": ("mla_attention_fwd_from_cq" if fused_q else "mla_attention_fwd") +
+                               " (rotated-key pre-pass + " +
                                ("attention_pair_kernel" if args.kernel_path == "pair" and cfg.n_heads % 2 == 0
                                 and cfg.d_c in (128, 192) else "attention_tc_kernel") + ")",
                      "peak_kind": f"{peak_kind} burst bf16",
@@ -811,6 +828,9 @@ def main(argv=None):
     ap.add_argument("--kernel-path", choices=("auto", "pair"), default="auto",
                     help="attention kernel: auto (one CTA per head and query tile) or pair (the "
                          "CTA-pair kernel, for comparison)")
+    ap.add_argument("--unfused-query", action="store_true",
+                    help="project Q' with its own GEMM (mla_project_chunk + mla_attention_fwd) "
+                         "instead of forming it inside the attention kernel")
     ap.add_argument("--bandwidth-only", action="store_true",
                     help="only time the memory-bound calls (append, RoPE, KV down-projection)")
     ap.add_argument("--backward", action="store_true",

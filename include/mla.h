@@ -239,6 +239,18 @@ mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w
                              const void* w_qcat, void* c_q, void* q, void* chunk_lat,
                              int32_t first_frame, void* stream);
 
+/* --------------------------------------------------------------------------------------------
+ * mla_project_latents: the two down-projections of mla_project_chunk without the query heads
+ * ([M]: the query latent c_Q and the content latent c_KV are down-projections of the token x,
+ * k_R = W_R^K x), in one pass over x:
+ *   c_q[b, n]       = W_down^Q x[b, n]                       device T [B, n_q, d_cq] (out)
+ *   chunk_lat[b, n] = [W_down^KV x[b, n] || W_R^K x[b, n]]   device T [B, n_q, D]    (out)
+ *   x device T [B, n_q, d_model]; w_x device T [d_cq + D, d_model] as in mla_project_chunk.
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_project_latents(const mla_config* cfg, const void* x, const void* w_x, void* c_q,
+                               void* chunk_lat, void* stream);
+
 /* mla_attention_uses_tensor_cores: 1 if mla_attention_fwd with this configuration (and with the
  * W_UV epilogue when with_w_uv != 0) runs the tcgen05 tensor-core kernel, 0 if it runs the
  * CUDA-core kernel, -1 for an invalid configuration.  The tensor-core kernel covers bf16 with
@@ -289,6 +301,29 @@ mla_status mla_attention_fwd(const mla_config* cfg, const void* q, const void* c
                              int32_t n_valid_frames, int32_t first_frame, const void* w_uv,
                              void* out, float* lse, void* workspace, size_t workspace_bytes,
                              int32_t* dev_status, void* stream);
+
+/* --------------------------------------------------------------------------------------------
+ * mla_attention_fwd_from_cq: mla_attention_fwd with the absorbed query heads computed inside the
+ * attention kernel from the query latent ([M]: the head-specific queries are computed from
+ * c_Q, the positional one rotated by 3D-RoPE).  Each CTA forms its own tile of
+ *   q[b, n, h, :] = [ w_qcat[h, 0:d_c] c_q[b, n] || RoPE3D(w_qcat[h, d_c:D] c_q[b, n], pos(b, n)) ]
+ * (fp32 accumulation, rounded once to bf16, exactly as mla_query_proj stores it) and attends
+ * with it; q never goes through device memory.  Results equal mla_query_proj followed by
+ * mla_attention_fwd on the same inputs.
+ *   c_q    device T [B, n_q, d_cq]   (mla_project_latents)
+ *   w_qcat device T [H, D, d_cq]     (mla_compose_query_weights)
+ *   the other arguments, results and the workspace as in mla_attention_fwd.
+ * Needs the tensor-core path: bf16, d_c in {128, 192}, d_rope in {16, 32, 64} with
+ * d_c + d_rope <= 256, d_cq a multiple of 64 (and d_head = 128 with w_uv); otherwise
+ * MLA_ERR_UNSUPPORTED (use mla_project_chunk and mla_attention_fwd).  Errors: those of
+ * mla_attention_fwd and MLA_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_attention_fwd_from_cq(const mla_config* cfg, const void* c_q, const void* w_qcat,
+                                     const void* chunk_lat, const void* cache,
+                                     const int32_t* slot_frame, int32_t n_valid_frames,
+                                     int32_t first_frame, const void* w_uv, void* out, float* lse,
+                                     void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream);
 
 /* --------------------------------------------------------------------------------------------
  * Frozen-ring attention.  While a chunk is denoised in several steps, every step attends to the

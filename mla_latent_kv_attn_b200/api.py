@@ -19,6 +19,7 @@ __all__ = [
     "make_config", "torch_dtype", "mla_config_check", "mla_cache_append", "mla_rope3d",
     "mla_key_positions", "mla_compose_query_weights", "mla_query_proj", "mla_project_chunk",
     "mla_attention_workspace_bytes", "mla_attention_fwd", "mla_attention_fwd_static_scratch",
+    "mla_project_latents", "mla_attention_fwd_from_cq",
     "mla_rotate_ring_keys", "mla_attention_fwd_cached_ring", "mla_attention_uses_tensor_cores",
     "mla_attention_bwd_workspace_bytes", "mla_attention_bwd",
     "mla_out_proj", "MLAError",
@@ -146,6 +147,17 @@ def mla_project_chunk(c: MLAConfigC, x, w_x, w_qcat, c_q, q, chunk_lat, first_fr
     _lib.check("mla_project_chunk", st)
 
 
+def mla_project_latents(c: MLAConfigC, x, w_x, c_q, chunk_lat, stream=None) -> None:
+    tpf, n_q, D = _geom(c)
+    dt = torch_dtype(c)
+    B = c.batch
+    st = _lib.lib().mla_project_latents(
+        ctypes.byref(c), _ptr(x, "x", dt, (B, n_q, c.d_model)),
+        _ptr(w_x, "w_x", dt, (c.d_cq + D, c.d_model)), _ptr(c_q, "c_q", dt, (B, n_q, c.d_cq)),
+        _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)), _stream(stream))
+    _lib.check("mla_project_latents", st)
+
+
 def mla_attention_uses_tensor_cores(c: MLAConfigC, with_w_uv: bool = True) -> bool:
     r = int(_lib.lib().mla_attention_uses_tensor_cores(ctypes.byref(c), 1 if with_w_uv else 0))
     if r < 0:
@@ -179,6 +191,27 @@ def mla_attention_fwd(c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_fr
                       stream=None) -> None:
     _attention("mla_attention_fwd", c, q, chunk_lat, cache, slot_frame, n_valid_frames,
                first_frame, w_uv, out, lse, workspace, dev_status, stream)
+
+
+def mla_attention_fwd_from_cq(c: MLAConfigC, c_q, w_qcat, chunk_lat, cache, slot_frame,
+                              n_valid_frames: int, first_frame: int, w_uv, out, lse=None,
+                              workspace=None, dev_status=None, stream=None) -> None:
+    """mla_attention_fwd with the query heads (and their 3D-RoPE) formed inside the attention
+    kernel from the query latent c_q and the composed weights w_qcat."""
+    tpf, n_q, D = _geom(c)
+    dt = torch_dtype(c)
+    B, H = c.batch, c.n_heads
+    out_shape = (B, n_q, H * c.d_head) if w_uv is not None else (B, n_q, H, c.d_c)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib.lib().mla_attention_fwd_from_cq(
+        ctypes.byref(c), _ptr(c_q, "c_q", dt, (B, n_q, c.d_cq)),
+        _ptr(w_qcat, "w_qcat", dt, (H, D, c.d_cq)), _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)),
+        _ptr(cache, "cache", dt, (B, c.window_frames * tpf, D)),
+        _ptr(slot_frame, "slot_frame", torch.int32, (B, c.window_frames)), n_valid_frames,
+        first_frame, _ptr(w_uv, "w_uv", dt, (H, c.d_head, c.d_c)), _ptr(out, "out", dt, out_shape),
+        _ptr(lse, "lse", torch.float32, (B, H, n_q)), _ptr(workspace, "workspace"), ws_bytes,
+        _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    _lib.check("mla_attention_fwd_from_cq", st)
 
 
 def mla_attention_fwd_cached_ring(c: MLAConfigC, q, chunk_lat, cache, slot_frame,

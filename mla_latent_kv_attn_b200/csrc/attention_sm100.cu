@@ -94,6 +94,12 @@ struct AttnShape {
 struct AttnParams {
   const bf16* q;        // [B, n_q, H, D] (read by the softmax threads when Q lives in TMEM)
   int n_q, H, nc, nc_pad, nt_ring, nt;
+  // Fused query heads: the K' ring first carries nqc chunk pairs (64 columns of the CTA's c_Q
+  // rows and of w_qcat[h]); their product Q'_h accumulates in TMEM, and the softmax threads
+  // rotate its positional part at (first_frame + n / tpf, row, column) and write Q as bf16.
+  int nqc;
+  int first_frame;
+  RopeGeom rope;
   float scale_log2;
   int has_w_uv;
   void* out;
@@ -156,18 +162,58 @@ __device__ __noinline__ void copy_q_row(uint32_t taddr, const bf16* row) {
   }
 }
 
+// Fused query heads: one row of Q'_h (fp32, TMEM columns kColO .. kColO+D of this thread's lane)
+// rotated by 3D-RoPE in its last D-DC columns at chunk token n's position, rounded once to
+// bf16 and stored as pairs from column kColS (zeros past D/2) - what the Q' GEMM's epilogue
+// stores.  16 columns at a time: D is a multiple of 16 and DC of 64.
+template <int DC>
+__device__ __forceinline__ void q_piece(uint32_t tlane, int c, const AttnParams& p, int t, int hh,
+                                        int ww, uint32_t* w8) {
+  uint32_t r[16];
+  tmem_ld16_wait(tlane + kColO + c, r);
+  float v[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+  if (c >= DC) {
+#pragma unroll
+    for (int k = 0; k < 16; k += 2)
+      rope_rotate(v[k], v[k + 1], rope_angle(p.rope, (c - DC + k) >> 1, t, hh, ww));
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) w8[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
+}
+
+template <int DC, int D, int kQWords>
+__device__ __noinline__ void q_row_from_accumulator(uint32_t tlane, const AttnParams& p, int n) {
+  const int nl = n < p.n_q ? n : 0;
+  const int i = nl % p.rope.tpf;
+  const int t = p.first_frame + nl / p.rope.tpf, hh = i / p.rope.frame_w, ww = i % p.rope.frame_w;
+#pragma unroll 1
+  for (int c = 0; c < kQWords * 2; c += 32) {     // 32 values = 16 bf16 pairs per store
+    uint32_t w[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) w[k] = 0u;
+    if (c < D) q_piece<DC>(tlane, c, p, t, hh, ww, w);
+    if (c + 16 < D) q_piece<DC>(tlane, c + 16, p, t, hh, ww, w + 8);
+    tmem_st16(tlane + kColS + c / 2, w);
+  }
+}
+
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          int32_t* dev_status) {
   return mbar_wait_or_abort(bar, parity, abort_flag, dev_status);
 }
 
-template <int DC, int DR>
+template <int DC, int DR, bool kFusedQ>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                         const __grid_constant__ CUtensorMap tm_cache,
                         const __grid_constant__ CUtensorMap tm_chunk,
                         const __grid_constant__ CUtensorMap tm_ws,
-                        const __grid_constant__ CUtensorMap tm_wuv, AttnParams p) {
+                        const __grid_constant__ CUtensorMap tm_wuv,
+                        const __grid_constant__ CUtensorMap tm_cq,
+                        const __grid_constant__ CUtensorMap tm_wq,
+                        const __grid_constant__ AttnParams p) {
   using Sh = AttnShape<DC, DR>;
   constexpr int kDc = DC;
   constexpr int kCBlk = Sh::kCBlk;
@@ -177,6 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kAliasP = Sh::kAliasP;
   constexpr uint32_t kColP = Sh::kColP;
   constexpr bool kQTmem = Sh::kQTmem;
+  static_assert(!kFusedQ || kQTmem, "fused query heads need the query tile in TMEM");
+  // a chunk pair of the fused query heads: 128 x 64 of c_Q, then D x 64 of w_qcat[h]
+  constexpr int kCqBytes = kBM * 128, kWqBytes = Sh::D * 128;
+  static_assert(!kFusedQ || kCqBytes + kWqBytes <= kKTile, "a query chunk pair fits a K' stage");
+  const int nqc = kFusedQ ? p.nqc : 0;   // ring uses before the first K' tile
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full;   // the Q tile landed (TMA) or is in TMEM (softmax)
   __shared__ __align__(8) uint64_t kv_full[kStages];
@@ -189,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t w_full;
   __shared__ __align__(8) uint64_t olat_full;
   __shared__ __align__(8) uint64_t epi_done;
+  __shared__ __align__(8) uint64_t qacc_full;   // fused query heads: Q'_h accumulated in TMEM
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -218,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&w_full), 1);
     mbar_init(smem_u32(&olat_full), kSoftmaxThreads);
     mbar_init(smem_u32(&epi_done), 1);
+    mbar_init(smem_u32(&qacc_full), 1);
 
     fence_barrier_init();
   }
@@ -243,9 +296,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(sQ + kCBlk * kQBlk, &tm_qr, qb, kDc, h, q0, b);
       }
       bool ok = true;
+      if constexpr (kFusedQ) {
+        // the query heads' operands first: chunk c = columns 64c.. of c_Q rows q0.. and of
+        // w_qcat[h] (its D rows), through the ring like K' tiles
+        tma_prefetch_desc(&tm_cq);
+        tma_prefetch_desc(&tm_wq);
+        for (int c = 0; c < nqc && ok; ++c) {
+          const int s = c % kStages;
+          ok = wait_bar(smem_u32(&kv_empty[s]), ((c / kStages) & 1) ^ 1, abort_flag, p.dev_status);
+          if (!ok) break;
+          const uint32_t dst = sK0 + s * kKTile;
+          const uint32_t fb = smem_u32(&kv_full[s]);
+          mbar_arrive_expect_tx(fb, kCqBytes + kWqBytes);
+          tma_load_3d(dst, &tm_cq, fb, 64 * c, q0, b);
+          tma_load_2d(dst + kCqBytes, &tm_wq, fb, 64 * c, h * Sh::D);
+        }
+      }
       for (int j = 0; j < p.nt && ok; ++j) {
-        const int s = j % kStages;
-        ok = wait_bar(smem_u32(&kv_empty[s]), ((j / kStages) & 1) ^ 1, abort_flag, p.dev_status);
+        const int u = nqc + j;                 // ring use of K' tile j
+        const int s = u % kStages;
+        ok = wait_bar(smem_u32(&kv_empty[s]), ((u / kStages) & 1) ^ 1, abort_flag, p.dev_status);
         if (!ok) break;
         const uint32_t dst = sK0 + s * kKTile;
         const uint32_t fb = smem_u32(&kv_full[s]);
@@ -262,8 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && p.has_w_uv) {
         // W_UV_h [128 x DC] goes into the stage a tile nt would use, once it is free.
-        const int s = p.nt % kStages;
-        if (wait_bar(smem_u32(&kv_empty[s]), ((p.nt / kStages) & 1) ^ 1, abort_flag, p.dev_status)) {
+        const int uw = nqc + p.nt;
+        const int s = uw % kStages;
+        if (wait_bar(smem_u32(&kv_empty[s]), ((uw / kStages) & 1) ^ 1, abort_flag, p.dev_status)) {
           const uint32_t wb = smem_u32(&w_full);
           mbar_arrive_expect_tx(wb, kCBlk * kQBlk);
           for (int i = 0; i < kCBlk; ++i)
@@ -294,10 +365,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t v_0 = smem_desc(sK0, kKBlk, 1024, kSwizzle128B);
       bool ok = true;
       if (warp == kQkWarp) {
-        ok = wait_bar(smem_u32(&q_full), 0, abort_flag, p.dev_status);
+        if constexpr (kFusedQ) {
+          // Q'_h = c_Q rows x w_qcat[h]^T (M=128, N=D, K=d_cq) into TMEM columns kColO.. (free
+          // until the first PV), then handed to the softmax threads
+          constexpr uint32_t idesc_q = idesc_bf16_f32(kBM, Sh::D, 0, 0);
+          for (int c = 0; c < nqc && ok; ++c) {
+            const int s = c % kStages;
+            ok = wait_bar(smem_u32(&kv_full[s]), (c / kStages) & 1, abort_flag, p.dev_status);
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t a0 = smem_desc(sK0 + s * kKTile, 16, 1024, kSwizzle128B);
+            const uint64_t b0 = smem_desc(sK0 + s * kKTile + kCqBytes, 16, 1024, kSwizzle128B);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem + kColO, a0 + 2 * kk, b0 + 2 * kk, idesc_q, (c | kk) != 0 ? 1u : 0u);
+            mma_commit(smem_u32(&kv_empty[s]));
+          }
+          if (ok) mma_commit(smem_u32(&qacc_full));
+        }
+        ok = ok && wait_bar(smem_u32(&q_full), 0, abort_flag, p.dev_status);
         for (int j = 0; j < p.nt && ok; ++j) {
-          const int s = j % kStages;
-          ok = wait_bar(smem_u32(&kv_full[s]), (j / kStages) & 1, abort_flag, p.dev_status);
+          const int u = nqc + j;
+          const int s = u % kStages;
+          ok = wait_bar(smem_u32(&kv_full[s]), (u / kStages) & 1, abort_flag, p.dev_status);
           if constexpr (kQTmem) {    // the softmax has loaded S(j-1) out of the one buffer
             if (ok && j >= 1)
               ok = wait_bar(smem_u32(&s_free[0]), (j - 1) & 1, abort_flag, p.dev_status);
@@ -344,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = wait_bar(smem_u32(&p_full), j & 1, abort_flag, p.dev_status);
           if (!ok) break;
           tc_fence_after();
-          const int s = j % kStages;
+          const int s = (nqc + j) % kStages;
           const uint64_t vd = v_0 + static_cast<uint32_t>(s) * kKTileD;
           const uint32_t pa = tmem + (kAliasP ? (j & 1) * kColS : kColP);
 #pragma unroll
@@ -360,11 +450,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                wait_bar(smem_u32(&olat_full), 0, abort_flag, p.dev_status);
           if (ok) {
             tc_fence_after();
-            const uint64_t w_c = smem_desc(sK0 + (p.nt % kStages) * kKTile, 16, 1024,
+            const uint64_t w_c = smem_desc(sK0 + ((nqc + p.nt) % kStages) * kKTile, 16, 1024,
                                            kSwizzle128B);
             // O_lat: in the dead Q tile, or (Q in TMEM) in the stage after W_UV's
             const uint64_t o_c =
-                kQTmem ? smem_desc(sK0 + ((p.nt + 1) % kStages) * kKTile, 16, 1024, kSwizzle128B)
+                kQTmem ? smem_desc(sK0 + ((nqc + p.nt + 1) % kStages) * kKTile, 16, 1024, kSwizzle128B)
                        : q_c;
 #pragma unroll
             for (int blk = 0; blk < kCBlk; ++blk)
@@ -382,7 +472,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = warp * 32 + lane;                 // TMEM lane and query row in the tile
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int n = q0 + row;
-    if constexpr (kQTmem) {
+    if constexpr (kFusedQ) {
+      // this row of Q'_h out of its fp32 accumulator, the positional part rotated at the row's
+      // position, into the query's TMEM columns as bf16 pairs
+      const bool okq = __all_sync(0xffffffffu, wait_bar(smem_u32(&qacc_full), 0, abort_flag,
+                                                        p.dev_status));
+      if (okq) {
+        tc_fence_after();
+        q_row_from_accumulator<DC, Sh::D, Sh::kQWords>(tmem + lane_off, p, n);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&q_full));
+    } else if constexpr (kQTmem) {
       // this row of the query tile into TMEM, bf16 pairs from column kColS (zeros past D/2
       // and for rows past n_q); the QK issuer waits for all 128 rows on q_full
       copy_q_row<Sh::D, Sh::kQWords>(tmem + lane_off + kColS,
@@ -513,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         // O_lat (bf16) -> shared memory, 128B-swizzled K-major, over the dead Q tile (or, with
         // Q in TMEM, into the K' stage after the one W_UV went to: all stages are free now).
-        const uint32_t so = kQTmem ? sK0 + ((p.nt + 1) % kStages) * kKTile : sQ;
+        const uint32_t so = kQTmem ? sK0 + ((nqc + p.nt + 1) % kStages) * kKTile : sQ;
         uint8_t* qsm = smem_raw + (so - smem_u32(smem_raw));
 #pragma unroll 1
         for (int c = 0; c < kDc; c += 32) {
@@ -566,14 +668,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DC, int DR>
-mla_status attention_tc_impl(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
+// Fused query heads (attention_tc_fused_q): c_q [B, n_q, d_cq] and w_qcat [H, D, d_cq] in place
+// of a.q, and the chunk's first frame for the query's 3D-RoPE.
+struct FusedQ {
+  const void* c_q;
+  const void* w_qcat;
+  int first_frame;
+};
+
+template <int DC, int DR, bool kFusedQ>
+mla_status attention_tc_impl(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s,
+                             const FusedQ* fq = nullptr) {
   using Sh = AttnShape<DC, DR>;
   constexpr int kD = Sh::D;
   const KeyWorkspace kw = key_workspace_layout(d, n_valid);
-  CUtensorMap tq, tqr, tcache, tchunk, tws, twuv;
+  CUtensorMap tq, tqr, tcache, tchunk, tws, twuv, tcq, twq;
   mla_status st;
-  {
+  if (kFusedQ) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(d.d_cq), static_cast<uint64_t>(d.n_q),
+                              static_cast<uint64_t>(d.B)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(d.d_cq) * 2,
+                                 static_cast<uint64_t>(d.n_q) * d.d_cq * 2};
+    const uint32_t box[3] = {64, kBM, 1};
+    if ((st = make_tmap_bf16(&tcq, fq->c_q, 3, dims, strides, box, 128)) != MLA_OK) return st;
+    const uint64_t wdims[2] = {static_cast<uint64_t>(d.d_cq), static_cast<uint64_t>(d.H) * kD};
+    const uint64_t wstrides[1] = {static_cast<uint64_t>(d.d_cq) * 2};
+    const uint32_t wbox[2] = {64, kD};
+    if ((st = make_tmap_bf16(&twq, fq->w_qcat, 2, wdims, wstrides, wbox, 128)) != MLA_OK) return st;
+    tq = tcq;    // never read: the query comes from the fused heads
+    tqr = tcq;
+  } else {
     const uint64_t dims[4] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.H),
                               static_cast<uint64_t>(d.n_q), static_cast<uint64_t>(d.B)};
     const uint64_t strides[3] = {kD * 2ull, static_cast<uint64_t>(d.H) * kD * 2,
@@ -583,6 +707,8 @@ mla_status attention_tc_impl(const Dims& d, const AttnArgs& a, int n_valid, cuda
     const uint32_t box_r[4] = {DR, 1, kBM, 1};
     if ((st = make_tmap_bf16(&tqr, a.q, 4, dims, strides, box_r, Sh::kRopeBytes)) != MLA_OK)
       return st;
+    tcq = tq;    // never read
+    twq = tq;
   }
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(d.n_q),
@@ -624,10 +750,14 @@ mla_status attention_tc_impl(const Dims& d, const AttnArgs& a, int n_valid, cuda
   p.scale_log2 = d.scale * 1.4426950408889634f;
   p.has_w_uv = a.w_uv != nullptr;
   p.out = a.out; p.lse = a.lse; p.dev_status = a.dev_status;
-  MLA_CUDA_TRY(cudaFuncSetAttribute(attention_tc_kernel<DC, DR>,
+  p.nqc = kFusedQ ? d.d_cq / 64 : 0;
+  p.first_frame = kFusedQ ? fq->first_frame : 0;
+  p.rope = rope_geom(d);
+  MLA_CUDA_TRY(cudaFuncSetAttribute(attention_tc_kernel<DC, DR, kFusedQ>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmem));
   dim3 grid(ceil_div(d.n_q, kBM), d.H, d.B);
-  attention_tc_kernel<DC, DR><<<grid, kThreads, Sh::kSmem, s>>>(tq, tqr, tcache, tchunk, tws, twuv, p);
+  attention_tc_kernel<DC, DR, kFusedQ><<<grid, kThreads, Sh::kSmem, s>>>(tq, tqr, tcache, tchunk,
+                                                                      tws, twuv, tcq, twq, p);
   MLA_LAUNCH_CHECK("attention_tc");
   return MLA_OK;
 }
@@ -641,12 +771,29 @@ bool tc_attention_supported(const Dims& d, bool has_w_uv) {
 
 mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
 #define MLA_ATTN_CASE(DC, DR) \
-  if (d.d_c == DC && d.d_rope == DR) return attention_tc_impl<DC, DR>(d, a, n_valid, s);
+  if (d.d_c == DC && d.d_rope == DR) return attention_tc_impl<DC, DR, false>(d, a, n_valid, s);
   MLA_ATTN_CASE(128, 16) MLA_ATTN_CASE(128, 32) MLA_ATTN_CASE(128, 64)
   MLA_ATTN_CASE(192, 16) MLA_ATTN_CASE(192, 32) MLA_ATTN_CASE(192, 64)
   MLA_ATTN_CASE(256, 16) MLA_ATTN_CASE(256, 32) MLA_ATTN_CASE(256, 64)
 #undef MLA_ATTN_CASE
   MLA_FAIL(MLA_ERR_UNSUPPORTED, "no tensor-core attention kernel for d_c %d, d_rope %d", d.d_c,
+           d.d_rope);
+}
+
+bool tc_attention_fused_q_supported(const Dims& d, bool has_w_uv) {
+  return tc_attention_supported(d, has_w_uv) && d.d_c <= 192 && d.d_c + d.d_rope <= 256 &&
+         d.d_cq % 64 == 0 && d.d_cq > 0;
+}
+
+mla_status attention_tc_fused_q(const Dims& d, const AttnArgs& a, int n_valid, const void* c_q,
+                                const void* w_qcat, int first_frame, cudaStream_t s) {
+  const FusedQ fq{c_q, w_qcat, first_frame};
+#define MLA_ATTN_FQ_CASE(DC, DR) \
+  if (d.d_c == DC && d.d_rope == DR) return attention_tc_impl<DC, DR, true>(d, a, n_valid, s, &fq);
+  MLA_ATTN_FQ_CASE(128, 16) MLA_ATTN_FQ_CASE(128, 32) MLA_ATTN_FQ_CASE(128, 64)
+  MLA_ATTN_FQ_CASE(192, 16) MLA_ATTN_FQ_CASE(192, 32) MLA_ATTN_FQ_CASE(192, 64)
+#undef MLA_ATTN_FQ_CASE
+  MLA_FAIL(MLA_ERR_UNSUPPORTED, "no fused-query attention kernel for d_c %d, d_rope %d", d.d_c,
            d.d_rope);
 }
 

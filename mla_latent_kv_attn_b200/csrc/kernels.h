@@ -151,6 +151,11 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s);
 
 bool tc_attention_supported(const Dims& d, bool has_w_uv);
 mla_status attention_tc(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);
+// The tensor-core attention with the query heads computed inside it from the query latent
+// (c_q [B, n_q, d_cq], w_qcat [H, D, d_cq]): d_c <= 192, D <= 256, d_cq a multiple of 64.
+bool tc_attention_fused_q_supported(const Dims& d, bool has_w_uv);
+mla_status attention_tc_fused_q(const Dims& d, const AttnArgs& a, int n_valid, const void* c_q,
+                                const void* w_qcat, int first_frame, cudaStream_t s);
 // CTA-pair tensor-core attention (attention_pair_sm100.cu): pairs of heads share each key tile.
 bool tc_attention_pair_supported(const Dims& d, bool has_w_uv);
 mla_status attention_tc_pair(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s);

@@ -147,6 +147,29 @@ mla_status query_heads(const Dims& d, const void* c_q, const void* w_qcat, void*
   return rope3d_inplace(d, q, d.B, d.n_q, N, d.d_c, d.H, d.D, nullptr, 0, first_frame, s);
 }
 
+// c_q = W_down^Q x and chunk_lat = [W_down^KV x || W_R^K x]: on the tensor cores one GEMM over
+// the stacked weights w_x with its columns split between the two outputs.
+mla_status project_latents(const Dims& d, const void* x, const void* w_x, void* c_q,
+                           void* chunk_lat, cudaStream_t s) {
+  const int M = d.B * d.n_q;
+  const int N = d.d_cq + d.D;
+  if (use_tc(d) && d.d_cq % 32 == 0 && tc_gemm_supported(M, N, d.d_model, d.d_model, d.d_model)) {
+    // one pass over x: columns 0..d_cq-1 are c_Q, the rest [c_KV || k_R]
+    TcGemmArgs g{};
+    g.A = x; g.a_sm = d.d_model; g.a_batch = 0;
+    g.B = w_x; g.b_sn = d.d_model; g.b_batch = 0;
+    g.C = c_q; g.c_sm = d.d_cq; g.c_batch = 0;
+    g.C2 = chunk_lat; g.c2_sm = d.D; g.c2_batch = 0; g.n_split = d.d_cq;
+    g.M = M; g.N = N; g.K = d.d_model; g.batch = 1;
+    g.epilogue = kEpiStore;
+    return gemm_tc(g, s);
+  }
+  const size_t es = dtype_size(d.dtype);
+  MLA_TRY(gemm(d, x, d.d_model, 0, w_x, d.d_model, 0, c_q, d.d_cq, 0, M, d.d_cq, d.d_model, 1, s));
+  return gemm(d, x, d.d_model, 0, static_cast<const char*>(w_x) + es * d.d_cq * d.d_model,
+              d.d_model, 0, chunk_lat, d.D, 0, M, d.D, d.d_model, 1, s);
+}
+
 mla_status check_workspace(const Dims& d, int n_valid, const void* workspace,
                            size_t workspace_bytes) {
   const KeyWorkspace kw = key_workspace_layout(d, n_valid);
@@ -373,25 +396,21 @@ mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w
   MLA_TRY(check_ptr(q, "q"));
   MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int M = d.B * d.n_q;
-  const int N = d.d_cq + d.D;
-  if (use_tc(d) && d.d_cq % 32 == 0 && tc_gemm_supported(M, N, d.d_model, d.d_model, d.d_model)) {
-    // one pass over x: columns 0..d_cq-1 are c_Q, the rest [c_KV || k_R]
-    TcGemmArgs g{};
-    g.A = x; g.a_sm = d.d_model; g.a_batch = 0;
-    g.B = w_x; g.b_sn = d.d_model; g.b_batch = 0;
-    g.C = c_q; g.c_sm = d.d_cq; g.c_batch = 0;
-    g.C2 = chunk_lat; g.c2_sm = d.D; g.c2_batch = 0; g.n_split = d.d_cq;
-    g.M = M; g.N = N; g.K = d.d_model; g.batch = 1;
-    g.epilogue = kEpiStore;
-    MLA_TRY(gemm_tc(g, s));
-  } else {
-    const size_t es = dtype_size(d.dtype);
-    MLA_TRY(gemm(d, x, d.d_model, 0, w_x, d.d_model, 0, c_q, d.d_cq, 0, M, d.d_cq, d.d_model, 1, s));
-    MLA_TRY(gemm(d, x, d.d_model, 0, static_cast<const char*>(w_x) + es * d.d_cq * d.d_model,
-                 d.d_model, 0, chunk_lat, d.D, 0, M, d.D, d.d_model, 1, s));
-  }
+  MLA_TRY(project_latents(d, x, w_x, c_q, chunk_lat, s));
   return query_heads(d, c_q, w_qcat, q, first_frame, s);
+}
+
+mla_status mla_project_latents(const mla_config* cfg, const void* x, const void* w_x, void* c_q,
+                               void* chunk_lat, void* stream) {
+  MLA_NVTX_RANGE("mla_project_latents");
+  set_last_error("");
+  MLA_TRY(check_cfg(cfg));
+  const Dims d = dims_of(*cfg);
+  MLA_TRY(check_ptr(x, "x"));
+  MLA_TRY(check_ptr(w_x, "w_x"));
+  MLA_TRY(check_ptr(c_q, "c_q"));
+  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
+  return project_latents(d, x, w_x, c_q, chunk_lat, static_cast<cudaStream_t>(stream));
 }
 
 int32_t mla_attention_uses_tensor_cores(const mla_config* cfg, int32_t with_w_uv) {
@@ -415,6 +434,43 @@ mla_status mla_attention_fwd(const mla_config* cfg, const void* q, const void* c
   MLA_NVTX_RANGE("mla_attention_fwd");
   return attention_entry(cfg, q, chunk_lat, cache, slot_frame, n_valid_frames, first_frame, w_uv,
                          out, lse, workspace, workspace_bytes, dev_status, stream, kRopeKeysAll);
+}
+
+mla_status mla_attention_fwd_from_cq(const mla_config* cfg, const void* c_q, const void* w_qcat,
+                                     const void* chunk_lat, const void* cache,
+                                     const int32_t* slot_frame, int32_t n_valid_frames,
+                                     int32_t first_frame, const void* w_uv, void* out, float* lse,
+                                     void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream) {
+  MLA_NVTX_RANGE("mla_attention_fwd_from_cq");
+  set_last_error("");
+  MLA_TRY(check_cfg(cfg));
+  const Dims d = dims_of(*cfg);
+  MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
+                d.W);
+  MLA_TRY(check_first_frame(first_frame, d.C));
+  if (!(use_tc(d) && tc_attention_fused_q_supported(d, w_uv != nullptr)))
+    MLA_FAIL(MLA_ERR_UNSUPPORTED,
+             "attention from the query latent needs the tensor-core path (bf16, d_c <= 192, "
+             "d_c + d_rope <= 256, d_cq a multiple of 64); use mla_project_chunk and "
+             "mla_attention_fwd");
+  MLA_TRY(check_ptr(c_q, "c_q"));
+  MLA_TRY(check_ptr(w_qcat, "w_qcat"));
+  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
+  MLA_TRY(check_ptr(slot_frame, "slot_frame"));
+  MLA_TRY(check_ptr(out, "out"));
+  MLA_TRY(check_ptr(cache, "cache", n_valid_frames > 0));
+  MLA_TRY(check_ptr(w_uv, "w_uv", false));
+  MLA_TRY(check_ptr(lse, "lse", false));
+  MLA_TRY(check_ptr(dev_status, "dev_status", false));
+  MLA_TRY(check_workspace(d, n_valid_frames, workspace, workspace_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MLA_TRY(build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid_frames, first_frame, workspace,
+                          s, kRopeKeysAll, dev_status, 1));
+  AttnArgs a{};
+  a.q = nullptr; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = workspace; a.w_uv = w_uv;
+  a.out = out; a.lse = lse; a.dev_status = dev_status;
+  return attention_tc_fused_q(d, a, n_valid_frames, c_q, w_qcat, first_frame, s);
 }
 
 mla_status mla_attention_fwd_cached_ring(const mla_config* cfg, const void* q,

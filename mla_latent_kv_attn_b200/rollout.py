@@ -93,14 +93,30 @@ class ChunkBuffers:
         self.dev_status = torch.zeros((1,), device=device, dtype=torch.int32)
 
 
+def fused_query_supported(c) -> bool:
+    """Whether mla_attention_fwd_from_cq (query heads formed inside the attention kernel) serves
+    this configuration."""
+    return (c.dtype == api.MLA_BF16 and c.kernel_path != api.MLA_PATH_SIMT
+            and c.d_c in (128, 192) and c.d_rope in (16, 32, 64) and c.d_c + c.d_rope <= 256
+            and c.d_cq % 64 == 0 and c.d_head == 128)
+
+
 def attend_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
-                 fuse_uv: bool = True, stream=None) -> torch.Tensor:
+                 fuse_uv: bool = True, stream=None, fused_q: bool = False) -> torch.Tensor:
     """Query path, chunk latents and attention of one chunk (buf.x holds its tokens).
-    Returns buf.o (fused W_UV) or buf.o_lat (latent output)."""
+    Returns buf.o (fused W_UV) or buf.o_lat (latent output).  With fused_q the attention kernel
+    forms the query heads itself from c_Q (buf.q is then not written)."""
     first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
+    out = buf.o if fuse_uv else buf.o_lat
+    if fused_q:
+        api.mla_project_latents(c, buf.x, w.w_x, buf.c_q, buf.chunk_lat, stream=stream)
+        api.mla_attention_fwd_from_cq(c, buf.c_q, w.w_qcat, buf.chunk_lat, ring.cache,
+                                      ring.slot_frame, n_valid, first,
+                                      w.w_uv if fuse_uv else None, out, buf.lse, buf.workspace,
+                                      buf.dev_status, stream=stream)
+        return out
     api.mla_project_chunk(c, buf.x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first,
                           stream=stream)
-    out = buf.o if fuse_uv else buf.o_lat
     api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid, first,
                           w.w_uv if fuse_uv else None, out, buf.lse, buf.workspace,
                           buf.dev_status, stream=stream)
@@ -123,9 +139,9 @@ def prefill_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int
 
 
 def run_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
-              fuse_uv: bool = True, stream=None) -> torch.Tensor:
+              fuse_uv: bool = True, stream=None, fused_q: bool = False) -> torch.Tensor:
     """One whole chunk: attend, then append."""
-    out = attend_chunk(c, w, ring, buf, chunk, fuse_uv=fuse_uv, stream=stream)
+    out = attend_chunk(c, w, ring, buf, chunk, fuse_uv=fuse_uv, stream=stream, fused_q=fused_q)
     append_chunk(c, ring, buf, chunk, stream=stream)
     return out
 
@@ -167,7 +183,7 @@ class HostStreamer:
         self.d2h.wait_event(event)
 
     def submit(self, chunk: int, x_host: torch.Tensor, o_host: torch.Tensor,
-               fuse_uv: bool = True) -> None:
+               fuse_uv: bool = True, fused_q: bool = False) -> None:
         """Enqueues chunk `chunk`: copy-in of x_host, attention, append, copy-out into o_host."""
         k = self.n % 2
         b = self.bufs[k]
@@ -180,7 +196,8 @@ class HostStreamer:
         self.compute.wait_event(x_ready)
         if self.o_free[k] is not None:
             self.compute.wait_event(self.o_free[k])
-        out = run_chunk(self.c, self.w, self.ring, b, chunk, fuse_uv=fuse_uv, stream=self.compute)
+        out = run_chunk(self.c, self.w, self.ring, b, chunk, fuse_uv=fuse_uv, stream=self.compute,
+                        fused_q=fused_q)
         done = torch.cuda.Event()
         done.record(self.compute)
         self.x_free[k] = done
@@ -217,7 +234,8 @@ class ChunkGraph:
     """
 
     def __init__(self, c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
-                 x: Optional[torch.Tensor] = None, events: bool = False, fuse_uv: bool = True):
+                 x: Optional[torch.Tensor] = None, events: bool = False, fuse_uv: bool = True,
+                 fused_q: bool = False):
         self.chunk = chunk
         first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
         x = buf.x if x is None else x
@@ -231,13 +249,22 @@ class ChunkGraph:
         with torch.cuda.graph(self.graph, stream=side, capture_error_mode="relaxed"):
             if events:
                 self.proj_start.record()
-            api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
+            if fused_q:
+                api.mla_project_latents(c, x, w.w_x, buf.c_q, buf.chunk_lat)
+            else:
+                api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
             if events:
                 self.attn_start.record()
             out = buf.o if fuse_uv else buf.o_lat
-            api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid,
-                                  first, w.w_uv if fuse_uv else None, out, buf.lse, buf.workspace,
-                                  buf.dev_status)
+            if fused_q:
+                api.mla_attention_fwd_from_cq(c, buf.c_q, w.w_qcat, buf.chunk_lat, ring.cache,
+                                              ring.slot_frame, n_valid, first,
+                                              w.w_uv if fuse_uv else None, out, buf.lse,
+                                              buf.workspace, buf.dev_status)
+            else:
+                api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame,
+                                      n_valid, first, w.w_uv if fuse_uv else None, out, buf.lse,
+                                      buf.workspace, buf.dev_status)
             if events:
                 self.attn_end.record()
             api.mla_cache_append(c, None, None, buf.chunk_lat, ring.cache, ring.slot_frame,

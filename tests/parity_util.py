@@ -55,20 +55,31 @@ class GpuRun:
         self.load_x(x)
         rollout.prefill_chunk(self.c, self.w, self.ring, self.buf, chunk)
 
-    def attend(self, chunk: int, x: np.ndarray, want_latent=True):
+    def attend(self, chunk: int, x: np.ndarray, want_latent=True, fused_q=False):
         """Runs the chunk's attention (fused W_UV and, optionally, latent output); returns numpy
-        copies of every intermediate.  Does not append."""
+        copies of every intermediate.  Does not append.  With fused_q the attention kernel forms
+        the query heads itself (no q in the result)."""
         self.load_x(x)
         self.buf.dev_status.zero_()
-        o = rollout.attend_chunk(self.c, self.w, self.ring, self.buf, chunk, fuse_uv=True)
-        res = dict(o=to_np(o), lse=to_np(self.buf.lse), q=to_np(self.buf.q),
-                   c_q=to_np(self.buf.c_q), chunk_lat=to_np(self.buf.chunk_lat))
+        o = rollout.attend_chunk(self.c, self.w, self.ring, self.buf, chunk, fuse_uv=True,
+                                 fused_q=fused_q)
+        res = dict(o=to_np(o), lse=to_np(self.buf.lse), c_q=to_np(self.buf.c_q),
+                   chunk_lat=to_np(self.buf.chunk_lat))
+        if not fused_q:
+            res["q"] = to_np(self.buf.q)
         if want_latent:
             first, n_valid = rollout.chunk_schedule(self.cfg.chunk_frames, self.cfg.window_frames,
                                                     chunk)
-            api.mla_attention_fwd(self.c, self.buf.q, self.buf.chunk_lat, self.ring.cache,
-                                  self.ring.slot_frame, n_valid, first, None, self.buf.o_lat,
-                                  None, self.buf.workspace, self.buf.dev_status)
+            if fused_q:
+                api.mla_attention_fwd_from_cq(self.c, self.buf.c_q, self.w.w_qcat,
+                                              self.buf.chunk_lat, self.ring.cache,
+                                              self.ring.slot_frame, n_valid, first, None,
+                                              self.buf.o_lat, None, self.buf.workspace,
+                                              self.buf.dev_status)
+            else:
+                api.mla_attention_fwd(self.c, self.buf.q, self.buf.chunk_lat, self.ring.cache,
+                                      self.ring.slot_frame, n_valid, first, None, self.buf.o_lat,
+                                      None, self.buf.workspace, self.buf.dev_status)
             res["o_lat"] = to_np(self.buf.o_lat)
         torch.cuda.synchronize()
         rollout.check_device_status(self.buf)
@@ -128,7 +139,8 @@ def check_chunk(name, cfg, g, o_res, rows, report=None, samples=None):
         lat_ref = np.concatenate([r["c_kv"], r["k_r"]], axis=1)
         compare(tag + ".chunk_lat", g["chunk_lat"][b], lat_ref, dt, report)
         compare(tag + ".c_q", g["c_q"][b][rows], r["c_q"], dt, report)
-        compare(tag + ".q", g["q"][b][rows], r["q_abs"], dt, report)
+        if "q" in g:
+            compare(tag + ".q", g["q"][b][rows], r["q_abs"], dt, report)
         compare(tag + ".o", g["o"][b][rows], r["o"], dt, report)
         if "o_lat" in g:
             compare(tag + ".o_lat", g["o_lat"][b][rows], r["o_lat"], dt, report)

@@ -160,6 +160,51 @@ def test_pair_and_single_cta_attention_agree_on_config1():
         assert np.linalg.norm(a - b) / np.linalg.norm(b) <= 1e-3, k
 
 
+FUSED_Q_SHAPES = [(dc, dr) for dc in (128, 192) for dr in (16, 32, 64)]
+
+
+@pytest.mark.parametrize("d_c,d_rope", FUSED_Q_SHAPES)
+def test_fused_query_heads_match_the_q_gemm(d_c, d_rope):
+    """mla_attention_fwd_from_cq forms each CTA's query tile inside the attention kernel (c_Q x
+    w_qcat[h] on the tensor cores, 3D-RoPE, one rounding to bf16) instead of reading Q' from the
+    Q' GEMM.  Same operands, same fp32 accumulation order, same rotation code: outputs and lse
+    agree with mla_project_chunk + mla_attention_fwd to the last place (checked to a bf16 ulp),
+    over a 4-chunk rollout whose ring wraps, with and without the W_UV epilogue; and both match
+    the oracle."""
+    cfg = inputs.with_latent_shape(inputs.small_bf16_config(), d_c, d_rope)
+    a, f = GpuRun(cfg), GpuRun(cfg)
+    o = OracleRun(cfg, a.lw)
+    rows = np.arange(cfg.n_q)
+    identical = True
+    for ch in range(cfg.n_chunks):
+        x = inputs.chunk_x(cfg, ch)
+        ra = a.attend(ch, x)
+        rf = f.attend(ch, x, fused_q=True)
+        for k in ("o", "o_lat", "lse", "c_q", "chunk_lat"):
+            err = np.abs(ra[k] - rf[k])
+            identical = identical and bool((err == 0).all())
+            assert err.max() <= 2.0 ** -8 * max(1.0, np.abs(ra[k]).max()), (ch, k, err.max())
+        check_chunk(f"fused.chunk{ch}", cfg, rf, o.step(ch, x, rows), rows)
+        a.append(ch)
+        f.append(ch)
+    print("fused query heads bit-identical to the Q' GEMM path:", identical)
+
+
+def test_fused_query_heads_config1_sampled_rows():
+    """The bench's step on config 1 (query heads formed in the attention kernel): 384 sampled
+    rows against the oracle, and every row against the unfused path."""
+    cfg = inputs.CONFIGS[1]
+    g, o = prefilled(cfg, api.MLA_PATH_AUTO, cfg.measured_chunk)
+    ch = cfg.measured_chunk
+    x = inputs.chunk_x(cfg, ch)
+    rows = inputs.sample_rows(cfg.n_q, 384, tag=1)
+    rf = g.attend(ch, x, fused_q=True)
+    check_chunk("cfg1.fused", cfg, rf, o.step(ch, x, rows, append=False), rows)
+    ra = g.attend(ch, x)
+    for k in ("o", "o_lat", "lse"):
+        assert np.abs(ra[k] - rf[k]).max() <= 2.0 ** -8 * max(1.0, np.abs(ra[k]).max()), k
+
+
 def test_tensor_core_and_cuda_core_paths_agree_on_config1():
     """Diagnostic cross-check on every row of config 1 (GPU against GPU)."""
     cfg = inputs.CONFIGS[1]
