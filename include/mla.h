@@ -324,6 +324,16 @@ mla_status mla_attention_fwd_from_cq(const mla_config* cfg, const void* c_q, con
                                      int32_t first_frame, const void* w_uv, void* out, float* lse,
                                      void* workspace, size_t workspace_bytes,
                                      int32_t* dev_status, void* stream);
+/* mla_attention_fwd_from_cq_cached_ring: mla_attention_fwd_from_cq for a workspace whose ring
+ * part already holds the rotated ring keys (mla_rotate_ring_keys, same cache, slot_frame and
+ * n_valid_frames, unchanged since), as mla_attention_fwd_cached_ring is to mla_attention_fwd:
+ * only the chunk's own positional keys are rotated.  Arguments, results and errors as in
+ * mla_attention_fwd_from_cq. */
+mla_status mla_attention_fwd_from_cq_cached_ring(
+    const mla_config* cfg, const void* c_q, const void* w_qcat, const void* chunk_lat,
+    const void* cache, const int32_t* slot_frame, int32_t n_valid_frames, int32_t first_frame,
+    const void* w_uv, void* out, float* lse, void* workspace, size_t workspace_bytes,
+    int32_t* dev_status, void* stream);
 
 /* --------------------------------------------------------------------------------------------
  * Frozen-ring attention.  While a chunk is denoised in several steps, every step attends to the

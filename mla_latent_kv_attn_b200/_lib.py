@@ -69,6 +69,8 @@ SIGNATURES = {
     "mla_project_latents": (c_int32, [_CFG, _P, _P, _P, _P, _P]),
     "mla_attention_fwd_from_cq": (c_int32, [_CFG, _P, _P, _P, _P, _P, c_int32, c_int32, _P, _P,
                                             _P, _P, c_size_t, _P, _P]),
+    "mla_attention_fwd_from_cq_cached_ring": (c_int32, [_CFG, _P, _P, _P, _P, _P, c_int32, c_int32,
+                                                        _P, _P, _P, _P, c_size_t, _P, _P]),
     "mla_attention_workspace_bytes": (c_size_t, [_CFG, c_int32]),
     "mla_attention_uses_tensor_cores": (c_int32, [_CFG, c_int32]),
     "mla_attention_bwd_workspace_bytes": (c_size_t, [_CFG, c_int32]),

@@ -195,15 +195,18 @@ def mla_attention_fwd(c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_fr
 
 def mla_attention_fwd_from_cq(c: MLAConfigC, c_q, w_qcat, chunk_lat, cache, slot_frame,
                               n_valid_frames: int, first_frame: int, w_uv, out, lse=None,
-                              workspace=None, dev_status=None, stream=None) -> None:
+                              workspace=None, dev_status=None, stream=None,
+                              cached_ring: bool = False) -> None:
     """mla_attention_fwd with the query heads (and their 3D-RoPE) formed inside the attention
-    kernel from the query latent c_q and the composed weights w_qcat."""
+    kernel from the query latent c_q and the composed weights w_qcat.  cached_ring: the
+    workspace already holds the ring's rotated keys (mla_rotate_ring_keys)."""
+    fn = "mla_attention_fwd_from_cq_cached_ring" if cached_ring else "mla_attention_fwd_from_cq"
     tpf, n_q, D = _geom(c)
     dt = torch_dtype(c)
     B, H = c.batch, c.n_heads
     out_shape = (B, n_q, H * c.d_head) if w_uv is not None else (B, n_q, H, c.d_c)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = _lib.lib().mla_attention_fwd_from_cq(
+    st = getattr(_lib.lib(), fn)(
         ctypes.byref(c), _ptr(c_q, "c_q", dt, (B, n_q, c.d_cq)),
         _ptr(w_qcat, "w_qcat", dt, (H, D, c.d_cq)), _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)),
         _ptr(cache, "cache", dt, (B, c.window_frames * tpf, D)),
@@ -211,7 +214,7 @@ def mla_attention_fwd_from_cq(c: MLAConfigC, c_q, w_qcat, chunk_lat, cache, slot
         first_frame, _ptr(w_uv, "w_uv", dt, (H, c.d_head, c.d_c)), _ptr(out, "out", dt, out_shape),
         _ptr(lse, "lse", torch.float32, (B, H, n_q)), _ptr(workspace, "workspace"), ws_bytes,
         _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
-    _lib.check("mla_attention_fwd_from_cq", st)
+    _lib.check(fn, st)
 
 
 def mla_attention_fwd_cached_ring(c: MLAConfigC, q, chunk_lat, cache, slot_frame,

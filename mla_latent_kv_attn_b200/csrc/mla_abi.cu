@@ -212,6 +212,44 @@ mla_status attention_entry(const mla_config* cfg, const void* q, const void* chu
   return attention_dispatch(d, a, n_valid_frames, s);
 }
 
+// Shared body of the attention-from-query-latent entry points (query heads formed inside the
+// attention kernel); rope_part as in attention_entry.
+mla_status attention_from_cq_entry(const mla_config* cfg, const void* c_q, const void* w_qcat,
+                                   const void* chunk_lat, const void* cache,
+                                   const int32_t* slot_frame, int32_t n_valid_frames,
+                                   int32_t first_frame, const void* w_uv, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                   void* stream, int rope_part) {
+  set_last_error("");
+  MLA_TRY(check_cfg(cfg));
+  const Dims d = dims_of(*cfg);
+  MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
+                d.W);
+  MLA_TRY(check_first_frame(first_frame, d.C));
+  if (!(use_tc(d) && tc_attention_fused_q_supported(d, w_uv != nullptr)))
+    MLA_FAIL(MLA_ERR_UNSUPPORTED,
+             "attention from the query latent needs the tensor-core path (bf16, d_c <= 192, "
+             "d_c + d_rope <= 256, d_cq a multiple of 64); use mla_project_chunk and "
+             "mla_attention_fwd");
+  MLA_TRY(check_ptr(c_q, "c_q"));
+  MLA_TRY(check_ptr(w_qcat, "w_qcat"));
+  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
+  MLA_TRY(check_ptr(slot_frame, "slot_frame"));
+  MLA_TRY(check_ptr(out, "out"));
+  MLA_TRY(check_ptr(cache, "cache", n_valid_frames > 0));
+  MLA_TRY(check_ptr(w_uv, "w_uv", false));
+  MLA_TRY(check_ptr(lse, "lse", false));
+  MLA_TRY(check_ptr(dev_status, "dev_status", false));
+  MLA_TRY(check_workspace(d, n_valid_frames, workspace, workspace_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MLA_TRY(build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid_frames, first_frame, workspace,
+                          s, rope_part, dev_status, 1));
+  AttnArgs a{};
+  a.q = nullptr; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = workspace; a.w_uv = w_uv;
+  a.out = out; a.lse = lse; a.dev_status = dev_status;
+  return attention_tc_fused_q(d, a, n_valid_frames, c_q, w_qcat, first_frame, s);
+}
+
 }  // namespace
 
 mla_status attention_dispatch(const Dims& d, const AttnArgs& a, int n_valid, cudaStream_t s) {
@@ -443,34 +481,20 @@ mla_status mla_attention_fwd_from_cq(const mla_config* cfg, const void* c_q, con
                                      void* workspace, size_t workspace_bytes,
                                      int32_t* dev_status, void* stream) {
   MLA_NVTX_RANGE("mla_attention_fwd_from_cq");
-  set_last_error("");
-  MLA_TRY(check_cfg(cfg));
-  const Dims d = dims_of(*cfg);
-  MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
-                d.W);
-  MLA_TRY(check_first_frame(first_frame, d.C));
-  if (!(use_tc(d) && tc_attention_fused_q_supported(d, w_uv != nullptr)))
-    MLA_FAIL(MLA_ERR_UNSUPPORTED,
-             "attention from the query latent needs the tensor-core path (bf16, d_c <= 192, "
-             "d_c + d_rope <= 256, d_cq a multiple of 64); use mla_project_chunk and "
-             "mla_attention_fwd");
-  MLA_TRY(check_ptr(c_q, "c_q"));
-  MLA_TRY(check_ptr(w_qcat, "w_qcat"));
-  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
-  MLA_TRY(check_ptr(slot_frame, "slot_frame"));
-  MLA_TRY(check_ptr(out, "out"));
-  MLA_TRY(check_ptr(cache, "cache", n_valid_frames > 0));
-  MLA_TRY(check_ptr(w_uv, "w_uv", false));
-  MLA_TRY(check_ptr(lse, "lse", false));
-  MLA_TRY(check_ptr(dev_status, "dev_status", false));
-  MLA_TRY(check_workspace(d, n_valid_frames, workspace, workspace_bytes));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  MLA_TRY(build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid_frames, first_frame, workspace,
-                          s, kRopeKeysAll, dev_status, 1));
-  AttnArgs a{};
-  a.q = nullptr; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = workspace; a.w_uv = w_uv;
-  a.out = out; a.lse = lse; a.dev_status = dev_status;
-  return attention_tc_fused_q(d, a, n_valid_frames, c_q, w_qcat, first_frame, s);
+  return attention_from_cq_entry(cfg, c_q, w_qcat, chunk_lat, cache, slot_frame, n_valid_frames,
+                                 first_frame, w_uv, out, lse, workspace, workspace_bytes,
+                                 dev_status, stream, kRopeKeysAll);
+}
+
+mla_status mla_attention_fwd_from_cq_cached_ring(
+    const mla_config* cfg, const void* c_q, const void* w_qcat, const void* chunk_lat,
+    const void* cache, const int32_t* slot_frame, int32_t n_valid_frames, int32_t first_frame,
+    const void* w_uv, void* out, float* lse, void* workspace, size_t workspace_bytes,
+    int32_t* dev_status, void* stream) {
+  MLA_NVTX_RANGE("mla_attention_fwd_from_cq_cached_ring");
+  return attention_from_cq_entry(cfg, c_q, w_qcat, chunk_lat, cache, slot_frame, n_valid_frames,
+                                 first_frame, w_uv, out, lse, workspace, workspace_bytes,
+                                 dev_status, stream, kRopeKeysChunk);
 }
 
 mla_status mla_attention_fwd_cached_ring(const mla_config* cfg, const void* q,

@@ -304,8 +304,11 @@ class LayerStack:
     appends) as one CUDA graph, with the step/layer inputs bound at capture time.
     """
 
-    def __init__(self, c, weights, device="cuda", fuse_uv: bool = True):
+    def __init__(self, c, weights, device="cuda", fuse_uv: bool = True,
+                 fused_q: Optional[bool] = None):
         self.c = c
+        # the query heads formed inside the attention kernel where the configuration allows
+        self.fused_q = fused_query_supported(c) if fused_q is None else fused_q
         self.w = list(weights)
         self.rings = [Ring(c, device=device) for _ in self.w]
         ws = max(api.mla_attention_workspace_bytes(c, c.window_frames), 256)
@@ -331,11 +334,21 @@ class LayerStack:
         chunk's latents afterwards.  Returns buf.o (or buf.o_lat without the W_UV epilogue)."""
         c, b, w, ring = self.c, self.buf, self.w[layer], self.rings[layer]
         first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
-        api.mla_project_chunk(c, x, w.w_x, w.w_qcat, b.c_q, b.q, b.chunk_lat, first, stream=stream)
         out = b.o if self.fuse_uv else b.o_lat
-        api.mla_attention_fwd_cached_ring(c, b.q, b.chunk_lat, ring.cache, ring.slot_frame, n_valid,
-                                          first, w.w_uv if self.fuse_uv else None, out, b.lse,
-                                          self.ws[layer], b.dev_status, stream=stream)
+        if self.fused_q:
+            api.mla_project_latents(c, x, w.w_x, b.c_q, b.chunk_lat, stream=stream)
+            api.mla_attention_fwd_from_cq(c, b.c_q, w.w_qcat, b.chunk_lat, ring.cache,
+                                          ring.slot_frame, n_valid, first,
+                                          w.w_uv if self.fuse_uv else None, out, b.lse,
+                                          self.ws[layer], b.dev_status, stream=stream,
+                                          cached_ring=True)
+        else:
+            api.mla_project_chunk(c, x, w.w_x, w.w_qcat, b.c_q, b.q, b.chunk_lat, first,
+                                  stream=stream)
+            api.mla_attention_fwd_cached_ring(c, b.q, b.chunk_lat, ring.cache, ring.slot_frame,
+                                              n_valid, first, w.w_uv if self.fuse_uv else None,
+                                              out, b.lse, self.ws[layer], b.dev_status,
+                                              stream=stream)
         if append:
             api.mla_cache_append(c, None, None, b.chunk_lat, ring.cache, ring.slot_frame, first,
                                  MLA_APPEND, stream=stream)

@@ -383,6 +383,30 @@ def test_layer_stack_graph_matches_eager():
     rollout.check_device_status(graphed.buf)
 
 
+def test_layer_stack_fused_query_matches_q_gemm():
+    """The layer stack's cached-ring attention with the query heads formed inside the kernel
+    (mla_attention_fwd_from_cq_cached_ring) against mla_project_chunk +
+    mla_attention_fwd_cached_ring: identical rings and outputs over 4 chunks (rings wrap)."""
+    cfg = inputs.small_bf16_config()
+    c = api.make_config(cfg)
+    n_layers, n_steps = 2, 2
+    lws = [inputs.layer_weights(cfg, l) for l in range(n_layers)]
+    xs = {(ch, s, l): torch.from_numpy(inputs.chunk_x(cfg, ch, s, l)).to(torch.bfloat16).cuda()
+          for ch in range(cfg.n_chunks) for s in range(n_steps) for l in range(n_layers)}
+    fused = rollout.LayerStack(c, [rollout.upload_weights(c, lw) for lw in lws], fused_q=True)
+    plain = rollout.LayerStack(c, [rollout.upload_weights(c, lw) for lw in lws], fused_q=False)
+    for ch in range(cfg.n_chunks):
+        x_of = lambda s, l, ch=ch: xs[(ch, s, l)]
+        fused.run_chunk(ch, n_steps, x_of)
+        plain.run_chunk(ch, n_steps, x_of)
+        torch.cuda.synchronize()
+        a, b = fused.buf.o.float(), plain.buf.o.float()
+        assert (a - b).abs().max().item() <= 2.0 ** -8 * max(1.0, b.abs().max().item()), ch
+        for l in range(n_layers):
+            assert torch.equal(fused.rings[l].cache, plain.rings[l].cache), (ch, l)
+    rollout.check_device_status(fused.buf)
+
+
 def test_standalone_rope3d_and_out_proj():
     cfg = inputs.small_bf16_config()
     g = GpuRun(cfg, api.MLA_PATH_AUTO)
