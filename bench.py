@@ -700,9 +700,10 @@ def run_stack(args, cfg):
                      "peak_kind": f"{peak_kind} sustained bf16",
                      "frac_of_burst": value / peaks["bf16_tflops"]},
         "e2e": None,
-        # per call: x-projection GEMM, Q' GEMM, chunk-key rotation, attention; per chunk and
-        # layer: the ring-key rotation (chunks with a non-empty window) and the append
-        "gpu_launches": steps * (calls * 4 + cfg.n_layers * (
+        # per call: x-projection GEMM, [Q' GEMM,] chunk-key rotation, attention (with the query
+        # heads formed inside it where supported); per chunk and layer: the ring-key rotation
+        # (chunks with a non-empty window) and the append
+        "gpu_launches": steps * (calls * (3 if stack.fused_q else 4) + cfg.n_layers * (
             cfg.n_chunks + sum(1 for ch in range(cfg.n_chunks) if cfg.valid_frames(ch) > 0))),
         "clocks": dict(clk.summary(), sm_mhz_device=clock_after()),
     }
