@@ -4,13 +4,14 @@
 
 One step = one chunk of an autoregressive rollout through the whole path, on one batch of
 synthetic Wan2.1-1.3B-shaped input (the 6-frame window full, a 3-frame chunk of 4680 queries):
-the projections of the chunk (query latent and chunk latents in one pass over x, then the
-absorbed query heads with fused 3D-RoPE), attention over the ring plus the chunk with the W_UV
-up-projection fused, and the ring append.  Steps advance
-the rollout (chunk 2, 3, 4, ... of a 6-frame window), so every step has the same work.
+the down-projections of the chunk (query latent and chunk latents in one pass over x), the
+rotated-key pre-pass, attention over the ring plus the chunk with the absorbed query heads
+(and their 3D-RoPE) formed inside the attention kernel and the W_UV up-projection fused, and
+the ring append.  (--unfused-query runs the query heads as their own GEMM instead.)  Steps
+advance the rollout (chunk 2, 3, 4, ... of a 6-frame window), so every step has the same work.
 
 Timing: W untimed warm-up steps, then K steps between a barrier + device synchronisation on
-both sides.  Each step's five kernels are captured beforehand as one CUDA graph per chunk
+both sides.  Each step's four kernels are captured beforehand as one CUDA graph per chunk
 (rollout.ChunkGraph) and replayed, so the device runs them back to back.  L2 is flushed before
 every step (a 256 MiB device memset, outside the per-step CUDA-event intervals).  Device time
 per step = sum of per-step event intervals on the launch stream; the job time is the max over
