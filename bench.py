@@ -542,7 +542,10 @@ def run_ours(args, cfg):
         else None
     # the step's three calls, timed by events inside the step graphs (means over the timed steps)
     n_x = cfg.d_cq + cfg.d_latent
-    proj_flops = 2.0 * cfg.batch * cfg.n_q * (cfg.d_model * n_x + cfg.d_cq * cfg.n_heads * cfg.d_latent)
+    # with the query heads formed inside the attention kernel the projection call is the
+    # x-projection alone; otherwise it also runs the Q' GEMM
+    proj_flops = 2.0 * cfg.batch * cfg.n_q * (
+        cfg.d_model * n_x + (0 if fused_q else cfg.d_cq * cfg.n_heads * cfg.d_latent))
     app_bytes = 2.0 * cfg.batch * cfg.n_q * cfg.d_latent * 2
     step_breakdown = {
         "projections_us": 1e3 * statistics.mean(proj_ms),
