@@ -4,14 +4,15 @@
 
 One step = one chunk of an autoregressive rollout through the whole path, on one batch of
 synthetic Wan2.1-1.3B-shaped input (the 6-frame window full, a 3-frame chunk of 4680 queries):
-the down-projections of the chunk (query latent and chunk latents in one pass over x), the
-rotated-key pre-pass, attention over the ring plus the chunk with the absorbed query heads
-(and their 3D-RoPE) formed inside the attention kernel and the W_UV up-projection fused, and
-the ring append.  (--unfused-query runs the query heads as their own GEMM instead.)  Steps
+the down-projections of the chunk (query latent and chunk latents in one pass over x, whose
+epilogue also writes the rotated positional keys of the ring and the chunk), attention over the
+ring plus the chunk with the absorbed query heads (and their 3D-RoPE) formed inside the
+attention kernel and the W_UV up-projection fused, and the ring append: three kernels.
+(--unfused-query runs the query heads as their own GEMM and the key rotation as its own pass.)  Steps
 advance the rollout (chunk 2, 3, 4, ... of a 6-frame window), so every step has the same work.
 
 Timing: W untimed warm-up steps, then K steps between a barrier + device synchronisation on
-both sides.  Each step's four kernels are captured beforehand as one CUDA graph per chunk
+both sides.  Each step's three kernels are captured beforehand as one CUDA graph per chunk
 (rollout.ChunkGraph) and replayed, so the device runs them back to back.  L2 is flushed before
 every step (a 256 MiB device memset, outside the per-step CUDA-event intervals).  Device time
 per step = sum of per-step event intervals on the launch stream; the job time is the max over
@@ -22,7 +23,7 @@ value      attention algorithmic TFLOP/s of the whole step: 2*(D + d_c) = 832 fl
            (query row, attended key, head), divided by the whole-step device time
 e2e        the same metric through the public API with host buffers: pinned host -> device copy
            of the step's tokens and device -> host copy of its output inside the timed interval
-roofline   the attention call (rotated-key pre-pass + tensor-core kernel), timed with CUDA
+roofline   the attention call (the tensor-core kernel alone), timed with CUDA
            events recorded inside each step's graph around that call, against the measured
            bf16 peak
 cpu_baseline  the float64 CPU oracle on a bounded sample of the same chunk (rank 0, N = 1)
@@ -410,9 +411,9 @@ def run_ours(args, cfg):
     stream = torch.cuda.current_stream(dev)
     # the query heads formed inside the attention kernel where the shape allows
     fused_q = rollout.fused_query_supported(c) and not args.unfused_query
-    # x GEMM (c_Q || chunk latents), [Q' GEMM + RoPE,] rope-key pre-pass, attention (+W_UV),
-    # ring append
-    launches_per_step = 4 if fused_q else 5
+    # fused: x GEMM (c_Q || chunk latents || rotated keys), attention (+W_UV), ring append;
+    # otherwise x GEMM, Q' GEMM + RoPE, rotated-key pass, attention (+W_UV), ring append
+    launches_per_step = 3 if fused_q else 5
 
     first_chunk = cfg.measured_chunk
     flops_step = cfg.attention_flops(first_chunk)   # same for every later chunk (window full)
@@ -422,7 +423,9 @@ def run_ours(args, cfg):
         x = pool[i % n_pool] if x is None else x
         first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, ch)
         if fused_q:
-            api.mla_project_latents(c, x, w.w_x, buf.c_q, buf.chunk_lat)
+            api.mla_project_latents_rotated(c, x, w.w_x, buf.c_q, buf.chunk_lat, ring.cache,
+                                            ring.slot_frame, n_valid, first, buf.workspace,
+                                            dev_status=buf.dev_status)
         else:
             api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
         if ev is not None:
@@ -430,7 +433,7 @@ def run_ours(args, cfg):
         if fused_q:
             api.mla_attention_fwd_from_cq(c, buf.c_q, w.w_qcat, buf.chunk_lat, ring.cache,
                                           ring.slot_frame, n_valid, first, w.w_uv, buf.o, buf.lse,
-                                          buf.workspace, buf.dev_status)
+                                          buf.workspace, buf.dev_status, prerotated=True)
         else:
             api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame, n_valid,
                                   first, w.w_uv, buf.o, buf.lse, buf.workspace, buf.dev_status)
@@ -439,10 +442,13 @@ def run_ours(args, cfg):
         api.mla_cache_append(c, None, None, buf.chunk_lat, ring.cache, ring.slot_frame, first,
                              api.MLA_APPEND)
 
-    # Each step is one CUDA graph (rollout.ChunkGraph): the chunk's five kernels replay back to
-    # back without per-launch host overhead.  Graphs are captured before the timed region (host
-    # set-up, like encoding a plan); capturing launches nothing.
-    graphs = [rollout.ChunkGraph(c, w, ring, buf, first_chunk + i, x=pool[i % n_pool], events=True,
+    # Each step is one CUDA graph (rollout.ChunkGraph): the chunk's kernels replay back to back
+    # without per-launch host overhead, each kernel's set-up overlapping the previous kernel's
+    # tail (programmatic launches).  Graphs are captured before the timed region (host set-up,
+    # like encoding a plan); capturing launches nothing.  The per-call breakdown is measured
+    # afterwards on graphs of further chunks with timing events between the calls (an event
+    # between two kernels keeps the second from starting early, so the timed steps have none).
+    graphs = [rollout.ChunkGraph(c, w, ring, buf, first_chunk + i, x=pool[i % n_pool],
                                  fused_q=fused_q)
               for i in range(args.warmup + args.steps)]
     # warm-up
@@ -476,14 +482,26 @@ def run_ours(args, cfg):
     if world > 1:
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(ev_s, ev_e)]
-    attn_ms = [graphs[args.warmup + i].attention_ms() for i in range(args.steps)]
-    proj_ms = [graphs[args.warmup + i].projection_ms() for i in range(args.steps)]
-    app_ms = [graphs[args.warmup + i].append_ms() for i in range(args.steps)]
     sm_mhz_device = clock_after()
     total_ms = max_over_ranks(sum(step_ms), device=dev)
     status = int(buf.dev_status.item())
     if status != 0:
         raise RuntimeError(f"a kernel reported status {status}")
+    base = args.warmup + args.steps
+
+    # ---- the step's calls, timed by events recorded inside the step graphs (further chunks of
+    # the same rollout, same work per chunk)
+    bd_graphs = [rollout.ChunkGraph(c, w, ring, buf, first_chunk + base + i, x=pool[i % n_pool],
+                                    events=True, fused_q=fused_q) for i in range(args.steps)]
+    for g in bd_graphs:
+        flush.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    attn_ms = [g.attention_ms() for g in bd_graphs]
+    proj_ms = [g.projection_ms() for g in bd_graphs]
+    app_ms = [g.append_ms() for g in bd_graphs]
+    base += args.steps
+    del bd_graphs
 
     # ---- end to end through the public API with host buffers
     # Pinned host tokens in, pinned host output back, every copy inside the timed interval.
@@ -495,7 +513,6 @@ def run_ours(args, cfg):
     o_host = [torch.empty(buf.o.shape, dtype=buf.o.dtype).pin_memory() for _ in range(2)]
     h2d = x_host[0].numel() * x_host[0].element_size()
     d2h = o_host[0].numel() * o_host[0].element_size()
-    base = args.warmup + args.steps
     streamer = rollout.HostStreamer(c, w, ring, device=dev, compute_stream=stream)
     for i in range(args.warmup):          # warm the streamer's own buffers and streams
         flush.zero_()
@@ -554,9 +571,9 @@ def run_ours(args, cfg):
         "append_us": 1e3 * statistics.mean(app_ms),
         "append_gbs": app_bytes / (statistics.mean(app_ms) * 1e-3) / 1e9,
         "step_us": 1e3 * statistics.mean(step_ms),
-        "calls": ("mla_project_latents (x-projection GEMM) | mla_attention_fwd_from_cq "
-                  "(rotated-key pre-pass + attention with the query heads formed inside it) | "
-                  "mla_cache_append(MLA_APPEND)") if fused_q else
+        "calls": ("mla_project_latents_rotated (x-projection GEMM, rotated keys from its "
+                  "epilogue) | mla_attention_fwd_from_cq_prerotated (attention with the query "
+                  "heads formed inside it) | mla_cache_append(MLA_APPEND)") if fused_q else
                  ("mla_project_chunk (x-projection GEMM, Q' GEMM + RoPE) | mla_attention_fwd "
                   "(rotated-key pre-pass + attention) | mla_cache_append(MLA_APPEND)")}
     n_units_all = world * cfg.batch
@@ -589,10 +606,11 @@ def run_ours(args, cfg):
         "attention_call_ms": attn_avg_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": ("mla_attention_fwd_from_cq" if fused_q else "mla_attention_fwd") +
-                               " (rotated-key pre-pass + " +
-                               ("attention_pair_kernel" if args.kernel_path == "pair" and cfg.n_heads % 2 == 0
-                                and cfg.d_c in (128, 192) else "attention_tc_kernel") + ")",
+                     "kernel": ("mla_attention_fwd_from_cq_prerotated (attention_tc_kernel)"
+                                if fused_q else "mla_attention_fwd (rotated-key pre-pass + " +
+                                ("attention_pair_kernel" if args.kernel_path == "pair"
+                                 and cfg.n_heads % 2 == 0 and cfg.d_c in (128, 192)
+                                 else "attention_tc_kernel") + ")"),
                      "peak_kind": f"{peak_kind} burst bf16",
                      "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
         "e2e": {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12,
@@ -704,10 +722,11 @@ def run_stack(args, cfg):
                      "peak_kind": f"{peak_kind} sustained bf16",
                      "frac_of_burst": value / peaks["bf16_tflops"]},
         "e2e": None,
-        # per call: x-projection GEMM, [Q' GEMM,] chunk-key rotation, attention (with the query
-        # heads formed inside it where supported); per chunk and layer: the ring-key rotation
-        # (chunks with a non-empty window) and the append
-        "gpu_launches": steps * (calls * (3 if stack.fused_q else 4) + cfg.n_layers * (
+        # per call: x-projection GEMM (with the chunk-key rotation in its epilogue) and attention
+        # with the query heads formed inside it where supported, else x-projection, Q' GEMM,
+        # chunk-key rotation and attention; per chunk and layer: the ring-key rotation (chunks
+        # with a non-empty window) and the append
+        "gpu_launches": steps * (calls * (2 if stack.fused_q else 4) + cfg.n_layers * (
             cfg.n_chunks + sum(1 for ch in range(cfg.n_chunks) if cfg.valid_frames(ch) > 0))),
         "clocks": dict(clk.summary(), sm_mhz_device=clock_after()),
     }

@@ -23,7 +23,11 @@
  *   exception is mla_attention_fwd_static_scratch: it uses a fixed array built into the library
  *   (reserved on every device that loads it) and keeps that array's device address (below).
  * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All work is
- *   enqueued on it, asynchronously.
+ *   enqueued on it, asynchronously.  The forward path's kernels are launched with programmatic
+ *   stream serialisation: each may begin its set-up while the previous kernel on the stream
+ *   drains and waits for that kernel's completion before it touches memory, so stream order is
+ *   kept.  Setting the environment variable MLA_NO_PDL (read once per process) launches them
+ *   plainly.
  * - Arguments are checked on the host before anything is launched.  A rejected call returns a
  *   non-zero mla_status, launches nothing and leaves every buffer untouched;
  *   mla_last_error() then describes the problem.  A launch that fails returns MLA_ERR_CUDA.
@@ -251,6 +255,36 @@ mla_status mla_project_chunk(const mla_config* cfg, const void* x, const void* w
 mla_status mla_project_latents(const mla_config* cfg, const void* x, const void* w_x, void* c_q,
                                void* chunk_lat, void* stream);
 
+/* --------------------------------------------------------------------------------------------
+ * mla_project_latents_rotated: mla_project_latents that also prepares the rotated positional
+ * keys of the chunk's attention ([M]: k_R is cached unrotated and rotated by 3D-RoPE when the
+ * chunk's attention runs), so that mla_attention_fwd_from_cq_prerotated needs no rotation pass.
+ * Into `workspace` (the layout of mla_attention_workspace_bytes(cfg, n_valid_frames)) it writes
+ * RoPE3D of every chunk token's k_R, as chunk_lat stores it, at the token's position (frame
+ * first_frame + frame within the chunk), and the zero padding after the chunk; with
+ * rotate_ring = 1 also RoPE3D of ring slots 0 .. n_valid_frames*tpf - 1 (t from slot_frame) and
+ * the ring part's padding, exactly as mla_rotate_ring_keys does; with rotate_ring = 0 the ring
+ * part is left as it is (a frozen ring whose keys mla_rotate_ring_keys rotated already).  On the
+ * tensor-core path (bf16, d_cq and d_cq + d_c multiples of 32, d_rope in {16, 32, 64}) this is
+ * one kernel: the projection GEMM's epilogue writes the chunk's rotated keys and its idle
+ * epilogue warps rotate the ring's while the first tile's MMAs run; otherwise the projection
+ * GEMMs and the rotation pass run one after the other, with the same results.
+ *   x, w_x, c_q, chunk_lat   as in mla_project_latents
+ *   cache, slot_frame        as in mla_attention_fwd (cache may be NULL when rotate_ring = 0 or
+ *                            n_valid_frames = 0)
+ *   n_valid_frames, first_frame  of the chunk's attention call
+ *   workspace, workspace_bytes   the attention call's workspace, 256-byte aligned
+ *   dev_status               as in mla_attention_fwd (MLA_DEBUG builds check the ring slots), or
+ *                            NULL
+ * Errors: MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+mla_status mla_project_latents_rotated(const mla_config* cfg, const void* x, const void* w_x,
+                                       void* c_q, void* chunk_lat, const void* cache,
+                                       const int32_t* slot_frame, int32_t n_valid_frames,
+                                       int32_t first_frame, int32_t rotate_ring, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status,
+                                       void* stream);
+
 /* mla_attention_uses_tensor_cores: 1 if mla_attention_fwd with this configuration (and with the
  * W_UV epilogue when with_w_uv != 0) runs the tcgen05 tensor-core kernel, 0 if it runs the
  * CUDA-core kernel, -1 for an invalid configuration.  The tensor-core kernel covers bf16 with
@@ -330,6 +364,16 @@ mla_status mla_attention_fwd_from_cq(const mla_config* cfg, const void* c_q, con
  * only the chunk's own positional keys are rotated.  Arguments, results and errors as in
  * mla_attention_fwd_from_cq. */
 mla_status mla_attention_fwd_from_cq_cached_ring(
+    const mla_config* cfg, const void* c_q, const void* w_qcat, const void* chunk_lat,
+    const void* cache, const int32_t* slot_frame, int32_t n_valid_frames, int32_t first_frame,
+    const void* w_uv, void* out, float* lse, void* workspace, size_t workspace_bytes,
+    int32_t* dev_status, void* stream);
+/* mla_attention_fwd_from_cq_prerotated: mla_attention_fwd_from_cq for a workspace that already
+ * holds every rotated positional key of the call (mla_project_latents_rotated with the same
+ * chunk_lat, cache, slot_frame, n_valid_frames and first_frame, none changed since): the
+ * attention kernel alone runs, with no rotation pass.  Results are bit-identical to
+ * mla_attention_fwd_from_cq.  Arguments, results and errors as in mla_attention_fwd_from_cq. */
+mla_status mla_attention_fwd_from_cq_prerotated(
     const mla_config* cfg, const void* c_q, const void* w_qcat, const void* chunk_lat,
     const void* cache, const int32_t* slot_frame, int32_t n_valid_frames, int32_t first_frame,
     const void* w_uv, void* out, float* lse, void* workspace, size_t workspace_bytes,

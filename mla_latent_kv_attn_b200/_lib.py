@@ -67,6 +67,11 @@ SIGNATURES = {
     "mla_query_proj": (c_int32, [_CFG, _P, _P, _P, _P, _P, c_int32, _P]),
     "mla_project_chunk": (c_int32, [_CFG, _P, _P, _P, _P, _P, _P, c_int32, _P]),
     "mla_project_latents": (c_int32, [_CFG, _P, _P, _P, _P, _P]),
+    "mla_project_latents_rotated": (c_int32, [_CFG, _P, _P, _P, _P, _P, _P, c_int32, c_int32,
+                                              c_int32, _P, c_size_t, _P, _P]),
+    "mla_attention_fwd_from_cq_prerotated": (c_int32, [_CFG, _P, _P, _P, _P, _P, c_int32,
+                                                       c_int32, _P, _P, _P, _P, c_size_t, _P,
+                                                       _P]),
     "mla_attention_fwd_from_cq": (c_int32, [_CFG, _P, _P, _P, _P, _P, c_int32, c_int32, _P, _P,
                                             _P, _P, c_size_t, _P, _P]),
     "mla_attention_fwd_from_cq_cached_ring": (c_int32, [_CFG, _P, _P, _P, _P, _P, c_int32, c_int32,

@@ -19,7 +19,7 @@ __all__ = [
     "make_config", "torch_dtype", "mla_config_check", "mla_cache_append", "mla_rope3d",
     "mla_key_positions", "mla_compose_query_weights", "mla_query_proj", "mla_project_chunk",
     "mla_attention_workspace_bytes", "mla_attention_fwd", "mla_attention_fwd_static_scratch",
-    "mla_project_latents", "mla_attention_fwd_from_cq",
+    "mla_project_latents", "mla_project_latents_rotated", "mla_attention_fwd_from_cq",
     "mla_rotate_ring_keys", "mla_attention_fwd_cached_ring", "mla_attention_uses_tensor_cores",
     "mla_attention_bwd_workspace_bytes", "mla_attention_bwd",
     "mla_out_proj", "MLAError",
@@ -158,6 +158,27 @@ def mla_project_latents(c: MLAConfigC, x, w_x, c_q, chunk_lat, stream=None) -> N
     _lib.check("mla_project_latents", st)
 
 
+def mla_project_latents_rotated(c: MLAConfigC, x, w_x, c_q, chunk_lat, cache, slot_frame,
+                                n_valid_frames: int, first_frame: int, workspace,
+                                rotate_ring: bool = True, dev_status=None, stream=None) -> None:
+    """mla_project_latents that also writes the chunk attention's rotated positional keys into
+    `workspace` (the ring's too with rotate_ring), for mla_attention_fwd_from_cq(...,
+    prerotated=True)."""
+    tpf, n_q, D = _geom(c)
+    dt = torch_dtype(c)
+    B = c.batch
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib.lib().mla_project_latents_rotated(
+        ctypes.byref(c), _ptr(x, "x", dt, (B, n_q, c.d_model)),
+        _ptr(w_x, "w_x", dt, (c.d_cq + D, c.d_model)), _ptr(c_q, "c_q", dt, (B, n_q, c.d_cq)),
+        _ptr(chunk_lat, "chunk_lat", dt, (B, n_q, D)),
+        _ptr(cache, "cache", dt, (B, c.window_frames * tpf, D)),
+        _ptr(slot_frame, "slot_frame", torch.int32, (B, c.window_frames)), n_valid_frames,
+        first_frame, 1 if rotate_ring else 0, _ptr(workspace, "workspace"), ws_bytes,
+        _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    _lib.check("mla_project_latents_rotated", st)
+
+
 def mla_attention_uses_tensor_cores(c: MLAConfigC, with_w_uv: bool = True) -> bool:
     r = int(_lib.lib().mla_attention_uses_tensor_cores(ctypes.byref(c), 1 if with_w_uv else 0))
     if r < 0:
@@ -196,11 +217,15 @@ def mla_attention_fwd(c: MLAConfigC, q, chunk_lat, cache, slot_frame, n_valid_fr
 def mla_attention_fwd_from_cq(c: MLAConfigC, c_q, w_qcat, chunk_lat, cache, slot_frame,
                               n_valid_frames: int, first_frame: int, w_uv, out, lse=None,
                               workspace=None, dev_status=None, stream=None,
-                              cached_ring: bool = False) -> None:
+                              cached_ring: bool = False, prerotated: bool = False) -> None:
     """mla_attention_fwd with the query heads (and their 3D-RoPE) formed inside the attention
     kernel from the query latent c_q and the composed weights w_qcat.  cached_ring: the
-    workspace already holds the ring's rotated keys (mla_rotate_ring_keys)."""
-    fn = "mla_attention_fwd_from_cq_cached_ring" if cached_ring else "mla_attention_fwd_from_cq"
+    workspace already holds the ring's rotated keys (mla_rotate_ring_keys); prerotated: it holds
+    every rotated key of the call (mla_project_latents_rotated), so no rotation pass runs."""
+    if cached_ring and prerotated:
+        raise ValueError("cached_ring and prerotated are exclusive")
+    fn = ("mla_attention_fwd_from_cq_prerotated" if prerotated else
+          "mla_attention_fwd_from_cq_cached_ring" if cached_ring else "mla_attention_fwd_from_cq")
     tpf, n_q, D = _geom(c)
     dt = torch_dtype(c)
     B, H = c.batch, c.n_heads

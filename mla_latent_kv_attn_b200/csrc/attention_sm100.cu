@@ -282,6 +282,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  // launched with programmatic serialisation: the set-up above may overlap the previous
+  // kernel's tail; nothing global is touched before it has completed
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
@@ -756,8 +760,8 @@ mla_status attention_tc_impl(const Dims& d, const AttnArgs& a, int n_valid, cuda
   MLA_CUDA_TRY(cudaFuncSetAttribute(attention_tc_kernel<DC, DR, kFusedQ>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmem));
   dim3 grid(ceil_div(d.n_q, kBM), d.H, d.B);
-  attention_tc_kernel<DC, DR, kFusedQ><<<grid, kThreads, Sh::kSmem, s>>>(tq, tqr, tcache, tchunk,
-                                                                      tws, twuv, tcq, twq, p);
+  MLA_CUDA_TRY(launch_pdl(attention_tc_kernel<DC, DR, kFusedQ>, grid, dim3(kThreads), Sh::kSmem,
+                          s, tq, tqr, tcache, tchunk, tws, twuv, tcq, twq, p));
   MLA_LAUNCH_CHECK("attention_tc");
   return MLA_OK;
 }

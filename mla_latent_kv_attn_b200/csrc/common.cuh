@@ -183,6 +183,99 @@ __device__ __forceinline__ void debug_check(bool ok, int32_t* dev_status) {
 #endif
 }
 
+// Rotated positional key of row r of sample b in the attention's key workspace (kPieces 16-byte
+// pieces of d_rope values per row):
+//   r <  nc                    ring slot r: RoPE3D of the cache row's k_R at its frame's position
+//   nc_pad <= r < nc_pad + n_q chunk token r - nc_pad (from chunk_lat)
+//   otherwise                  zeros (tile padding)
+// The unrotated values are read as stored (already rounded to T); each pair is rotated in fp32
+// and rounded once.  With MLA_DEBUG, ring slots must hold a frame (t >= 0) and, with
+// check_window, one of the chunk's window (first_frame - W <= t < first_frame).
+template <typename T, int kPieces>
+__device__ __forceinline__ void rope_key_row(const T* __restrict__ cache,
+                                             const T* __restrict__ chunk_lat,
+                                             const int32_t* __restrict__ slot_frame,
+                                             T* __restrict__ ws, int b, int r, int W, int D,
+                                             int d_c, int n_q, int nc, int nc_pad, int rows_ws,
+                                             int first_frame, const RopeGeom& g,
+                                             int32_t* dev_status, int check_window) {
+  constexpr int kPer = 16 / sizeof(T);          // elements per piece
+  constexpr int kDr = kPieces * kPer;
+  uint4* dst = reinterpret_cast<uint4*>(ws + (static_cast<int64_t>(b) * rows_ws + r) * kDr);
+  const T* src = nullptr;
+  int m = -1;
+  if (r < nc) {
+    m = r;
+    src = cache + (static_cast<int64_t>(b) * W * g.tpf + r) * D;
+  } else if (r >= nc_pad && r - nc_pad < n_q) {
+    m = nc + (r - nc_pad);
+    src = chunk_lat + (static_cast<int64_t>(b) * n_q + (r - nc_pad)) * D;
+  }
+  if (src == nullptr) {
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  uint4 raw[kPieces];
+  const uint4* s4 = reinterpret_cast<const uint4*>(src + d_c);
+#pragma unroll
+  for (int k = 0; k < kPieces; ++k) raw[k] = s4[k];
+  int t, h, w;
+  key_position(slot_frame, b, W, g.tpf, g.frame_w, nc, first_frame, m, t, h, w);
+  if (m < nc)
+    debug_check(t >= 0 && (!check_window || (t < first_frame && t >= first_frame - W)), dev_status);
+#pragma unroll
+  for (int k = 0; k < kPieces; ++k) {
+    T* x = reinterpret_cast<T*>(&raw[k]);
+#pragma unroll
+    for (int q = 0; q < kPer; q += 2) {
+      float x0 = Elem<T>::to_f(x[q]), x1 = Elem<T>::to_f(x[q + 1]);
+      rope_rotate(x0, x1, rope_angle(g, (k * kPer + q) / 2, t, h, w));
+      x[q] = Elem<T>::from_f(x0);
+      x[q + 1] = Elem<T>::from_f(x1);
+    }
+    dst[k] = raw[k];
+  }
+}
+
+// ---- programmatic dependent launch ---------------------------------------------------------
+// The forward path's kernels are launched with programmatic stream serialisation: a kernel's
+// CTAs may be scheduled while the previous kernel on the stream is still draining, set up
+// shared memory, barriers and TMEM, and then block in grid_dep_wait() until that kernel has
+// completed and its memory writes are visible.  Every CTA calls grid_dep_wait() before its first
+// access to global memory and unconditionally (so a kernel never completes before the one it
+// follows), then grid_dep_launch() to let the next kernel be scheduled.  Both are no-ops in a
+// kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Host: whether launches carry the programmatic-serialisation attribute (on unless the
+// environment sets MLA_NO_PDL; read once per process).
+bool pdl_enabled();
+
+// Launches kernel<<<grid, block, smem, s>>>(args...) through cudaLaunchKernelEx with the
+// programmatic-serialisation attribute (when pdl_enabled()).  Only for kernels that call
+// grid_dep_wait() as described above.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int round_up(int a, int b) { return ceil_div(a, b) * b; }
 

@@ -26,7 +26,12 @@
 // in long runs instead of one 128-byte piece per row and K-slice.
 // Optionally the columns n >= n_split go to a second output C2 (column n - n_split): one GEMM
 // over [W_1; W_2] then writes x W_1^T and x W_2^T to their own arrays.  Optionally every output
-// row is also stored into a ring of frames (the fused down-projection and cache append).
+// row is also stored into a ring of frames (the fused down-projection and cache append), and
+// optionally the epilogue writes the rotated positional keys the chunk's attention reads (the
+// chunk's own from the k_R columns of each row, the ring's from the cache while the first
+// tile's MMAs run), so that attention needs no separate rotation pass.
+// Launched with programmatic serialisation (launch_pdl): barrier set-up and the TMEM allocation
+// may overlap the previous kernel's tail.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -83,7 +88,54 @@ struct GemmParams {
   bf16* ring;                // ring append (see TcGemmArgs), or null
   int32_t* slot_frame;
   int ring_W, ring_tpf, ring_n_q, ring_first, ring_B;
+  bf16* rk;                  // rotated positional keys (see TcGemmArgs), or null
+  const bf16* rk_cache;
+  const int32_t* rk_slot_frame;
+  int32_t* rk_dev_status;
+  int rk_col, rk_dr, rk_D, rk_dc, rk_n_q, rk_B, rk_W, rk_nc, rk_nc_pad, rk_rows, rk_first, rk_ring;
 };
+
+// Row r of sample b of the rotated-key workspace (ring slot, padding or tail row).
+__device__ __forceinline__ void gemm_key_row(const GemmParams& p, int b, int r) {
+  switch (p.rk_dr) {
+#define MLA_GEMM_KEY_ROW(DR)                                                                     \
+  case DR:                                                                                       \
+    rope_key_row<bf16, DR / 8>(p.rk_cache, nullptr, p.rk_slot_frame, p.rk, b, r, p.rk_W, p.rk_D, \
+                               p.rk_dc, p.rk_n_q, p.rk_nc, p.rk_nc_pad, p.rk_rows, p.rk_first,   \
+                               p.rope, p.rk_dev_status, 1);                                      \
+    break;
+    MLA_GEMM_KEY_ROW(16)
+    MLA_GEMM_KEY_ROW(32)
+    MLA_GEMM_KEY_ROW(64)
+#undef MLA_GEMM_KEY_ROW
+    default: break;
+  }
+}
+
+// The chunk token's rotated positional key from the 32 accumulator columns v of one epilogue
+// chunk starting at output column n (rk_col <= n < rk_col + rk_dr): each value is taken as
+// chunk_lat stores it (rounded to bf16), rotated in fp32 and rounded once, as rope_key_row does.
+__device__ __forceinline__ void gemm_chunk_key(const GemmParams& p, int m, int n, const float* v) {
+  const int bs = m / p.rk_n_q, j = m % p.rk_n_q;
+  const int i = j % p.rope.tpf;
+  const int t = p.rk_first + j / p.rope.tpf, h = i / p.rope.frame_w, w = i % p.rope.frame_w;
+  const int c0 = n - p.rk_col;                       // a multiple of 32
+  const int npairs = min(16, (p.rk_dr - c0) / 2);    // 8 or 16
+  uint32_t packed[16];
+#pragma unroll
+  for (int pr = 0; pr < 16; ++pr) {
+    float x0 = __bfloat162float(__float2bfloat16_rn(v[2 * pr]));
+    float x1 = __bfloat162float(__float2bfloat16_rn(v[2 * pr + 1]));
+    if (pr < npairs) rope_rotate(x0, x1, rope_angle(p.rope, c0 / 2 + pr, t, h, w));
+    packed[pr] = pack_bf16x2(x0, x1);
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(
+      p.rk + (static_cast<int64_t>(bs) * p.rk_rows + p.rk_nc_pad + j) * p.rk_dr + c0);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (4 * q < npairs)
+      d4[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+}
 
 __device__ __forceinline__ void store_row32(bf16* dst, const float* v, int valid, bool vec_ok) {
   if (vec_ok && valid >= 32) {
@@ -155,6 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  grid_dep_wait();     // the previous kernel on the stream has completed (programmatic launch)
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -245,6 +299,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const bool ring_vec = p.ring != nullptr && ((reinterpret_cast<uintptr_t>(p.ring) & 15u) == 0) &&
                           (p.N % 8 == 0);
+    if (p.rk != nullptr) {
+      // the rotated-key rows that do not come from this GEMM's output: the ring part (with
+      // rk_ring) and the zero rows after the chunk, spread over every epilogue thread of the grid
+      // while the first tile's MMAs run
+      const int ring_rows = p.rk_ring ? p.rk_nc_pad : 0;
+      const int tail0 = p.rk_nc_pad + p.rk_n_q;
+      const int per = ring_rows + (p.rk_rows - tail0);
+      const int total = p.rk_B * per;                // < 2^31 (host check)
+      for (int e = blockIdx.x * kEpiThreads + (threadIdx.x - 64); e < total;
+           e += gridDim.x * kEpiThreads) {
+        const int b = e / per, i = e % per;
+        gemm_key_row(p, b, i < ring_rows ? i : tail0 + (i - ring_rows));
+      }
+    }
     int lt = 0, chunk = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
       const int acc = lt & 1;
@@ -289,6 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const bool second = p.n_split > 0 && n >= p.n_split;
+        if (p.rk != nullptr && n >= p.rk_col && n < p.rk_col + p.rk_dr && m < p.M)
+          gemm_chunk_key(p, m, n, v);
         if (p.ring != nullptr && m < p.M) {
           // the same row into its ring slot (whole frames wrap; row width N)
           const int bs = m / p.ring_n_q, r = m % p.ring_n_q;
@@ -418,6 +488,12 @@ mla_status launch_gemm(const TcGemmArgs& g, cudaStream_t s) {
   p.ring = static_cast<bf16*>(g.ring); p.slot_frame = g.slot_frame;
   p.ring_W = g.ring_W; p.ring_tpf = g.ring_tpf; p.ring_n_q = g.ring_n_q;
   p.ring_first = g.ring_first; p.ring_B = g.ring_B;
+  p.rk = static_cast<bf16*>(g.rk); p.rk_cache = static_cast<const bf16*>(g.rk_cache);
+  p.rk_slot_frame = g.rk_slot_frame; p.rk_dev_status = g.rk_dev_status;
+  p.rk_col = g.rk_col; p.rk_dr = g.rk_dr; p.rk_D = g.rk_D; p.rk_dc = g.rk_dc;
+  p.rk_n_q = g.rk_n_q; p.rk_B = g.rk_B; p.rk_W = g.rk_W; p.rk_nc = g.rk_nc;
+  p.rk_nc_pad = g.rk_nc_pad; p.rk_rows = g.rk_rows; p.rk_first = g.rk_first;
+  p.rk_ring = g.rk_ring;
   // output maps: 32 x 128 boxes, 64B swizzle (the staging layout)
   CUtensorMap tc, tc2;
   p.tma_store = tma_storable(g.C, g.c_sm, g.c_batch, g.batch) &&
@@ -442,8 +518,8 @@ mla_status launch_gemm(const TcGemmArgs& g, cudaStream_t s) {
                                     Cfg::kSmem));
   const long long tiles = static_cast<long long>(p.n_tiles_m) * p.n_tiles_n * g.batch;
   const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
-  gemm_tc_kernel<BN><<<grid, kThreads, Cfg::kSmem, s>>>(ta, tb, tc, tc2, p);
-  MLA_LAUNCH_CHECK("gemm_tc");
+  MLA_CUDA_TRY(launch_pdl(gemm_tc_kernel<BN>, dim3(grid), dim3(kThreads), Cfg::kSmem, s, ta, tb,
+                          tc, tc2, p));
   return MLA_OK;
 }
 
@@ -462,6 +538,17 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s) {
        g.ring_tpf <= 0 || g.ring_n_q % g.ring_tpf != 0 ||
        static_cast<int64_t>(g.ring_B) * g.ring_n_q != g.M))
     MLA_FAIL(MLA_ERR_INVALID_ARG, "GEMM ring epilogue: inconsistent ring geometry");
+  if (g.rk != nullptr &&
+      (g.batch != 1 || g.rk_col % 32 != 0 || g.rk_col < 0 || g.rk_col + g.rk_dr > g.N ||
+       (g.rk_dr != 16 && g.rk_dr != 32 && g.rk_dr != 64) || g.rk_dr != 2 * (g.rope.pt + g.rope.ph + g.rope.pw) ||
+       g.rk_D != g.rk_dc + g.rk_dr || g.rk_n_q <= 0 || g.rk_n_q % g.rope.tpf != 0 ||
+       static_cast<int64_t>(g.rk_B) * g.rk_n_q != g.M || g.rk_nc_pad < g.rk_nc ||
+       g.rk_rows < g.rk_nc_pad + g.rk_n_q || (g.rk_ring && g.rk_nc > 0 && g.rk_cache == nullptr) ||
+       g.rk_slot_frame == nullptr || (reinterpret_cast<uintptr_t>(g.rk) & 15u) != 0 ||
+       (g.rk_cache != nullptr && (reinterpret_cast<uintptr_t>(g.rk_cache) & 15u) != 0) ||
+       (g.rk_D * 2) % 16 != 0 || (g.rk_dc * 2) % 16 != 0 ||
+       static_cast<int64_t>(g.rk_B) * g.rk_rows >= (int64_t{1} << 31)))
+    MLA_FAIL(MLA_ERR_INVALID_ARG, "GEMM rotated-key epilogue: inconsistent key geometry");
   if (g.epilogue == kEpiRopeQ &&
       (g.rope_D <= 0 || g.N % g.rope_D != 0 || g.rope_dr % 2 != 0 || g.rope_dr > g.rope_D ||
        g.rope_dr / 2 > kMaxRopePairs))

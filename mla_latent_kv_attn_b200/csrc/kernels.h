@@ -93,8 +93,9 @@ mla_status ring_append(const Dims& d, const void* chunk_lat, void* cache, int32_
 mla_status key_positions(const Dims& d, const int32_t* slot_frame, int n_valid, int first_frame,
                          int32_t* out, cudaStream_t s);
 // Which rows of the rotated-key workspace build_rope_keys writes: all, the ring part (rows
-// [0, nc_pad)) or the chunk part (rows [nc_pad, rows)).
-enum RopeKeysPart : int { kRopeKeysAll = 0, kRopeKeysRing = 1, kRopeKeysChunk = 2 };
+// [0, nc_pad)) or the chunk part (rows [nc_pad, rows)); kRopeKeysNone tells the attention entry
+// points that the workspace is complete already (written by the x-projection's epilogue).
+enum RopeKeysPart : int { kRopeKeysAll = 0, kRopeKeysRing = 1, kRopeKeysChunk = 2, kRopeKeysNone = 3 };
 // dev_status (optional): with MLA_DEBUG builds the kernel checks that every attended ring slot
 // holds a frame (t >= 0) and, with check_window, one of the chunk's window
 // (first_frame - W <= t < first_frame), writing MLA_ERR_DEVICE_CHECK there otherwise.
@@ -144,6 +145,19 @@ struct TcGemmArgs {
   void* ring;
   int32_t* slot_frame;
   int ring_W, ring_tpf, ring_n_q, ring_first, ring_B;
+  // Optional rotated positional keys for the attention's key workspace (batch 1; rk_col a
+  // multiple of 32; rk_dr 16, 32 or 64; M = rk_B * rk_n_q; geometry from `rope`): row m = chunk
+  // token j = m mod rk_n_q of sample b = m / rk_n_q at frame rk_first + j / tpf.  The epilogue
+  // stores RoPE3D of output columns [rk_col, rk_col + rk_dr) of row m, taken as rounded to bf16,
+  // to workspace row rk_nc_pad + j of sample b; the epilogue warps also write the zero rows after
+  // the chunk and, with rk_ring, the ring part (rows [0, rk_nc_pad): the rotated k_R of ring
+  // slots from rk_cache / rk_slot_frame, zeros from rk_nc on) before the first accumulator is
+  // ready.  Rows are laid out as key_workspace_layout() gives them (rk_rows per sample).
+  void* rk;
+  const void* rk_cache;
+  const int32_t* rk_slot_frame;
+  int32_t* rk_dev_status;
+  int rk_col, rk_dr, rk_D, rk_dc, rk_n_q, rk_B, rk_W, rk_nc, rk_nc_pad, rk_rows, rk_first, rk_ring;
 };
 
 bool tc_gemm_supported(int M, int N, int K, int64_t a_sm, int64_t b_sn);

@@ -1,6 +1,7 @@
 // mla_abi.cu - the extern "C" entry points of include/mla.h: host-side validation, then launches
 // on the caller's stream.  No allocation, no synchronisation.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 
@@ -13,6 +14,11 @@ thread_local std::string g_last_error;
 }
 
 void set_last_error(const std::string& msg) { g_last_error = msg; }
+
+bool pdl_enabled() {
+  static const bool on = std::getenv("MLA_NO_PDL") == nullptr;
+  return on;
+}
 
 namespace {
 
@@ -181,6 +187,40 @@ mla_status check_workspace(const Dims& d, int n_valid, const void* workspace,
   return check_ptr(workspace, "workspace");
 }
 
+// project_latents plus the rotated positional keys of the chunk's attention in the key
+// workspace: on the tensor cores one GEMM whose epilogue writes them (the ring's too with
+// rotate_ring), otherwise the GEMMs and the rotation pass.
+mla_status project_latents_rotated(const Dims& d, const void* x, const void* w_x, void* c_q,
+                                   void* chunk_lat, const void* cache, const int32_t* slot_frame,
+                                   int n_valid, int first_frame, int rotate_ring, void* workspace,
+                                   int32_t* dev_status, cudaStream_t s) {
+  const int M = d.B * d.n_q;
+  const int N = d.d_cq + d.D;
+  const KeyWorkspace kw = key_workspace_layout(d, n_valid);
+  if (use_tc(d) && d.d_cq % 32 == 0 && (d.d_cq + d.d_c) % 32 == 0 &&
+      (d.d_rope == 16 || d.d_rope == 32 || d.d_rope == 64) && d.tpf > 0 &&
+      static_cast<int64_t>(d.B) * kw.rows < (int64_t{1} << 31) &&
+      tc_gemm_supported(M, N, d.d_model, d.d_model, d.d_model)) {
+    TcGemmArgs g{};
+    g.A = x; g.a_sm = d.d_model; g.a_batch = 0;
+    g.B = w_x; g.b_sn = d.d_model; g.b_batch = 0;
+    g.C = c_q; g.c_sm = d.d_cq; g.c_batch = 0;
+    g.C2 = chunk_lat; g.c2_sm = d.D; g.c2_batch = 0; g.n_split = d.d_cq;
+    g.M = M; g.N = N; g.K = d.d_model; g.batch = 1;
+    g.epilogue = kEpiStore;
+    g.rope = rope_geom(d);
+    g.rk = workspace; g.rk_cache = cache; g.rk_slot_frame = slot_frame;
+    g.rk_dev_status = dev_status;
+    g.rk_col = d.d_cq + d.d_c; g.rk_dr = d.d_rope; g.rk_D = d.D; g.rk_dc = d.d_c;
+    g.rk_n_q = d.n_q; g.rk_B = d.B; g.rk_W = d.W; g.rk_nc = kw.nc; g.rk_nc_pad = kw.nc_pad;
+    g.rk_rows = kw.rows; g.rk_first = first_frame; g.rk_ring = rotate_ring ? 1 : 0;
+    return gemm_tc(g, s);
+  }
+  MLA_TRY(project_latents(d, x, w_x, c_q, chunk_lat, s));
+  return build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid, first_frame, workspace, s,
+                         rotate_ring ? kRopeKeysAll : kRopeKeysChunk, dev_status, 1);
+}
+
 // Shared body of the attention entry points: checks, the rotated-key pre-pass (all of it, or
 // only the chunk's keys when the ring's rotated keys are already in the workspace), attention.
 mla_status attention_entry(const mla_config* cfg, const void* q, const void* chunk_lat,
@@ -242,8 +282,9 @@ mla_status attention_from_cq_entry(const mla_config* cfg, const void* c_q, const
   MLA_TRY(check_ptr(dev_status, "dev_status", false));
   MLA_TRY(check_workspace(d, n_valid_frames, workspace, workspace_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  MLA_TRY(build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid_frames, first_frame, workspace,
-                          s, rope_part, dev_status, 1));
+  if (rope_part != kRopeKeysNone)
+    MLA_TRY(build_rope_keys(d, cache, chunk_lat, slot_frame, n_valid_frames, first_frame,
+                            workspace, s, rope_part, dev_status, 1));
   AttnArgs a{};
   a.q = nullptr; a.chunk_lat = chunk_lat; a.cache = cache; a.ws = workspace; a.w_uv = w_uv;
   a.out = out; a.lse = lse; a.dev_status = dev_status;
@@ -451,6 +492,33 @@ mla_status mla_project_latents(const mla_config* cfg, const void* x, const void*
   return project_latents(d, x, w_x, c_q, chunk_lat, static_cast<cudaStream_t>(stream));
 }
 
+mla_status mla_project_latents_rotated(const mla_config* cfg, const void* x, const void* w_x,
+                                       void* c_q, void* chunk_lat, const void* cache,
+                                       const int32_t* slot_frame, int32_t n_valid_frames,
+                                       int32_t first_frame, int32_t rotate_ring, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status,
+                                       void* stream) {
+  MLA_NVTX_RANGE("mla_project_latents_rotated");
+  set_last_error("");
+  MLA_TRY(check_cfg(cfg));
+  const Dims d = dims_of(*cfg);
+  MLA_CHECK_ARG(n_valid_frames >= 0 && n_valid_frames <= d.W, "n_valid_frames must be in [0, %d]",
+                d.W);
+  MLA_CHECK_ARG(rotate_ring == 0 || rotate_ring == 1, "rotate_ring must be 0 or 1");
+  MLA_TRY(check_first_frame(first_frame, d.C));
+  MLA_TRY(check_ptr(x, "x"));
+  MLA_TRY(check_ptr(w_x, "w_x"));
+  MLA_TRY(check_ptr(c_q, "c_q"));
+  MLA_TRY(check_ptr(chunk_lat, "chunk_lat"));
+  MLA_TRY(check_ptr(slot_frame, "slot_frame"));
+  MLA_TRY(check_ptr(cache, "cache", rotate_ring && n_valid_frames > 0));
+  MLA_TRY(check_ptr(dev_status, "dev_status", false));
+  MLA_TRY(check_workspace(d, n_valid_frames, workspace, workspace_bytes));
+  return project_latents_rotated(d, x, w_x, c_q, chunk_lat, cache, slot_frame, n_valid_frames,
+                                 first_frame, rotate_ring, workspace, dev_status,
+                                 static_cast<cudaStream_t>(stream));
+}
+
 int32_t mla_attention_uses_tensor_cores(const mla_config* cfg, int32_t with_w_uv) {
   if (check_cfg(cfg) != MLA_OK) return -1;
   const Dims d = dims_of(*cfg);
@@ -495,6 +563,17 @@ mla_status mla_attention_fwd_from_cq_cached_ring(
   return attention_from_cq_entry(cfg, c_q, w_qcat, chunk_lat, cache, slot_frame, n_valid_frames,
                                  first_frame, w_uv, out, lse, workspace, workspace_bytes,
                                  dev_status, stream, kRopeKeysChunk);
+}
+
+mla_status mla_attention_fwd_from_cq_prerotated(
+    const mla_config* cfg, const void* c_q, const void* w_qcat, const void* chunk_lat,
+    const void* cache, const int32_t* slot_frame, int32_t n_valid_frames, int32_t first_frame,
+    const void* w_uv, void* out, float* lse, void* workspace, size_t workspace_bytes,
+    int32_t* dev_status, void* stream) {
+  MLA_NVTX_RANGE("mla_attention_fwd_from_cq_prerotated");
+  return attention_from_cq_entry(cfg, c_q, w_qcat, chunk_lat, cache, slot_frame, n_valid_frames,
+                                 first_frame, w_uv, out, lse, workspace, workspace_bytes,
+                                 dev_status, stream, kRopeKeysNone);
 }
 
 mla_status mla_attention_fwd_cached_ring(const mla_config* cfg, const void* q,

@@ -236,6 +236,8 @@ namespace {
 __global__ void ring_append_kernel(const uint4* __restrict__ lat, uint4* __restrict__ cache,
                                    int32_t* __restrict__ slot_frame, int B, int C, int W,
                                    int vec_per_frame, int first_frame) {
+  grid_dep_wait();     // launched with programmatic serialisation (launch_pdl)
+  grid_dep_launch();
   const int64_t per_sample = static_cast<int64_t>(C) * vec_per_frame;
   const int64_t total = per_sample * B;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
@@ -262,9 +264,9 @@ mla_status ring_append(const Dims& d, const void* chunk_lat, void* cache, int32_
   const int64_t total = static_cast<int64_t>(d.B) * d.C * vec_per_frame;
   const int threads = 256;
   const int blocks = static_cast<int>(std::min<int64_t>((total + threads - 1) / threads, 148 * 8));
-  ring_append_kernel<<<blocks, threads, 0, s>>>(static_cast<const uint4*>(chunk_lat),
-                                                static_cast<uint4*>(cache), slot_frame, d.B, d.C,
-                                                d.W, vec_per_frame, first_frame);
+  launch_pdl(ring_append_kernel, dim3(blocks), dim3(threads), 0, s,
+             static_cast<const uint4*>(chunk_lat), static_cast<uint4*>(cache), slot_frame, d.B,
+             d.C, d.W, vec_per_frame, first_frame);
   MLA_LAUNCH_CHECK("ring_append");
   return MLA_OK;
 }
@@ -355,9 +357,10 @@ __global__ void rope_keys_kernel(const T* __restrict__ cache, const T* __restric
   }
 }
 
-// The same rows with 16-byte vectors: one thread per rotated key (kPieces 16-byte pieces of
-// d_rope values); every piece is loaded before the first is rotated and stored, and the key's
-// position is computed once.  Needs d_c, d_rope and D at whole 16-byte multiples (host check).
+// The same rows with 16-byte vectors: one thread per rotated key (rope_key_row: every piece is
+// loaded before the first is rotated and stored, and the key's position is computed once).
+// Needs d_c, d_rope and D at whole 16-byte multiples (host check).  Launched with programmatic
+// serialisation (launch_pdl).
 template <typename T, int kPieces>
 __global__ void __launch_bounds__(256)
     rope_keys_vec_kernel(const T* __restrict__ cache, const T* __restrict__ chunk_lat,
@@ -365,49 +368,14 @@ __global__ void __launch_bounds__(256)
                          int D, int d_c, int n_q, int nc, int nc_pad, int rows_ws, int row_begin,
                          int row_end, int first_frame, RopeGeom g, int32_t* dev_status,
                          int check_window) {
-  constexpr int kPer = 16 / sizeof(T);          // elements per piece
-  constexpr int kDr = kPieces * kPer;
+  grid_dep_wait();
+  grid_dep_launch();
   const int span = row_end - row_begin;
   const int total = B * span;                   // < 2^31 (host check)
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-    const int r = row_begin + e % span;
-    const int b = e / span;
-    uint4* dst = reinterpret_cast<uint4*>(ws + (static_cast<int64_t>(b) * rows_ws + r) * kDr);
-    const T* src = nullptr;
-    int m = -1;
-    if (r < nc) {
-      m = r;
-      src = cache + (static_cast<int64_t>(b) * W * g.tpf + r) * D;
-    } else if (r >= nc_pad && r - nc_pad < n_q) {
-      m = nc + (r - nc_pad);
-      src = chunk_lat + (static_cast<int64_t>(b) * n_q + (r - nc_pad)) * D;
-    }
-    if (src == nullptr) {
-#pragma unroll
-      for (int k = 0; k < kPieces; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
-      continue;
-    }
-    uint4 raw[kPieces];
-    const uint4* s4 = reinterpret_cast<const uint4*>(src + d_c);
-#pragma unroll
-    for (int k = 0; k < kPieces; ++k) raw[k] = s4[k];
-    int t, h, w;
-    key_position(slot_frame, b, W, g.tpf, g.frame_w, nc, first_frame, m, t, h, w);
-    if (m < nc)
-      debug_check(t >= 0 && (!check_window || (t < first_frame && t >= first_frame - W)), dev_status);
-#pragma unroll
-    for (int k = 0; k < kPieces; ++k) {
-      T* x = reinterpret_cast<T*>(&raw[k]);
-#pragma unroll
-      for (int q = 0; q < kPer; q += 2) {
-        float x0 = Elem<T>::to_f(x[q]), x1 = Elem<T>::to_f(x[q + 1]);
-        rope_rotate(x0, x1, rope_angle(g, (k * kPer + q) / 2, t, h, w));
-        x[q] = Elem<T>::from_f(x0);
-        x[q + 1] = Elem<T>::from_f(x1);
-      }
-      dst[k] = raw[k];
-    }
-  }
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x)
+    rope_key_row<T, kPieces>(cache, chunk_lat, slot_frame, ws, e / span, row_begin + e % span, W,
+                             D, d_c, n_q, nc, nc_pad, rows_ws, first_frame, g, dev_status,
+                             check_window);
 }
 
 }  // namespace
@@ -427,6 +395,7 @@ mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_l
   const KeyWorkspace k = key_workspace_layout(d, n_valid);
   const int n_pairs = d.d_rope / 2;
   // the ring part is rows [0, nc_pad) (its padding rows included), the chunk part the rest
+  if (part == kRopeKeysNone) return MLA_OK;
   const int row_begin = part == kRopeKeysChunk ? k.nc_pad : 0;
   const int row_end = part == kRopeKeysRing ? k.nc_pad : k.rows;
   if (row_end <= row_begin) return MLA_OK;
@@ -443,10 +412,10 @@ mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_l
     const int64_t vtotal = static_cast<int64_t>(d.B) * (row_end - row_begin);
     const int vblocks = static_cast<int>(std::min<int64_t>((vtotal + 255) / 256, 148 * 16));
 #define MLA_KEYS_VEC(T, P)                                                                       \
-  rope_keys_vec_kernel<T, P><<<vblocks, 256, 0, s>>>(                                          \
-      static_cast<const T*>(cache), static_cast<const T*>(chunk_lat), slot_frame,               \
-      static_cast<T*>(ws), d.B, d.W, d.D, d.d_c, d.n_q, k.nc, k.nc_pad, k.rows, row_begin,      \
-      row_end, first_frame, g, dev_status, check_window)
+  launch_pdl(rope_keys_vec_kernel<T, P>, dim3(vblocks), dim3(256), 0, s,                       \
+             static_cast<const T*>(cache), static_cast<const T*>(chunk_lat), slot_frame,       \
+             static_cast<T*>(ws), d.B, d.W, d.D, d.d_c, d.n_q, k.nc, k.nc_pad, k.rows,         \
+             row_begin, row_end, first_frame, g, dev_status, check_window)
     if (d.dtype == MLA_FP32) {
       if (pieces == 2) MLA_KEYS_VEC(float, 2);
       else if (pieces == 4) MLA_KEYS_VEC(float, 4);

@@ -104,16 +104,14 @@ def fused_query_supported(c) -> bool:
 def attend_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
                  fuse_uv: bool = True, stream=None, fused_q: bool = False) -> torch.Tensor:
     """Query path, chunk latents and attention of one chunk (buf.x holds its tokens).
-    Returns buf.o (fused W_UV) or buf.o_lat (latent output).  With fused_q the attention kernel
-    forms the query heads itself from c_Q (buf.q is then not written)."""
+    Returns buf.o (fused W_UV) or buf.o_lat (latent output).  With fused_q the x-projection also
+    writes every rotated positional key of the call and the attention kernel forms the query
+    heads itself from c_Q (buf.q is then not written): two launches."""
     first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
     out = buf.o if fuse_uv else buf.o_lat
     if fused_q:
-        api.mla_project_latents(c, buf.x, w.w_x, buf.c_q, buf.chunk_lat, stream=stream)
-        api.mla_attention_fwd_from_cq(c, buf.c_q, w.w_qcat, buf.chunk_lat, ring.cache,
-                                      ring.slot_frame, n_valid, first,
-                                      w.w_uv if fuse_uv else None, out, buf.lse, buf.workspace,
-                                      buf.dev_status, stream=stream)
+        _attend_from_cq(c, w, ring, buf, buf.x, n_valid, first, out, fuse_uv, buf.workspace,
+                        rotate_ring=True, stream=stream)
         return out
     api.mla_project_chunk(c, buf.x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first,
                           stream=stream)
@@ -121,6 +119,22 @@ def attend_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
                           w.w_uv if fuse_uv else None, out, buf.lse, buf.workspace,
                           buf.dev_status, stream=stream)
     return out
+
+
+def _attend_from_cq(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, x, n_valid: int,
+                    first: int, out, fuse_uv: bool, workspace, rotate_ring: bool,
+                    stream=None) -> None:
+    """The two calls of a chunk's attention with the query heads formed in the attention kernel:
+    the x-projection with the rotated keys (mla_project_latents_rotated) and the attention with
+    no rotation pass."""
+    api.mla_project_latents_rotated(c, x, w.w_x, buf.c_q, buf.chunk_lat, ring.cache,
+                                    ring.slot_frame, n_valid, first, workspace,
+                                    rotate_ring=rotate_ring, dev_status=buf.dev_status,
+                                    stream=stream)
+    api.mla_attention_fwd_from_cq(c, buf.c_q, w.w_qcat, buf.chunk_lat, ring.cache,
+                                  ring.slot_frame, n_valid, first, w.w_uv if fuse_uv else None,
+                                  out, buf.lse, workspace, buf.dev_status, stream=stream,
+                                  prerotated=True)
 
 
 def append_chunk(c, ring: Ring, buf: ChunkBuffers, chunk: int, stream=None) -> None:
@@ -250,7 +264,9 @@ class ChunkGraph:
             if events:
                 self.proj_start.record()
             if fused_q:
-                api.mla_project_latents(c, x, w.w_x, buf.c_q, buf.chunk_lat)
+                api.mla_project_latents_rotated(c, x, w.w_x, buf.c_q, buf.chunk_lat, ring.cache,
+                                                ring.slot_frame, n_valid, first, buf.workspace,
+                                                dev_status=buf.dev_status)
             else:
                 api.mla_project_chunk(c, x, w.w_x, w.w_qcat, buf.c_q, buf.q, buf.chunk_lat, first)
             if events:
@@ -260,7 +276,7 @@ class ChunkGraph:
                 api.mla_attention_fwd_from_cq(c, buf.c_q, w.w_qcat, buf.chunk_lat, ring.cache,
                                               ring.slot_frame, n_valid, first,
                                               w.w_uv if fuse_uv else None, out, buf.lse,
-                                              buf.workspace, buf.dev_status)
+                                              buf.workspace, buf.dev_status, prerotated=True)
             else:
                 api.mla_attention_fwd(c, buf.q, buf.chunk_lat, ring.cache, ring.slot_frame,
                                       n_valid, first, w.w_uv if fuse_uv else None, out, buf.lse,
@@ -295,8 +311,10 @@ class LayerStack:
     Every step of a chunk runs every layer's attention against that layer's ring, which stays
     frozen until the chunk is finished (hyper.ai summary of VideoMLA, "Introduction": the cache
     rolls forward chunk by chunk).  So the positional keys of each ring are rotated once per
-    chunk (mla_rotate_ring_keys into the layer's own workspace) and every step's attention only
-    rotates the chunk's keys (mla_attention_fwd_cached_ring).  At the last step each layer
+    chunk (mla_rotate_ring_keys into the layer's own workspace) and every step only rotates the
+    chunk's keys: in the x-projection's epilogue with the fused query heads
+    (mla_project_latents_rotated with rotate_ring=False, then the attention with no rotation
+    pass), else in mla_attention_fwd_cached_ring.  At the last step each layer
     appends the chunk's latents to its ring right after its attention.
 
     One set of chunk activations (buf) is shared by all layers: a call's outputs are valid until
@@ -336,12 +354,10 @@ class LayerStack:
         first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
         out = b.o if self.fuse_uv else b.o_lat
         if self.fused_q:
-            api.mla_project_latents(c, x, w.w_x, b.c_q, b.chunk_lat, stream=stream)
-            api.mla_attention_fwd_from_cq(c, b.c_q, w.w_qcat, b.chunk_lat, ring.cache,
-                                          ring.slot_frame, n_valid, first,
-                                          w.w_uv if self.fuse_uv else None, out, b.lse,
-                                          self.ws[layer], b.dev_status, stream=stream,
-                                          cached_ring=True)
+            # the ring part of the layer's workspace was rotated by begin_chunk; the projection
+            # writes the chunk's rotated keys next to it
+            _attend_from_cq(c, w, ring, b, x, n_valid, first, out, self.fuse_uv, self.ws[layer],
+                            rotate_ring=False, stream=stream)
         else:
             api.mla_project_chunk(c, x, w.w_x, w.w_qcat, b.c_q, b.q, b.chunk_lat, first,
                                   stream=stream)

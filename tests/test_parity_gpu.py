@@ -190,6 +190,53 @@ def test_fused_query_heads_match_the_q_gemm(d_c, d_rope):
     print("fused query heads bit-identical to the Q' GEMM path:", identical)
 
 
+@pytest.mark.parametrize("d_c,d_rope", FUSED_Q_SHAPES)
+def test_rotated_keys_from_the_projection_epilogue(d_c, d_rope):
+    """mla_project_latents_rotated writes the chunk's rotated positional keys from the
+    x-projection's epilogue and the ring's from its idle epilogue warps.  Over a 4-chunk rollout
+    of 2 samples whose ring fills and wraps (chunk 0 has no ring keys): c_q and chunk_lat equal
+    mla_project_latents; the workspace equals what the rotation pass of mla_attention_fwd_from_cq
+    writes (padding rows included), with rotate_ring=1 from a poisoned workspace and with
+    rotate_ring=0 on top of mla_rotate_ring_keys; and mla_attention_fwd_from_cq_prerotated gives
+    exactly the outputs and lse of mla_attention_fwd_from_cq."""
+    cfg = inputs.with_latent_shape(inputs.small_bf16_config(), d_c, d_rope)
+    g = GpuRun(cfg)
+    c, b, w = g.c, g.buf, g.w
+    cq2, lat2 = torch.empty_like(b.c_q), torch.empty_like(b.chunk_lat)
+    o2, lse2 = torch.empty_like(b.o), torch.empty_like(b.lse)
+    for ch in range(cfg.n_chunks):
+        first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, ch)
+        nbytes = api.mla_attention_workspace_bytes(c, n_valid)
+        g.load_x(inputs.chunk_x(cfg, ch))
+        b.dev_status.zero_()
+        # reference: plain projection, then the attention with its own rotation pass
+        ws_ref = torch.full_like(b.workspace, 0x5A)
+        api.mla_project_latents(c, b.x, w.w_x, b.c_q, b.chunk_lat)
+        api.mla_attention_fwd_from_cq(c, b.c_q, w.w_qcat, b.chunk_lat, g.ring.cache,
+                                      g.ring.slot_frame, n_valid, first, w.w_uv, b.o, b.lse,
+                                      ws_ref, b.dev_status)
+        # the fused projection, from a poisoned workspace
+        ws = torch.full_like(b.workspace, 0xA5)
+        api.mla_project_latents_rotated(c, b.x, w.w_x, cq2, lat2, g.ring.cache, g.ring.slot_frame,
+                                        n_valid, first, ws, dev_status=b.dev_status)
+        api.mla_attention_fwd_from_cq(c, cq2, w.w_qcat, lat2, g.ring.cache, g.ring.slot_frame,
+                                      n_valid, first, w.w_uv, o2, lse2, ws, b.dev_status,
+                                      prerotated=True)
+        # frozen ring: ring part from mla_rotate_ring_keys, the rest from the projection
+        ws_frozen = torch.full_like(b.workspace, 0x3C)
+        api.mla_rotate_ring_keys(c, g.ring.cache, g.ring.slot_frame, n_valid, ws_frozen)
+        api.mla_project_latents_rotated(c, b.x, w.w_x, cq2, lat2, g.ring.cache, g.ring.slot_frame,
+                                        n_valid, first, ws_frozen, rotate_ring=False,
+                                        dev_status=b.dev_status)
+        torch.cuda.synchronize()
+        assert torch.equal(cq2, b.c_q) and torch.equal(lat2, b.chunk_lat), ch
+        assert torch.equal(ws[:nbytes], ws_ref[:nbytes]), ch
+        assert torch.equal(ws_frozen[:nbytes], ws_ref[:nbytes]), ch
+        assert torch.equal(o2, b.o) and torch.equal(lse2, b.lse), ch
+        rollout.check_device_status(b)
+        g.append(ch)
+
+
 def test_fused_query_heads_config1_sampled_rows():
     """The bench's step on config 1 (query heads formed in the attention kernel): 384 sampled
     rows against the oracle, and every row against the unfused path."""
