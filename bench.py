@@ -329,7 +329,9 @@ def measure_bandwidth(cfg, flush, stream, hbm_gbs: float, reps: int = 20):
     bandwidth.  Algorithmic bytes: ring append 2 * D * sizeof(T) per chunk token (read the chunk
     latent, write the ring row); ring-key rotation 2 * d_rope * sizeof(T) per ring key (read k_R,
     write the rotated key); query RoPE 2 * d_rope * sizeof(T) per (token, head); KV
-    down-projection x + [W_down^KV; W_R^K] read, [c_KV || k_R] written once."""
+    down-projection x + [W_down^KV; W_R^K] read, [c_KV || k_R] written once; the step's
+    x-projection x + w_x read, [c_Q || c_KV || k_R] written once, and with the rotated keys also
+    k_R of every ring key read and the rotated key of every ring and chunk key written."""
     import torch
     from mla_latent_kv_attn_b200 import api, rollout
     res = {}
@@ -373,7 +375,22 @@ def measure_bandwidth(cfg, flush, stream, hbm_gbs: float, reps: int = 20):
             flops = 2.0 * batch * n_q * cfg.d_model * D
             res[f"kv_down_projection_{tag}"] = bandwidth_entry(
                 nbytes, ms, hbm_gbs, wl, kernel="gemm_tc_kernel", tflops=flops / (ms * 1e-3) / 1e12)
-            del x, wkv
+            # the step's x-projection (c_Q || chunk latents in one pass over x), without and with
+            # the rotated keys of the ring and the chunk written from its epilogue
+            wx = torch.randn((cfg.d_cq + D, cfg.d_model), device="cuda").to(dt)
+            cq = torch.empty((batch, n_q, cfg.d_cq), device="cuda", dtype=dt)
+            n_x = cfg.d_cq + D
+            nbytes = (batch * n_q * cfg.d_model + n_x * cfg.d_model + batch * n_q * n_x) * es
+            flops = 2.0 * batch * n_q * cfg.d_model * n_x
+            ms = time_calls(lambda: api.mla_project_latents(c, x, wx, cq, lat), flush, stream, reps)
+            res[f"x_projection_{tag}"] = bandwidth_entry(
+                nbytes, ms, hbm_gbs, wl, kernel="gemm_tc_kernel", tflops=flops / (ms * 1e-3) / 1e12)
+            ms = time_calls(lambda: api.mla_project_latents_rotated(
+                c, x, wx, cq, lat, ring.cache, ring.slot_frame, W, first, ws), flush, stream, reps)
+            nbytes += batch * (W * tpf * 2 + n_q) * cfg.d_rope * es
+            res[f"x_projection_rotated_keys_{tag}"] = bandwidth_entry(
+                nbytes, ms, hbm_gbs, wl, kernel="gemm_tc_kernel", tflops=flops / (ms * 1e-3) / 1e12)
+            del x, wkv, wx, cq
         del ring, lat, ws, q, q3
         torch.cuda.empty_cache()
     return res

@@ -143,14 +143,21 @@ __device__ __forceinline__ void rope_sincos(float a, float* s, float* c) {
   __sincosf(r, s, c);
 }
 
+// Rotates one pair (x0, x1) by the angle whose sine and cosine are s and c.  The rounding steps
+// are spelled out (one product rounded, then one fused multiply-add), so every kernel that
+// rotates gets the same bits whatever the compiler would contract.
+__device__ __forceinline__ void rope_apply(float& x0, float& x1, float s, float c) {
+  const float y0 = __fmaf_rn(x0, c, -__fmul_rn(x1, s));
+  const float y1 = __fmaf_rn(x0, s, __fmul_rn(x1, c));
+  x0 = y0;
+  x1 = y1;
+}
+
 // Rotates one pair (x0, x1) by angle a.
 __device__ __forceinline__ void rope_rotate(float& x0, float& x1, float a) {
   float s, c;
   rope_sincos(a, &s, &c);
-  const float y0 = x0 * c - x1 * s;
-  const float y1 = x0 * s + x1 * c;
-  x0 = y0;
-  x1 = y1;
+  rope_apply(x0, x1, s, c);
 }
 
 // (t, h, w) of key m in the walk order of the attention kernels: ring slots 0 .. nc-1 (their

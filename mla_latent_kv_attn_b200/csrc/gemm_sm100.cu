@@ -112,13 +112,32 @@ __device__ __forceinline__ void gemm_key_row(const GemmParams& p, int b, int r) 
   }
 }
 
-// The chunk token's rotated positional key from the 32 accumulator columns v of one epilogue
-// chunk starting at output column n (rk_col <= n < rk_col + rk_dr): each value is taken as
-// chunk_lat stores it (rounded to bf16), rotated in fp32 and rounded once, as rope_key_row does.
-__device__ __forceinline__ void gemm_chunk_key(const GemmParams& p, int m, int n, const float* v) {
-  const int bs = m / p.rk_n_q, j = m % p.rk_n_q;
+// Sine and cosine of the rotary pairs of the rotated-key chunk at output column n (rk_col <= n <
+// rk_col + rk_dr, a multiple of 32) for row m = chunk token j of sample m / rk_n_q, at frame
+// rk_first + j / tpf.  They depend on the row's position only, so the epilogue computes them
+// before the tile's accumulator is ready.
+__device__ __forceinline__ void gemm_key_sincos(const GemmParams& p, int m, int n, float* sn,
+                                                float* cs) {
+  const int j = m % p.rk_n_q;
   const int i = j % p.rope.tpf;
   const int t = p.rk_first + j / p.rope.tpf, h = i / p.rope.frame_w, w = i % p.rope.frame_w;
+  const int c0 = n - p.rk_col;
+  const int npairs = min(16, (p.rk_dr - c0) / 2);    // 8 or 16
+#pragma unroll
+  for (int pr = 0; pr < 16; ++pr) {
+    sn[pr] = 0.f;
+    cs[pr] = 1.f;
+    if (pr < npairs) rope_sincos(rope_angle(p.rope, c0 / 2 + pr, t, h, w), &sn[pr], &cs[pr]);
+  }
+}
+
+// The chunk token's rotated positional key from the 32 accumulator columns v of the epilogue
+// chunk at output column n, with its pairs' sine and cosine from gemm_key_sincos: each value is
+// taken as chunk_lat stores it (rounded to bf16), rotated in fp32 and rounded once, as
+// rope_key_row does.
+__device__ __forceinline__ void gemm_chunk_key(const GemmParams& p, int m, int n, const float* v,
+                                               const float* sn, const float* cs) {
+  const int bs = m / p.rk_n_q, j = m % p.rk_n_q;
   const int c0 = n - p.rk_col;                       // a multiple of 32
   const int npairs = min(16, (p.rk_dr - c0) / 2);    // 8 or 16
   uint32_t packed[16];
@@ -126,7 +145,7 @@ __device__ __forceinline__ void gemm_chunk_key(const GemmParams& p, int m, int n
   for (int pr = 0; pr < 16; ++pr) {
     float x0 = __bfloat162float(__float2bfloat16_rn(v[2 * pr]));
     float x1 = __bfloat162float(__float2bfloat16_rn(v[2 * pr + 1]));
-    if (pr < npairs) rope_rotate(x0, x1, rope_angle(p.rope, c0 / 2 + pr, t, h, w));
+    rope_apply(x0, x1, sn[pr], cs[pr]);
     packed[pr] = pack_bf16x2(x0, x1);
   }
   uint4* d4 = reinterpret_cast<uint4*>(
@@ -316,6 +335,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     int lt = 0, chunk = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
       const int acc = lt & 1;
+      // the rotated-key chunk this group drains in this tile, if any (output column rk_n), with
+      // its rotary sines and cosines for this thread's row, while the tile's MMAs run
+      int rk_n = -1;
+      float rk_sin[16], rk_cos[16];
+      if (p.rk != nullptr) {
+        const TileCoord tk = tile_coord(p, t);
+        const int kn0 = tk.n0 * BN;
+        for (int c = p.rk_col; c < p.rk_col + p.rk_dr; c += kEpiCols)
+          if (c >= kn0 && c < kn0 + BN && (((c - kn0) / kEpiCols) & 1) == grp) rk_n = c;
+        if (rk_n >= 0 && tk.m0 + row < p.M) gemm_key_sincos(p, tk.m0 + row, rk_n, rk_sin, rk_cos);
+      }
       const bool ok = __all_sync(0xffffffffu, mbar_wait_or_abort(smem_u32(&acc_full[acc]),
                                                                   (lt >> 1) & 1, abort_flag, nullptr));
       if (!ok) break;
@@ -357,8 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const bool second = p.n_split > 0 && n >= p.n_split;
-        if (p.rk != nullptr && n >= p.rk_col && n < p.rk_col + p.rk_dr && m < p.M)
-          gemm_chunk_key(p, m, n, v);
+        if (n == rk_n && m < p.M) gemm_chunk_key(p, m, n, v, rk_sin, rk_cos);
         if (p.ring != nullptr && m < p.M) {
           // the same row into its ring slot (whole frames wrap; row width N)
           const int bs = m / p.ring_n_q, r = m % p.ring_n_q;
