@@ -104,6 +104,33 @@ def test_null_pointers_rejected_without_a_device():
     assert st == _lib.MLA_ERR_INVALID_ARG
 
 
+def test_projection_with_rotated_keys_checks_without_a_device():
+    """mla_project_latents_rotated and mla_attention_fwd_from_cq_prerotated refuse bad
+    arguments on the host before any device call."""
+    c = api.make_config(inputs.CONFIGS[1])
+    lib = _lib.lib()
+    st = lib.mla_project_latents_rotated(ctypes.byref(c), None, None, None, None, None, None, 7,
+                                         0, 1, None, 0, None, None)
+    assert st == _lib.MLA_ERR_INVALID_ARG and "n_valid_frames" in _lib.last_error()
+    st = lib.mla_project_latents_rotated(ctypes.byref(c), None, None, None, None, None, None, 6,
+                                         0, 2, None, 0, None, None)
+    assert st == _lib.MLA_ERR_INVALID_ARG and "rotate_ring" in _lib.last_error()
+    st = lib.mla_project_latents_rotated(ctypes.byref(c), None, None, None, None, None, None, 6,
+                                         -1, 1, None, 0, None, None)
+    assert st == _lib.MLA_ERR_INVALID_ARG and "first_frame" in _lib.last_error()
+    st = lib.mla_project_latents_rotated(ctypes.byref(c), None, None, None, None, None, None, 6,
+                                         6, 1, None, 0, None, None)
+    assert st == _lib.MLA_ERR_INVALID_ARG and "x is null" in _lib.last_error()
+    st = lib.mla_attention_fwd_from_cq_prerotated(ctypes.byref(c), None, None, None, None, None,
+                                                  7, 0, None, None, None, None, 0, None, None)
+    assert st == _lib.MLA_ERR_INVALID_ARG and "n_valid_frames" in _lib.last_error()
+    fp32 = api.make_config(inputs.CONFIGS[0])
+    st = lib.mla_attention_fwd_from_cq_prerotated(ctypes.byref(fp32), None, None, None, None,
+                                                  None, 0, 0, None, None, None, None, 0, None,
+                                                  None)
+    assert st == _lib.MLA_ERR_UNSUPPORTED
+
+
 def test_frame_index_overflow_rejected_without_a_device():
     c = api.make_config(inputs.CONFIGS[1])              # chunk_frames 3
     lib = _lib.lib()

@@ -98,9 +98,11 @@ def test_wan_config1_sampled_rows():
 
 
 def test_wan_config3_batch8_sampled_rows():
-    """Config 3: 8 independent samples, window 9 frames, chunk 3 frames; 512 sampled rows of
-    every sample (every 128-row query tile holds some), then the append and every sample's ring
-    (slots bit-exact, contents within tolerance)."""
+    """Config 3: 8 independent samples, window 9 frames, chunk 3 frames, on the bench's path
+    (rotated keys from the x-projection, query heads formed in the attention kernel); 512
+    sampled rows of every sample (every 128-row query tile holds some) against the oracle, every
+    row against the unfused path, then the append and every sample's ring (slots bit-exact,
+    contents within tolerance)."""
     cfg = inputs.CONFIGS[3]
     g, o = prefilled(cfg, api.MLA_PATH_AUTO, cfg.measured_chunk)
     check_ring(cfg, g, o)
@@ -111,14 +113,20 @@ def test_wan_config3_batch8_sampled_rows():
     pos = g.key_positions(ch)
     for b in range(cfg.batch):
         np.testing.assert_array_equal(pos[b], expected_key_positions(cfg, o.windows[b], cfg.first_frame(ch)))
-    check_chunk("cfg3", cfg, g.attend(ch, x), o.step(ch, x, rows), rows)
+    rf = g.attend(ch, x, fused_q=True)
+    check_chunk("cfg3", cfg, rf, o.step(ch, x, rows), rows)
+    ra = g.attend(ch, x)
+    for k in ("o", "o_lat", "lse"):
+        assert np.abs(ra[k] - rf[k]).max() <= 2.0 ** -8 * max(1.0, np.abs(ra[k]).max()), k
     g.append(ch)
     check_ring(cfg, g, o)
 
 
 def test_wan_config2_long_rollout_sampled():
     """Config 2: 80 chunks, window 21 frames; temporal positions reach t = 239 and the ring
-    wraps every 7 chunks.  Every chunk runs the whole path on the GPU.  The oracle evaluates 512
+    wraps every 7 chunks.  Every chunk runs the whole path on the GPU as the bench runs it
+    (rotated keys from the x-projection, query heads formed in the attention kernel).  The
+    oracle evaluates 512
     sampled rows (every query tile holds some) with all heads at chunks 0-8 (the window fills,
     then the first wraps) and 76-79 (t up to 239), with the key positions; after every chunk's
     append the whole ring is compared (slots bit-exact, contents within tolerance)."""
@@ -133,10 +141,10 @@ def test_wan_config2_long_rollout_sampled():
         if ch in checked:
             pos = g.key_positions(ch)
             np.testing.assert_array_equal(pos[0], expected_key_positions(cfg, o.windows[0], cfg.first_frame(ch)))
-            check_chunk(f"cfg2.chunk{ch}", cfg, g.attend(ch, x, want_latent=False),
+            check_chunk(f"cfg2.chunk{ch}", cfg, g.attend(ch, x, want_latent=False, fused_q=True),
                         o.step(ch, x, rows), rows)
         else:
-            g.attend(ch, x, want_latent=False)
+            g.attend(ch, x, want_latent=False, fused_q=True)
             o.prefill(ch, x)
         g.append(ch)
         check_ring(cfg, g, o)
@@ -233,6 +241,34 @@ def test_rotated_keys_from_the_projection_epilogue(d_c, d_rope):
         assert torch.equal(ws[:nbytes], ws_ref[:nbytes]), ch
         assert torch.equal(ws_frozen[:nbytes], ws_ref[:nbytes]), ch
         assert torch.equal(o2, b.o) and torch.equal(lse2, b.lse), ch
+        rollout.check_device_status(b)
+        g.append(ch)
+
+
+@pytest.mark.parametrize("which", ["fp32_toy", "bf16_cuda_cores"])
+def test_rotated_keys_without_the_fused_epilogue(which):
+    """Where the tensor-core GEMM does not serve (fp32, or the CUDA-core path forced),
+    mla_project_latents_rotated runs the projection GEMMs and then the rotation pass; over a
+    rollout whose ring wraps, its outputs and workspace equal those of mla_project_chunk and the
+    rotation pass inside mla_attention_fwd."""
+    cfg = inputs.CONFIGS[0] if which == "fp32_toy" else inputs.small_bf16_config()
+    g = GpuRun(cfg, api.MLA_PATH_SIMT if which == "bf16_cuda_cores" else api.MLA_PATH_AUTO)
+    c, b, w = g.c, g.buf, g.w
+    cq2, lat2 = torch.empty_like(b.c_q), torch.empty_like(b.chunk_lat)
+    for ch in range(cfg.n_chunks):
+        first, n_valid = rollout.chunk_schedule(cfg.chunk_frames, cfg.window_frames, ch)
+        nbytes = api.mla_attention_workspace_bytes(c, n_valid)
+        g.load_x(inputs.chunk_x(cfg, ch))
+        ws_ref = torch.full_like(b.workspace, 0x5A)
+        api.mla_project_chunk(c, b.x, w.w_x, w.w_qcat, b.c_q, b.q, b.chunk_lat, first)
+        api.mla_attention_fwd(c, b.q, b.chunk_lat, g.ring.cache, g.ring.slot_frame, n_valid,
+                              first, w.w_uv, b.o, b.lse, ws_ref, b.dev_status)
+        ws = torch.full_like(b.workspace, 0xA5)
+        api.mla_project_latents_rotated(c, b.x, w.w_x, cq2, lat2, g.ring.cache, g.ring.slot_frame,
+                                        n_valid, first, ws, dev_status=b.dev_status)
+        torch.cuda.synchronize()
+        assert torch.equal(cq2, b.c_q) and torch.equal(lat2, b.chunk_lat), ch
+        assert torch.equal(ws[:nbytes], ws_ref[:nbytes]), ch
         rollout.check_device_status(b)
         g.append(ch)
 
