@@ -101,15 +101,21 @@ def fused_query_supported(c) -> bool:
             and c.d_cq % 64 == 0 and c.d_head == 128)
 
 
+def _use_fused_q(c, fused_q: Optional[bool]) -> bool:
+    """fused_q as given, or (None) the fused form wherever the configuration allows it."""
+    return fused_query_supported(c) if fused_q is None else bool(fused_q)
+
+
 def attend_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
-                 fuse_uv: bool = True, stream=None, fused_q: bool = False) -> torch.Tensor:
+                 fuse_uv: bool = True, stream=None, fused_q: Optional[bool] = None) -> torch.Tensor:
     """Query path, chunk latents and attention of one chunk (buf.x holds its tokens).
     Returns buf.o (fused W_UV) or buf.o_lat (latent output).  With fused_q the x-projection also
     writes every rotated positional key of the call and the attention kernel forms the query
-    heads itself from c_Q (buf.q is then not written): two launches."""
+    heads itself from c_Q (buf.q is then not written): two launches.  fused_q=None picks the
+    fused form wherever the configuration allows it."""
     first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
     out = buf.o if fuse_uv else buf.o_lat
-    if fused_q:
+    if _use_fused_q(c, fused_q):
         _attend_from_cq(c, w, ring, buf, buf.x, n_valid, first, out, fuse_uv, buf.workspace,
                         rotate_ring=True, stream=stream)
         return out
@@ -153,7 +159,7 @@ def prefill_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int
 
 
 def run_chunk(c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
-              fuse_uv: bool = True, stream=None, fused_q: bool = False) -> torch.Tensor:
+              fuse_uv: bool = True, stream=None, fused_q: Optional[bool] = None) -> torch.Tensor:
     """One whole chunk: attend, then append."""
     out = attend_chunk(c, w, ring, buf, chunk, fuse_uv=fuse_uv, stream=stream, fused_q=fused_q)
     append_chunk(c, ring, buf, chunk, stream=stream)
@@ -197,7 +203,7 @@ class HostStreamer:
         self.d2h.wait_event(event)
 
     def submit(self, chunk: int, x_host: torch.Tensor, o_host: torch.Tensor,
-               fuse_uv: bool = True, fused_q: bool = False) -> None:
+               fuse_uv: bool = True, fused_q: Optional[bool] = None) -> None:
         """Enqueues chunk `chunk`: copy-in of x_host, attention, append, copy-out into o_host."""
         k = self.n % 2
         b = self.bufs[k]
@@ -249,8 +255,9 @@ class ChunkGraph:
 
     def __init__(self, c, w: DeviceWeights, ring: Ring, buf: ChunkBuffers, chunk: int,
                  x: Optional[torch.Tensor] = None, events: bool = False, fuse_uv: bool = True,
-                 fused_q: bool = False):
+                 fused_q: Optional[bool] = None):
         self.chunk = chunk
+        fused_q = _use_fused_q(c, fused_q)
         first, n_valid = chunk_schedule(c.chunk_frames, c.window_frames, chunk)
         x = buf.x if x is None else x
         # external events: recorded by the graph at replay time (a plain event recorded during
