@@ -582,22 +582,24 @@ mla_status gemm_tc(const TcGemmArgs& g, cudaStream_t s) {
       (g.rope_D <= 0 || g.N % g.rope_D != 0 || g.rope_dr % 2 != 0 || g.rope_dr > g.rope_D ||
        g.rope_dr / 2 > kMaxRopePairs))
     MLA_FAIL(MLA_ERR_UNSUPPORTED, "query RoPE epilogue needs whole head blocks and even d_rope");
-  // Tile width: the one whose tiles spread most evenly over the SMs (each persistent CTA takes
-  // ceil(tiles / SMs) tiles) with the least padding in N; ties go to the wider tile, which
-  // re-reads A fewer times.  Projections here have few 128-row tiles, so a narrower N tile is
-  // often what puts every SM to work.
+  // Tile width: the one with the least modelled time.  A persistent CTA takes ceil(tiles / SMs)
+  // tiles one after another, and a tile's main loop is paced by the operand bytes it streams
+  // into shared memory, K * (128 + width) * 2 (measured: these GEMMs run far below the tensor
+  // rate), so the model is rounds * (128 + width); ties go to the wider tile.  Few rows (one
+  // chunk) favour a width that fills every SM in one round; many rows favour wide tiles, which
+  // re-read the A panel fewer times (x-projection of 32 chunks: 263 us with 256-wide tiles
+  // against 728 us with 64-wide ones, which an SM-fill criterion alone had picked).
   const int sms = num_sms();
   const int widths[5] = {256, 224, 192, 128, 64};
   int best = 256;
-  double best_eff = -1.0;
+  long long best_cost = -1;
   for (int w : widths) {
     const long long tiles =
         static_cast<long long>(ceil_div(g.M, kBM)) * ceil_div(g.N, w) * g.batch;
     const long long rounds = (tiles + sms - 1) / sms;
-    const double eff = static_cast<double>(tiles) / static_cast<double>(rounds * sms) *
-                       (static_cast<double>(g.N) / (ceil_div(g.N, w) * w));
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
+    const long long cost = rounds * (kBM + w);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
       best = w;
     }
   }
