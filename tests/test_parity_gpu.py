@@ -467,9 +467,11 @@ def test_layer_stack_graph_matches_eager():
 
 
 def test_layer_stack_fused_query_matches_q_gemm():
-    """The layer stack's cached-ring attention with the query heads formed inside the kernel
-    (mla_attention_fwd_from_cq_cached_ring) against mla_project_chunk +
-    mla_attention_fwd_cached_ring: identical rings and outputs over 4 chunks (rings wrap)."""
+    """The layer stack's default form (the chunk's rotated keys from the x-projection,
+    mla_project_latents_rotated with rotate_ring=0 beside the ring keys rotated once per chunk,
+    then the attention forming the query heads itself) against mla_project_chunk +
+    mla_attention_fwd_cached_ring: identical rings and outputs to a bf16 ulp over 4 chunks (rings
+    wrap)."""
     cfg = inputs.small_bf16_config()
     c = api.make_config(cfg)
     n_layers, n_steps = 2, 2
