@@ -264,10 +264,9 @@ mla_status ring_append(const Dims& d, const void* chunk_lat, void* cache, int32_
   const int64_t total = static_cast<int64_t>(d.B) * d.C * vec_per_frame;
   const int threads = 256;
   const int blocks = static_cast<int>(std::min<int64_t>((total + threads - 1) / threads, 148 * 8));
-  launch_pdl(ring_append_kernel, dim3(blocks), dim3(threads), 0, s,
-             static_cast<const uint4*>(chunk_lat), static_cast<uint4*>(cache), slot_frame, d.B,
-             d.C, d.W, vec_per_frame, first_frame);
-  MLA_LAUNCH_CHECK("ring_append");
+  MLA_CUDA_TRY(launch_pdl(ring_append_kernel, dim3(blocks), dim3(threads), 0, s,
+                          static_cast<const uint4*>(chunk_lat), static_cast<uint4*>(cache),
+                          slot_frame, d.B, d.C, d.W, vec_per_frame, first_frame));
   return MLA_OK;
 }
 
@@ -412,10 +411,11 @@ mla_status build_rope_keys(const Dims& d, const void* cache, const void* chunk_l
     const int64_t vtotal = static_cast<int64_t>(d.B) * (row_end - row_begin);
     const int vblocks = static_cast<int>(std::min<int64_t>((vtotal + 255) / 256, 148 * 16));
 #define MLA_KEYS_VEC(T, P)                                                                       \
-  launch_pdl(rope_keys_vec_kernel<T, P>, dim3(vblocks), dim3(256), 0, s,                       \
-             static_cast<const T*>(cache), static_cast<const T*>(chunk_lat), slot_frame,       \
-             static_cast<T*>(ws), d.B, d.W, d.D, d.d_c, d.n_q, k.nc, k.nc_pad, k.rows,         \
-             row_begin, row_end, first_frame, g, dev_status, check_window)
+  MLA_CUDA_TRY(launch_pdl(rope_keys_vec_kernel<T, P>, dim3(vblocks), dim3(256), 0, s,          \
+                          static_cast<const T*>(cache), static_cast<const T*>(chunk_lat),      \
+                          slot_frame, static_cast<T*>(ws), d.B, d.W, d.D, d.d_c, d.n_q, k.nc,  \
+                          k.nc_pad, k.rows, row_begin, row_end, first_frame, g, dev_status,    \
+                          check_window))
     if (d.dtype == MLA_FP32) {
       if (pieces == 2) MLA_KEYS_VEC(float, 2);
       else if (pieces == 4) MLA_KEYS_VEC(float, 4);
