@@ -203,8 +203,12 @@ class HostStreamer:
         self.d2h.wait_event(event)
 
     def submit(self, chunk: int, x_host: torch.Tensor, o_host: torch.Tensor,
-               fuse_uv: bool = True, fused_q: Optional[bool] = None) -> None:
-        """Enqueues chunk `chunk`: copy-in of x_host, attention, append, copy-out into o_host."""
+               fuse_uv: bool = True, fused_q: Optional[bool] = None,
+               ring: Optional[Ring] = None) -> None:
+        """Enqueues chunk `chunk`: copy-in of x_host, attention, append, copy-out into o_host.
+        `ring` (default: the streamer's own) lets one streamer serve several independent
+        rollouts, each with its ring; chunks of one ring still run in submission order."""
+        ring = self.ring if ring is None else ring
         k = self.n % 2
         b = self.bufs[k]
         with torch.cuda.stream(self.h2d):
@@ -216,7 +220,7 @@ class HostStreamer:
         self.compute.wait_event(x_ready)
         if self.o_free[k] is not None:
             self.compute.wait_event(self.o_free[k])
-        out = run_chunk(self.c, self.w, self.ring, b, chunk, fuse_uv=fuse_uv, stream=self.compute,
+        out = run_chunk(self.c, self.w, ring, b, chunk, fuse_uv=fuse_uv, stream=self.compute,
                         fused_q=fused_q)
         done = torch.cuda.Event()
         done.record(self.compute)
