@@ -390,6 +390,41 @@ def test_host_streamer_matches_serial_rollout():
     assert torch.equal(a.ring.slot_frame, b.ring.slot_frame)
 
 
+def test_host_streamer_serves_independent_rollouts_in_turn():
+    """One HostStreamer serving two rollouts with their own rings, chunks interleaved (the
+    bench's end-to-end form): each rollout's outputs and ring are bit-identical to that rollout
+    run alone with run_chunk."""
+    cfg = inputs.small_bf16_config()
+    xs = [[torch.from_numpy(inputs.chunk_x(cfg, ch, layer=r)).to(torch.bfloat16)
+           for ch in range(cfg.n_chunks)] for r in range(2)]
+    a = GpuRun(cfg)
+    refs, rings = [], []
+    for r in range(2):
+        ring = rollout.Ring(a.c)
+        out = []
+        for ch in range(cfg.n_chunks):
+            a.buf.x.copy_(xs[r][ch])
+            out.append(rollout.run_chunk(a.c, a.w, ring, a.buf, ch).cpu().clone())
+        refs.append(out)
+        rings.append(ring)
+    b = GpuRun(cfg)
+    served = [rollout.Ring(b.c) for _ in range(2)]
+    st = rollout.HostStreamer(b.c, b.w, b.ring)
+    outs = [[torch.empty_like(refs[0][0]).pin_memory() for _ in range(cfg.n_chunks)]
+            for _ in range(2)]
+    for ch in range(cfg.n_chunks):
+        for r in range(2):
+            st.submit(ch, xs[r][ch].pin_memory(), outs[r][ch], ring=served[r])
+    st.finish()
+    torch.cuda.synchronize()
+    st.check_device_status()
+    for r in range(2):
+        for ch in range(cfg.n_chunks):
+            assert torch.equal(outs[r][ch], refs[r][ch]), (r, ch)
+        assert torch.equal(served[r].cache, rings[r].cache), r
+        assert torch.equal(served[r].slot_frame, rings[r].slot_frame), r
+
+
 def test_chunk_graph_replay_matches_eager_rollout():
     """rollout.ChunkGraph (a chunk's projections, attention and append captured as one CUDA
     graph per chunk index) replays to bit-identical outputs and ring state as the eager calls."""
