@@ -97,6 +97,47 @@ def test_wan_config1_sampled_rows():
     check_ring(cfg, g, o)
 
 
+def test_largest_accepted_batch_on_the_bench_path():
+    """The largest batch the library accepts for the Wan preset (170 samples; at 171 the unfused
+    path's Q' array would reach 2^31 elements) through the bench's 3-launch step, one chunk after
+    the window filled: the kernels' address arithmetic at the largest legal offsets.  The first
+    and the last sample get their seeded inputs and are compared with the oracle on sampled rows
+    (every 128-row query tile represented); the other samples get arbitrary values, which
+    cannot reach the checked ones (samples are independent)."""
+    cfg = inputs.CONFIGS[1]
+    top = 170
+    c = api.make_config(cfg, batch=top)
+    lw = inputs.layer_weights(cfg)
+    w = rollout.upload_weights(c, lw)
+    ring, buf = rollout.Ring(c), rollout.ChunkBuffers(c)
+    d = oracle.dims_from(cfg)
+    checked = (0, top - 1)
+    windows = {b: oracle.SlidingWindow(d) for b in checked}
+    gen = torch.Generator(device="cuda").manual_seed(1234)
+    rows = inputs.sample_rows(cfg.n_q, 128, tag=170)
+    assert len(set(rows // 128)) == -(-cfg.n_q // 128)
+    for ch in range(cfg.measured_chunk + 1):
+        buf.x.normal_(generator=gen)
+        xs = {}
+        for b in checked:
+            xs[b] = inputs.chunk_x(cfg, ch, samples=range(b, b + 1))[0]
+            buf.x[b].copy_(torch.from_numpy(xs[b]).to(torch.bfloat16))
+        first = cfg.first_frame(ch)
+        if ch < cfg.measured_chunk:
+            rollout.prefill_chunk(c, w, ring, buf, ch)
+            for b in checked:
+                c_kv, k_r = oracle.down_project(xs[b], lw.w_dkv, lw.w_kr)
+                windows[b].append_chunk(first, c_kv, k_r)
+            continue
+        out = rollout.attend_chunk(c, w, ring, buf, ch)
+        torch.cuda.synchronize()
+        rollout.check_device_status(buf)
+        for b in checked:
+            r = oracle.chunk_step(d, lw, xs[b], windows[b], first, rows=rows, append=False)
+            compare(f"batch{top}.o[b{b}]", to_np(out[b])[rows], r["o"], cfg.dtype)
+            compare(f"batch{top}.lse[b{b}]", to_np(buf.lse[b])[:, rows], r["lse"], "bf16")
+
+
 def test_wan_config3_batch8_sampled_rows():
     """Config 3: 8 independent samples, window 9 frames, chunk 3 frames, on the bench's path
     (rotated keys from the x-projection, query heads formed in the attention kernel); 512
