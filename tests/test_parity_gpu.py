@@ -114,7 +114,7 @@ def test_largest_accepted_batch_on_the_bench_path():
     checked = (0, top - 1)
     windows = {b: oracle.SlidingWindow(d) for b in checked}
     gen = torch.Generator(device="cuda").manual_seed(1234)
-    rows = inputs.sample_rows(cfg.n_q, 128, tag=170)
+    rows = inputs.sample_rows(cfg.n_q, 192, tag=170)
     assert len(set(rows // 128)) == -(-cfg.n_q // 128)
     for ch in range(cfg.measured_chunk + 1):
         buf.x.normal_(generator=gen)
