@@ -5,6 +5,8 @@ Floating point: bf16 workloads within max-abs 2e-2 and rel-L2 5e-3, fp32 within 
 for every intermediate the ABI exposes (chunk latents, query latent, absorbed query, latent
 output, output, lse).  Integer work (key positions, ring slots) is bit-exact.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -53,6 +55,25 @@ def test_small_frames_bf16_rollout(path):
 
 
 LATENT_SHAPES = [(dc, dr) for dc in (128, 192, 256) for dr in (16, 32, 64)]
+
+
+@pytest.mark.parametrize("fused_q", [False, True])
+def test_window_of_one_chunk_replaces_the_whole_ring(fused_q):
+    """Degenerate window: W = C = 3 frames, so every append overwrites every slot of the ring and
+    each chunk attends to exactly the previous chunk plus itself.  A 5-chunk rollout of 2
+    samples on both paths (unfused; the 3-launch step), every row and the ring against the
+    oracle."""
+    cfg = dataclasses.replace(inputs.small_bf16_config(), window_frames=3, n_chunks=5,
+                              name="wan_layer_small_frames_w3")
+    g = GpuRun(cfg)
+    o = OracleRun(cfg, g.lw)
+    rows = np.arange(cfg.n_q)
+    for ch in range(cfg.n_chunks):
+        x = inputs.chunk_x(cfg, ch)
+        check_chunk(f"w3.chunk{ch}", cfg, g.attend(ch, x, fused_q=fused_q), o.step(ch, x, rows), rows)
+        g.append(ch)
+        check_ring(cfg, g, o)
+    assert int(g.ring.slot_frame.min()) == 3 * (cfg.n_chunks - 1)
 
 
 @pytest.mark.parametrize("path", ["tc", "pair"])
