@@ -233,15 +233,20 @@ class OracleRows:
         self.k_rope = o.rope3d(k_r_all, pos_all, self.d)
         self.setup_s = time.perf_counter() - t0
 
-    def __call__(self, rows: int, seed_tag: int = 7):
-        o, cfg, lw, d = self.o, self.cfg, self.lw, self.d
-        sel = self.sample.inputs.sample_rows(cfg.n_q, rows, tag=seed_tag)
-        t0 = time.perf_counter()
+    def evaluate(self, sel):
+        """The rows' part of chunk_step for the query rows `sel`: their attention results."""
+        o, lw, d = self.o, self.lw, self.d
         c_q = o.query_latent(self.sample.x[sel], lw.w_dq)
         q_nope, q_r = o.query_heads(c_q, lw.w_uq, lw.w_qr)
         q_rope = o.rope3d(q_r, self.pos_chunk[sel], d)
-        o.attend(q_nope, q_rope, self.k_nope, self.k_rope, self.v, d.softmax_scale,
-                 c_keys=self.c_all)
+        return o.attend(q_nope, q_rope, self.k_nope, self.k_rope, self.v, d.softmax_scale,
+                        c_keys=self.c_all)
+
+    def __call__(self, rows: int, seed_tag: int = 7):
+        cfg = self.cfg
+        sel = self.sample.inputs.sample_rows(cfg.n_q, rows, tag=seed_tag)
+        t0 = time.perf_counter()
+        self.evaluate(sel)
         dt = time.perf_counter() - t0
         flops = 2.0 * (cfg.d_latent + cfg.d_c) * len(sel) * \
             cfg.keys_per_query(cfg.measured_chunk) * cfg.n_heads

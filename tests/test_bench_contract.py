@@ -7,6 +7,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -109,3 +110,20 @@ def test_clock_summary_uses_the_samples_stamped_inside_the_timed_region():
                           "1965, 1965, 200.0, 0x0000000000000001, 0"]
     s = clk.summary()
     assert s["sm_mhz"] == 1700 and s["from"] == "utilisation >= 50 %" and s["samples"] == 2
+
+
+def test_reference_split_computes_what_one_oracle_call_does():
+    """The reference arm builds the chunk's keys once and evaluates sampled rows per step
+    (bench.OracleRows); for the same rows that is exactly oracle.chunk_step's result."""
+    import bench
+    import oracle
+    from mla_latent_kv_attn_b200 import inputs
+    cfg = inputs.small_bf16_config()
+    sample = bench.OracleSample(cfg)
+    prep = bench.OracleRows(sample)
+    rows = inputs.sample_rows(cfg.n_q, 37, tag=5)
+    got = prep.evaluate(rows)
+    ref = oracle.chunk_step(sample.d, sample.lw, sample.x, sample.win,
+                            cfg.first_frame(cfg.measured_chunk), rows=rows, append=False)
+    for k in ("o", "o_lat", "lse"):
+        assert np.array_equal(got[k], ref[k]), k
